@@ -1,0 +1,50 @@
+"""FP8 (e4m3fn) per-tensor quantisation, fp64 emulation — test infrastructure.
+
+[AP-lin]: with --fp8 "most layers" become Float8Linear with per-tensor
+scaling.  The pages give nothing more; the reading used here is dynamic
+scaling from the tensor's own absolute maximum, s = 448 / amax, values
+rounded to the nearest e4m3fn value (ties to even) and saturated at ±448.
+
+e4m3fn: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no
+infinities; largest finite 448; smallest normal 2^-6; subnormal spacing 2^-9.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+E4M3_MAX = 448.0
+_MIN_NORMAL_EXP = -6   # smallest normal is 2^-6
+_MANT_BITS = 3
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Nearest e4m3fn value to each element (ties to even), saturating to ±448."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    # binade exponent e with 2^e <= a < 2^(e+1); below the normal range the
+    # spacing stays that of the smallest binade (subnormals)
+    _, ex = np.frexp(np.maximum(a, 2.0 ** _MIN_NORMAL_EXP))
+    e = ex.astype(np.float64) - 1.0
+    ulp = np.exp2(e - _MANT_BITS)
+    y = np.round(a / ulp) * ulp          # numpy rounds halves to even
+    y = np.minimum(y, E4M3_MAX)
+    return np.copysign(y, x)
+
+
+def fp8_scale(t: np.ndarray) -> float:
+    """Per-tensor scale: 448 / max|t| (a floor keeps an all-zero tensor finite)."""
+    amax = float(np.max(np.abs(t))) if t.size else 0.0
+    return E4M3_MAX / max(amax, 1e-12)
+
+
+def quantize_e4m3(t: np.ndarray) -> tuple[np.ndarray, float]:
+    """Return (codes as fp64 values, scale) with t ~= codes / scale."""
+    s = fp8_scale(t)
+    return e4m3_round(np.asarray(t, dtype=np.float64) * s), s
+
+
+def fp8_matmul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """a @ b with both operands quantised per tensor to e4m3, fp64 accumulate."""
+    qa, sa = quantize_e4m3(a)
+    qb, sb = quantize_e4m3(b)
+    return (qa @ qb) / (sa * sb)
