@@ -1,0 +1,237 @@
+"""Python binding of libgptblock.so (the C ABI declared in include/gptblock.h).
+
+Argument marshalling only: every step of the block runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the stream.  There is no CPU or
+PyTorch fallback: if the library is missing the import of the binding raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgptblock.so")
+MAX_LAYERS = 64
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+F32, BF16, FP8_E4M3 = 0, 1, 2
+WS_BLOCK_SAVED, WS_BLOCK_SCRATCH, WS_LM_HEAD, WS_STACK = 0, 1, 2, 3
+DTYPES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3}
+
+EXPORTS = [
+    "gptb_workspace_bytes", "gpt_block_forward", "gpt_block_backward", "lm_head_xent",
+    "gpt_stack_step", "gptb_gemm_bf16", "gptb_device_error", "gptb_set_wait_limit_ns",
+    "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
+    "gptb_error_string",
+]
+
+_vp = ctypes.c_void_p
+_fp = ctypes.POINTER(ctypes.c_float)
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("d", ctypes.c_int),
+        ("n_head", ctypes.c_int), ("n_kv_head", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("mlp_hidden", ctypes.c_int), ("vocab", ctypes.c_int), ("n_layer", ctypes.c_int),
+        ("window", ctypes.c_int * MAX_LAYERS), ("has_ve", ctypes.c_int * MAX_LAYERS),
+        ("ve_gate_ch", ctypes.c_int), ("smear_ch", ctypes.c_int), ("backout_layer", ctypes.c_int),
+        ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float), ("dtype", ctypes.c_int),
+    ]
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [("w_qkv", _vp), ("w_o", _vp), ("w_fc", _vp), ("w_proj", _vp),
+                ("w_ve_gate", _vp), ("ve_table", _vp), ("lambdas", _vp)]
+
+
+class BlockGrads(ctypes.Structure):
+    _fields_ = [("w_qkv", _vp), ("w_o", _vp), ("w_fc", _vp), ("w_proj", _vp),
+                ("w_ve_gate", _vp), ("ve_table", _vp), ("lambdas", _vp)]
+
+
+class ModelWeights(ctypes.Structure):
+    _fields_ = [("wte", _vp), ("w_lm", _vp), ("w_smear_gate", _vp), ("smear_lambda", _vp),
+                ("backout_lambda", _vp), ("layers", BlockWeights * MAX_LAYERS)]
+
+
+class ModelGrads(ctypes.Structure):
+    _fields_ = [("wte", _vp), ("w_lm", _vp), ("w_smear_gate", _vp), ("smear_lambda", _vp),
+                ("backout_lambda", _vp), ("layers", BlockGrads * MAX_LAYERS)]
+
+
+_LIB = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it was not built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m gpt_transformer_block_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER
+    lib.gptb_workspace_bytes.argtypes = [P(Config), ctypes.c_int]
+    lib.gptb_workspace_bytes.restype = ctypes.c_size_t
+    lib.gpt_block_forward.argtypes = [P(Config), ctypes.c_int, P(BlockWeights), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.gpt_block_backward.argtypes = [P(Config), ctypes.c_int, P(BlockWeights), _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, P(BlockGrads), _vp, _vp]
+    lib.lm_head_xent.argtypes = [P(Config), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.gpt_stack_step.argtypes = [P(Config), P(ModelWeights), _vp, _vp, _vp, P(ModelGrads), _vp, _vp]
+    lib.gptb_gemm_bf16.argtypes = [_vp, ctypes.c_int, ctypes.c_longlong, _vp, ctypes.c_int, ctypes.c_longlong,
+                                   _vp, ctypes.c_int, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_int, _vp]
+    lib.gptb_device_error.argtypes = [_vp]
+    lib.gptb_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.gptb_reset_counters.restype = None
+    lib.gptb_launch_count.restype = ctypes.c_longlong
+    lib.gptb_set_gemm_timing.argtypes = [ctypes.c_int]
+    lib.gptb_gemm_timing.argtypes = [P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_longlong)]
+    lib.gptb_error_string.argtypes = [ctypes.c_int]
+    lib.gptb_error_string.restype = ctypes.c_char_p
+    for name in EXPORTS:
+        if name not in ("gptb_workspace_bytes", "gptb_error_string", "gptb_reset_counters",
+                        "gptb_launch_count"):
+            getattr(lib, name).restype = ctypes.c_int
+    _LIB = lib
+    return lib
+
+
+class GPTBError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        msg = load().gptb_error_string(code).decode()
+        super().__init__(f"{what}: {msg} ({code})")
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise GPTBError(rc, what)
+
+
+def ptr(t) -> int | None:
+    """Device address of a tensor (None for None)."""
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def make_config(c: dict) -> Config:
+    """Build the C config from a plain dict (keys of the workload presets)."""
+    cfg = Config()
+    for k in ("B", "T", "d", "n_head", "n_kv_head", "head_dim", "mlp_hidden", "vocab", "n_layer",
+              "ve_gate_ch", "smear_ch", "backout_layer"):
+        setattr(cfg, k, int(c[k]))
+    L = int(c["n_layer"])
+    if L > MAX_LAYERS:
+        raise ValueError("too many layers")
+    for i in range(L):
+        cfg.window[i] = int(c["window"][i])
+        cfg.has_ve[i] = int(c["has_ve"][i])
+    cfg.rope_base = float(c["rope_base"])
+    cfg.norm_eps = float(c["norm_eps"])
+    cfg.dtype = DTYPES[c["dtype"]] if isinstance(c["dtype"], str) else int(c["dtype"])
+    return cfg
+
+
+def block_weights(lw: dict) -> BlockWeights:
+    """lw: device tensors w_qkv, w_o, w_fc, w_proj, lambdas [2] fp32, optional w_ve_gate, ve_table."""
+    return BlockWeights(ptr(lw["w_qkv"]), ptr(lw["w_o"]), ptr(lw["w_fc"]), ptr(lw["w_proj"]),
+                        ptr(lw.get("w_ve_gate")), ptr(lw.get("ve_table")), ptr(lw["lambdas"]))
+
+
+def block_grads(lg: dict) -> BlockGrads:
+    return BlockGrads(ptr(lg["w_qkv"]), ptr(lg["w_o"]), ptr(lg["w_fc"]), ptr(lg["w_proj"]),
+                      ptr(lg.get("w_ve_gate")), ptr(lg.get("ve_table")), ptr(lg["lambdas"]))
+
+
+def model_weights(w: dict) -> ModelWeights:
+    mw = ModelWeights()
+    mw.wte, mw.w_lm = ptr(w["wte"]), ptr(w["w_lm"])
+    mw.w_smear_gate = ptr(w.get("w_smear_gate"))
+    mw.smear_lambda = ptr(w.get("smear_lambda"))
+    mw.backout_lambda = ptr(w.get("backout_lambda"))
+    for i, lw in enumerate(w["layers"]):
+        mw.layers[i] = block_weights(lw)
+    return mw
+
+
+def model_grads(g: dict) -> ModelGrads:
+    mg = ModelGrads()
+    mg.wte, mg.w_lm = ptr(g["wte"]), ptr(g["w_lm"])
+    mg.w_smear_gate = ptr(g.get("w_smear_gate"))
+    mg.smear_lambda = ptr(g.get("smear_lambda"))
+    mg.backout_lambda = ptr(g.get("backout_lambda"))
+    for i, lg in enumerate(g["layers"]):
+        mg.layers[i] = block_grads(lg)
+    return mg
+
+
+# ---------------------------------------------------------------- entry points
+
+def gptb_workspace_bytes(cfg: Config, kind: int) -> int:
+    return int(load().gptb_workspace_bytes(ctypes.byref(cfg), kind))
+
+
+def gpt_block_forward(cfg, layer, w: BlockWeights, x, x0, idx, x_out, saved, scratch, stream=None):
+    _check(load().gpt_block_forward(ctypes.byref(cfg), layer, ctypes.byref(w), ptr(x), ptr(x0), ptr(idx),
+                                    ptr(x_out), ptr(saved), ptr(scratch), _stream(stream)), "gpt_block_forward")
+
+
+def gpt_block_backward(cfg, layer, w: BlockWeights, x, x0, idx, saved, dx_out, dx_extra, dx, dx0_accum,
+                       g: BlockGrads, scratch, stream=None):
+    _check(load().gpt_block_backward(ctypes.byref(cfg), layer, ctypes.byref(w), ptr(x), ptr(x0), ptr(idx),
+                                     ptr(saved), ptr(dx_out), ptr(dx_extra), ptr(dx), ptr(dx0_accum),
+                                     ctypes.byref(g), ptr(scratch), _stream(stream)), "gpt_block_backward")
+
+
+def lm_head_xent(cfg, h, w_lm, targets, loss_out, dh, dw_lm, ws, stream=None):
+    _check(load().lm_head_xent(ctypes.byref(cfg), ptr(h), ptr(w_lm), ptr(targets), ptr(loss_out), ptr(dh),
+                               ptr(dw_lm), ptr(ws), _stream(stream)), "lm_head_xent")
+
+
+def gpt_stack_step(cfg, w: ModelWeights, idx, targets, loss_out, g: ModelGrads, ws, stream=None):
+    _check(load().gpt_stack_step(ctypes.byref(cfg), ctypes.byref(w), ptr(idx), ptr(targets), ptr(loss_out),
+                                 ctypes.byref(g), ptr(ws), _stream(stream)), "gpt_stack_step")
+
+
+def gptb_gemm_bf16(A, a_mn, lda, B, b_mn, ldb, C, c_f32, ldc, M, N, K, stream=None):
+    _check(load().gptb_gemm_bf16(ptr(A), int(a_mn), lda, ptr(B), int(b_mn), ldb, ptr(C), int(c_f32), ldc,
+                                 M, N, K, _stream(stream)), "gptb_gemm_bf16")
+
+
+def gptb_device_error(stream=None) -> int:
+    return int(load().gptb_device_error(_stream(stream)))
+
+
+def gptb_set_wait_limit_ns(ns: int):
+    _check(load().gptb_set_wait_limit_ns(int(ns)), "gptb_set_wait_limit_ns")
+
+
+def gptb_reset_counters():
+    load().gptb_reset_counters()
+
+
+def gptb_launch_count() -> int:
+    return int(load().gptb_launch_count())
+
+
+def gptb_set_gemm_timing(enable: bool):
+    _check(load().gptb_set_gemm_timing(1 if enable else 0), "gptb_set_gemm_timing")
+
+
+def gptb_gemm_timing():
+    ms, fl, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_longlong()
+    _check(load().gptb_gemm_timing(ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(n)), "gptb_gemm_timing")
+    return ms.value, fl.value, n.value
+
+
+from .model import GPTStack, BlockRunner, to_device_weights  # noqa: E402,F401

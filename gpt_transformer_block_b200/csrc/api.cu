@@ -1,0 +1,741 @@
+// C ABI of the GPT block library: argument checks, workspace layout and the
+// launch sequence of one block / one stack training step.  All compute runs
+// in the kernels included below (single translation unit).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/gptblock.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+
+using namespace gptb;
+
+namespace {
+
+// ------------------------------------------------------------ accounting --
+std::atomic<long long> g_launches{0};
+std::mutex g_timing_mu;
+bool g_timing = false;
+struct TimedLaunch {
+  cudaEvent_t a, b;
+  double flops;
+};
+std::vector<TimedLaunch> g_timed;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+#define LAUNCHED() g_launches.fetch_add(1, std::memory_order_relaxed)
+#define CK(x)                                   \
+  do {                                          \
+    if ((x) != cudaSuccess) return GPTB_ERR_CUDA; \
+  } while (0)
+#define CKL()                                                  \
+  do {                                                         \
+    LAUNCHED();                                                \
+    if (cudaPeekAtLastError() != cudaSuccess) {                \
+      cudaGetLastError();                                      \
+      return GPTB_ERR_CUDA;                                    \
+    }                                                          \
+  } while (0)
+// instantiate a row kernel for NC = ceil(d / 256) chunks per lane
+#define ROWK(NCV, ...)                                     \
+  switch (NCV) {                                           \
+    case 1: { constexpr int NC = 1; __VA_ARGS__; } break;  \
+    case 2: { constexpr int NC = 2; __VA_ARGS__; } break;  \
+    case 3: { constexpr int NC = 3; __VA_ARGS__; } break;  \
+    case 4: { constexpr int NC = 4; __VA_ARGS__; } break;  \
+    case 5: { constexpr int NC = 5; __VA_ARGS__; } break;  \
+    case 6: { constexpr int NC = 6; __VA_ARGS__; } break;  \
+    case 7: { constexpr int NC = 7; __VA_ARGS__; } break;  \
+    case 8: { constexpr int NC = 8; __VA_ARGS__; } break;  \
+    default: return GPTB_ERR_UNSUPPORTED;                  \
+  }
+#define TRY(x)                     \
+  do {                             \
+    int _r = (x);                  \
+    if (_r != GPTB_OK) return _r;  \
+  } while (0)
+
+// ------------------------------------------------------------ device info --
+struct DevInfo {
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+DevInfo dev_info() {
+  static DevInfo cache[64];
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  DevInfo& d = cache[dev & 63];
+  if (d.sms == 0) {
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+  }
+  return d;
+}
+
+// ------------------------------------------------------------ tensor maps --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D tensor map with 128-byte swizzle: inner extent `inner`, `outer` rows of
+// `ld` elements; box = box_inner x box_outer.  Out-of-range reads fill zeros.
+bool make_tmap(CUtensorMap* m, const void* ptr, bool fp8, uint64_t inner, uint64_t outer, uint64_t ld,
+               uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t esz = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * esz};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// --------------------------------------------------------------- GEMM ----
+struct Op {
+  const void* p;
+  long long ld;  // row stride (elements) of the stored matrix
+  bool mn;       // false: stored [rows, K] (K-major); true: stored [K, rows]
+};
+
+// split count for weight-gradient GEMMs: minimise waves * (k blocks per split
+// + a fixed per-unit epilogue cost)
+int plan_splits(int tiles, int kb_total, int sms) {
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= 16 && s <= kb_total; ++s) {
+    const long long units = (long long)tiles * s;
+    const long long waves = (units + sms - 1) / sms;
+    const long long cost = waves * ((kb_total + s - 1) / s + 8);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+template <bool AM, bool BM>
+int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, int splits, const EpiParams& ep,
+              cudaStream_t st, int sms) {
+  auto kern = gemm_tc_kernel<AM, BM, false>;
+  const int smem = tc_smem_bytes();
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const long long units = (long long)((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN) * splits;
+  const int grid = (int)std::min<long long>(units, sms);
+  kern<<<grid, TC_THREADS, smem, st>>>(ta, tb, M, N, K, splits, ep);
+  CKL();
+  return GPTB_OK;
+}
+
+int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t st) {
+  if (M <= 0 || N <= 0) return GPTB_OK;
+  if (K <= 0) return ep.kind == EPI_ACCUM_F32 ? GPTB_OK : GPTB_ERR_INVALID_ARG;
+  cudaEvent_t ea = nullptr, eb = nullptr;
+  bool timed = false;
+  {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    if (g_timing) {
+      ea = take_event();
+      eb = take_event();
+      timed = ea && eb;
+    }
+  }
+  if (timed) cudaEventRecord(ea, st);
+  int rc = GPTB_OK;
+  if (dtype == GPTB_F32) {
+    dim3 grid((N + 63) / 64, (M + 63) / 64);
+    const float* a = static_cast<const float*>(A.p);
+    const float* b = static_cast<const float*>(B.p);
+    if (!A.mn && !B.mn) gemm_simt_f32_kernel<false, false><<<grid, 256, 0, st>>>(a, A.ld, b, B.ld, M, N, K, ep);
+    else if (!A.mn && B.mn) gemm_simt_f32_kernel<false, true><<<grid, 256, 0, st>>>(a, A.ld, b, B.ld, M, N, K, ep);
+    else if (A.mn && B.mn) gemm_simt_f32_kernel<true, true><<<grid, 256, 0, st>>>(a, A.ld, b, B.ld, M, N, K, ep);
+    else gemm_simt_f32_kernel<true, false><<<grid, 256, 0, st>>>(a, A.ld, b, B.ld, M, N, K, ep);
+    LAUNCHED();
+    if (cudaPeekAtLastError() != cudaSuccess) {
+      cudaGetLastError();
+      rc = GPTB_ERR_CUDA;
+    }
+  } else {
+    const DevInfo di = dev_info();
+    if (di.cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+    if (!aligned16(A.p) || !aligned16(B.p) || !aligned16(ep.out) || (A.ld % 8) || (B.ld % 8) || (ep.ldo % 8) ||
+        (N % 8))
+      return GPTB_ERR_INVALID_ARG;
+    CUtensorMap ta, tb;
+    bool ok = A.mn ? make_tmap(&ta, A.p, false, M, K, A.ld, 64, 64) : make_tmap(&ta, A.p, false, K, M, A.ld, 64, TC_BM);
+    ok = ok && (B.mn ? make_tmap(&tb, B.p, false, N, K, B.ld, 64, 64)
+                     : make_tmap(&tb, B.p, false, K, N, B.ld, 64, TC_BN));
+    if (!ok) return GPTB_ERR_CUDA;
+    int splits = 1;
+    if (ep.kind == EPI_ACCUM_F32) {
+      const int tiles = ((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN);
+      splits = plan_splits(tiles, (K + 63) / 64, di.sms);
+    }
+    if (!A.mn && !B.mn) rc = launch_tc<false, false>(ta, tb, M, N, K, splits, ep, st, di.sms);
+    else if (!A.mn && B.mn) rc = launch_tc<false, true>(ta, tb, M, N, K, splits, ep, st, di.sms);
+    else if (A.mn && B.mn) rc = launch_tc<true, true>(ta, tb, M, N, K, splits, ep, st, di.sms);
+    else rc = launch_tc<true, false>(ta, tb, M, N, K, splits, ep, st, di.sms);
+  }
+  if (timed) {
+    cudaEventRecord(eb, st);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timed.push_back({ea, eb, 2.0 * M * (double)N * K});
+  }
+  return rc;
+}
+
+EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = nullptr, long long ld_aux = 0,
+              void* out2 = nullptr, long long ldo2 = 0) {
+  EpiParams e;
+  e.kind = kind;
+  e.out_f32 = (kind == EPI_ACCUM_F32 || dtype == GPTB_F32) ? 1 : 0;
+  e.out = out;
+  e.ldo = ldo;
+  e.aux = aux;
+  e.ld_aux = ld_aux;
+  e.out2 = out2;
+  e.ldo2 = ldo2;
+  e.alpha = nullptr;
+  return e;
+}
+
+// ---------------------------------------------------------- workspace -----
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  void* take(size_t bytes) {
+    off = (off + 255) & ~size_t(255);
+    void* p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct Dims {
+  long long N;
+  int B, T, d, H, Hkv, hd, F, V, L, Wq, NH, esz;
+};
+Dims dims_of(const gptb_config& c) {
+  Dims m;
+  m.B = c.B;
+  m.T = c.T;
+  m.N = (long long)c.B * c.T;
+  m.d = c.d;
+  m.H = c.n_head;
+  m.Hkv = c.n_kv_head;
+  m.hd = c.head_dim;
+  m.F = c.mlp_hidden;
+  m.V = c.vocab;
+  m.L = c.n_layer;
+  m.Wq = (c.n_head + 2 * c.n_kv_head) * c.head_dim;
+  m.NH = c.n_head + c.n_kv_head;
+  m.esz = c.dtype == GPTB_F32 ? 4 : 2;
+  return m;
+}
+
+struct Saved {
+  void *h, *qkv, *o, *h2, *u, *act;
+  float *rstd1, *sg, *rstd_qk, *lse, *rstd2;
+};
+Saved carve_saved(Carve& cv, const Dims& m) {
+  Saved s;
+  const size_t e = m.esz;
+  s.h = cv.take(m.N * m.d * e);
+  s.rstd1 = (float*)cv.take(m.N * 4);
+  s.sg = (float*)cv.take(m.N * m.Hkv * 4);
+  s.qkv = cv.take(m.N * m.Wq * e);
+  s.rstd_qk = (float*)cv.take(m.N * m.NH * 4);
+  s.o = cv.take(m.N * (long long)m.H * m.hd * e);
+  s.lse = (float*)cv.take((size_t)m.B * m.H * m.T * 4);
+  s.h2 = cv.take(m.N * m.d * e);
+  s.rstd2 = (float*)cv.take(m.N * 4);
+  s.u = cv.take(m.N * m.F * e);
+  s.act = cv.take(m.N * m.F * e);
+  return s;
+}
+
+struct Scratch {
+  float2* rope;
+  // forward
+  void *xm, *x1;
+  // backward
+  void *du, *dh2, *dx1, *dO, *dqkv, *dh;
+  float *D, *dq, *dk, *dv, *dz;
+};
+Scratch carve_scratch(Carve& cv, const Dims& m) {
+  Scratch s;
+  const size_t e = m.esz;
+  s.rope = (float2*)cv.take((size_t)m.T * (m.hd / 2) * sizeof(float2));
+  const size_t start = cv.off;
+  s.xm = cv.take(m.N * m.d * e);
+  s.x1 = cv.take(m.N * m.d * e);
+  const size_t fwd_end = cv.off;
+  cv.off = start;  // backward temporaries reuse the forward's space
+  s.du = cv.take(m.N * m.F * e);
+  s.dh2 = cv.take(m.N * m.d * e);
+  s.dx1 = cv.take(m.N * m.d * e);
+  s.dO = cv.take(m.N * (long long)m.H * m.hd * e);
+  s.dqkv = cv.take(m.N * m.Wq * e);
+  s.dh = cv.take(m.N * m.d * e);
+  s.D = (float*)cv.take((size_t)m.B * m.H * m.T * 4);
+  s.dq = (float*)cv.take(m.N * (long long)m.H * m.hd * 4);
+  s.dk = (float*)cv.take(m.N * (long long)m.Hkv * m.hd * 4);
+  s.dv = (float*)cv.take(m.N * (long long)m.Hkv * m.hd * 4);
+  s.dz = (float*)cv.take(m.N * m.Hkv * 4);
+  cv.off = std::max(cv.off, fwd_end);
+  return s;
+}
+
+struct LmWs {
+  void* logits;
+  float* row_loss;
+  int chunk;
+};
+LmWs carve_lm(Carve& cv, const Dims& m) {
+  LmWs l;
+  l.chunk = (int)std::min<long long>(m.N, 8192);
+  l.logits = cv.take((size_t)l.chunk * m.V * m.esz);
+  l.row_loss = (float*)cv.take(m.N * 4);
+  return l;
+}
+
+struct StackWs {
+  std::vector<void*> x_in;
+  std::vector<Saved> saved;
+  void *xL, *hf, *dhf, *dxA, *dxB, *dx_bo;
+  float *rstd_f, *dx0;
+  Scratch scr;
+  LmWs lm;
+};
+StackWs carve_stack(Carve& cv, const Dims& m) {
+  StackWs s;
+  const size_t row = m.N * m.d * m.esz;
+  for (int i = 0; i < m.L; ++i) s.x_in.push_back(cv.take(row));
+  for (int i = 0; i < m.L; ++i) s.saved.push_back(carve_saved(cv, m));
+  s.xL = cv.take(row);
+  s.hf = cv.take(row);
+  s.rstd_f = (float*)cv.take(m.N * 4);
+  s.dhf = cv.take(row);
+  s.dxA = cv.take(row);
+  s.dxB = cv.take(row);
+  s.dx_bo = cv.take(row);
+  s.dx0 = (float*)cv.take(m.N * m.d * 4);
+  s.scr = carve_scratch(cv, m);
+  s.lm = carve_lm(cv, m);
+  return s;
+}
+
+// ------------------------------------------------------------ checks ------
+int check_config(const gptb_config* c) {
+  if (!c) return GPTB_ERR_INVALID_ARG;
+  if (c->dtype != GPTB_F32 && c->dtype != GPTB_BF16 && c->dtype != GPTB_FP8_E4M3) return GPTB_ERR_UNSUPPORTED;
+  if (c->dtype == GPTB_FP8_E4M3) return GPTB_ERR_UNSUPPORTED;
+  if (c->B < 1 || c->T < 1 || c->d < 8 || c->d % 8 || c->d > 8 * 32 * EW_MAXC) return GPTB_ERR_INVALID_ARG;
+  if (c->n_head < 1 || c->n_kv_head < 1 || c->n_head % c->n_kv_head) return GPTB_ERR_INVALID_ARG;
+  if (c->mlp_hidden < 8 || c->mlp_hidden % 8 || c->vocab < 8 || c->vocab % 8) return GPTB_ERR_INVALID_ARG;
+  if (c->n_layer < 1 || c->n_layer > GPTB_MAX_LAYERS) return GPTB_ERR_INVALID_ARG;
+  if (c->backout_layer < -1 || c->backout_layer >= c->n_layer) return GPTB_ERR_INVALID_ARG;
+  if (c->smear_ch < 0 || c->smear_ch > 256 || c->smear_ch > c->d) return GPTB_ERR_INVALID_ARG;
+  if (!(c->norm_eps >= 0.f) || !(c->rope_base > 0.f)) return GPTB_ERR_INVALID_ARG;
+  for (int i = 0; i < c->n_layer; ++i) {
+    if (c->window[i] < -1) return GPTB_ERR_INVALID_ARG;
+    if (c->has_ve[i] && (c->ve_gate_ch < 1 || c->ve_gate_ch > 256 || c->ve_gate_ch > c->d)) return GPTB_ERR_INVALID_ARG;
+  }
+  if (c->dtype == GPTB_F32) {
+    if (c->head_dim < 2 || c->head_dim % 2 || c->head_dim > 128 || c->T > 1024) return GPTB_ERR_UNSUPPORTED;
+  } else {
+    if (c->head_dim != 128) return GPTB_ERR_UNSUPPORTED;
+    if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  }
+  if (((long long)c->B * c->T) > (1ll << 31) / 4) return GPTB_ERR_INVALID_ARG;
+  return GPTB_OK;
+}
+
+int grid_rows(long long rows) {
+  const long long wpb = EW_THREADS / 32;
+  const long long need = (rows + wpb - 1) / wpb;
+  const long long cap = (long long)dev_info().sms * 8;
+  return (int)std::max<long long>(1, std::min(need, cap));
+}
+
+template <class T>
+int rope_init(const gptb_config& c, float2* tab, cudaStream_t st) {
+  const long long n = (long long)c.T * (c.head_dim / 2);
+  rope_table_kernel<<<(int)std::min<long long>((n + 255) / 256, 4096), 256, 0, st>>>(tab, c.T, c.head_dim / 2,
+                                                                                     (double)c.rope_base);
+  CKL();
+  return GPTB_OK;
+}
+
+// ------------------------------------------------------ block forward -----
+template <class T>
+int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w, const T* x, const T* x0,
+                   const int32_t* idx, T* x_out, const Saved& S, const Scratch& X, cudaStream_t st) {
+  const Dims m = dims_of(c);
+  const int nc = (m.d + 255) / 256;
+  const bool ve = c.has_ve[layer] != 0;
+  if (!w.w_qkv || !w.w_o || !w.w_fc || !w.w_proj || !w.lambdas || (ve && (!w.w_ve_gate || !w.ve_table)))
+    return GPTB_ERR_INVALID_ARG;
+  const int gr = grid_rows(m.N);
+  ROWK(nc, mix_norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(x, x0, w.lambdas, (T*)X.xm, (T*)S.h, S.rstd1, m.N, m.d, c.norm_eps,
+                                                ve ? (const T*)w.w_ve_gate : nullptr, S.sg, m.Hkv, c.ve_gate_ch));
+  CKL();
+  TRY(gemm(c.dtype, {S.h, m.d, false}, {w.w_qkv, m.d, false}, (int)m.N, m.Wq, m.d,
+           epi(EPI_STORE, c.dtype, S.qkv, m.Wq), st));
+  qkv_post_kernel<T><<<grid_rows(m.N * (m.NH + (ve ? m.Hkv : 0))), EW_THREADS, 0, st>>>(
+      (T*)S.qkv, m.Wq, S.rstd_qk, X.rope, m.T, m.N, m.H, m.Hkv, m.hd, c.norm_eps, ve ? (const T*)w.ve_table : nullptr,
+      idx, S.sg);
+  CKL();
+  const int W = c.window[layer];
+  if (c.dtype == GPTB_F32) {
+    attn_fwd_simt_kernel<T><<<dim3(m.T, m.H, m.B), 128, 0, st>>>((const T*)S.qkv, m.Wq, (T*)S.o,
+                                                                 (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, m.hd, W);
+    CKL();
+  } else {
+    CK(cudaFuncSetAttribute(attn_fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AF_SMEM));
+    attn_fwd_bf16_kernel<<<dim3((m.T + AF_BR - 1) / AF_BR, m.H, m.B), AF_THREADS, AF_SMEM, st>>>(
+        (const bf16*)S.qkv, m.Wq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W);
+    CKL();
+  }
+  TRY(gemm(c.dtype, {S.o, (long long)m.H * m.hd, false}, {w.w_o, (long long)m.H * m.hd, false}, (int)m.N, m.d,
+           m.H * m.hd, epi(EPI_RESID, c.dtype, X.x1, m.d, X.xm, m.d), st));
+  ROWK(nc, norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
+                                            c.norm_eps));
+  CKL();
+  TRY(gemm(c.dtype, {S.h2, m.d, false}, {w.w_fc, m.d, false}, (int)m.N, m.F, m.d,
+           epi(EPI_RELU2, c.dtype, S.u, m.F, nullptr, 0, S.act, m.F), st));
+  TRY(gemm(c.dtype, {S.act, m.F, false}, {w.w_proj, m.F, false}, (int)m.N, m.d, m.F,
+           epi(EPI_RESID, c.dtype, x_out, m.d, X.x1, m.d), st));
+  return GPTB_OK;
+}
+
+// ----------------------------------------------------- block backward -----
+template <class T>
+int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w, const T* x, const T* x0,
+                   const int32_t* idx, const Saved& S, const T* dx2, const T* dx_extra, T* dx, float* dx0_acc,
+                   const gptb_block_grads& g, const Scratch& X, cudaStream_t st) {
+  const Dims m = dims_of(c);
+  const int nc = (m.d + 255) / 256;
+  const bool ve = c.has_ve[layer] != 0;
+  if (!g.w_qkv || !g.w_o || !g.w_fc || !g.w_proj || !g.lambdas || (ve && (!g.w_ve_gate || !g.ve_table)))
+    return GPTB_ERR_INVALID_ARG;
+  const int dt = c.dtype;
+  const int N = (int)m.N;
+  const long long Ho = (long long)m.H * m.hd, Kv = (long long)m.Hkv * m.hd;
+  // MLP
+  TRY(gemm(dt, {dx2, m.d, true}, {S.act, m.F, true}, m.d, m.F, N, epi(EPI_ACCUM_F32, dt, g.w_proj, m.F), st));
+  TRY(gemm(dt, {dx2, m.d, false}, {w.w_proj, m.F, true}, N, m.F, m.d, epi(EPI_DRELU2, dt, X.du, m.F, S.u, m.F), st));
+  TRY(gemm(dt, {X.du, m.F, true}, {S.h2, m.d, true}, m.F, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
+  TRY(gemm(dt, {X.du, m.F, false}, {w.w_fc, m.d, true}, N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
+  const int gr = grid_rows(m.N);
+  ROWK(nc, norm_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d));
+  CKL();
+  // attention output projection
+  TRY(gemm(dt, {X.dx1, m.d, true}, {S.o, Ho, true}, m.d, (int)Ho, N, epi(EPI_ACCUM_F32, dt, g.w_o, Ho), st));
+  TRY(gemm(dt, {X.dx1, m.d, false}, {w.w_o, Ho, true}, N, (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
+  // attention
+  attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
+                                                                     m.B, m.T, m.H, m.hd);
+  CKL();
+  CK(cudaMemsetAsync(X.dq, 0, m.N * Ho * 4, st));
+  const int W = c.window[layer];
+  if (dt == GPTB_F32) {
+    CK(cudaMemsetAsync(X.dk, 0, m.N * Kv * 4, st));
+    CK(cudaMemsetAsync(X.dv, 0, m.N * Kv * 4, st));
+    attn_bwd_simt_kernel<T><<<dim3(m.T, m.H, m.B), 128, 0, st>>>((const T*)S.qkv, m.Wq, (const T*)X.dO, Ho, S.lse,
+                                                                 X.D, X.dq, Ho, X.dk, X.dv, Kv, m.T, m.H, m.Hkv, m.hd,
+                                                                 W);
+    CKL();
+  } else {
+    CK(cudaFuncSetAttribute(attn_bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AB_SMEM));
+    attn_bwd_bf16_kernel<<<dim3((m.T + AB_BC - 1) / AB_BC, m.Hkv, m.B), AB_THREADS, AB_SMEM, st>>>(
+        (const bf16*)S.qkv, m.Wq, (const bf16*)X.dO, Ho, S.lse, X.D, X.dq, Ho, X.dk, X.dv, Kv, m.T, m.H, m.Hkv, W);
+    CKL();
+  }
+  qkv_post_bwd_kernel<T><<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(
+      (const T*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (T*)X.dqkv, m.T, m.N, m.H, m.Hkv, m.hd,
+      ve ? (const T*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz);
+  CKL();
+  // QKV projection
+  TRY(gemm(dt, {X.dqkv, m.Wq, true}, {S.h, m.d, true}, m.Wq, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_qkv, m.d), st));
+  TRY(gemm(dt, {X.dqkv, m.Wq, false}, {w.w_qkv, m.d, true}, N, m.d, m.Wq, epi(EPI_STORE, dt, X.dh, m.d), st));
+  if (ve) {
+    const int nthreads = ((m.Hkv * c.ve_gate_ch + 31) / 32) * 32;
+    if (nthreads > 1024) return GPTB_ERR_UNSUPPORTED;
+    ve_gate_wgrad_kernel<T><<<dev_info().sms * 4, nthreads, 0, st>>>(X.dz, (const T*)S.h, m.N, m.d, m.Hkv,
+                                                                     c.ve_gate_ch, g.w_ve_gate);
+    CKL();
+  }
+  ROWK(nc, mix_norm_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)X.dh, ve ? X.dz : nullptr,
+                                                    ve ? (const T*)w.w_ve_gate : nullptr, m.Hkv, c.ve_gate_ch,
+                                                    (const T*)S.h, S.rstd1, (const T*)X.dx1, x, x0, w.lambdas, dx_extra,
+                                                    dx, dx0_acc, g.lambdas, m.N, m.d));
+  CKL();
+  return GPTB_OK;
+}
+
+// -------------------------------------------------------------- lm head ---
+template <class T>
+int lm_head_impl(const gptb_config& c, const T* h, const T* w_lm, const int32_t* targets, float* loss_out, T* dh,
+                 float* dw_lm, const LmWs& lw, cudaStream_t st) {
+  const Dims m = dims_of(c);
+  const int nc = (m.d + 255) / 256;
+  const int dt = c.dtype;
+  for (long long c0 = 0; c0 < m.N; c0 += lw.chunk) {
+    const int rows = (int)std::min<long long>(lw.chunk, m.N - c0);
+    const T* hc = h + c0 * m.d;
+    TRY(gemm(dt, {hc, m.d, false}, {w_lm, m.d, false}, rows, m.V, m.d, epi(EPI_STORE, dt, lw.logits, m.V), st));
+    xent_rows_kernel<T><<<rows, 512, 0, st>>>((T*)lw.logits, m.V, m.V, targets + c0, lw.row_loss + c0,
+                                              1.f / (float)m.N, rows);
+    CKL();
+    TRY(gemm(dt, {lw.logits, m.V, false}, {w_lm, m.d, true}, rows, m.d, m.V, epi(EPI_STORE, dt, dh + c0 * m.d, m.d),
+             st));
+    TRY(gemm(dt, {lw.logits, m.V, true}, {hc, m.d, true}, m.V, m.d, rows, epi(EPI_ACCUM_F32, dt, dw_lm, m.d), st));
+  }
+  mean_kernel<<<1, 1024, 0, st>>>(lw.row_loss, m.N, loss_out);
+  CKL();
+  return GPTB_OK;
+}
+
+// --------------------------------------------------------------- stack ----
+template <class T>
+int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t* idx, const int32_t* targets,
+               float* loss_out, const gptb_model_grads& g, const StackWs& S, cudaStream_t st) {
+  const Dims m = dims_of(c);
+  const int nc = (m.d + 255) / 256;
+  if (!w.wte || !w.w_lm || !g.wte || !g.w_lm) return GPTB_ERR_INVALID_ARG;
+  if (c.smear_ch > 0 && (!w.w_smear_gate || !w.smear_lambda || !g.w_smear_gate || !g.smear_lambda))
+    return GPTB_ERR_INVALID_ARG;
+  if (c.backout_layer >= 0 && (!w.backout_lambda || !g.backout_lambda)) return GPTB_ERR_INVALID_ARG;
+  TRY(rope_init<T>(c, S.scr.rope, st));
+  const int gr = grid_rows(m.N);
+  ROWK(nc, embed_smear_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(idx, (const T*)w.wte, (const T*)w.w_smear_gate, w.smear_lambda,
+                                                   (T*)S.x_in[0], m.B, m.T, m.d, c.smear_ch));
+  CKL();
+  const T* x0 = (const T*)S.x_in[0];
+  for (int i = 0; i < m.L; ++i) {
+    T* xo = (T*)(i + 1 < m.L ? S.x_in[i + 1] : S.xL);
+    TRY(block_fwd_impl<T>(c, i, w.layers[i], (const T*)S.x_in[i], x0, idx, xo, S.saved[i], S.scr, st));
+  }
+  const T* x_bo = c.backout_layer >= 0 ? (const T*)S.x_in[c.backout_layer] : nullptr;
+  ROWK(nc, norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)S.xL, x_bo, w.backout_lambda, (T*)S.hf, S.rstd_f, m.N, m.d,
+                                            c.norm_eps));
+  CKL();
+  TRY(lm_head_impl<T>(c, (const T*)S.hf, (const T*)w.w_lm, targets, loss_out, (T*)S.dhf, g.w_lm, S.lm, st));
+  ROWK(nc, final_norm_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)S.dhf, (const T*)S.hf, S.rstd_f, x_bo,
+                                                      w.backout_lambda, (T*)S.dxA, (T*)S.dx_bo, g.backout_lambda,
+                                                      m.N, m.d));
+  CKL();
+  CK(cudaMemsetAsync(S.dx0, 0, m.N * m.d * 4, st));
+  T* cur = (T*)S.dxA;
+  T* nxt = (T*)S.dxB;
+  for (int i = m.L - 1; i >= 0; --i) {
+    const T* extra = (i == c.backout_layer) ? (const T*)S.dx_bo : nullptr;
+    TRY(block_bwd_impl<T>(c, i, w.layers[i], (const T*)S.x_in[i], x0, idx, S.saved[i], cur, extra, nxt, S.dx0,
+                          g.layers[i], S.scr, st));
+    std::swap(cur, nxt);
+  }
+  ROWK(nc, smear_embed_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(cur, S.dx0, idx, (const T*)w.wte, (const T*)w.w_smear_gate,
+                                                       w.smear_lambda, g.wte, g.w_smear_gate, g.smear_lambda, m.B, m.T,
+                                                       m.d, c.smear_ch));
+  CKL();
+  return GPTB_OK;
+}
+
+}  // namespace
+
+// ================================================================ C ABI ====
+extern "C" {
+
+size_t gptb_workspace_bytes(const gptb_config* cfg, int kind) {
+  if (!cfg || cfg->B < 1 || cfg->T < 1 || cfg->n_layer < 1 || cfg->n_layer > GPTB_MAX_LAYERS) return 0;
+  const Dims m = dims_of(*cfg);
+  Carve cv(nullptr);
+  switch (kind) {
+    case GPTB_WS_BLOCK_SAVED: carve_saved(cv, m); break;
+    case GPTB_WS_BLOCK_SCRATCH: carve_scratch(cv, m); break;
+    case GPTB_WS_LM_HEAD: carve_lm(cv, m); break;
+    case GPTB_WS_STACK: carve_stack(cv, m); break;
+    default: return 0;
+  }
+  return (cv.off + 255) & ~size_t(255);
+}
+
+int gpt_block_forward(const gptb_config* cfg, int layer, const gptb_block_weights* w, const void* x, const void* x0,
+                      const int32_t* idx, void* x_out, void* saved, void* scratch, gptb_stream_t stream) {
+  TRY(check_config(cfg));
+  if (!w || !x || !x0 || !idx || !x_out || !saved || !scratch || layer < 0 || layer >= cfg->n_layer)
+    return GPTB_ERR_INVALID_ARG;
+  const Dims m = dims_of(*cfg);
+  Carve cs(saved), cx(scratch);
+  const Saved S = carve_saved(cs, m);
+  const Scratch X = carve_scratch(cx, m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == GPTB_F32) {
+    TRY(rope_init<float>(*cfg, X.rope, st));
+    return block_fwd_impl<float>(*cfg, layer, *w, (const float*)x, (const float*)x0, idx, (float*)x_out, S, X, st);
+  }
+  TRY(rope_init<bf16>(*cfg, X.rope, st));
+  return block_fwd_impl<bf16>(*cfg, layer, *w, (const bf16*)x, (const bf16*)x0, idx, (bf16*)x_out, S, X, st);
+}
+
+int gpt_block_backward(const gptb_config* cfg, int layer, const gptb_block_weights* w, const void* x, const void* x0,
+                       const int32_t* idx, const void* saved, const void* dx_out, const void* dx_extra, void* dx,
+                       float* dx0_accum, gptb_block_grads* g, void* scratch, gptb_stream_t stream) {
+  TRY(check_config(cfg));
+  if (!w || !x || !x0 || !idx || !saved || !dx_out || !dx || !dx0_accum || !g || !scratch || layer < 0 ||
+      layer >= cfg->n_layer)
+    return GPTB_ERR_INVALID_ARG;
+  const Dims m = dims_of(*cfg);
+  Carve cs(const_cast<void*>(saved)), cx(scratch);
+  const Saved S = carve_saved(cs, m);
+  const Scratch X = carve_scratch(cx, m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == GPTB_F32) {
+    TRY(rope_init<float>(*cfg, X.rope, st));
+    return block_bwd_impl<float>(*cfg, layer, *w, (const float*)x, (const float*)x0, idx, S, (const float*)dx_out,
+                                 (const float*)dx_extra, (float*)dx, dx0_accum, *g, X, st);
+  }
+  TRY(rope_init<bf16>(*cfg, X.rope, st));
+  return block_bwd_impl<bf16>(*cfg, layer, *w, (const bf16*)x, (const bf16*)x0, idx, S, (const bf16*)dx_out,
+                              (const bf16*)dx_extra, (bf16*)dx, dx0_accum, *g, X, st);
+}
+
+int lm_head_xent(const gptb_config* cfg, const void* h, const void* w_lm, const int32_t* targets, float* loss_out,
+                 void* dh, float* dw_lm, void* ws, gptb_stream_t stream) {
+  TRY(check_config(cfg));
+  if (!h || !w_lm || !targets || !loss_out || !dh || !dw_lm || !ws) return GPTB_ERR_INVALID_ARG;
+  const Dims m = dims_of(*cfg);
+  Carve cv(ws);
+  const LmWs lw = carve_lm(cv, m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == GPTB_F32)
+    return lm_head_impl<float>(*cfg, (const float*)h, (const float*)w_lm, targets, loss_out, (float*)dh, dw_lm, lw, st);
+  return lm_head_impl<bf16>(*cfg, (const bf16*)h, (const bf16*)w_lm, targets, loss_out, (bf16*)dh, dw_lm, lw, st);
+}
+
+int gpt_stack_step(const gptb_config* cfg, const gptb_model_weights* w, const int32_t* idx, const int32_t* targets,
+                   float* loss_out, gptb_model_grads* g, void* ws, gptb_stream_t stream) {
+  TRY(check_config(cfg));
+  if (!w || !idx || !targets || !loss_out || !g || !ws) return GPTB_ERR_INVALID_ARG;
+  const Dims m = dims_of(*cfg);
+  Carve cv(ws);
+  const StackWs S = carve_stack(cv, m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == GPTB_F32) return stack_impl<float>(*cfg, *w, idx, targets, loss_out, *g, S, st);
+  return stack_impl<bf16>(*cfg, *w, idx, targets, loss_out, *g, S, st);
+}
+
+int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, void* C, int c_f32,
+                   long long ldc, int M, int N, int K, gptb_stream_t stream) {
+  if (!A || !B || !C || M < 0 || N < 0 || K < 0) return GPTB_ERR_INVALID_ARG;
+  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  EpiParams e = epi(c_f32 ? EPI_ACCUM_F32 : EPI_STORE, GPTB_BF16, C, ldc);
+  return gemm(GPTB_BF16, {A, lda, a_mn != 0}, {B, ldb, b_mn != 0}, M, N, K, e, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gptb_device_error(gptb_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GPTB_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(int)) != cudaSuccess) return GPTB_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return GPTB_ERR_CUDA;
+    return GPTB_ERR_TIMEOUT;
+  }
+  return GPTB_OK;
+}
+
+int gptb_set_wait_limit_ns(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns)) == cudaSuccess ? GPTB_OK : GPTB_ERR_CUDA;
+}
+
+void gptb_reset_counters(void) {
+  g_launches.store(0);
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  for (auto& t : g_timed) {
+    g_event_pool.push_back(t.a);
+    g_event_pool.push_back(t.b);
+  }
+  g_timed.clear();
+}
+
+long long gptb_launch_count(void) { return g_launches.load(); }
+
+int gptb_set_gemm_timing(int enable) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  g_timing = enable != 0;
+  return GPTB_OK;
+}
+
+int gptb_gemm_timing(double* ms, double* flops, long long* launches) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  double tms = 0, tf = 0;
+  for (auto& t : g_timed) {
+    if (cudaEventSynchronize(t.b) != cudaSuccess) return GPTB_ERR_CUDA;
+    float e = 0.f;
+    if (cudaEventElapsedTime(&e, t.a, t.b) != cudaSuccess) return GPTB_ERR_CUDA;
+    tms += e;
+    tf += t.flops;
+  }
+  if (ms) *ms = tms;
+  if (flops) *flops = tf;
+  if (launches) *launches = (long long)g_timed.size();
+  return GPTB_OK;
+}
+
+const char* gptb_error_string(int code) {
+  switch (code) {
+    case GPTB_OK: return "ok";
+    case GPTB_ERR_INVALID_ARG: return "invalid argument";
+    case GPTB_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case GPTB_ERR_CUDA: return "CUDA error";
+    case GPTB_ERR_TIMEOUT: return "bounded device wait expired";
+    case GPTB_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,373 @@
+// GEMMs of the block: C = A * B^T with A [M,K], B [N,K] and a fused epilogue.
+//
+// Every projection of the block is an nn.Linear (y = x W^T with W [out,in]),
+// so the three products of training map onto one kernel with per-operand
+// majorness:
+//   forward   y  = x  W^T : A = x  (K-major),  B = W  (K-major)
+//   dgrad     dx = dy W   : A = dy (K-major),  B = W  (N-major, W is [K,N])
+//   wgrad     dW = dy^T x : A = dy (M-major),  B = x  (N-major)
+//
+// bf16 / e4m3 path (tcgen05): persistent, warp-specialised kernel.
+//   warp 0   TMA producer (128-byte swizzled tiles, 4-stage mbarrier ring)
+//   warp 1   TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-5 epilogue: tcgen05.ld 32 lanes x 32 columns per warp, fused
+//             elementwise op, direct 16-byte global stores / fp32 atomics
+//   Tile 128 x 256, two TMEM accumulators (2 x 256 columns) so the epilogue
+//   of tile i overlaps the MMAs of tile i+1.  Split-K over the K blocks is
+//   used for weight gradients (long K, few tiles); partial sums meet in the
+//   fp32 gradient through vector atomics.
+// fp32 path (SIMT, FFMA): a plain tiled kernel with the same epilogues, for
+//   the fp32 configuration whose 1e-5 tolerance tensor-core fp32 (tf32)
+//   inputs cannot meet.
+#pragma once
+#include "common.cuh"
+
+namespace gptb {
+
+enum EpiKind : int {
+  EPI_STORE = 0,      // out = alpha*acc
+  EPI_RESID = 1,      // out = aux + alpha*acc                (residual add)
+  EPI_RELU2 = 2,      // out = u = alpha*acc, out2 = relu(u)^2 (MLP activation)
+  EPI_DRELU2 = 3,     // out = alpha*acc * 2*relu(aux)         (aux = saved u)
+  EPI_ACCUM_F32 = 4,  // out(f32) += alpha*acc, atomic          (weight grads)
+};
+
+struct EpiParams {
+  int kind;
+  int out_f32;  // element type of out/out2/aux: 1 = float, 0 = bf16
+  void* out;
+  long long ldo;
+  const void* aux;
+  long long ld_aux;
+  void* out2;
+  long long ldo2;
+  const float* alpha;  // device scalar or nullptr (= 1)
+};
+
+// ---------------------------------------------------------------- epilogue
+template <class T>
+__device__ __forceinline__ void epi_store8_t(const EpiParams& ep, long long r, int c, float (&v)[8]) {
+  T* o = reinterpret_cast<T*>(ep.out) + r * ep.ldo + c;
+  switch (ep.kind) {
+    case EPI_RESID: {
+      float a[8];
+      load8(reinterpret_cast<const T*>(ep.aux) + r * ep.ld_aux + c, a);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += a[i];
+      store8(o, v);
+    } break;
+    case EPI_RELU2: {
+      float a[8];
+      store8(o, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float t = fmaxf(v[i], 0.f);
+        a[i] = t * t;
+      }
+      store8(reinterpret_cast<T*>(ep.out2) + r * ep.ldo2 + c, a);
+    } break;
+    case EPI_DRELU2: {
+      float u[8];
+      load8(reinterpret_cast<const T*>(ep.aux) + r * ep.ld_aux + c, u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] *= 2.f * fmaxf(u[i], 0.f);
+      store8(o, v);
+    } break;
+    default:
+      store8(o, v);
+  }
+}
+
+__device__ __forceinline__ void epi_apply8(const EpiParams& ep, long long r, int c, float (&v)[8]) {
+  if (ep.kind == EPI_ACCUM_F32) {
+    float* o = reinterpret_cast<float*>(ep.out) + r * ep.ldo + c;
+    atomicAdd(reinterpret_cast<float4*>(o), make_float4(v[0], v[1], v[2], v[3]));
+    atomicAdd(reinterpret_cast<float4*>(o + 4), make_float4(v[4], v[5], v[6], v[7]));
+  } else if (ep.out_f32) {
+    epi_store8_t<float>(ep, r, c, v);
+  } else {
+    epi_store8_t<bf16>(ep, r, c, v);
+  }
+}
+
+template <class T>
+__device__ __forceinline__ void epi_scalar_t(const EpiParams& ep, long long r, int c, float v) {
+  T* o = reinterpret_cast<T*>(ep.out) + r * ep.ldo + c;
+  switch (ep.kind) {
+    case EPI_RESID: *o = from_f<T>(to_f(reinterpret_cast<const T*>(ep.aux)[r * ep.ld_aux + c]) + v); break;
+    case EPI_RELU2: {
+      *o = from_f<T>(v);
+      float t = fmaxf(v, 0.f);
+      reinterpret_cast<T*>(ep.out2)[r * ep.ldo2 + c] = from_f<T>(t * t);
+    } break;
+    case EPI_DRELU2:
+      *o = from_f<T>(v * 2.f * fmaxf(to_f(reinterpret_cast<const T*>(ep.aux)[r * ep.ld_aux + c]), 0.f));
+      break;
+    default: *o = from_f<T>(v);
+  }
+}
+__device__ __forceinline__ void epi_apply1(const EpiParams& ep, long long r, int c, float v) {
+  if (ep.kind == EPI_ACCUM_F32) atomicAdd(reinterpret_cast<float*>(ep.out) + r * ep.ldo + c, v);
+  else if (ep.out_f32) epi_scalar_t<float>(ep, r, c, v);
+  else epi_scalar_t<bf16>(ep, r, c, v);
+}
+
+// ------------------------------------------------------ tcgen05 kernel ----
+constexpr int TC_BM = 128;
+constexpr int TC_BN = 256;
+constexpr int TC_STAGES = 4;
+constexpr int TC_THREADS = 192;
+constexpr int TC_GROUP_M = 8;
+
+__host__ __device__ constexpr int tc_smem_bytes() {
+  // stages * (A 16 KB + B 32 KB) + barriers + 1 KB alignment slack
+  return TC_STAGES * (TC_BM * 128 + TC_BN * 128) + 256 + 1024;
+}
+
+__device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, int& tm, int& tn, int& split) {
+  const int tiles = tiles_m * tiles_n;
+  split = u / tiles;
+  const int t = u - split * tiles;
+  const int per_group = TC_GROUP_M * tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * TC_GROUP_M;
+  const int gsize = min(tiles_m - first_m, TC_GROUP_M);
+  const int r = t - g * per_group;
+  tm = first_m + r % gsize;
+  tn = r / gsize;
+}
+
+template <bool A_MN, bool B_MN, bool FP8>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                   int K, int splits, EpiParams ep) {
+  constexpr int ELEM = FP8 ? 1 : 2;
+  constexpr int BK = 128 / ELEM;      // one 128-byte swizzle row of K (64 bf16 / 128 e4m3)
+  constexpr int MMA_K = 32 / ELEM;    // K per tcgen05.mma (16 bf16 / 32 e4m3)
+  constexpr int ATOM = BK;            // MN extent of one swizzle atom for MN-major operands
+  constexpr int A_BYTES = TC_BM * 128;
+  constexpr int B_BYTES = TC_BN * 128;
+  constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
+  constexpr uint32_t IDESC = make_idesc(TC_BM, TC_BN, A_MN, B_MN, FP8);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + TC_STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + TC_STAGES * B_BYTES);
+  uint64_t* empty = full + TC_STAGES;
+  uint64_t* tfull = empty + TC_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (M + TC_BM - 1) / TC_BM, tiles_n = (N + TC_BN - 1) / TC_BN;
+  const int units = tiles_m * tiles_n * splits;
+  const int kb_total = (K + BK - 1) / BK;
+  const int kb_per = (kb_total + splits - 1) / splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tm, tn, split;
+        tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
+        const int kb0 = split * kb_per, kb1 = min(kb_total, kb0 + kb_per);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, ERRW_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], STAGE_TX);
+          uint8_t* a = sA + stage * A_BYTES;
+          uint8_t* b = sB + stage * B_BYTES;
+          const int k0 = kb * BK;
+          if (!A_MN) {
+            tma_load_2d(a, &tmA, &full[stage], k0, tm * TC_BM);
+          } else {
+#pragma unroll
+            for (int i = 0; i < TC_BM / ATOM; ++i) tma_load_2d(a + i * BK * 128, &tmA, &full[stage], tm * TC_BM + i * ATOM, k0);
+          }
+          if (!B_MN) {
+            tma_load_2d(b, &tmB, &full[stage], k0, tn * TC_BN);
+          } else {
+#pragma unroll
+            for (int i = 0; i < TC_BN / ATOM; ++i) tma_load_2d(b + i * BK * 128, &tmB, &full[stage], tn * TC_BN + i * ATOM, k0);
+          }
+          if (++stage == TC_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // drain: wait (bounded) until the MMA side consumed every stage we filled
+      if (!ok) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+          uint64_t* bar = &full[s];
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar, phase) && !mbar_try_wait(bar, phase ^ 1u)) {
+            if (globaltimer_ns() - t0 > 100000000ull) {
+              record_error(ERRW_TIMEOUT_DRAIN);
+              break;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tm, tn, split;
+        tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
+        const int kb0 = split * kb_per, kb1 = min(kb_total, kb0 + kb_per);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, ERRW_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / MMA_K; ++k) {
+            // K-major: advance 32 bytes along the swizzled row; MN-major: MMA_K rows of 128 bytes
+            const uint64_t ad = A_MN ? smem_desc_sw128(a_addr + k * MMA_K * 128, BK * 128, 1024)
+                                     : smem_desc_sw128(a_addr + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + k * MMA_K * 128, BK * 128, 1024)
+                                     : smem_desc_sw128(b_addr + k * 32, 16, 1024);
+            const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
+            if (FP8) mma_f8_ss(d_tmem, ad, bd, IDESC, accum);
+            else mma_bf16_ss(d_tmem, ad, bd, IDESC, accum);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == TC_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const float alpha = ep.alpha ? *ep.alpha : 1.f;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      int tm, tn, split;
+      tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      const long long row = (long long)tm * TC_BM + q * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < TC_BN; c += 32) {
+        const int col = tn * TC_BN + c;
+        if (col >= N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + c), r);
+        tmem_ld_wait();
+        if (row < M) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (col + g * 8 < N) {
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[g * 8 + i]) * alpha;
+              epi_apply8(ep, row, col + g * 8, v);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ---------------------------------------------------------- SIMT kernel ---
+// fp32 FFMA GEMM, 64x64 tile, 256 threads with 4x4 outputs each.
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(256) gemm_simt_f32_kernel(const float* __restrict__ A, long long lda,
+                                                            const float* __restrict__ B, long long ldb, int M, int N,
+                                                            int K, EpiParams ep) {
+  __shared__ float sa[16][64 + 4];
+  __shared__ float sb[16][64 + 4];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      const int kk = i / 64, mm = i % 64;
+      const int gm = m0 + mm, gk = k0 + kk, gn = n0 + mm;
+      sa[kk][mm] = (gm < M && gk < K) ? (A_MN ? A[(long long)gk * lda + gm] : A[(long long)gm * lda + gk]) : 0.f;
+      sb[kk][mm] = (gn < N && gk < K) ? (B_MN ? B[(long long)gk * ldb + gn] : B[(long long)gn * ldb + gk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = sa[kk][ty + 16 * i];
+        b[i] = sb[kk][tx + 16 * i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const float alpha = ep.alpha ? *ep.alpha : 1.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = m0 + ty + 16 * i, c = n0 + tx + 16 * j;
+      if (r < M && c < N) epi_apply1(ep, r, c, acc[i][j] * alpha);
+    }
+}
+
+}  // namespace gptb

@@ -1,0 +1,199 @@
+/* gptblock.h — C ABI of the B200 (sm_100a) GPT block library.
+ *
+ * One training step (forward + backward) of the nanochat GPT transformer
+ * block stack, as described on the source pages:
+ *   apidog.com/fr "Comment Entraîner Votre Propre ChatGPT Pour 50€ ?",
+ *   § "Comment nanochat fonctionne" › 1. Le modèle GPT (feature list: RoPE,
+ *   QK normalisation, untied embedding / output projection, ReLU², GQA,
+ *   sliding-window attention; value-embedding snippet; "efficiency tricks"
+ *   snippets: per-layer residual lambdas, smear, backout) and § 3 "Gestion de
+ *   la précision" (Linear casts the weight to the activation dtype; FP8 with
+ *   per-tensor scaling).
+ *
+ * Conventions for every entry point
+ *   - Every tensor pointer is a DEVICE pointer allocated by the caller (for
+ *     example through PyTorch).  The library never allocates or frees device
+ *     memory; buffers it needs beyond inputs and outputs come from a
+ *     caller-owned workspace whose size gptb_workspace_bytes() reports.
+ *   - Activations are row-major and token-major: [B, T, features].  Weights
+ *     follow nn.Linear, [out, in], and every projection is y = x W^T.
+ *   - Storage dtype (cfg.dtype): GPTB_F32 -> float; GPTB_BF16 and
+ *     GPTB_FP8_E4M3 -> bf16 storage (FP8 only changes the GEMM operands).
+ *   - Scalars (lambdas) are fp32 device values.  All gradients are fp32 and
+ *     ACCUMULATED (+=); the caller zeroes them before the first micro-step,
+ *     which makes gradient accumulation free.
+ *   - All work is enqueued on `stream`; no call synchronises the host except
+ *     gptb_device_error().  Pointers must be 16-byte aligned.
+ *   - Return value: GPTB_OK (0) or a negative GPTB_ERR_* code; nothing is
+ *     enqueued when an argument check fails.  No exceptions cross the ABI.
+ */
+#ifndef GPTBLOCK_H
+#define GPTBLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* gptb_stream_t; /* same type as cudaStream_t */
+
+enum {
+  GPTB_OK = 0,
+  GPTB_ERR_INVALID_ARG = -1, /* null / misaligned pointer, inconsistent shape */
+  GPTB_ERR_UNSUPPORTED = -2, /* dtype, head_dim or device not supported      */
+  GPTB_ERR_CUDA = -3,        /* a CUDA call or kernel launch failed          */
+  GPTB_ERR_TIMEOUT = -4,     /* a bounded device wait expired (see below)    */
+  GPTB_ERR_WORKSPACE = -5    /* workspace too small                          */
+};
+
+enum { GPTB_F32 = 0, GPTB_BF16 = 1, GPTB_FP8_E4M3 = 2 };
+
+#define GPTB_MAX_LAYERS 64
+
+/* Model shape and options.  Plain data, passed by pointer, copied by callee. */
+typedef struct {
+  int B, T;            /* batch rows, tokens per row                              */
+  int d;               /* model width, multiple of 8, <= 2048                     */
+  int n_head;          /* query heads H                                           */
+  int n_kv_head;       /* key/value heads Hkv, H % Hkv == 0 (GQA)                 */
+  int head_dim;        /* hd: 128 for bf16/fp8; <= 128 and even for f32           */
+  int mlp_hidden;      /* F (4*d in nanochat), multiple of 8                      */
+  int vocab;           /* V, multiple of 8                                        */
+  int n_layer;         /* L <= GPTB_MAX_LAYERS                                    */
+  int window[GPTB_MAX_LAYERS]; /* per layer: -1 full causal, else W: keys t-W..t  */
+  int has_ve[GPTB_MAX_LAYERS]; /* per layer: 1 = gated value embedding            */
+  int ve_gate_ch;      /* channels feeding the VE gate (32)                       */
+  int smear_ch;        /* channels feeding the smear gate (24); 0 = smear off     */
+  int backout_layer;   /* layer whose input is subtracted after the last; -1 off  */
+  float rope_base;     /* 10000                                                   */
+  float norm_eps;      /* RMSNorm epsilon inside the rsqrt (1e-6)                 */
+  int dtype;           /* GPTB_F32 | GPTB_BF16 | GPTB_FP8_E4M3                    */
+} gptb_config;
+
+/* Weights of one block (storage dtype).  w_ve_gate / ve_table only on
+ * value-embedding layers (NULL elsewhere). */
+typedef struct {
+  const void* w_qkv;      /* [(H+2Hkv)*hd, d]: rows q heads, then k, then v     */
+  const void* w_o;        /* [d, H*hd]                                          */
+  const void* w_fc;       /* [F, d]                                             */
+  const void* w_proj;     /* [d, F]                                             */
+  const void* w_ve_gate;  /* [Hkv, ve_gate_ch]                                  */
+  const void* ve_table;   /* [V, Hkv*hd]                                        */
+  const float* lambdas;   /* device fp32 [2]: resid_lambda, x0_lambda           */
+} gptb_block_weights;
+
+/* Gradients of one block, fp32, accumulated (+=), same shapes as above. */
+typedef struct {
+  float* w_qkv;
+  float* w_o;
+  float* w_fc;
+  float* w_proj;
+  float* w_ve_gate;  /* may be NULL on layers without VE                         */
+  float* ve_table;   /* dense [V, Hkv*hd] scatter-add target; NULL without VE    */
+  float* lambdas;    /* [2]                                                      */
+} gptb_block_grads;
+
+typedef struct {
+  const void* wte;           /* [V, d] token embedding                         */
+  const void* w_lm;          /* [V, d] untied output projection                */
+  const void* w_smear_gate;  /* [smear_ch]                                     */
+  const float* smear_lambda; /* device fp32 scalar                             */
+  const float* backout_lambda; /* device fp32 scalar                           */
+  gptb_block_weights layers[GPTB_MAX_LAYERS];
+} gptb_model_weights;
+
+typedef struct {
+  float* wte;
+  float* w_lm;
+  float* w_smear_gate;
+  float* smear_lambda;
+  float* backout_lambda;
+  gptb_block_grads layers[GPTB_MAX_LAYERS];
+} gptb_model_grads;
+
+/* Workspace kinds for gptb_workspace_bytes(). */
+enum {
+  GPTB_WS_BLOCK_SAVED = 0,   /* activations one block saves for its backward    */
+  GPTB_WS_BLOCK_SCRATCH = 1, /* temporaries of one block forward/backward        */
+  GPTB_WS_LM_HEAD = 2,       /* temporaries of lm_head_xent                      */
+  GPTB_WS_STACK = 3          /* everything gpt_stack_step needs                  */
+};
+
+/* Bytes of workspace of the given kind for this config (0 on a bad config). */
+size_t gptb_workspace_bytes(const gptb_config* cfg, int kind);
+
+/* One block forward (layer `layer` of cfg; its window / has_ve apply).
+ *   x, x0  [B,T,d]  block input and the stack's x0 (the smeared embedding)
+ *   idx    [B,T] int32 token ids (value-embedding lookup)
+ *   x_out  [B,T,d]  block output
+ *   saved  GPTB_WS_BLOCK_SAVED bytes, filled here, read by the backward
+ *   scratch GPTB_WS_BLOCK_SCRATCH bytes
+ * Computes xm = a x + b x0; h = rmsnorm(xm); q,k,v = h Wqkv^T;
+ * v += 3 sigmoid(h[:, :C] Wg^T) VE[idx]; q,k = rope(rmsnorm_per_head(q,k));
+ * x1 = xm + attn(q,k,v) Wo^T; x_out = x1 + relu(rmsnorm(x1) Wfc^T)^2 Wproj^T. */
+int gpt_block_forward(const gptb_config* cfg, int layer, const gptb_block_weights* w, const void* x,
+                      const void* x0, const int32_t* idx, void* x_out, void* saved, void* scratch,
+                      gptb_stream_t stream);
+
+/* One block backward from dL/dx_out.  Needs the forward's x, x0, idx and
+ * saved buffer.  Writes dx [B,T,d] (storage dtype), ACCUMULATES dx0_accum
+ * [B,T,d] (fp32) and every gradient in g.  dx_extra (nullable, storage dtype)
+ * is added to dx (used for the backout term). */
+int gpt_block_backward(const gptb_config* cfg, int layer, const gptb_block_weights* w, const void* x,
+                       const void* x0, const int32_t* idx, const void* saved, const void* dx_out,
+                       const void* dx_extra, void* dx, float* dx0_accum, gptb_block_grads* g, void* scratch,
+                       gptb_stream_t stream);
+
+/* Untied lm_head + mean next-token cross-entropy over N = B*T rows without
+ * materialising the full [N, V] logits (row chunks of at most 8192 tokens).
+ *   h [N,d] (normed final hidden state), w_lm [V,d], targets [N] int32
+ *   loss_out: device fp32 scalar (written, the mean over N)
+ *   dh [N,d] storage dtype (written); dw_lm [V,d] fp32 (accumulated)
+ *   ws: GPTB_WS_LM_HEAD bytes.  bf16/fp8 configs only. */
+int lm_head_xent(const gptb_config* cfg, const void* h, const void* w_lm, const int32_t* targets, float* loss_out,
+                 void* dh, float* dw_lm, void* ws, gptb_stream_t stream);
+
+/* Whole training step of the stack: embed -> smear -> L blocks -> backout ->
+ * final RMSNorm -> lm_head + cross-entropy, then the full backward.  Writes
+ * loss_out (device fp32 scalar) and accumulates every gradient in g.
+ * ws: GPTB_WS_STACK bytes.  bf16/fp8 configs (lm_head present). */
+int gpt_stack_step(const gptb_config* cfg, const gptb_model_weights* w, const int32_t* idx, const int32_t* targets,
+                   float* loss_out, gptb_model_grads* g, void* ws, gptb_stream_t stream);
+
+/* Plain GEMM entry point used by the tests of the tensor-core kernel:
+ * C[M,N] (+)= A[M,K] B[N,K]^T (bf16 operands, fp32 accumulate).
+ *   a_mn / b_mn: 0 = operand stored K-major (row-major [M,K] / [N,K]),
+ *                1 = stored MN-major (row-major [K,M] / [K,N]);
+ *   lda, ldb: row strides in elements of the stored matrices;
+ *   c_f32: 1 -> C is float and ACCUMULATED (+=, split-K allowed),
+ *          0 -> C is bf16 and overwritten; ldc in elements. */
+int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, void* C,
+                   int c_f32, long long ldc, int M, int N, int K, gptb_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns GPTB_OK, GPTB_ERR_TIMEOUT if a bounded wait inside a kernel expired
+ * (the kernel recorded it, drained and returned), or GPTB_ERR_CUDA. */
+int gptb_device_error(gptb_stream_t stream);
+
+/* Wait limit (nanoseconds) of every bounded device wait; default 2 s.
+ * Applies to kernels launched afterwards on the current device. */
+int gptb_set_wait_limit_ns(unsigned long long ns);
+
+/* Kernel accounting: every kernel this library launches increments a host
+ * counter; with timing enabled, the GEMM launches are also bracketed by CUDA
+ * events on their stream and their device time and FLOPs are accumulated. */
+void gptb_reset_counters(void);
+long long gptb_launch_count(void);
+int gptb_set_gemm_timing(int enable);
+/* Sum of GEMM device milliseconds and FLOPs since the last reset (syncs). */
+int gptb_gemm_timing(double* ms, double* flops, long long* launches);
+
+/* Human-readable text for a return code. */
+const char* gptb_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTBLOCK_H */

@@ -1,0 +1,49 @@
+"""Shared helpers for the parity tests (no method arithmetic here)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+
+TOL = {"bf16": 2e-2, "fp8": 6e-2, "f32": 1e-5}
+
+
+def relerr(gpu, ref) -> float:
+    """Normwise max relative error: max|gpu - ref| / max|ref|."""
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    denom = np.max(np.abs(r)) if r.size else 0.0
+    if denom == 0.0:
+        return float(np.max(np.abs(g))) if g.size else 0.0
+    return float(np.max(np.abs(g - r)) / denom)
+
+
+def np64(t) -> np.ndarray:
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().double().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def oracle_layer(w: dict, i: int) -> dict:
+    """Synthetic layer weights as fp64 numpy arrays / floats for the oracle."""
+    out = {}
+    for k, v in w["layers"][i].items():
+        out[k] = v if isinstance(v, float) else np64(v)
+    return out
+
+
+def oracle_weights(w: dict) -> dict:
+    out = {"layers": [oracle_layer(w, i) for i in range(len(w["layers"]))]}
+    for k, v in w.items():
+        if k != "layers":
+            out[k] = v if isinstance(v, float) else np64(v)
+    return out
+
+
+def small_bf16(**kw) -> dict:
+    """A small bf16 stack that spans several GEMM tiles with ragged tails."""
+    base = dict(B=2, T=200, d=256, n_head=2, n_kv_head=1, n_layer=3, vocab=512, mlp_hidden=1024,
+                window=[-1, 48, -1], has_ve=[0, 1, 0], backout_layer=1)
+    base.update(kw)
+    return synth.config("d24", **base)

@@ -1,0 +1,80 @@
+"""Block forward/backward parity through the C ABI against the fp64 oracle.
+
+Inputs are the same seeded values on both sides (rounded to the storage
+dtype, widened to fp64 for the oracle).  Tolerance: normwise max relative
+error <= 2e-2 for bf16 storage, <= 1e-5 for the fp32 configuration."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import model as om
+from helpers import TOL, np64, oracle_layer, relerr, small_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def run_block(gb, c, w, inp, layer):
+    from gpt_transformer_block_b200.model import BlockRunner, to_device_weights, zero_grads_like, storage_torch_dtype
+    dt = storage_torch_dtype(c)
+    dw = to_device_weights(c, w)
+    lw = dw["layers"][layer]
+    x = inp["x"].to("cuda", dt)
+    x0 = inp["x0"].to("cuda", dt)
+    dy = inp["dy"].to("cuda", dt)
+    idx = inp["idx"].cuda()
+    r = BlockRunner(c)
+    x_out = torch.empty_like(x)
+    r.forward(layer, lw, x, x0, idx, x_out)
+    g = zero_grads_like(c, dw)["layers"][layer]
+    dx = torch.empty_like(x)
+    dx0 = torch.zeros(x.shape, dtype=torch.float32, device="cuda")
+    r.backward(layer, lw, x, x0, idx, dy, dx, dx0, g)
+    torch.cuda.synchronize()
+    assert gb.gptb_device_error() == 0
+    return x_out, dx, dx0, g
+
+
+def check_block(gb, c, layer, seed=1, x_std=1.0, exact_keys=()):
+    w = synth.make_weights(c, seed=seed)
+    inp = synth.make_block_inputs(c, seed=seed + 1, x_std=x_std)
+    x_out, dx, dx0, g = run_block(gb, c, w, inp, layer)
+    lw = oracle_layer(w, layer)
+    y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), inp["idx"].numpy(), layer)
+    rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), inp["idx"].numpy(), layer)
+    tol = TOL[c["dtype"]]
+    errs = {"x_out": relerr(np64(x_out), y), "dx": relerr(np64(dx), rdx), "dx0": relerr(np64(dx0), rdx0)}
+    for k in ("w_qkv", "w_o", "w_fc", "w_proj", "w_ve_gate", "ve_table"):
+        if k in rg:
+            errs[k] = relerr(np64(g[k]), rg[k])
+    lam = np64(g["lambdas"])
+    errs["resid_lambda"] = relerr(lam[0:1], [rg["resid_lambda"]])
+    errs["x0_lambda"] = relerr(lam[1:2], [rg["x0_lambda"]])
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (bad, errs)
+    return errs
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2])
+def test_block_bf16_small(cuda_lib, layer):
+    # layer 0: full causal; layer 1: window 48 + value embedding; layer 2: full
+    check_block(cuda_lib, small_bf16(), layer)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_block_bf16_gqa_window(cuda_lib, layer):
+    # H=4, Hkv=2 (G=2), H*hd != d, T not a multiple of any tile
+    c = small_bf16(n_head=4, n_kv_head=2, T=333, B=1, window=[100, 0, -1], has_ve=[1, 1, 0], n_layer=3)
+    check_block(cuda_lib, c, layer)
+
+
+def test_block_fp32_config(cuda_lib):
+    # the fp32 block as specified: B=2, T=64, d=128, H=2, Hkv=1, hd=64, window 32
+    c = synth.config("block_fp32")
+    check_block(cuda_lib, c, 0)
+
+
+def test_block_fp32_all_terms(cuda_lib):
+    # same block with every term on: value embedding, random lambdas
+    c = synth.config("block_fp32", has_ve=[1])
+    check_block(cuda_lib, c, 0)

@@ -1,0 +1,107 @@
+"""lm_head_xent and gpt_stack_step parity through the C ABI against the
+fp64 oracle (loss and every gradient)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import model as om
+from helpers import TOL, np64, oracle_weights, relerr, small_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_lm_head_xent(cuda_lib, dtype):
+    from gpt_transformer_block_b200.model import lm_head
+    g = torch.Generator().manual_seed(3)
+    N, d, V = 300, 256, 1024
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    h = torch.randn(N, d, generator=g).to(tdt)
+    w = (torch.randn(V, d, generator=g) * 0.05).to(tdt)
+    y = torch.randint(0, V, (N,), generator=g, dtype=torch.int32)
+    c = small_bf16(B=1, T=N, vocab=V, dtype=dtype, head_dim=128 if dtype == "bf16" else 64)
+    dh = torch.empty(N, d, dtype=tdt, device="cuda")
+    dw = torch.zeros(V, d, dtype=torch.float32, device="cuda")
+    loss = lm_head(c, h.cuda(), w.cuda(), y.cuda(), dh, dw)
+    torch.cuda.synchronize()
+    rl, rdh, rdw = om.lm_head_xent(np64(h), np64(w), y.numpy())
+    tol = TOL[dtype]
+    assert abs(loss.item() - rl) / abs(rl) <= tol
+    assert relerr(np64(dh), rdh) <= tol
+    assert relerr(np64(dw), rdw) <= tol
+
+
+def run_stack(gb, c, w, batch):
+    from gpt_transformer_block_b200.model import GPTStack
+    st = GPTStack(c, w)
+    loss = st.step(batch["idx"].cuda(), batch["targets"].cuda())
+    torch.cuda.synchronize()
+    assert gb.gptb_device_error() == 0
+    return loss.item(), st.g
+
+
+def compare_stack(c, w, batch, loss, g):
+    ow = oracle_weights(w)
+    rl, cache = om.stack_forward(c, ow, batch["idx"].numpy(), batch["targets"].numpy())
+    rg = om.stack_backward(c, ow, cache, batch["idx"].numpy())
+    tol = TOL[c["dtype"]]
+    errs = {"loss": abs(loss - rl) / abs(rl)}
+    for k in ("wte", "w_lm", "w_smear_gate"):
+        if k in rg:
+            errs[k] = relerr(np64(g[k]), rg[k])
+    for k in ("smear_lambda", "backout_lambda"):
+        if k in rg:
+            errs[k] = relerr(np64(g[k]), [rg[k]])
+    for i, lg in enumerate(rg["layers"]):
+        for k, v in lg.items():
+            if k in ("resid_lambda", "x0_lambda"):
+                errs[f"L{i}.{k}"] = relerr(np64(g["layers"][i]["lambdas"])[0 if k == "resid_lambda" else 1:][:1], [v])
+            else:
+                errs[f"L{i}.{k}"] = relerr(np64(g["layers"][i][k]), v)
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (bad, errs)
+    return errs
+
+
+def test_stack_bf16_small(cuda_lib):
+    c = small_bf16()
+    w = synth.make_weights(c, seed=11)
+    b = synth.make_batch(c, seed=12)
+    loss, g = run_stack(cuda_lib, c, w, b)
+    compare_stack(c, w, b, loss, g)
+
+
+def test_stack_bf16_gqa_backout0(cuda_lib):
+    c = small_bf16(n_head=4, n_kv_head=2, n_layer=2, window=[64, -1], has_ve=[1, 0], backout_layer=0, T=130)
+    w = synth.make_weights(c, seed=21)
+    b = synth.make_batch(c, seed=22)
+    loss, g = run_stack(cuda_lib, c, w, b)
+    compare_stack(c, w, b, loss, g)
+
+
+def test_stack_fp32_all_terms(cuda_lib):
+    # the fp32 block width/heads at stack level with VE, smear, backout on
+    c = synth.config("block_fp32", n_layer=2, has_ve=[0, 1], smear_ch=24, backout_layer=1, lm_head=True,
+                     vocab=512, window=[32, -1])
+    w = synth.make_weights(c, seed=31)
+    b = synth.make_batch(c, seed=32)
+    loss, g = run_stack(cuda_lib, c, w, b)
+    compare_stack(c, w, b, loss, g)
+
+
+def test_grad_accumulation_equals_sum(cuda_lib):
+    """Two steps without zeroing accumulate exactly twice one step's gradients
+    (the property gradient accumulation relies on)."""
+    from gpt_transformer_block_b200.model import GPTStack
+    c = small_bf16(n_layer=2, window=[-1, 32], has_ve=[0, 1])
+    w = synth.make_weights(c, seed=41)
+    b = synth.make_batch(c, seed=42)
+    st = GPTStack(c, w)
+    idx, tg = b["idx"].cuda(), b["targets"].cuda()
+    st.step(idx, tg)
+    one = st.g["layers"][1]["w_qkv"].clone()
+    st.step(idx, tg)
+    torch.cuda.synchronize()
+    two = st.g["layers"][1]["w_qkv"]
+    assert relerr(two.cpu().numpy(), 2 * one.cpu().numpy()) < 1e-5
