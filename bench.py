@@ -1,0 +1,350 @@
+#!/usr/bin/env python
+"""Training-step throughput of the GPT block stack on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload d24]
+
+One step = one gpt_stack_step (embedding, smear, L blocks forward, backout,
+final norm, lm_head + cross-entropy, and the whole backward) over one batch of
+synthetic token ids, with weights, ids and targets resident in HBM.  Rank 0
+prints one JSON line.  Under torchrun (N > 1) every rank runs its own batch
+(weak scaling, one replica per GPU, no collective in the data path); the
+timed region is bracketed by barriers and the max over ranks is reported.
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only)
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+PAGES_FLOPS_NOTE = "6*(N_mat + d*V) + 12*L*H*hd*T_eff"
+
+
+# ------------------------------------------------------------------ FLOPs --
+
+def attention_pairs(T: int, window: int) -> int:
+    """Visible (query, key) pairs of one causal row of length T."""
+    if window < 0 or window >= T - 1:
+        return T * (T + 1) // 2
+    W = window
+    # rows t <= W see t+1 keys; later rows see W+1 keys
+    return (W + 1) * (W + 2) // 2 + (T - W - 1) * (W + 1)
+
+
+def flops_per_token(c: dict) -> dict:
+    """Algorithmic training FLOPs per token (forward + backward = 3x forward).
+
+    Matmul parameters count 6 FLOPs per token; attention counts only the
+    visible pairs (4*hd per pair and head forward: QK^T and PV), times 3.
+    The pages-convention count uses 12*L*H*hd*T_eff with T_eff the average
+    attended length T/2-ish convention of the source (T for full layers,
+    window for windowed layers, averaged)."""
+    d, H, Hk, hd, F, V, L, T = (c["d"], c["n_head"], c["n_kv_head"], c["head_dim"], c["mlp_hidden"],
+                                c["vocab"], c["n_layer"], c["T"])
+    n_mat = L * (d * (H + 2 * Hk) * hd + H * hd * d + 2 * d * F)
+    n_lm = d * V if c.get("lm_head", True) else 0
+    att = sum(12 * hd * H * attention_pairs(T, c["window"][i]) for i in range(L)) / T
+    t_eff = sum((T if c["window"][i] < 0 else min(T, c["window"][i])) for i in range(L)) / L
+    pages = 6 * (n_mat + n_lm) + 12 * L * H * hd * t_eff
+    return {"algorithmic": 6 * (n_mat + n_lm) + att, "pages_convention": pages,
+            "matmul_params": n_mat + n_lm}
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
+        loaded = sorted(sm)[len(sm) // 4:] if len(sm) > 4 else sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------- peaks ---------
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def profile_traffic(workload: str) -> float | None:
+    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", f"gemm_tc_{workload}.json")
+    if os.path.exists(p):
+        try:
+            return float(json.load(open(p))["dram_bytes_per_launch"])
+        except Exception:
+            return None
+    return None
+
+
+# -------------------------------------------------------------- oracle arm -
+
+def oracle_sample(c: dict, seed: int = 7) -> dict:
+    """Time the fp64 oracle on one block slice (B=1, full T) forward+backward
+    plus the lm_head on 512 tokens, and extrapolate to one full step."""
+    import numpy as np
+    from oracle import model as om
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    cs = dict(c, B=1)
+    w = synth.make_weights(cs, seed=seed, mode="random")
+    inp = synth.make_block_inputs(cs, seed=seed + 1)
+    layer = max(i for i in range(cs["n_layer"]) if True)  # last layer: value embedding on
+    lw = {k: (v if isinstance(v, float) else np.asarray(v, dtype=np.float64)) for k, v in w["layers"][layer].items()}
+    x = inp["x"].double().numpy()
+    x0 = inp["x0"].double().numpy()
+    dy = inp["dy"].double().numpy()
+    idx = inp["idx"].numpy()
+    t0 = time.perf_counter()
+    _, cache = om.block_forward(cs, lw, x, x0, idx, layer)
+    om.block_backward(cs, lw, cache, dy, idx, layer)
+    t_block = time.perf_counter() - t0
+    n_lm = min(512, cs["T"])
+    h = np.random.default_rng(seed).standard_normal((n_lm, cs["d"]))
+    wl = np.asarray(w["w_lm"], dtype=np.float64)
+    y = np.random.default_rng(seed + 1).integers(0, cs["vocab"], n_lm)
+    t0 = time.perf_counter()
+    om.lm_head_xent(h, wl, y)
+    t_lm = (time.perf_counter() - t0) * (cs["T"] / n_lm)
+    t_step_row = cs["n_layer"] * t_block + t_lm   # one batch row of T tokens
+    return {"tok_per_s": cs["T"] / t_step_row, "cores": cores, "t_block_s": t_block, "t_lm_s": t_lm,
+            "sample": f"one block fwd+bwd at B=1,T={cs['T']},d={cs['d']} (layer {layer}) x {cs['n_layer']} layers "
+                      f"+ lm_head fwd+bwd on {n_lm} tokens scaled to {cs['T']}; fp64 numpy"}
+
+
+def run_reference(args, c: dict, fl: dict):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    vals = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        info = oracle_sample(c, seed=7 + i)
+        if i >= args.warmup:
+            vals.append(info["tok_per_s"])
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "training tokens/sec (fwd+bwd)", "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": c["name"], "global_batch": c["B"], "seq_len": c["T"], "parallelism": "cpu"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+                         "sample": info["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "mfu_algorithmic": None, "flops_per_token": fl,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="d24", choices=list(synth.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    c = synth.config(args.workload)
+    fl = flops_per_token(c)
+    if args.impl == "reference":
+        run_reference(args, c, fl)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    import gpt_transformer_block_b200 as gb
+    from gpt_transformer_block_b200.model import GPTStack
+    gb.load()
+
+    w = synth.make_weights(c, seed=1234 + rank, mode="init")
+    batch = synth.make_batch(c, seed=4321 + rank)
+    model = GPTStack(c, w)
+    idx = batch["idx"].cuda()
+    tg = batch["targets"].cuda()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        model.step(idx, tg)
+    torch.cuda.synchronize()
+    if gb.gptb_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- timed region: device-resident inputs
+    gb.gptb_reset_counters()
+    gb.gptb_set_gemm_timing(True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        model.step(idx, tg)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ck = clocks.stop()
+    gb.gptb_set_gemm_timing(False)
+    ms = e0.elapsed_time(e1)
+    launches = gb.gptb_launch_count()
+    gemm_ms, gemm_flops, gemm_n = gb.gptb_gemm_timing()
+    err = gb.gptb_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {err} in timed region")
+    loss = model.loss.item()
+
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+
+    tokens_per_step = c["B"] * c["T"]
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    ms_step = ms / args.steps
+
+    # ---- end to end through the public API, inputs from pinned host memory
+    idx_h = batch["idx"].pin_memory()
+    tg_h = batch["targets"].pin_memory()
+    loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(args.e2e_steps):
+        idx.copy_(idx_h, non_blocking=True)
+        tg.copy_(tg_h, non_blocking=True)
+        model.step(idx, tg)
+        loss_h.copy_(model.loss, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    e2e_s = time.perf_counter() - t0
+    if dist is not None:
+        t = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = t.item()
+    e2e_val = world * tokens_per_step * args.e2e_steps / e2e_s
+
+    peaks = measured_peaks()
+    flops_s = value / world * fl["algorithmic"]
+    gemm_tflops = gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    peak_t = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": "training tokens/sec (fwd+bwd) on 1 B200 and MFU vs bf16 tensor peak",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": c["name"], "global_batch": c["B"] * world, "seq_len": c["T"],
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "n_layer": c["n_layer"], "d_model": c["d"], "vocab": c["vocab"],
+                   "l2": "working set (~40 GB of saved activations) far larger than L2; no flush"},
+        "mfu": {"algorithmic_flops_per_token": fl["algorithmic"],
+                "pages_flops_per_token": fl["pages_convention"],
+                "vs_nominal_2250": flops_s / 2.25e15,
+                "vs_measured_sustained": flops_s / (peak_t * 1e12),
+                "pages_convention_vs_nominal": value / world * fl["pages_convention"] / 2.25e15},
+        "roofline": {"kernel": "gemm_tc_kernel (tcgen05, all GEMMs of the step)", "bound": "tensor",
+                     "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": (gemm_tflops / peak_t) if gemm_tflops else None,
+                     "peak_source": f"{peaks['source']} bf16 sustained",
+                     "traffic": profile_traffic(c["name"]),
+                     "share_of_step": gemm_ms / ms if ms > 0 else None, "launches": gemm_n},
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": 2 * tokens_per_step * 4,
+                "d2h_bytes_per_step": 4},
+        "gpu_launches": launches,
+        "clocks": ck,
+        "loss": loss,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        info = oracle_sample(c)
+        line["cpu_baseline"] = {"value": info["tok_per_s"], "unit": "tokens/s", "cores": info["cores"],
+                                "kind": "oracle", "sample": info["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del model
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -253,6 +253,10 @@ def block_backward(c, lw, cache, dx2, idx, layer, fp8=False):
     a, b = float(lw["resid_lambda"]), float(lw["x0_lambda"])
     g["resid_lambda"] = float(np.sum(dxm * cache["x"]))
     g["x0_lambda"] = float(np.sum(dxm * cache["x0"]))
+    # conditioning of the two scalar sums: sum of |terms| (used to judge a
+    # rounded evaluation of a cancelling sum; not a gradient)
+    g["_scale"] = {"resid_lambda": float(np.sum(np.abs(dxm * cache["x"]))),
+                   "x0_lambda": float(np.sum(np.abs(dxm * cache["x0"])))}
     return a * dxm, b * dxm, g
 
 
@@ -271,7 +275,7 @@ def smear_forward(x, w_gate, lam):
 
 
 def smear_backward(dy, x, sg, w_gate, lam):
-    """Returns (dx, d w_gate, d lambda)."""
+    """Returns (dx, d w_gate, d lambda, sum of |terms| of d lambda)."""
     x = _f64(x)
     C = np.asarray(w_gate).shape[0]
     dx = dy.copy()
@@ -282,7 +286,7 @@ def smear_backward(dy, x, sg, w_gate, lam):
     dz = lam * s * sg * (1.0 - sg)
     dw = np.einsum("bt,btc->c", dz, x[..., :C])
     dx[..., :C] += dz[..., None] * _f64(w_gate)[None, None, :]
-    return dx, dw, dlam
+    return dx, dw, dlam, float(np.sum(np.abs(sg[:, 1:, None] * dy[:, 1:, :] * x[:, :-1, :])))
 
 
 # ---------------------------------------------------------------------------
@@ -347,13 +351,14 @@ def stack_backward(c, w, cache, idx, fp8=False):
     """Gradients of the mean loss w.r.t. every parameter of the stack."""
     idx = np.asarray(idx)
     L = c["n_layer"]
-    grads = {"w_lm": cache["dw_lm"], "layers": [None] * L}
+    grads = {"w_lm": cache["dw_lm"], "layers": [None] * L, "_scale": {}}
     dxf = rmsnorm_backward(cache["dhf"], cache["hf"], cache["rf"])
     dx = dxf
     dx_bo = None
     if cache["x_bo"] is not None:
         lam = float(w["backout_lambda"])
         grads["backout_lambda"] = float(-np.sum(dxf * cache["x_bo"]))
+        grads["_scale"]["backout_lambda"] = float(np.sum(np.abs(dxf * cache["x_bo"])))
         dx_bo = -lam * dxf
     dx0 = np.zeros_like(dx)
     for i in reversed(range(L)):
@@ -364,9 +369,10 @@ def stack_backward(c, w, cache, idx, fp8=False):
         grads["layers"][i] = gi
     dxs = dx + dx0                     # x0 is the smeared embedding itself
     if c["smear_ch"] > 0:
-        demb, dws, dlam = smear_backward(dxs, cache["emb"], cache["smear_sg"],
-                                         w["w_smear_gate"], float(w["smear_lambda"]))
+        demb, dws, dlam, dlam_scale = smear_backward(dxs, cache["emb"], cache["smear_sg"],
+                                                     w["w_smear_gate"], float(w["smear_lambda"]))
         grads["w_smear_gate"], grads["smear_lambda"] = dws, dlam
+        grads["_scale"]["smear_lambda"] = dlam_scale
     else:
         demb = dxs
     V, d = np.asarray(w["wte"]).shape

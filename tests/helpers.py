@@ -19,6 +19,12 @@ def relerr(gpu, ref) -> float:
     return float(np.max(np.abs(g - r)) / denom)
 
 
+def scalar_err(gpu: float, ref: float, scale: float) -> float:
+    """Error of a scalar sum judged against the sum of its terms' magnitudes
+    (forward-error bound of a rounded dot product): |gpu - ref| / sum|terms|."""
+    return abs(float(gpu) - float(ref)) / max(float(scale), 1e-300)
+
+
 def np64(t) -> np.ndarray:
     if isinstance(t, torch.Tensor):
         return t.detach().float().cpu().double().numpy()

@@ -9,7 +9,7 @@ import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, np64, oracle_layer, relerr, small_bf16
+from helpers import TOL, np64, oracle_layer, relerr, scalar_err, small_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -48,8 +48,8 @@ def check_block(gb, c, layer, seed=1, x_std=1.0, exact_keys=()):
         if k in rg:
             errs[k] = relerr(np64(g[k]), rg[k])
     lam = np64(g["lambdas"])
-    errs["resid_lambda"] = relerr(lam[0:1], [rg["resid_lambda"]])
-    errs["x0_lambda"] = relerr(lam[1:2], [rg["x0_lambda"]])
+    errs["resid_lambda"] = scalar_err(lam[0], rg["resid_lambda"], rg["_scale"]["resid_lambda"])
+    errs["x0_lambda"] = scalar_err(lam[1], rg["x0_lambda"], rg["_scale"]["x0_lambda"])
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, (bad, errs)
     return errs

@@ -6,7 +6,7 @@ import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, np64, oracle_weights, relerr, small_bf16
+from helpers import TOL, np64, oracle_weights, relerr, scalar_err, small_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -52,11 +52,14 @@ def compare_stack(c, w, batch, loss, g):
             errs[k] = relerr(np64(g[k]), rg[k])
     for k in ("smear_lambda", "backout_lambda"):
         if k in rg:
-            errs[k] = relerr(np64(g[k]), [rg[k]])
+            errs[k] = scalar_err(np64(g[k])[0], rg[k], rg["_scale"][k])
     for i, lg in enumerate(rg["layers"]):
+        lam = np64(g["layers"][i]["lambdas"])
         for k, v in lg.items():
+            if k == "_scale":
+                continue
             if k in ("resid_lambda", "x0_lambda"):
-                errs[f"L{i}.{k}"] = relerr(np64(g["layers"][i]["lambdas"])[0 if k == "resid_lambda" else 1:][:1], [v])
+                errs[f"L{i}.{k}"] = scalar_err(lam[0 if k == "resid_lambda" else 1], v, lg["_scale"][k])
             else:
                 errs[f"L{i}.{k}"] = relerr(np64(g["layers"][i][k]), v)
     bad = {k: v for k, v in errs.items() if not v <= tol}
