@@ -22,7 +22,7 @@ EXPORTS = [
     "gptb_workspace_bytes", "gpt_block_forward", "gpt_block_backward", "lm_head_xent",
     "gpt_stack_step", "gptb_gemm_bf16", "gptb_device_error", "gptb_set_wait_limit_ns",
     "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
-    "gptb_error_string",
+    "gptb_error_string", "lm_head_xent_noalloc",
 ]
 
 _vp = ctypes.c_void_p
@@ -78,6 +78,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gpt_block_backward.argtypes = [P(Config), ctypes.c_int, P(BlockWeights), _vp, _vp, _vp, _vp, _vp, _vp,
                                        _vp, _vp, P(BlockGrads), _vp, _vp]
     lib.lm_head_xent.argtypes = [P(Config), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.lm_head_xent_noalloc.argtypes = [P(Config), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     lib.gpt_stack_step.argtypes = [P(Config), P(ModelWeights), _vp, _vp, _vp, P(ModelGrads), _vp, _vp]
     lib.gptb_gemm_bf16.argtypes = [_vp, ctypes.c_int, ctypes.c_longlong, _vp, ctypes.c_int, ctypes.c_longlong,
                                    _vp, ctypes.c_int, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
@@ -196,6 +197,12 @@ def gpt_block_backward(cfg, layer, w: BlockWeights, x, x0, idx, saved, dx_out, d
 def lm_head_xent(cfg, h, w_lm, targets, loss_out, dh, dw_lm, ws, stream=None):
     _check(load().lm_head_xent(ctypes.byref(cfg), ptr(h), ptr(w_lm), ptr(targets), ptr(loss_out), ptr(dh),
                                ptr(dw_lm), ptr(ws), _stream(stream)), "lm_head_xent")
+
+
+def lm_head_xent_noalloc(cfg, h, w_lm, targets, loss_out, dh, dw_lm, stream=None):
+    """lm_head_xent with the library's own static scratch (no workspace argument)."""
+    _check(load().lm_head_xent_noalloc(ctypes.byref(cfg), ptr(h), ptr(w_lm), ptr(targets), ptr(loss_out), ptr(dh),
+                                       ptr(dw_lm), _stream(stream)), "lm_head_xent_noalloc")
 
 
 def gpt_stack_step(cfg, w: ModelWeights, idx, targets, loss_out, g: ModelGrads, ws, stream=None):

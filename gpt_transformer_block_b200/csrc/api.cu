@@ -739,3 +739,56 @@ const char* gptb_error_string(int code) {
 }
 
 }  // extern "C"
+
+// ======================================================= no-alloc lm_head ==
+// lm_head_xent for callers that cannot allocate device memory: its scratch
+// (one chunk of logits and the per-row losses) lives in this file-scope
+// device array instead of a caller-provided workspace.  Every GPU that loads
+// the library holds the array until the process exits.
+namespace {
+
+constexpr size_t NOALLOC_LOGITS_BYTES = size_t(8) << 20;  // logits of one row chunk
+constexpr long long NOALLOC_MAX_ROWS = 65536;             // B*T limit (row losses)
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_LOGITS_BYTES + NOALLOC_MAX_ROWS * 4];
+
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (host code only sees a host-side stand-in under the name).
+int noalloc_scratch(unsigned char** out) {
+  static std::mutex mu;
+  static unsigned char* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTB_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return GPTB_ERR_CUDA;
+    }
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = addr[dev];
+  return GPTB_OK;
+}
+
+}  // namespace
+
+extern "C" int lm_head_xent_noalloc(const gptb_config* cfg, const void* h, const void* w_lm, const int32_t* targets,
+                                    float* loss_out, void* dh, float* dw_lm, gptb_stream_t stream) {
+  TRY(check_config(cfg));
+  if (!h || !w_lm || !targets || !loss_out || !dh || !dw_lm) return GPTB_ERR_INVALID_ARG;
+  const Dims m = dims_of(*cfg);
+  if (m.N > NOALLOC_MAX_ROWS) return GPTB_ERR_WORKSPACE;
+  const long long rows = (long long)(NOALLOC_LOGITS_BYTES / ((size_t)m.V * m.esz));
+  if (rows < 1) return GPTB_ERR_WORKSPACE;
+  unsigned char* base = nullptr;
+  TRY(noalloc_scratch(&base));
+  LmWs lw;
+  lw.logits = base;
+  lw.row_loss = reinterpret_cast<float*>(base + NOALLOC_LOGITS_BYTES);
+  lw.chunk = (int)std::min<long long>(rows, m.N);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == GPTB_F32)
+    return lm_head_impl<float>(*cfg, (const float*)h, (const float*)w_lm, targets, loss_out, (float*)dh, dw_lm, lw, st);
+  return lm_head_impl<bf16>(*cfg, (const bf16*)h, (const bf16*)w_lm, targets, loss_out, (bf16*)dh, dw_lm, lw, st);
+}

@@ -155,6 +155,27 @@ int gpt_block_backward(const gptb_config* cfg, int layer, const gptb_block_weigh
 int lm_head_xent(const gptb_config* cfg, const void* h, const void* w_lm, const int32_t* targets, float* loss_out,
                  void* dh, float* dw_lm, void* ws, gptb_stream_t stream);
 
+/* lm_head_xent without a workspace, for callers that cannot allocate device
+ * memory themselves: for example a plugin or C caller that is handed tensors
+ * and a stream by a host framework whose allocator owns all device memory, or
+ * a latency-critical path that must not call cudaMalloc (which can
+ * synchronise the device).  No counterpart on the source pages: this is a
+ * convenience of this library.
+ *   Same arguments, results and accumulation (+= into dw_lm) as lm_head_xent,
+ *   minus `ws`.  Its scratch is one file-scope device array of 8 MiB of
+ *   logits plus 256 KiB of row losses, held by every GPU that loads the
+ *   library until the process exits.  Limits: B*T <= 65536 and
+ *   vocab * element size <= 8 MiB (otherwise GPTB_ERR_WORKSPACE, nothing
+ *   enqueued).  Rows are processed in chunks of 8 MiB / (vocab * element
+ *   size) rows (128 rows for vocab 32768 in bf16).
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Nothing is allocated or freed.  All calls share the one array and every
+ *   call overwrites it: calls that overlap on the GPU (other streams, other
+ *   threads) race and give wrong results; serialise them. */
+int lm_head_xent_noalloc(const gptb_config* cfg, const void* h, const void* w_lm, const int32_t* targets,
+                         float* loss_out, void* dh, float* dw_lm, gptb_stream_t stream);
+
 /* Whole training step of the stack: embed -> smear -> L blocks -> backout ->
  * final RMSNorm -> lm_head + cross-entropy, then the full backward.  Writes
  * loss_out (device fp32 scalar) and accumulates every gradient in g.
