@@ -13,6 +13,7 @@
 
 #include "../../include/gptblock.h"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "elementwise.cuh"
 #include "gemm.cuh"
@@ -155,10 +156,10 @@ int plan_splits(int tiles, int kb_total, int sms) {
   return best;
 }
 
-template <bool AM, bool BM>
+template <bool AM, bool BM, bool F8>
 int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, int splits, const EpiParams& ep,
               cudaStream_t st, int sms) {
-  auto kern = gemm_tc_kernel<AM, BM, false>;
+  auto kern = gemm_tc_kernel<AM, BM, F8>;
   const int smem = tc_smem_bytes();
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const long long units = (long long)((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN) * splits;
@@ -197,25 +198,35 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
       rc = GPTB_ERR_CUDA;
     }
   } else {
+    // tcgen05 path: bf16 operands, or e4m3 operands when dtype == GPTB_FP8_E4M3
     const DevInfo di = dev_info();
     if (di.cc_major != 10) return GPTB_ERR_UNSUPPORTED;
-    if (!aligned16(A.p) || !aligned16(B.p) || !aligned16(ep.out) || (A.ld % 8) || (B.ld % 8) || (ep.ldo % 8) ||
-        (N % 8))
+    const bool f8 = dtype == GPTB_FP8_E4M3;
+    const int align = f8 ? 16 : 8;  // row strides must be multiples of 16 bytes
+    const uint32_t bk = f8 ? 128 : 64;
+    if (!aligned16(A.p) || !aligned16(B.p) || !aligned16(ep.out) || (A.ld % align) || (B.ld % align) ||
+        (ep.ldo % 8) || (N % 8))
       return GPTB_ERR_INVALID_ARG;
     CUtensorMap ta, tb;
-    bool ok = A.mn ? make_tmap(&ta, A.p, false, M, K, A.ld, 64, 64) : make_tmap(&ta, A.p, false, K, M, A.ld, 64, TC_BM);
-    ok = ok && (B.mn ? make_tmap(&tb, B.p, false, N, K, B.ld, 64, 64)
-                     : make_tmap(&tb, B.p, false, K, N, B.ld, 64, TC_BN));
+    bool ok = A.mn ? make_tmap(&ta, A.p, f8, M, K, A.ld, bk, bk) : make_tmap(&ta, A.p, f8, K, M, A.ld, bk, TC_BM);
+    ok = ok && (B.mn ? make_tmap(&tb, B.p, f8, N, K, B.ld, bk, bk) : make_tmap(&tb, B.p, f8, K, N, B.ld, bk, TC_BN));
     if (!ok) return GPTB_ERR_CUDA;
     int splits = 1;
     if (ep.kind == EPI_ACCUM_F32) {
       const int tiles = ((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN);
-      splits = plan_splits(tiles, (K + 63) / 64, di.sms);
+      splits = plan_splits(tiles, (K + (int)bk - 1) / (int)bk, di.sms);
     }
-    if (!A.mn && !B.mn) rc = launch_tc<false, false>(ta, tb, M, N, K, splits, ep, st, di.sms);
-    else if (!A.mn && B.mn) rc = launch_tc<false, true>(ta, tb, M, N, K, splits, ep, st, di.sms);
-    else if (A.mn && B.mn) rc = launch_tc<true, true>(ta, tb, M, N, K, splits, ep, st, di.sms);
-    else rc = launch_tc<true, false>(ta, tb, M, N, K, splits, ep, st, di.sms);
+    const int sel = (A.mn ? 1 : 0) | (B.mn ? 2 : 0) | (f8 ? 4 : 0);
+    switch (sel) {
+      case 0: rc = launch_tc<false, false, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      case 1: rc = launch_tc<true, false, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      case 2: rc = launch_tc<false, true, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      case 3: rc = launch_tc<true, true, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      case 4: rc = launch_tc<false, false, true>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      case 6: rc = launch_tc<false, true, true>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      case 7: rc = launch_tc<true, true, true>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      default: rc = GPTB_ERR_UNSUPPORTED;  // e4m3 with A M-major and B K-major: not used
+    }
   }
   if (timed) {
     cudaEventRecord(eb, st);
@@ -229,7 +240,7 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
               void* out2 = nullptr, long long ldo2 = 0) {
   EpiParams e;
   e.kind = kind;
-  e.out_f32 = (kind == EPI_ACCUM_F32 || dtype == GPTB_F32) ? 1 : 0;
+  e.out_f32 = (kind == EPI_ACCUM_F32 || dtype == GPTB_F32) ? 1 : 0;  // FP8 configs store bf16
   e.out = out;
   e.ldo = ldo;
   e.aux = aux;
@@ -237,6 +248,13 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
   e.out2 = out2;
   e.ldo2 = ldo2;
   e.alpha = nullptr;
+  e.amax_a = nullptr;
+  e.amax_b = nullptr;
+  return e;
+}
+EpiParams epi8(EpiParams e, const float* amax_a, const float* amax_b) {
+  e.amax_a = amax_a;
+  e.amax_b = amax_b;
   return e;
 }
 
@@ -256,6 +274,7 @@ struct Carve {
 struct Dims {
   long long N;
   int B, T, d, H, Hkv, hd, F, V, L, Wq, NH, esz;
+  bool fp8;
 };
 Dims dims_of(const gptb_config& c) {
   Dims m;
@@ -272,12 +291,17 @@ Dims dims_of(const gptb_config& c) {
   m.Wq = (c.n_head + 2 * c.n_kv_head) * c.head_dim;
   m.NH = c.n_head + c.n_kv_head;
   m.esz = c.dtype == GPTB_F32 ? 4 : 2;
+  m.fp8 = c.dtype == GPTB_FP8_E4M3;
   return m;
 }
 
 struct Saved {
   void *h, *qkv, *o, *h2, *u, *act;
   float *rstd1, *sg, *rstd_qk, *lse, *rstd2;
+  // FP8 only: e4m3 copies of the four weights (reused by the input-gradient
+  // GEMMs) and the amax of the four GEMM activations and four weights
+  uint8_t *wqkv8, *wo8, *wfc8, *wproj8;
+  float* amax;  // [h, o, h2, act, wqkv, wo, wfc, wproj]
 };
 Saved carve_saved(Carve& cv, const Dims& m) {
   Saved s;
@@ -293,6 +317,16 @@ Saved carve_saved(Carve& cv, const Dims& m) {
   s.rstd2 = (float*)cv.take(m.N * 4);
   s.u = cv.take(m.N * m.F * e);
   s.act = cv.take(m.N * m.F * e);
+  s.wqkv8 = s.wo8 = s.wfc8 = s.wproj8 = nullptr;
+  s.amax = nullptr;
+  if (m.fp8) {
+    const long long Ho = (long long)m.H * m.hd;
+    s.wqkv8 = (uint8_t*)cv.take((size_t)m.Wq * m.d);
+    s.wo8 = (uint8_t*)cv.take((size_t)m.d * Ho);
+    s.wfc8 = (uint8_t*)cv.take((size_t)m.F * m.d);
+    s.wproj8 = (uint8_t*)cv.take((size_t)m.d * m.F);
+    s.amax = (float*)cv.take(8 * 4);
+  }
   return s;
 }
 
@@ -300,9 +334,12 @@ struct Scratch {
   float2* rope;
   // forward
   void *xm, *x1;
+  uint8_t* a8;  // FP8: e4m3 copy of the activation feeding a forward GEMM
   // backward
   void *du, *dh2, *dx1, *dO, *dqkv, *dh;
   float *D, *dq, *dk, *dv, *dz;
+  uint8_t* g8;   // FP8: e4m3 copy of the gradient feeding a GEMM pair
+  float* gamax;  // FP8: its amax
 };
 Scratch carve_scratch(Carve& cv, const Dims& m) {
   Scratch s;
@@ -311,6 +348,11 @@ Scratch carve_scratch(Carve& cv, const Dims& m) {
   const size_t start = cv.off;
   s.xm = cv.take(m.N * m.d * e);
   s.x1 = cv.take(m.N * m.d * e);
+  s.a8 = nullptr;
+  if (m.fp8) {
+    const long long w = std::max<long long>(std::max<long long>(m.d, m.F), (long long)m.H * m.hd);
+    s.a8 = (uint8_t*)cv.take(m.N * w);
+  }
   const size_t fwd_end = cv.off;
   cv.off = start;  // backward temporaries reuse the forward's space
   s.du = cv.take(m.N * m.F * e);
@@ -324,6 +366,13 @@ Scratch carve_scratch(Carve& cv, const Dims& m) {
   s.dk = (float*)cv.take(m.N * (long long)m.Hkv * m.hd * 4);
   s.dv = (float*)cv.take(m.N * (long long)m.Hkv * m.hd * 4);
   s.dz = (float*)cv.take(m.N * m.Hkv * 4);
+  s.g8 = nullptr;
+  s.gamax = nullptr;
+  if (m.fp8) {
+    const long long w = std::max<long long>(std::max<long long>(m.Wq, m.F), std::max<long long>(m.d, (long long)m.H * m.hd));
+    s.g8 = (uint8_t*)cv.take(m.N * w);
+    s.gamax = (float*)cv.take(4);
+  }
   cv.off = std::max(cv.off, fwd_end);
   return s;
 }
@@ -371,7 +420,6 @@ StackWs carve_stack(Carve& cv, const Dims& m) {
 int check_config(const gptb_config* c) {
   if (!c) return GPTB_ERR_INVALID_ARG;
   if (c->dtype != GPTB_F32 && c->dtype != GPTB_BF16 && c->dtype != GPTB_FP8_E4M3) return GPTB_ERR_UNSUPPORTED;
-  if (c->dtype == GPTB_FP8_E4M3) return GPTB_ERR_UNSUPPORTED;
   if (c->B < 1 || c->T < 1 || c->d < 8 || c->d % 8 || c->d > 8 * 32 * EW_MAXC) return GPTB_ERR_INVALID_ARG;
   if (c->n_head < 1 || c->n_kv_head < 1 || c->n_head % c->n_kv_head) return GPTB_ERR_INVALID_ARG;
   if (c->mlp_hidden < 8 || c->mlp_hidden % 8 || c->vocab < 8 || c->vocab % 8) return GPTB_ERR_INVALID_ARG;
@@ -409,6 +457,46 @@ int rope_init(const gptb_config& c, float2* tab, cudaStream_t st) {
   return GPTB_OK;
 }
 
+
+// per-tensor e4m3 quantisation: amax (fp32 bits, atomicMax) then codes
+template <class T>
+int quant(const T* x, long long n, uint8_t* out, float* amax, cudaStream_t st) {
+  CK(cudaMemsetAsync(amax, 0, sizeof(float), st));
+  const long long n8 = n / 8;
+  const int grid = (int)std::max<long long>(1, std::min<long long>((n8 + 255) / 256, (long long)dev_info().sms * 8));
+  amax_kernel<T><<<grid, 256, 0, st>>>(x, n8, reinterpret_cast<unsigned int*>(amax));
+  CKL();
+  quantize_e4m3_kernel<T><<<grid, 256, 0, st>>>(x, n8, amax, out);
+  CKL();
+  return GPTB_OK;
+}
+
+// One GEMM operand: the storage-dtype matrix and, for FP8 configs, its e4m3
+// copy and amax slot (quant = produce the copy now; false = already produced).
+struct Operand {
+  const void* p;
+  long long ld;
+  bool mn;
+  long long elems;
+  uint8_t* q;
+  float* amax;
+  bool quant;
+};
+
+// A projection GEMM of the block in the config's arithmetic: f32 (SIMT) or
+// bf16 (tcgen05) operands as stored, or per-tensor e4m3 operands (FP8).  In
+// FP8 configs an operand without an e4m3 slot (q == nullptr) selects the bf16
+// GEMM: the weight-gradient products keep high-precision operands.
+template <class T>
+int proj(const gptb_config& c, const Operand& A, const Operand& B, int M, int N, int K, const EpiParams& e,
+         cudaStream_t st) {
+  if (c.dtype != GPTB_FP8_E4M3) return gemm(c.dtype, {A.p, A.ld, A.mn}, {B.p, B.ld, B.mn}, M, N, K, e, st);
+  if (!A.q) return gemm(GPTB_BF16, {A.p, A.ld, A.mn}, {B.p, B.ld, B.mn}, M, N, K, e, st);  // high-precision GEMM
+  if (A.quant) TRY(quant<T>((const T*)A.p, A.elems, A.q, A.amax, st));
+  if (B.quant) TRY(quant<T>((const T*)B.p, B.elems, B.q, B.amax, st));
+  return gemm(GPTB_FP8_E4M3, {A.q, A.ld, A.mn}, {B.q, B.ld, B.mn}, M, N, K, epi8(e, A.amax, B.amax), st);
+}
+
 // ------------------------------------------------------ block forward -----
 template <class T>
 int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w, const T* x, const T* x0,
@@ -422,8 +510,10 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   ROWK(nc, mix_norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(x, x0, w.lambdas, (T*)X.xm, (T*)S.h, S.rstd1, m.N, m.d, c.norm_eps,
                                                 ve ? (const T*)w.w_ve_gate : nullptr, S.sg, m.Hkv, c.ve_gate_ch));
   CKL();
-  TRY(gemm(c.dtype, {S.h, m.d, false}, {w.w_qkv, m.d, false}, (int)m.N, m.Wq, m.d,
-           epi(EPI_STORE, c.dtype, S.qkv, m.Wq), st));
+  const long long Ho = (long long)m.H * m.hd;
+  TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, X.a8, S.amax + 0, true},
+              {w.w_qkv, m.d, false, (long long)m.Wq * m.d, S.wqkv8, S.amax + 4, true}, (int)m.N, m.Wq, m.d,
+              epi(EPI_STORE, c.dtype, S.qkv, m.Wq), st));
   qkv_post_kernel<T><<<grid_rows(m.N * (m.NH + (ve ? m.Hkv : 0))), EW_THREADS, 0, st>>>(
       (T*)S.qkv, m.Wq, S.rstd_qk, X.rope, m.T, m.N, m.H, m.Hkv, m.hd, c.norm_eps, ve ? (const T*)w.ve_table : nullptr,
       idx, S.sg);
@@ -434,20 +524,27 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
                                                                  (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, m.hd, W);
     CKL();
   } else {
-    CK(cudaFuncSetAttribute(attn_fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AF_SMEM));
-    attn_fwd_bf16_kernel<<<dim3((m.T + AF_BR - 1) / AF_BR, m.H, m.B), AF_THREADS, AF_SMEM, st>>>(
-        (const bf16*)S.qkv, m.Wq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W);
+    // tcgen05 flash attention: one tensor map (64-column boxes of 128 rows)
+    // over the packed qkv buffer serves the Q, K and V tiles
+    CUtensorMap tq;
+    if (!make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128)) return GPTB_ERR_CUDA;
+    CK(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM));
+    attn_fwd_tc_kernel<<<dim3((m.T + FA_BM - 1) / FA_BM, m.H, m.B), FA_THREADS, FA_SMEM, st>>>(
+        tq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W);
     CKL();
   }
-  TRY(gemm(c.dtype, {S.o, (long long)m.H * m.hd, false}, {w.w_o, (long long)m.H * m.hd, false}, (int)m.N, m.d,
-           m.H * m.hd, epi(EPI_RESID, c.dtype, X.x1, m.d, X.xm, m.d), st));
+  TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, X.a8, S.amax + 1, true},
+              {w.w_o, Ho, false, m.d * Ho, S.wo8, S.amax + 5, true}, (int)m.N, m.d, (int)Ho,
+              epi(EPI_RESID, c.dtype, X.x1, m.d, X.xm, m.d), st));
   ROWK(nc, norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
                                             c.norm_eps));
   CKL();
-  TRY(gemm(c.dtype, {S.h2, m.d, false}, {w.w_fc, m.d, false}, (int)m.N, m.F, m.d,
-           epi(EPI_RELU2, c.dtype, S.u, m.F, nullptr, 0, S.act, m.F), st));
-  TRY(gemm(c.dtype, {S.act, m.F, false}, {w.w_proj, m.F, false}, (int)m.N, m.d, m.F,
-           epi(EPI_RESID, c.dtype, x_out, m.d, X.x1, m.d), st));
+  TRY(proj<T>(c, {S.h2, m.d, false, m.N * m.d, X.a8, S.amax + 2, true},
+              {w.w_fc, m.d, false, (long long)m.F * m.d, S.wfc8, S.amax + 6, true}, (int)m.N, m.F, m.d,
+              epi(EPI_RELU2, c.dtype, S.u, m.F, nullptr, 0, S.act, m.F), st));
+  TRY(proj<T>(c, {S.act, m.F, false, m.N * m.F, X.a8, S.amax + 3, true},
+              {w.w_proj, m.F, false, (long long)m.d * m.F, S.wproj8, S.amax + 7, true}, (int)m.N, m.d, m.F,
+              epi(EPI_RESID, c.dtype, x_out, m.d, X.x1, m.d), st));
   return GPTB_OK;
 }
 
@@ -465,16 +562,25 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   const int N = (int)m.N;
   const long long Ho = (long long)m.H * m.hd, Kv = (long long)m.Hkv * m.hd;
   // MLP
-  TRY(gemm(dt, {dx2, m.d, true}, {S.act, m.F, true}, m.d, m.F, N, epi(EPI_ACCUM_F32, dt, g.w_proj, m.F), st));
-  TRY(gemm(dt, {dx2, m.d, false}, {w.w_proj, m.F, true}, N, m.F, m.d, epi(EPI_DRELU2, dt, X.du, m.F, S.u, m.F), st));
-  TRY(gemm(dt, {X.du, m.F, true}, {S.h2, m.d, true}, m.F, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
-  TRY(gemm(dt, {X.du, m.F, false}, {w.w_fc, m.d, true}, N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
+  // (FP8: the input-gradient GEMMs quantise the gradient and reuse the
+  // forward's e4m3 weights; the weight-gradient GEMMs run on the bf16 tensors)
+  const long long Nd = m.N * m.d;
+  TRY(proj<T>(c, {dx2, m.d, true, Nd, nullptr, nullptr, false}, {S.act, m.F, true, 0, nullptr, nullptr, false}, m.d,
+              m.F, N, epi(EPI_ACCUM_F32, dt, g.w_proj, m.F), st));
+  TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false},
+              N, m.F, m.d, epi(EPI_DRELU2, dt, X.du, m.F, S.u, m.F), st));
+  TRY(proj<T>(c, {X.du, m.F, true, 0, nullptr, nullptr, false}, {S.h2, m.d, true, 0, nullptr, nullptr, false}, m.F,
+              m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
+  TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, X.gamax, true}, {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false},
+              N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
   const int gr = grid_rows(m.N);
   ROWK(nc, norm_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d));
   CKL();
   // attention output projection
-  TRY(gemm(dt, {X.dx1, m.d, true}, {S.o, Ho, true}, m.d, (int)Ho, N, epi(EPI_ACCUM_F32, dt, g.w_o, Ho), st));
-  TRY(gemm(dt, {X.dx1, m.d, false}, {w.w_o, Ho, true}, N, (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
+  TRY(proj<T>(c, {X.dx1, m.d, true, 0, nullptr, nullptr, false}, {S.o, Ho, true, 0, nullptr, nullptr, false}, m.d,
+              (int)Ho, N, epi(EPI_ACCUM_F32, dt, g.w_o, Ho), st));
+  TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+              (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
   // attention
   attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
                                                                      m.B, m.T, m.H, m.hd);
@@ -499,8 +605,10 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
       ve ? (const T*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz);
   CKL();
   // QKV projection
-  TRY(gemm(dt, {X.dqkv, m.Wq, true}, {S.h, m.d, true}, m.Wq, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_qkv, m.d), st));
-  TRY(gemm(dt, {X.dqkv, m.Wq, false}, {w.w_qkv, m.d, true}, N, m.d, m.Wq, epi(EPI_STORE, dt, X.dh, m.d), st));
+  TRY(proj<T>(c, {X.dqkv, m.Wq, true, 0, nullptr, nullptr, false}, {S.h, m.d, true, 0, nullptr, nullptr, false},
+              m.Wq, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_qkv, m.d), st));
+  TRY(proj<T>(c, {X.dqkv, m.Wq, false, m.N * m.Wq, X.g8, X.gamax, true},
+              {w.w_qkv, m.d, true, 0, S.wqkv8, S.amax + 4, false}, N, m.d, m.Wq, epi(EPI_STORE, dt, X.dh, m.d), st));
   if (ve) {
     const int nthreads = ((m.Hkv * c.ve_gate_ch + 31) / 32) * 32;
     if (nthreads > 1024) return GPTB_ERR_UNSUPPORTED;
@@ -522,7 +630,7 @@ int lm_head_impl(const gptb_config& c, const T* h, const T* w_lm, const int32_t*
                  float* dw_lm, const LmWs& lw, cudaStream_t st) {
   const Dims m = dims_of(c);
   const int nc = (m.d + 255) / 256;
-  const int dt = c.dtype;
+  const int dt = c.dtype == GPTB_FP8_E4M3 ? GPTB_BF16 : c.dtype;  // lm_head stays bf16
   for (long long c0 = 0; c0 < m.N; c0 += lw.chunk) {
     const int rows = (int)std::min<long long>(lw.chunk, m.N - c0);
     const T* hc = h + c0 * m.d;

@@ -51,10 +51,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 // smem tile of R rows x 128 bf16 (256 B per row); 16-byte chunk c of row r
 // lives at chunk c ^ (r & 7) so that ldmatrix row groups hit distinct banks
@@ -74,8 +70,6 @@ __device__ __forceinline__ void load_tile128(uint32_t sbase, const bf16* g, long
   }
 }
 
-constexpr float LOG2E = 1.4426950408889634f;
-constexpr float LN2 = 0.6931471805599453f;
 
 // ------------------------------------------------------ forward (bf16) ----
 constexpr int AF_BR = 128, AF_BC = 64, AF_THREADS = 256;

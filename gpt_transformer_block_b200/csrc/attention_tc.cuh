@@ -1,0 +1,313 @@
+// Attention forward on the 5th-generation tensor cores (tcgen05 + TMEM), bf16,
+// hd = 128.  Same math as attention.cuh (causal GQA, sliding window, LSE).
+//
+// CTA = 128 queries of one head; 10 warps:
+//   warp 0    TMA producer: Q once, then K and V tiles of 128 keys into two
+//             2-stage rings (a K slot is refilled once its S MMA is done, a V
+//             slot once its PV MMA is done; all loads are 64-column boxes of
+//             the packed qkv buffer, 128-byte swizzle)
+//   warp 1    TMEM owner + single-thread MMA issuer:
+//               S_j = Q K_j^T   (M=128, N=128, K=128) into one of two TMEM
+//                               score buffers (columns 0..127 / 128..255)
+//               O  += P_j V_j   (M=128, N=128, K=128; V as MN-major operand)
+//                               into TMEM columns 256..383
+//             S_{j+1} is issued before O += P_j V_j so the scores of the next
+//             tile are ready when the softmax finishes the current one.
+//   warps 2-9 softmax: two warps per TMEM lane quarter; thread = one query
+//             row (its TMEM lane) and one half (64 keys) of the score tile.
+//             Masks (causal / window / sequence end), combines the two halves'
+//             row max through shared memory, keeps a running max in base 2 and
+//             rescales O in TMEM only when the max grows by more than 8 (a
+//             factor 256; P stays below 256 in bf16 and the final
+//             normalisation uses the same max, so the result is exact), writes
+//             P (bf16) into a swizzled smem tile for the PV MMA, and at the end
+//             normalises its half of O and writes o and the LSE.
+// Only key tiles that intersect [q0 - W, q0 + 127] are visited.
+#pragma once
+#include "common.cuh"
+
+namespace gptb {
+
+constexpr int FA_BM = 128, FA_BN = 128;
+constexpr int FA_THREADS = 320;
+constexpr int FA_SOFTMAX_THREADS = 256;
+constexpr int FA_TILE = 128 * 128 * 2;  // one 128x128 bf16 tile: 32 KB (two 64-column swizzled halves)
+constexpr int FA_SMEM = 1024 /*align*/ + FA_TILE /*Q*/ + 4 * FA_TILE /*K,V x2*/ + FA_TILE /*P*/ + 256 /*barriers*/ +
+                        2 * 2 * 128 * 4 /*row max exchange, 2 tiles in flight*/ + 2 * 128 * 4 /*row sums*/;
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// K-major SW128 descriptor of a 128-row tile, k-th 16-element K step
+__device__ __forceinline__ uint64_t fa_desc_k(uint32_t tile, int k) {
+  return smem_desc_sw128(tile + (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), 16, 1024);
+}
+// MN-major SW128 descriptor (two 64-wide MN halves 16 KB apart), k-th 16-row K step
+__device__ __forceinline__ uint64_t fa_desc_mn(uint32_t tile, int k) {
+  return smem_desc_sw128(tile + (uint32_t)(k * 2048), 16384, 1024);
+}
+
+__global__ void __launch_bounds__(FA_THREADS, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ o, long long ldo,
+                       float* __restrict__ lse, int T, int H, int Hkv, int window) {
+  extern __shared__ uint8_t fa_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + FA_TILE;          // 2 stages
+  uint8_t* sV = sK + 2 * FA_TILE;      // 2 stages
+  uint8_t* sP = sV + 2 * FA_TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + FA_TILE);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]  K ring: a slot is free once S_j = Q K_j^T is done
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_empty = bars + 7;   // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint64_t* v_full = bars + 12;   // [2]  V ring: a slot is free once O += P_j V_j is done
+  uint64_t* v_empty = bars + 14;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xmax = reinterpret_cast<float*>(bars + 32);  // [2 tile parities][2 halves][128 rows] (after 256 B of barriers)
+  float* xsum = xmax + 2 * 2 * 128;                   // [2 halves][128 rows]
+
+  const int nqb = (T + FA_BM - 1) / FA_BM;
+  const int qb = nqb - 1 - (int)blockIdx.x;  // heavy (late) query tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (H / Hkv);
+  const int q0 = qb * FA_BM;
+  const int kb_lo = (window >= 0) ? max(0, q0 - window) / FA_BN : 0;
+  const int kb_hi = min(T - 1, q0 + FA_BM - 1) / FA_BN;
+  const int ntiles = kb_hi - kb_lo + 1;
+  const int row_base = b * T;  // row of token (b, 0) in the packed [B*T, Wq] buffer
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 8);
+    }
+    mbar_init(p_full, 8);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, FA_TILE);
+      tma_load_2d(sQ, &tm_qkv, q_full, h * 128, row_base + q0);
+      tma_load_2d(sQ + 16384, &tm_qkv, q_full, h * 128 + 64, row_base + q0);
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = j & 1;
+        const uint32_t par = ((j >> 1) & 1) ^ 1u;
+        const int kr = row_base + (kb_lo + j) * FA_BN;
+        if (!mbar_wait(&k_empty[st], par, abort_flag, ERRW_TIMEOUT_PRODUCER)) break;
+        mbar_arrive_expect_tx(&k_full[st], FA_TILE);
+        uint8_t* k = sK + st * FA_TILE;
+        tma_load_2d(k, &tm_qkv, &k_full[st], (H + kvh) * 128, kr);
+        tma_load_2d(k + 16384, &tm_qkv, &k_full[st], (H + kvh) * 128 + 64, kr);
+        if (!mbar_wait(&v_empty[st], par, abort_flag, ERRW_TIMEOUT_PRODUCER)) break;
+        mbar_arrive_expect_tx(&v_full[st], FA_TILE);
+        uint8_t* v = sV + st * FA_TILE;
+        tma_load_2d(v, &tm_qkv, &v_full[st], (H + Hkv + kvh) * 128, kr);
+        tma_load_2d(v + 16384, &tm_qkv, &v_full[st], (H + Hkv + kvh) * 128 + 64, kr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = make_idesc(128, 128, false, false, false);
+      constexpr uint32_t IDESC_O = make_idesc(128, 128, false, true, false);
+      const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP);
+      bool ok = mbar_wait(q_full, 0, abort_flag, ERRW_TIMEOUT_MMA);
+      auto issue_pv = [&](int i) -> bool {
+        if (!mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
+        if (!mbar_wait(p_full, i & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t aV = smem_u32(sV + (i & 1) * FA_TILE);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mma_bf16_ss(tmem + 256, fa_desc_k(aP, k), fa_desc_mn(aV, k), IDESC_O, (i > 0 || k > 0) ? 1u : 0u);
+        mma_commit(pv_done);
+        mma_commit(&v_empty[i & 1]);
+        return true;
+      };
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int sb = j & 1;
+        if (!mbar_wait(&k_full[sb], (j >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
+        if (!mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aK = smem_u32(sK + sb * FA_TILE);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mma_bf16_ss(tmem + sb * 128, fa_desc_k(aQ, k), fa_desc_k(aK, k), IDESC_S, k > 0 ? 1u : 0u);
+        mma_commit(&s_full[sb]);
+        mma_commit(&k_empty[sb]);
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = issue_pv(ntiles - 1);
+      if (*abort_flag) {
+        mma_commit(drain);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0))
+          if (globaltimer_ns() - t0 > 100000000ull) { record_error(ERRW_TIMEOUT_DRAIN); break; }
+      }
+    }
+  } else {
+    // softmax warps: TMEM lane quarter qw = warp % 4 -> query rows 32*qw ..
+    // 32*qw+31; half hf -> score / output columns 64*hf .. 64*hf+63
+    const int qw = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    const int r = qw * 32 + lane;  // row within the tile
+    const int t = q0 + r;          // query position
+    const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
+    const float sl2 = LOG2E / sqrtf(128.f);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    // Every softmax warp runs every iteration and passes every named barrier,
+    // also after a failed (timed-out) wait: then it only skips the work, so no
+    // warp can be left waiting at a barrier that another warp never reaches.
+    for (int j = 0; j < ntiles; ++j) {
+      const int sb = j & 1;
+      const int k0 = (kb_lo + j) * FA_BN + hf * 64;  // first key of this half
+      ok = ok && mbar_wait_warp(&s_full[sb], (j >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+      tc_fence_after();
+      const bool need_mask = (k0 + 63 > q0) || (k0 + 64 > T) || (window >= 0 && q0 + FA_BM - 1 - k0 > window);
+      // pass 1: max of this half of the row (masked), 4 independent partials
+      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64 + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int jk = k0 + c * 32 + i;
+            const bool vis = !need_mask || ((jk <= t) && (jk < T) && (window < 0 || t - jk <= window));
+            mp[i & 3] = vis ? fmaxf(mp[i & 3], __uint_as_float(v[i])) : mp[i & 3];
+          }
+        }
+      }
+      float* xm = xmax + sb * 256;
+      xm[hf * 128 + r] = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+      named_bar_sync(1, FA_SOFTMAX_THREADS);
+      const float mx = fmaxf(xm[r], xm[128 + r]) * sl2;
+      // the previous PV product must be done before P is overwritten or O rescaled
+      if (j > 0) ok = ok && mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+      if (!ok) continue;
+      // rescale decision is per row (identical in both halves) but the TMEM
+      // accesses are warp-collective: the whole warp enters, rows that keep
+      // their max use a factor of 1
+      const bool grow = mx > m_used + 8.f;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float corr = grow ? fast_exp2(m_used - mx) : 1.f;  // 0 when m_used is -inf
+        if (j > 0) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(lane_addr + 256 + hf * 64 + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * corr);
+            tmem_st_32x32b_x32(lane_addr + 256 + hf * 64 + c * 32, v);
+          }
+          tmem_st_wait();
+        }
+        if (grow) {
+          l *= corr;
+          m_used = mx;
+        }
+      }
+      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+      // pass 2: P = exp2(s*scale - m) (bf16) into K-block hf of the K-major
+      // swizzled P tile; 16-byte chunk cc of row r sits at cc ^ (r & 7)
+      uint8_t* prow = sP + hf * 16384 + r * 128;
+      float lp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64 + c * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int i = g * 8 + e;
+            const int jk = k0 + c * 32 + i;
+            const bool vis = !need_mask || ((jk <= t) && (jk < T) && (window < 0 || t - jk <= window));
+            p[e] = vis ? fast_exp2(fmaf(__uint_as_float(v[i]), sl2, -mu)) : 0.f;
+            lp[e & 3] += p[e];
+          }
+          const int cc = c * 4 + g;  // 0..7
+          uint4 u;
+          u.x = pack_bf16(p[0], p[1]);
+          u.y = pack_bf16(p[2], p[3]);
+          u.z = pack_bf16(p[4], p[5]);
+          u.w = pack_bf16(p[6], p[7]);
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = u;
+        }
+      }
+      l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+      // scores consumed; P visible to the tensor core
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_empty[sb]);
+        mbar_arrive(p_full);
+      }
+    }
+    // the two halves' sums share the same running max: add them
+    xsum[hf * 128 + r] = l;
+    named_bar_sync(1, FA_SOFTMAX_THREADS);
+    const float lt = xsum[r] + xsum[128 + r];
+    if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(pv_done, (ntiles - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
+      tc_fence_after();
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      bf16* orow = o + ((long long)b * T + t) * ldo + h * 128 + hf * 64;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(lane_addr + 256 + hf * 64 + c * 32, v);
+        tmem_ld_wait();
+        if (t < T) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint4 u;
+            u.x = pack_bf16(__uint_as_float(v[g * 8 + 0]) * inv, __uint_as_float(v[g * 8 + 1]) * inv);
+            u.y = pack_bf16(__uint_as_float(v[g * 8 + 2]) * inv, __uint_as_float(v[g * 8 + 3]) * inv);
+            u.z = pack_bf16(__uint_as_float(v[g * 8 + 4]) * inv, __uint_as_float(v[g * 8 + 5]) * inv);
+            u.w = pack_bf16(__uint_as_float(v[g * 8 + 6]) * inv, __uint_as_float(v[g * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = u;
+          }
+        }
+      }
+      if (t < T && hf == 0) lse[((long long)b * H + h) * T + t] = (m_used + log2f(lt)) * LN2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace gptb

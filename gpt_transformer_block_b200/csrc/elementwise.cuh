@@ -626,3 +626,50 @@ __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ x,
 }
 
 }  // namespace gptb
+
+namespace gptb {
+
+// ------------------------------------------------- FP8 (e4m3) per tensor --
+// Per-tensor dynamic scaling: s = 448 / max|x|; codes = RNE-satfinite(x * s).
+// amax is kept as float bits so that atomicMax on the unsigned pattern orders
+// non-negative floats correctly.
+template <class T>
+__global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, long long n8, unsigned int* __restrict__ amax) {
+  __shared__ float sred[8];
+  float m = 0.f;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    float v[8];
+    load8(x + i * 8, v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) sred[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, sred[w]);
+    atomicMax(amax, __float_as_uint(m));
+  }
+}
+
+__device__ __forceinline__ float fp8_inv_scale(const float* amax) { return fmaxf(*amax, 1e-12f) / 448.f; }
+
+template <class T>
+__global__ void __launch_bounds__(256)
+    quantize_e4m3_kernel(const T* __restrict__ x, long long n8, const float* __restrict__ amax, uint8_t* __restrict__ out) {
+  const float s = 448.f / fmaxf(*amax, 1e-12f);
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    float v[8];
+    load8(x + i * 8, v);
+    uint2 o;
+    __nv_fp8x2_storage_t p[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      p[k] = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * k] * s, v[2 * k + 1] * s), __NV_SATFINITE, __NV_E4M3);
+    o.x = (uint32_t)p[0] | ((uint32_t)p[1] << 16);
+    o.y = (uint32_t)p[2] | ((uint32_t)p[3] << 16);
+    *reinterpret_cast<uint2*>(out + i * 8) = o;
+  }
+}
+
+}  // namespace gptb

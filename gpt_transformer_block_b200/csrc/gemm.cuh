@@ -42,7 +42,17 @@ struct EpiParams {
   void* out2;
   long long ldo2;
   const float* alpha;  // device scalar or nullptr (= 1)
+  // e4m3 operands: per-tensor amax of A and B; the product is rescaled by
+  // (amax_a / 448) * (amax_b / 448), the inverse of the two quantisation scales
+  const float* amax_a;
+  const float* amax_b;
 };
+
+__device__ __forceinline__ float epi_alpha(const EpiParams& ep) {
+  float a = ep.alpha ? *ep.alpha : 1.f;
+  if (ep.amax_a) a *= (fmaxf(*ep.amax_a, 1e-12f) / 448.f) * (fmaxf(*ep.amax_b, 1e-12f) / 448.f);
+  return a;
+}
 
 // ---------------------------------------------------------------- epilogue
 template <class T>
@@ -158,7 +168,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* empty = full + TC_STAGES;
   uint64_t* tfull = empty + TC_STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,6 +187,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -191,6 +203,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // stages with a load in flight, and the phase they complete
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         int tm, tn, split;
@@ -202,6 +215,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], STAGE_TX);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           uint8_t* a = sA + stage * A_BYTES;
           uint8_t* b = sB + stage * B_BYTES;
           const int k0 = kb * BK;
@@ -223,12 +238,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
       }
-      // drain: wait (bounded) until the MMA side consumed every stage we filled
+      // after an abort, wait (bounded) for the loads this thread issued to land
+      // before the CTA exits; a consumed stage's phase has already completed
       if (!ok) {
-        for (int s = 0; s < TC_STAGES; ++s) {
-          uint64_t* bar = &full[s];
+        for (int s2 = 0; s2 < TC_STAGES; ++s2) {
+          if (!(armed & (1u << s2))) continue;
+          const uint32_t par = (armed_par >> s2) & 1u;
           const unsigned long long t0 = globaltimer_ns();
-          while (!mbar_try_wait(bar, phase) && !mbar_try_wait(bar, phase ^ 1u)) {
+          while (!mbar_try_wait(&full[s2], par)) {
             if (globaltimer_ns() - t0 > 100000000ull) {
               record_error(ERRW_TIMEOUT_DRAIN);
               break;
@@ -281,16 +298,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
+      if (*abort_flag) {
+        // let every MMA this thread issued finish before TMEM is released
+        mma_commit(drain);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0)) {
+          if (globaltimer_ns() - t0 > 100000000ull) {
+            record_error(ERRW_TIMEOUT_DRAIN);
+            break;
+          }
+        }
+      }
     }
   } else {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    const float alpha = ep.alpha ? *ep.alpha : 1.f;
+    const float alpha = epi_alpha(ep);
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       int tm, tn, split;
       tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
+      if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
       const long long row = (long long)tm * TC_BM + q * 32 + lane;
 #pragma unroll 1
@@ -360,7 +388,7 @@ __global__ void __launch_bounds__(256) gemm_simt_f32_kernel(const float* __restr
     }
     __syncthreads();
   }
-  const float alpha = ep.alpha ? *ep.alpha : 1.f;
+  const float alpha = epi_alpha(ep);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll

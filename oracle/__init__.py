@@ -36,7 +36,8 @@ reads the first 32 channels of the normed block input; smear adds the previous
 token's embedding, gated from the current token's first 24 channels; backout
 subtracts the residual entering layer L/2 after the last layer; the loss is the
 mean next-token cross-entropy over all B*T positions; FP8 quantises each GEMM
-operand per tensor with scale 448/amax, round-to-nearest-even, saturating.
+operand of the forward and input-gradient GEMMs per tensor with scale
+448/amax, round-to-nearest-even, saturating (weight-gradient GEMMs exact).
 
 Parity status: every function here is pinned by the "not gpu" tests in
 tests/test_oracle_*.py (finite differences, closed forms, invariants, and

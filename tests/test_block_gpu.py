@@ -40,8 +40,9 @@ def check_block(gb, c, layer, seed=1, x_std=1.0, exact_keys=()):
     inp = synth.make_block_inputs(c, seed=seed + 1, x_std=x_std)
     x_out, dx, dx0, g = run_block(gb, c, w, inp, layer)
     lw = oracle_layer(w, layer)
-    y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), inp["idx"].numpy(), layer)
-    rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), inp["idx"].numpy(), layer)
+    f8 = c["dtype"] == "fp8"
+    y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), inp["idx"].numpy(), layer, fp8=f8)
+    rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), inp["idx"].numpy(), layer, fp8=f8)
     tol = TOL[c["dtype"]]
     errs = {"x_out": relerr(np64(x_out), y), "dx": relerr(np64(dx), rdx), "dx0": relerr(np64(dx0), rdx0)}
     for k in ("w_qkv", "w_o", "w_fc", "w_proj", "w_ve_gate", "ve_table"):
@@ -78,3 +79,11 @@ def test_block_fp32_all_terms(cuda_lib):
     # same block with every term on: value embedding, random lambdas
     c = synth.config("block_fp32", has_ve=[1])
     check_block(cuda_lib, c, 0)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_block_fp8(cuda_lib, layer):
+    # e4m3 operands with per-tensor scales on the four block GEMMs (fwd, dgrad,
+    # wgrad); the oracle quantises the same operands the same way
+    c = small_bf16(dtype="fp8", n_layer=2, window=[-1, 48], has_ve=[0, 1])
+    check_block(cuda_lib, c, layer)

@@ -41,10 +41,11 @@ def run_stack(gb, c, w, batch):
     return loss.item(), st.g
 
 
-def compare_stack(c, w, batch, loss, g):
+def compare_stack(c, w, batch, loss, g, layers=None):
     ow = oracle_weights(w)
-    rl, cache = om.stack_forward(c, ow, batch["idx"].numpy(), batch["targets"].numpy())
-    rg = om.stack_backward(c, ow, cache, batch["idx"].numpy())
+    f8 = c["dtype"] == "fp8"
+    rl, cache = om.stack_forward(c, ow, batch["idx"].numpy(), batch["targets"].numpy(), fp8=f8)
+    rg = om.stack_backward(c, ow, cache, batch["idx"].numpy(), fp8=f8)
     tol = TOL[c["dtype"]]
     errs = {"loss": abs(loss - rl) / abs(rl)}
     for k in ("wte", "w_lm", "w_smear_gate"):
@@ -54,6 +55,8 @@ def compare_stack(c, w, batch, loss, g):
         if k in rg:
             errs[k] = scalar_err(np64(g[k])[0], rg[k], rg["_scale"][k])
     for i, lg in enumerate(rg["layers"]):
+        if layers is not None and i not in layers:
+            continue
         lam = np64(g["layers"][i]["lambdas"])
         for k, v in lg.items():
             if k == "_scale":
@@ -108,3 +111,16 @@ def test_grad_accumulation_equals_sum(cuda_lib):
     torch.cuda.synchronize()
     two = st.g["layers"][1]["w_qkv"]
     assert relerr(two.cpu().numpy(), 2 * one.cpu().numpy()) < 1e-5
+
+
+def test_stack_fp8_small(cuda_lib):
+    """FP8 end to end: loss, lm_head / embedding / smear / backout gradients and
+    the top layer.  Below the top layer every input-gradient GEMM re-quantises a
+    gradient that already differs from the oracle's, so e4m3 code flips (one ulp
+    = 12.5 %) compound layer by layer; the deeper layers are checked with the
+    same tolerance by the teacher-forced block tests (test_block_fp8)."""
+    c = small_bf16(dtype="fp8")
+    w = synth.make_weights(c, seed=51)
+    b = synth.make_batch(c, seed=52)
+    loss, g = run_stack(cuda_lib, c, w, b)
+    compare_stack(c, w, b, loss, g, layers=(c["n_layer"] - 1,))
