@@ -130,6 +130,21 @@ bool make_tmap(CUtensorMap* m, const void* ptr, bool fp8, uint64_t inner, uint64
   return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor map without swizzle (TMA bulk reduce-add target)
+bool make_tmap_f32_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                         uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // --------------------------------------------------------------- GEMM ----
@@ -595,9 +610,17 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
                                                                  W);
     CKL();
   } else {
-    CK(cudaFuncSetAttribute(attn_bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AB_SMEM));
-    attn_bwd_bf16_kernel<<<dim3((m.T + AB_BC - 1) / AB_BC, m.Hkv, m.B), AB_THREADS, AB_SMEM, st>>>(
-        (const bf16*)S.qkv, m.Wq, (const bf16*)X.dO, Ho, S.lse, X.D, X.dq, Ho, X.dk, X.dv, Kv, m.T, m.H, m.Hkv, W);
+    // tcgen05 flash backward: K/V tiles (128 rows) and Q/dO tiles (64 rows) by
+    // TMA, dQ accumulated with TMA bulk reduce-add into the fp32 buffer
+    CUtensorMap tkv, tq, tdo, tdq;
+    bool okm = make_tmap(&tkv, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128);
+    okm = okm && make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 64);
+    okm = okm && make_tmap(&tdo, X.dO, false, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 64, 64);
+    okm = okm && make_tmap_f32_plain(&tdq, X.dq, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 128, 64);
+    if (!okm) return GPTB_ERR_CUDA;
+    CK(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AB2_SMEM));
+    attn_bwd_tc_kernel<<<dim3((m.T + AB2_BK - 1) / AB2_BK, m.Hkv, m.B), AB2_THREADS, AB2_SMEM, st>>>(
+        tkv, tq, tdo, tdq, S.lse, X.D, X.dk, X.dv, Kv, m.T, m.H, m.Hkv, W);
     CKL();
   }
   qkv_post_bwd_kernel<T><<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(

@@ -311,3 +311,323 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 }
 
 }  // namespace gptb
+
+namespace gptb {
+
+// ---------------------------------------------- backward (bf16, tcgen05) ---
+// CTA = 128 keys of one kv head; loops over the G query heads of the group
+// and over the 64-query tiles that can see its keys (causal + window).
+// Per step (one query head, one 64-query tile), on the tensor core:
+//   S^T  = K Q^T      (M=128 keys, N=64, K=128)      -> TMEM cols 256..319
+//   dP^T = V dO^T     (M=128 keys, N=64, K=128)      -> TMEM cols 320..383
+//   dV  += P^T dO     (M=128, N=128, K=64 queries)   -> TMEM cols 128..255
+//   dK  += dS^T Q     (M=128, N=128, K=64)           -> TMEM cols   0..127
+//   dQ^T = K^T dS^T   (M=128 hd, N=64, K=128 keys)   -> TMEM cols 384..447
+// Warps: 0 TMA producer (K, V once; Q, dO, LSE, D per step in a 2-stage
+// ring), 1 MMA issuer, 2-9 softmax backward (thread = key row, 32 of the 64
+// queries): P^T = exp2(S^T*scale*log2e - LSE*log2e), dS^T = P^T (dP^T - D)/sqrt(hd)
+// written as bf16 into swizzled smem tiles that are both the K-major A
+// operand of dV/dK and the MN-major B operand of dQ^T; 10-13 dQ epilogue:
+// thread = hd lane, dQ^T row -> smem [64 q][128 hd] fp32 -> one TMA bulk
+// reduce-add into the fp32 dQ accumulator (no per-element atomics).
+// At the end the softmax warps write dK, dV (fp32) for the CTA's keys.
+constexpr int AB2_BK = 128, AB2_BQ = 64;
+constexpr int AB2_THREADS = 448;
+constexpr int AB2_KV_TILE = 128 * 128 * 2;  // 32 KB
+constexpr int AB2_Q_TILE = 64 * 128 * 2;    // 16 KB
+constexpr int AB2_PS_TILE = 128 * 64 * 2;   // 16 KB
+constexpr int AB2_DQ_STAGE = 64 * 128 * 4;  // 32 KB
+constexpr int AB2_SMEM = 1024 + 2 * AB2_KV_TILE + 4 * AB2_Q_TILE + 2 * AB2_PS_TILE + AB2_DQ_STAGE + 256 + 2 * 2 * 64 * 4;
+
+__global__ void __launch_bounds__(AB2_THREADS, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dq,
+                       const float* __restrict__ lse, const float* __restrict__ Dd, float* __restrict__ dk_out,
+                       float* __restrict__ dv_out, long long lddkv, int T, int H, int Hkv, int window) {
+  extern __shared__ uint8_t ab_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ab_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + AB2_KV_TILE;
+  uint8_t* sQ = sV + AB2_KV_TILE;        // 2 stages
+  uint8_t* sDO = sQ + 2 * AB2_Q_TILE;    // 2 stages
+  uint8_t* sP = sDO + 2 * AB2_Q_TILE;
+  uint8_t* sDS = sP + AB2_PS_TILE;
+  float* sDQ = reinterpret_cast<float*>(sDS + AB2_PS_TILE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sDQ) + AB2_DQ_STAGE);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* qdo_full = bars + 1;   // [2]
+  uint64_t* qdo_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_empty = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* ds_free = bars + 8;
+  uint64_t* dq_full = bars + 9;
+  uint64_t* dq_free = bars + 10;
+  uint64_t* acc_done = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sLD = reinterpret_cast<float*>(bars + 32);  // [2 stages][lse*log2e 64 | D 64]
+
+  const int kb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int G = H / Hkv;
+  const int k0 = kb * AB2_BK;
+  const int row_base = b * T;
+  const int qt_lo = k0 / AB2_BQ;
+  const int q_hi = (window >= 0) ? min(T - 1, k0 + AB2_BK - 1 + window) : T - 1;
+  const int nq = q_hi / AB2_BQ - qt_lo + 1;
+  const int steps = G * nq;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qdo_full[i], 1);
+      mbar_init(&qdo_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 8);
+    mbar_init(p_full, 8);
+    mbar_init(ds_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 4);
+    mbar_init(acc_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_kv);
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * AB2_KV_TILE);
+      tma_load_2d(sK, &tm_kv, kv_full, (H + kvh) * 128, row_base + k0);
+      tma_load_2d(sK + 16384, &tm_kv, kv_full, (H + kvh) * 128 + 64, row_base + k0);
+      tma_load_2d(sV, &tm_kv, kv_full, (H + Hkv + kvh) * 128, row_base + k0);
+      tma_load_2d(sV + 16384, &tm_kv, kv_full, (H + Hkv + kvh) * 128 + 64, row_base + k0);
+    }
+    bool ok = true;
+    for (int i = 0; i < steps && ok; ++i) {
+      const int st = i & 1;
+      const int hh = kvh * G + i / nq;
+      const int q0 = (qt_lo + i % nq) * AB2_BQ;
+      ok = mbar_wait_warp(&qdo_empty[st], ((i >> 1) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_PRODUCER);
+      if (!ok) break;
+      float* ld = sLD + st * 128;
+      for (int e = lane; e < 64; e += 32) {
+        const int t = q0 + e;
+        const long long li = ((long long)b * H + hh) * T + t;
+        ld[e] = (t < T) ? lse[li] * LOG2E : 0.f;
+        ld[64 + e] = (t < T) ? Dd[li] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&qdo_full[st], 2 * AB2_Q_TILE);
+        uint8_t* q = sQ + st * AB2_Q_TILE;
+        uint8_t* d = sDO + st * AB2_Q_TILE;
+        tma_load_2d(q, &tm_q, &qdo_full[st], hh * 128, row_base + q0);
+        tma_load_2d(q + 8192, &tm_q, &qdo_full[st], hh * 128 + 64, row_base + q0);
+        tma_load_2d(d, &tm_do, &qdo_full[st], hh * 128, row_base + q0);
+        tma_load_2d(d + 8192, &tm_do, &qdo_full[st], hh * 128 + 64, row_base + q0);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_S = make_idesc(128, 64, false, false, false);   // S^T, dP^T
+      constexpr uint32_t ID_G = make_idesc(128, 128, false, true, false);   // dV, dK
+      constexpr uint32_t ID_Q = make_idesc(128, 64, true, true, false);     // dQ^T
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP), aDS = smem_u32(sDS);
+      bool ok = mbar_wait(kv_full, 0, abort_flag, ERRW_TIMEOUT_MMA);
+      auto grads = [&](int i) -> bool {
+        const int st = i & 1;
+        if (!mbar_wait(p_full, i & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t aQ = smem_u32(sQ + st * AB2_Q_TILE), aDO = smem_u32(sDO + st * AB2_Q_TILE);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
+          // A: P^T / dS^T tile (128 key rows x 64 queries, K-major, one 128-byte K block)
+          // B: dO / Q as MN-major (hd halves 8 KB apart), K step = 16 query rows
+          mma_bf16_ss(tmem + 128, smem_desc_sw128(aP + k * 32, 16, 1024), smem_desc_sw128(aDO + k * 2048, 8192, 1024),
+                      ID_G, acc);
+          mma_bf16_ss(tmem + 0, smem_desc_sw128(aDS + k * 32, 16, 1024), smem_desc_sw128(aQ + k * 2048, 8192, 1024),
+                      ID_G, acc);
+        }
+        if (!mbar_wait(dq_free, (i & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          // A = K^T (MN-major over hd, halves 16 KB apart), B = dS (MN-major over queries), K step = 16 keys
+          mma_bf16_ss(tmem + 384, smem_desc_sw128(aK + k * 2048, 16384, 1024),
+                      smem_desc_sw128(aDS + k * 2048, 8192, 1024), ID_Q, k > 0 ? 1u : 0u);
+        }
+        mma_commit(ds_free);
+        mma_commit(&qdo_empty[st]);
+        mma_commit(dq_full);
+        return true;
+      };
+      for (int i = 0; ok && i < steps; ++i) {
+        const int st = i & 1;
+        if (!mbar_wait(&qdo_full[st], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
+        if (!mbar_wait(s_empty, (i & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aQ = smem_u32(sQ + st * AB2_Q_TILE), aDO = smem_u32(sDO + st * AB2_Q_TILE);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          // K-major over hd: A rows = keys (halves 16 KB apart), B rows = queries (halves 8 KB apart)
+          const uint32_t ka = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), kq = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
+          mma_bf16_ss(tmem + 256, smem_desc_sw128(aK + ka, 16, 1024), smem_desc_sw128(aQ + kq, 16, 1024), ID_S, k > 0);
+          mma_bf16_ss(tmem + 320, smem_desc_sw128(aV + ka, 16, 1024), smem_desc_sw128(aDO + kq, 16, 1024), ID_S, k > 0);
+        }
+        mma_commit(s_full);
+        if (i > 0 && !grads(i - 1)) { ok = false; break; }
+      }
+      if (ok && steps > 0) ok = grads(steps - 1);
+      mma_commit(acc_done);
+      if (*abort_flag) {
+        mma_commit(drain);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0))
+          if (globaltimer_ns() - t0 > 100000000ull) { record_error(ERRW_TIMEOUT_DRAIN); break; }
+      }
+    }
+  } else if (warp < 10) {
+    // ---------------------------------------------------- softmax backward
+    const int qw = warp & 3;
+    const int cb = (warp - 2) >> 2;          // queries cb*32 .. cb*32+31 of the tile
+    const int r = qw * 32 + lane;            // key row within the tile
+    const int key = k0 + r;
+    const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
+    const float scale = rsqrtf(128.f);
+    const float sl2 = LOG2E * scale;
+    bool ok = true;
+    for (int i = 0; i < steps && ok; ++i) {
+      const int st = i & 1;
+      const int q0 = (qt_lo + i % nq) * AB2_BQ;
+      ok = mbar_wait_warp(s_full, i & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[32], dv[32];
+      tmem_ld_32x32b_x32(lane_addr + 256 + cb * 32, sv);
+      tmem_ld_32x32b_x32(lane_addr + 320 + cb * 32, dv);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty);
+      const float* l2 = sLD + st * 128 + cb * 32;
+      const float* Dq = sLD + st * 128 + 64 + cb * 32;
+      const int tq = q0 + cb * 32;  // first query of this warp's columns
+      const bool need_mask = (key > tq) || (k0 + AB2_BK - 1 > tq) || (tq + 32 > T) || (k0 + AB2_BK > T) ||
+                             (window >= 0 && tq + 31 - k0 > window);
+      // the previous step's dV/dK/dQ MMAs must be done reading P^T / dS^T
+      if (i > 0) {
+        ok = mbar_wait_warp(ds_free, (i - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+        if (!ok) break;
+      }
+      uint8_t* prow = sP + r * 128;
+      uint8_t* drow = sDS + r * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pu[4], du[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          float pe[2], de[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = c * 8 + e2 * 2 + h2;
+            const int t = tq + e;
+            const bool vis = !need_mask || ((key <= t) && (t < T) && (key < T) && (window < 0 || t - key <= window));
+            pe[h2] = vis ? fast_exp2(fmaf(__uint_as_float(sv[e]), sl2, -l2[e])) : 0.f;
+            de[h2] = pe[h2] * (__uint_as_float(dv[e]) - Dq[e]) * scale;
+          }
+          pu[e2] = pack_bf16(pe[0], pe[1]);
+          du[e2] = pack_bf16(de[0], de[1]);
+        }
+        const int cc = cb * 4 + c;  // 16-byte chunk (8 queries) within the 128-byte row
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+        *reinterpret_cast<uint4*>(drow + ((cc ^ (r & 7)) << 4)) = make_uint4(du[0], du[1], du[2], du[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // dK, dV rows (fp32) for this CTA's keys: columns cb*64 .. cb*64+63
+    if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(acc_done, 0, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        float* dst = (which == 0 ? dk_out : dv_out) + ((long long)row_base + key) * lddkv + kvh * 128 + cb * 64;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_addr + which * 128 + cb * 64 + c * 32, v);
+          tmem_ld_wait();
+          if (key < T) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+              *reinterpret_cast<float4*>(dst + c * 32 + g * 4) =
+                  make_float4(__uint_as_float(v[g * 4]), __uint_as_float(v[g * 4 + 1]), __uint_as_float(v[g * 4 + 2]),
+                              __uint_as_float(v[g * 4 + 3]));
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------- dQ epilogue
+    const int qw = warp & 3;
+    const int hdl = qw * 32 + lane;  // hd column this thread holds
+    const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
+    const bool issuer = (warp == 10 && lane == 0);
+    bool ok = true;
+    for (int i = 0; i < steps; ++i) {
+      const int hh = kvh * G + i / nq;
+      const int q0 = (qt_lo + i % nq) * AB2_BQ;
+      ok = ok && mbar_wait_warp(dq_full, i & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+      uint32_t v0[32], v1[32];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld_32x32b_x32(lane_addr + 384, v0);
+        tmem_ld_32x32b_x32(lane_addr + 416, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+      // staging buffer: the previous reduction must have finished reading it
+      if (issuer) bulk_wait_read0();
+      named_bar_sync(2, 128);
+      if (ok) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) sDQ[q * 128 + hdl] = __uint_as_float(v0[q]);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) sDQ[(32 + q) * 128 + hdl] = __uint_as_float(v1[q]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(2, 128);
+      if (issuer && ok) {
+        tma_reduce_add_2d(&tm_dq, sDQ, hh * 128, row_base + q0);
+        bulk_commit_group();
+      }
+    }
+    if (issuer) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace gptb
