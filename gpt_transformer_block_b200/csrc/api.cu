@@ -130,9 +130,9 @@ bool make_tmap(CUtensorMap* m, const void* ptr, bool fp8, uint64_t inner, uint64
   return r == CUDA_SUCCESS;
 }
 
-// 2-D fp32 tensor map without swizzle (TMA bulk reduce-add target)
-bool make_tmap_f32_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
-                         uint32_t box_inner, uint32_t box_outer) {
+// 2-D fp32 tensor map (TMA store / bulk reduce-add target), optional 128-byte swizzle
+bool make_tmap_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
+                   uint32_t box_outer, bool sw128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -140,8 +140,8 @@ bool make_tmap_f32_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -172,14 +172,14 @@ int plan_splits(int tiles, int kb_total, int sms) {
 }
 
 template <bool AM, bool BM, bool F8>
-int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, int splits, const EpiParams& ep,
-              cudaStream_t st, int sms) {
+int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const CUtensorMap& to2,
+              const CUtensorMap& tx, int M, int N, int K, int splits, const EpiParams& ep, cudaStream_t st, int sms) {
   auto kern = gemm_tc_kernel<AM, BM, F8>;
   const int smem = tc_smem_bytes();
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const long long units = (long long)((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN) * splits;
   const int grid = (int)std::min<long long>(units, sms);
-  kern<<<grid, TC_THREADS, smem, st>>>(ta, tb, M, N, K, splits, ep);
+  kern<<<grid, TC_THREADS, smem, st>>>(ta, tb, to, to2, tx, M, N, K, splits, ep);
   CKL();
   return GPTB_OK;
 }
@@ -219,12 +219,24 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
     const bool f8 = dtype == GPTB_FP8_E4M3;
     const int align = f8 ? 16 : 8;  // row strides must be multiples of 16 bytes
     const uint32_t bk = f8 ? 128 : 64;
+    const bool acc32 = ep.kind == EPI_ACCUM_F32;
+    const bool has_aux = ep.kind == EPI_RESID || ep.kind == EPI_DRELU2;
+    if (ep.out_f32 && !acc32) return GPTB_ERR_UNSUPPORTED;  // tensor-core outputs are bf16 or fp32 accumulations
     if (!aligned16(A.p) || !aligned16(B.p) || !aligned16(ep.out) || (A.ld % align) || (B.ld % align) ||
-        (ep.ldo % 8) || (N % 8))
+        (ep.ldo % (acc32 ? 4 : 8)) || (N % 8))
       return GPTB_ERR_INVALID_ARG;
-    CUtensorMap ta, tb;
+    if (has_aux && (!aligned16(ep.aux) || ep.ld_aux % 8)) return GPTB_ERR_INVALID_ARG;
+    if (ep.kind == EPI_RELU2 && (!aligned16(ep.out2) || ep.ldo2 % 8)) return GPTB_ERR_INVALID_ARG;
+    CUtensorMap ta, tb, to, to2, tx;
     bool ok = A.mn ? make_tmap(&ta, A.p, f8, M, K, A.ld, bk, bk) : make_tmap(&ta, A.p, f8, K, M, A.ld, bk, TC_BM);
     ok = ok && (B.mn ? make_tmap(&tb, B.p, f8, N, K, B.ld, bk, bk) : make_tmap(&tb, B.p, f8, K, N, B.ld, bk, TC_BN));
+    // epilogue maps: 32-row boxes of 64 bf16 / 32 fp32 columns, 128-byte swizzle
+    ok = ok && (acc32 ? make_tmap_f32(&to, ep.out, N, M, ep.ldo, 32, 32, true)
+                      : make_tmap(&to, ep.out, false, N, M, ep.ldo, 64, 32));
+    to2 = to;
+    tx = to;
+    if (ok && ep.kind == EPI_RELU2) ok = make_tmap(&to2, ep.out2, false, N, M, ep.ldo2, 64, 32);
+    if (ok && has_aux) ok = make_tmap(&tx, ep.aux, false, N, M, ep.ld_aux, 64, 32);
     if (!ok) return GPTB_ERR_CUDA;
     int splits = 1;
     if (ep.kind == EPI_ACCUM_F32) {
@@ -233,13 +245,13 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
     }
     const int sel = (A.mn ? 1 : 0) | (B.mn ? 2 : 0) | (f8 ? 4 : 0);
     switch (sel) {
-      case 0: rc = launch_tc<false, false, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
-      case 1: rc = launch_tc<true, false, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
-      case 2: rc = launch_tc<false, true, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
-      case 3: rc = launch_tc<true, true, false>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
-      case 4: rc = launch_tc<false, false, true>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
-      case 6: rc = launch_tc<false, true, true>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
-      case 7: rc = launch_tc<true, true, true>(ta, tb, M, N, K, splits, ep, st, di.sms); break;
+      case 0: rc = launch_tc<false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
+      case 1: rc = launch_tc<true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
+      case 2: rc = launch_tc<false, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
+      case 3: rc = launch_tc<true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
+      case 4: rc = launch_tc<false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
+      case 6: rc = launch_tc<false, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
+      case 7: rc = launch_tc<true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
       default: rc = GPTB_ERR_UNSUPPORTED;  // e4m3 with A M-major and B K-major: not used
     }
   }
@@ -616,7 +628,7 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     bool okm = make_tmap(&tkv, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128);
     okm = okm && make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 64);
     okm = okm && make_tmap(&tdo, X.dO, false, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 64, 64);
-    okm = okm && make_tmap_f32_plain(&tdq, X.dq, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 128, 64);
+    okm = okm && make_tmap_f32(&tdq, X.dq, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 128, 64, false);
     if (!okm) return GPTB_ERR_CUDA;
     CK(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AB2_SMEM));
     attn_bwd_tc_kernel<<<dim3((m.T + AB2_BK - 1) / AB2_BK, m.Hkv, m.B), AB2_THREADS, AB2_SMEM, st>>>(

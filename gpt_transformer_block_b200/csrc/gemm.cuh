@@ -10,8 +10,10 @@
 // bf16 / e4m3 path (tcgen05): persistent, warp-specialised kernel.
 //   warp 0   TMA producer (128-byte swizzled tiles, 4-stage mbarrier ring)
 //   warp 1   TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-5 epilogue: tcgen05.ld 32 lanes x 32 columns per warp, fused
-//             elementwise op, direct 16-byte global stores / fp32 atomics
+//   warps 2-5 epilogue: tcgen05.ld 32 lanes x 64 columns per step, fused
+//             elementwise op into a swizzled per-warp smem tile, written by
+//             TMA bulk stores (bf16) or TMA bulk reduce-add (fp32 weight
+//             gradients); residual / saved-u inputs arrive by TMA loads
 //   Tile 128 x 256, two TMEM accumulators (2 x 256 columns) so the epilogue
 //   of tile i overlaps the MMAs of tile i+1.  Split-K over the K blocks is
 //   used for weight gradients (long K, few tiles); partial sums meet in the
@@ -129,9 +131,10 @@ constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 192;
 constexpr int TC_GROUP_M = 8;
 
+constexpr int TC_EPI_BYTES = 4 * 8192;  // per epilogue warp: two 32-row x 128-byte staging tiles
 __host__ __device__ constexpr int tc_smem_bytes() {
-  // stages * (A 16 KB + B 32 KB) + barriers + 1 KB alignment slack
-  return TC_STAGES * (TC_BM * 128 + TC_BN * 128) + 256 + 1024;
+  // stages * (A 16 KB + B 32 KB) + epilogue staging + barriers + 1 KB alignment slack
+  return TC_STAGES * (TC_BM * 128 + TC_BN * 128) + TC_EPI_BYTES + 256 + 1024;
 }
 
 __device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, int& tm, int& tn, int& split) {
@@ -149,8 +152,9 @@ __device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, 
 
 template <bool A_MN, bool B_MN, bool FP8>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                   int K, int splits, EpiParams ep) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
+                   const __grid_constant__ CUtensorMap tmX, int M, int N, int K, int splits, EpiParams ep) {
   constexpr int ELEM = FP8 ? 1 : 2;
   constexpr int BK = 128 / ELEM;      // one 128-byte swizzle row of K (64 bf16 / 128 e4m3)
   constexpr int MMA_K = 32 / ELEM;    // K per tcgen05.mma (16 bf16 / 32 e4m3)
@@ -164,12 +168,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + TC_STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + TC_STAGES * B_BYTES);
+  uint8_t* sEpi = sB + TC_STAGES * B_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + TC_EPI_BYTES);
   uint64_t* empty = full + TC_STAGES;
   uint64_t* tfull = empty + TC_STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* aux_bar = drain + 1;  // [4] one per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,6 +194,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&tempty[b], 4);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&aux_bar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -312,32 +319,101 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t* stg0 = sEpi + (warp - 2) * 8192;  // this warp's two staging tiles
+    uint8_t* stg1 = stg0 + 4096;
+    uint64_t* abar = &aux_bar[warp - 2];
+    uint32_t aphase = 0;
+    const bool has_aux = (ep.kind == EPI_RESID || ep.kind == EPI_DRELU2);
+    const bool acc32 = (ep.kind == EPI_ACCUM_F32);
+    const int swz = (lane & 7);  // 16-byte chunk swizzle of this lane's 128-byte staging row
     int acc = 0;
     uint32_t acc_phase = 0;
     const float alpha = epi_alpha(ep);
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int tm, tn, split;
       tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
       if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const long long row = (long long)tm * TC_BM + q * 32 + lane;
+      const int row0 = tm * TC_BM + q * 32;
 #pragma unroll 1
-      for (int c = 0; c < TC_BN; c += 32) {
-        const int col = tn * TC_BN + c;
-        if (col >= N) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + c), r);
+      for (int cc = 0; cc < TC_BN / 64; ++cc) {
+        const int col0 = tn * TC_BN + cc * 64;
+        if (col0 >= N) break;  // warp-uniform
+        uint32_t r0[32], r1[32];
+        const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + cc * 64);
+        tmem_ld_32x32b_x32(ta, r0);
+        tmem_ld_32x32b_x32(ta + 32, r1);
+        // the staging tiles are free once this warp's previous bulk copies have read them
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        if (has_aux && lane == 0) {
+          mbar_arrive_expect_tx(abar, 4096);
+          tma_load_2d(stg1, &tmX, abar, col0, row0);
+        }
         tmem_ld_wait();
-        if (row < M) {
+        if (has_aux) {
+          if (!mbar_wait_warp(abar, aphase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
+            ok = false;
+            break;
+          }
+          aphase ^= 1u;
+        }
+        uint8_t* p0 = stg0 + lane * 128;
+        uint8_t* p1 = stg1 + lane * 128;
+        if (acc32) {
+          // fp32: columns 0..31 -> tile 0, 32..63 -> tile 1 (32 x 128-byte rows each)
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (col + g * 8 < N) {
-              float v[8];
+          for (int g = 0; g < 8; ++g) {
+            *reinterpret_cast<float4*>(p0 + ((g ^ swz) << 4)) =
+                make_float4(__uint_as_float(r0[4 * g]) * alpha, __uint_as_float(r0[4 * g + 1]) * alpha,
+                            __uint_as_float(r0[4 * g + 2]) * alpha, __uint_as_float(r0[4 * g + 3]) * alpha);
+            *reinterpret_cast<float4*>(p1 + ((g ^ swz) << 4)) =
+                make_float4(__uint_as_float(r1[4 * g]) * alpha, __uint_as_float(r1[4 * g + 1]) * alpha,
+                            __uint_as_float(r1[4 * g + 2]) * alpha, __uint_as_float(r1[4 * g + 3]) * alpha);
+          }
+        } else {
+          // bf16: 8 chunks of 8 columns; aux (if any) sits in tile 1 with the same swizzle
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[g * 8 + i]) * alpha;
-              epi_apply8(ep, row, col + g * 8, v);
+          for (int g = 0; g < 8; ++g) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(g < 4 ? r0[g * 8 + i] : r1[(g - 4) * 8 + i]) * alpha;
+            uint8_t* cp0 = p0 + ((g ^ swz) << 4);
+            uint8_t* cp1 = p1 + ((g ^ swz) << 4);
+            if (has_aux) {
+              float a[8];
+              load8(reinterpret_cast<const bf16*>(cp1), a);
+              if (ep.kind == EPI_RESID) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] += a[i];
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] *= 2.f * fmaxf(a[i], 0.f);
+              }
+            }
+            store8(reinterpret_cast<bf16*>(cp0), v);
+            if (ep.kind == EPI_RELU2) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float t = fmaxf(v[i], 0.f);
+                v[i] = t * t;
+              }
+              store8(reinterpret_cast<bf16*>(cp1), v);
             }
           }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (acc32) {
+            tma_reduce_add_2d(&tmO, stg0, col0, row0);
+            tma_reduce_add_2d(&tmO, stg1, col0 + 32, row0);
+          } else {
+            tma_store_2d(&tmO, stg0, col0, row0);
+            if (ep.kind == EPI_RELU2) tma_store_2d(&tmO2, stg1, col0, row0);
+          }
+          bulk_commit_group();
         }
       }
       tc_fence_before();
@@ -346,6 +422,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait0();
   }
   __syncthreads();
   if (warp == 1) {
