@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "../../include/gptblock.h"
@@ -541,9 +542,16 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, X.a8, S.amax + 0, true},
               {w.w_qkv, m.d, false, (long long)m.Wq * m.d, S.wqkv8, S.amax + 4, true}, (int)m.N, m.Wq, m.d,
               epi(EPI_STORE, c.dtype, S.qkv, m.Wq), st));
-  qkv_post_kernel<T><<<grid_rows(m.N * (m.NH + (ve ? m.Hkv : 0))), EW_THREADS, 0, st>>>(
-      (T*)S.qkv, m.Wq, S.rstd_qk, X.rope, m.T, m.N, m.H, m.Hkv, m.hd, c.norm_eps, ve ? (const T*)w.ve_table : nullptr,
-      idx, S.sg);
+  if constexpr (std::is_same<T, bf16>::value) {
+    // bf16 storage always has hd = 128: vectorised per-(token, head) kernel
+    qkv_post_h128_kernel<<<grid_rows(m.N * (m.NH + (ve ? m.Hkv : 0))), EW_THREADS, 0, st>>>(
+        (bf16*)S.qkv, m.Wq, S.rstd_qk, X.rope, m.T, m.N, m.H, m.Hkv, c.norm_eps,
+        ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg);
+  } else {
+    qkv_post_kernel<T><<<grid_rows(m.N * (m.NH + (ve ? m.Hkv : 0))), EW_THREADS, 0, st>>>(
+        (T*)S.qkv, m.Wq, S.rstd_qk, X.rope, m.T, m.N, m.H, m.Hkv, m.hd, c.norm_eps,
+        ve ? (const T*)w.ve_table : nullptr, idx, S.sg);
+  }
   CKL();
   const int W = c.window[layer];
   if (c.dtype == GPTB_F32) {
@@ -609,8 +617,14 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
               (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
   // attention
-  attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
-                                                                     m.B, m.T, m.H, m.hd);
+  if constexpr (std::is_same<T, bf16>::value) {
+    attn_bwd_pre_h128_kernel<<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const bf16*)S.o, Ho, (const bf16*)X.dO, Ho,
+                                                                        X.D, m.T, m.N, m.H);
+  } else {
+    attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
+                                                                       m.B, m.T, m.H, m.hd);
+  
+  }
   CKL();
   CK(cudaMemsetAsync(X.dq, 0, m.N * Ho * 4, st));
   const int W = c.window[layer];
@@ -635,9 +649,15 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
         tkv, tq, tdo, tdq, S.lse, X.D, X.dk, X.dv, Kv, m.T, m.H, m.Hkv, W);
     CKL();
   }
-  qkv_post_bwd_kernel<T><<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(
-      (const T*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (T*)X.dqkv, m.T, m.N, m.H, m.Hkv, m.hd,
-      ve ? (const T*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz);
+  if constexpr (std::is_same<T, bf16>::value) {
+    qkv_post_bwd_h128_kernel<<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(
+        (const bf16*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (bf16*)X.dqkv, m.T, m.N, m.H, m.Hkv,
+        ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz);
+  } else {
+    qkv_post_bwd_kernel<T><<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(
+        (const T*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (T*)X.dqkv, m.T, m.N, m.H, m.Hkv, m.hd,
+        ve ? (const T*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz);
+  }
   CKL();
   // QKV projection
   TRY(proj<T>(c, {X.dqkv, m.Wq, true, 0, nullptr, nullptr, false}, {S.h, m.d, true, 0, nullptr, nullptr, false},

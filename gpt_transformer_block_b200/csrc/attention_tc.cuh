@@ -176,6 +176,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const int t = q0 + r;          // query position
     const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
     const float sl2 = LOG2E / sqrtf(128.f);
+    // keys visible from query t: [t - W, t] (or [0, t]) clipped to the sequence
+    const int kv_lo = (window >= 0) ? t - window : 0;
+    const int kv_hi = min(t, T - 1);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     // Every softmax warp runs every iteration and passes every named barrier,
@@ -187,22 +190,28 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       ok = ok && mbar_wait_warp(&s_full[sb], (j >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
       tc_fence_after();
       const bool need_mask = (k0 + 63 > q0) || (k0 + 64 > T) || (window >= 0 && q0 + FA_BM - 1 - k0 > window);
-      // pass 1: max of this half of the row (masked), 4 independent partials
-      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // both 32-column chunks of this half go to registers at once; the score
+      // buffer is released right after, so the next-but-one S MMA can start
+      uint32_t v[64];
       if (ok) {
+        tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      // masked scores become -inf; visible keys of row t: kv_lo..kv_hi
+      if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64 + c * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int jk = k0 + c * 32 + i;
-            const bool vis = !need_mask || ((jk <= t) && (jk < T) && (window < 0 || t - jk <= window));
-            mp[i & 3] = vis ? fmaxf(mp[i & 3], __uint_as_float(v[i])) : mp[i & 3];
-          }
+        for (int i = 0; i < 64; ++i) {
+          const int jk = k0 + i;
+          v[i] = (jk >= kv_lo && jk <= kv_hi) ? v[i] : __float_as_uint(-INFINITY);
         }
       }
+      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < 64; ++i) mp[i & 3] = fmaxf(mp[i & 3], __uint_as_float(v[i]));
       float* xm = xmax + sb * 256;
       xm[hf * 128 + r] = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
       named_bar_sync(1, FA_SOFTMAX_THREADS);
@@ -240,39 +249,25 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       uint8_t* prow = sP + hf * 16384 + r * 128;
       float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64 + c * 32, v);
-        tmem_ld_wait();
+      for (int cc = 0; cc < 8; ++cc) {
+        float p[8];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = g * 8 + e;
-            const int jk = k0 + c * 32 + i;
-            const bool vis = !need_mask || ((jk <= t) && (jk < T) && (window < 0 || t - jk <= window));
-            p[e] = vis ? fast_exp2(fmaf(__uint_as_float(v[i]), sl2, -mu)) : 0.f;
-            lp[e & 3] += p[e];
-          }
-          const int cc = c * 4 + g;  // 0..7
-          uint4 u;
-          u.x = pack_bf16(p[0], p[1]);
-          u.y = pack_bf16(p[2], p[3]);
-          u.z = pack_bf16(p[4], p[5]);
-          u.w = pack_bf16(p[6], p[7]);
-          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = u;
+        for (int e = 0; e < 8; ++e) {
+          p[e] = fast_exp2(fmaf(__uint_as_float(v[cc * 8 + e]), sl2, -mu));  // exp2(-inf) = 0 for masked keys
+          lp[e & 3] += p[e];
         }
+        uint4 u;
+        u.x = pack_bf16(p[0], p[1]);
+        u.y = pack_bf16(p[2], p[3]);
+        u.z = pack_bf16(p[4], p[5]);
+        u.w = pack_bf16(p[6], p[7]);
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = u;
       }
       l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-      // scores consumed; P visible to the tensor core
-      tc_fence_before();
+      // P visible to the tensor core
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&s_empty[sb]);
-        mbar_arrive(p_full);
-      }
+      if (lane == 0) mbar_arrive(p_full);
     }
     // the two halves' sums share the same running max: add them
     xsum[hf * 128 + r] = l;
@@ -511,6 +506,9 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
     const float scale = rsqrtf(128.f);
     const float sl2 = LOG2E * scale;
+    // queries that see this key: [key, key + W] (or [key, T)) inside the sequence
+    const int q_vis_lo = key;
+    const int q_vis_hi = (key < T) ? ((window >= 0) ? min(T - 1, key + window) : T - 1) : -1;
     bool ok = true;
     for (int i = 0; i < steps && ok; ++i) {
       const int st = i & 1;
@@ -547,7 +545,7 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
           for (int h2 = 0; h2 < 2; ++h2) {
             const int e = c * 8 + e2 * 2 + h2;
             const int t = tq + e;
-            const bool vis = !need_mask || ((key <= t) && (t < T) && (key < T) && (window < 0 || t - key <= window));
+            const bool vis = !need_mask || (t >= q_vis_lo && t <= q_vis_hi);
             pe[h2] = vis ? fast_exp2(fmaf(__uint_as_float(sv[e]), sl2, -l2[e])) : 0.f;
             de[h2] = pe[h2] * (__uint_as_float(dv[e]) - Dq[e]) * scale;
           }

@@ -673,3 +673,155 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace gptb
+
+namespace gptb {
+
+// ------------------------------------------- vectorised hd = 128 variants --
+// One warp per (token, head).  Lane l holds elements 4l..4l+3 of the head:
+// lanes 0-15 the first half (rotation partner j), lanes 16-31 the second half
+// (j + 64); the partner value is one shuffle (lane ^ 16) away.
+
+__device__ __forceinline__ void ld4(const bf16* p, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+__device__ __forceinline__ void st4(bf16* p, const float (&v)[4]) {
+  uint2 u;
+  u.x = pack_bf16(v[0], v[1]);
+  u.y = pack_bf16(v[2], v[3]);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    qkv_post_h128_kernel(bf16* __restrict__ qkv, long long ld, float* __restrict__ rstd_qk,
+                         const float2* __restrict__ rope, int Tn, long long N, int H, int Hkv, float eps,
+                         const bf16* __restrict__ ve_table, const int32_t* __restrict__ idx,
+                         const float* __restrict__ sg) {
+  const int lane = threadIdx.x & 31;
+  const int nh_norm = H + Hkv;
+  const int nh = nh_norm + (ve_table ? Hkv : 0);
+  const bool hi = lane >= 16;
+  const int j0 = (lane & 15) * 4;
+  for (RowLoop it(N * nh); it.row < it.nrows; it.row += it.stride) {
+    const long long n = it.row / nh;
+    const int hh = (int)(it.row - n * nh);
+    bf16* p = qkv + n * ld + (long long)hh * 128 + lane * 4;
+    float x[4];
+    ld4(p, x);
+    if (hh < nh_norm) {
+      float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+      const float r = rsqrtf(warp_sum(ss) * (1.f / 128.f) + eps);
+      const int t = (int)(n % Tn);
+      const float4 c01 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + j0);
+      const float4 c23 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + j0 + 2);
+      const float cs[4][2] = {{c01.x, c01.y}, {c01.z, c01.w}, {c23.x, c23.y}, {c23.z, c23.w}};
+      float y[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float mine = x[e] * r;
+        const float other = __shfl_xor_sync(0xffffffffu, x[e], 16) * r;
+        // first half: x1 c - x2 s ; second half: x1 s + x2 c  (x1 = first-half value)
+        y[e] = hi ? (other * cs[e][1] + mine * cs[e][0]) : (mine * cs[e][0] - other * cs[e][1]);
+      }
+      st4(p, y);
+      if (lane == 0) rstd_qk[n * nh_norm + hh] = r;
+    } else {
+      const int kv = hh - nh_norm;
+      const float gate = 3.f * sg[n * Hkv + kv];
+      float e[4];
+      ld4(ve_table + (long long)idx[n] * Hkv * 128 + (long long)kv * 128 + lane * 4, e);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[i] = fmaf(gate, e[i], x[i]);
+      st4(p, x);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(EW_THREADS)
+    qkv_post_bwd_h128_kernel(const bf16* __restrict__ qkv, long long ld, const float* __restrict__ rstd_qk,
+                             const float2* __restrict__ rope, const float* __restrict__ dq, long long lddq,
+                             const float* __restrict__ dk, const float* __restrict__ dv, long long lddkv,
+                             bf16* __restrict__ dqkv, int Tn, long long N, int H, int Hkv,
+                             const bf16* __restrict__ ve_table, const int32_t* __restrict__ idx,
+                             const float* __restrict__ sg, float* __restrict__ dve_table, float* __restrict__ dz) {
+  const int lane = threadIdx.x & 31;
+  const int nh = H + 2 * Hkv;
+  const bool hi = lane >= 16;
+  const int j0 = (lane & 15) * 4;
+  for (RowLoop it(N * nh); it.row < it.nrows; it.row += it.stride) {
+    const long long n = it.row / nh;
+    const int hh = (int)(it.row - n * nh);
+    bf16* out = dqkv + n * ld + (long long)hh * 128 + lane * 4;
+    if (hh < H + Hkv) {
+      const float* gp = (hh < H) ? dq + n * lddq + (long long)hh * 128 : dk + n * lddkv + (long long)(hh - H) * 128;
+      const float4 g4 = *reinterpret_cast<const float4*>(gp + lane * 4);
+      const float g[4] = {g4.x, g4.y, g4.z, g4.w};
+      float y[4];
+      ld4(qkv + n * ld + (long long)hh * 128 + lane * 4, y);
+      const int t = (int)(n % Tn);
+      const float4 c01 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + j0);
+      const float4 c23 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + j0 + 2);
+      const float cs[4][2] = {{c01.x, c01.y}, {c01.z, c01.w}, {c23.x, c23.y}, {c23.z, c23.w}};
+      // undo the rotation on the gradient and on the stored (rotated) output:
+      // first half: a1 c + a2 s ; second half: -a1 s + a2 c  (a1 = first-half value)
+      float gu[4], yu[4], dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float go = __shfl_xor_sync(0xffffffffu, g[e], 16);
+        const float yo = __shfl_xor_sync(0xffffffffu, y[e], 16);
+        gu[e] = hi ? (g[e] * cs[e][0] - go * cs[e][1]) : (g[e] * cs[e][0] + go * cs[e][1]);
+        yu[e] = hi ? (y[e] * cs[e][0] - yo * cs[e][1]) : (y[e] * cs[e][0] + yo * cs[e][1]);
+        dot = fmaf(gu[e], yu[e], dot);
+      }
+      const float m = warp_sum(dot) * (1.f / 128.f);
+      const float r = rstd_qk[n * (H + Hkv) + hh];
+      float o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = r * (gu[e] - yu[e] * m);
+      st4(out, o);
+    } else {
+      const int kv = hh - H - Hkv;
+      const float4 g4 = *reinterpret_cast<const float4*>(dv + n * lddkv + (long long)kv * 128 + lane * 4);
+      float g[4] = {g4.x, g4.y, g4.z, g4.w};
+      if (ve_table) {
+        const long long row = (long long)idx[n] * Hkv * 128 + (long long)kv * 128 + lane * 4;
+        const float s = sg[n * Hkv + kv];
+        const float gate = 3.f * s;
+        float e[4];
+        ld4(ve_table + row, e);
+        const float dg = warp_sum(g[0] * e[0] + g[1] * e[1] + g[2] * e[2] + g[3] * e[3]);
+        atomicAdd(reinterpret_cast<float4*>(dve_table + row), make_float4(gate * g[0], gate * g[1], gate * g[2], gate * g[3]));
+        if (lane == 0) dz[n * Hkv + kv] = dg * 3.f * s * (1.f - s);
+      }
+      st4(out, g);
+    }
+  }
+}
+
+}  // namespace gptb
+
+namespace gptb {
+
+// D[b,h,t] = sum_c dO[t,h,c] * o[t,h,c] for hd = 128: one warp per (token, head),
+// 8-byte loads per lane
+__global__ void __launch_bounds__(EW_THREADS)
+    attn_bwd_pre_h128_kernel(const bf16* __restrict__ o, long long ldo, const bf16* __restrict__ dO, long long lddo,
+                             float* __restrict__ D, int Tn, long long N, int H) {
+  const int lane = threadIdx.x & 31;
+  for (RowLoop it(N * H); it.row < it.nrows; it.row += it.stride) {
+    const long long n = it.row / H;
+    const int h = (int)(it.row - n * H);
+    float a[4], g[4];
+    ld4(o + n * ldo + (long long)h * 128 + lane * 4, a);
+    ld4(dO + n * lddo + (long long)h * 128 + lane * 4, g);
+    const float s = warp_sum(a[0] * g[0] + a[1] * g[1] + a[2] * g[2] + a[3] * g[3]);
+    if (lane == 0) {
+      const long long b = n / Tn, t = n - b * Tn;
+      D[(b * H + h) * Tn + t] = s;
+    }
+  }
+}
+
+}  // namespace gptb
