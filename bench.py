@@ -46,13 +46,14 @@ def attention_pairs(T: int, window: int) -> int:
 
 
 def flops_per_token(c: dict) -> dict:
-    """Algorithmic training FLOPs per token (forward + backward = 3x forward).
+    """Training FLOPs per token (forward + backward = 3x forward).
 
-    Matmul parameters count 6 FLOPs per token; attention counts only the
-    visible pairs (4*hd per pair and head forward: QK^T and PV), times 3.
-    The pages-convention count uses 12*L*H*hd*T_eff with T_eff the average
-    attended length T/2-ish convention of the source (T for full layers,
-    window for windowed layers, averaged)."""
+    algorithmic: 6 per matmul parameter (block projections and lm_head) plus
+    attention over the visible (query, key) pairs only: 4*hd FLOPs per pair
+    and head forward (QK^T and PV), times 3.
+    pages_convention: 6 per matmul parameter plus 12*L*H*hd*T_eff, with T_eff
+    the mean attended context per layer (T for full layers, W for windowed
+    ones); this count reproduces the pages' total for their depth-24 run."""
     d, H, Hk, hd, F, V, L, T = (c["d"], c["n_head"], c["n_kv_head"], c["head_dim"], c["mlp_hidden"],
                                 c["vocab"], c["n_layer"], c["T"])
     n_mat = L * (d * (H + 2 * Hk) * hd + H * hd * d + 2 * d * F)
@@ -115,6 +116,22 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
+# ------------------------------------------------------- multi-rank ---------
+
+def max_over_ranks(value: float, dist=None, device="cuda") -> float:
+    """Max of a per-rank timing over all ranks (the job is as slow as its slowest rank)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch (weak scaling)."""
+    return world * tokens_per_step * steps / (ms_max / 1e3)
+
+
 # ----------------------------------------------------------- peaks ---------
 
 def measured_peaks() -> dict:
@@ -152,7 +169,7 @@ def oracle_sample(c: dict, seed: int = 7) -> dict:
     cs = dict(c, B=1)
     w = synth.make_weights(cs, seed=seed, mode="random")
     inp = synth.make_block_inputs(cs, seed=seed + 1)
-    layer = max(i for i in range(cs["n_layer"]) if True)  # last layer: value embedding on
+    layer = cs["n_layer"] - 1  # the last layer carries a value embedding
     lw = {k: (v if isinstance(v, float) else np.asarray(v, dtype=np.float64)) for k, v in w["layers"][layer].items()}
     x = inp["x"].double().numpy()
     x0 = inp["x0"].double().numpy()
@@ -275,13 +292,9 @@ def main():
         raise RuntimeError(f"device error {err} in timed region")
     loss = model.loss.item()
 
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-
+    ms = max_over_ranks(ms, dist)
     tokens_per_step = c["B"] * c["T"]
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = job_throughput(world, tokens_per_step, args.steps, ms)
     ms_step = ms / args.steps
 
     # ---- end to end through the public API, inputs from pinned host memory
@@ -297,12 +310,8 @@ def main():
         model.step(idx, tg)
         loss_h.copy_(model.loss, non_blocking=True)
         torch.cuda.current_stream().synchronize()
-    e2e_s = time.perf_counter() - t0
-    if dist is not None:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = t.item()
-    e2e_val = world * tokens_per_step * args.e2e_steps / e2e_s
+    e2e_s = max_over_ranks(time.perf_counter() - t0, dist)
+    e2e_val = job_throughput(world, tokens_per_step, args.e2e_steps, e2e_s * 1e3)
 
     peaks = measured_peaks()
     flops_s = value / world * fl["algorithmic"]

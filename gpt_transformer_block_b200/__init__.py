@@ -22,7 +22,7 @@ EXPORTS = [
     "gptb_workspace_bytes", "gpt_block_forward", "gpt_block_backward", "lm_head_xent",
     "gpt_stack_step", "gptb_gemm_bf16", "gptb_device_error", "gptb_set_wait_limit_ns",
     "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
-    "gptb_error_string", "lm_head_xent_noalloc",
+    "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
 ]
 
 _vp = ctypes.c_void_p
@@ -85,6 +85,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                    ctypes.c_int, _vp]
     lib.gptb_device_error.argtypes = [_vp]
     lib.gptb_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.gptb_probe_bounded_wait.argtypes = [ctypes.c_ulonglong, _vp]
     lib.gptb_reset_counters.restype = None
     lib.gptb_launch_count.restype = ctypes.c_longlong
     lib.gptb_set_gemm_timing.argtypes = [ctypes.c_int]
@@ -217,6 +218,11 @@ def gptb_gemm_bf16(A, a_mn, lda, B, b_mn, ldb, C, c_f32, ldc, M, N, K, stream=No
 
 def gptb_device_error(stream=None) -> int:
     return int(load().gptb_device_error(_stream(stream)))
+
+
+def gptb_probe_bounded_wait(limit_ns: int, stream=None) -> int:
+    """Run the bounded-wait self-test; GPTB_ERR_TIMEOUT is the expected result."""
+    return int(load().gptb_probe_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 def gptb_set_wait_limit_ns(ns: int):

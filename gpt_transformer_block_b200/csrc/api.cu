@@ -17,6 +17,7 @@
 #include "attention_tc.cuh"
 #include "common.cuh"
 #include "elementwise.cuh"
+#include "rows.cuh"
 #include "gemm.cuh"
 
 using namespace gptb;
@@ -58,19 +59,6 @@ cudaEvent_t take_event() {
       return GPTB_ERR_CUDA;                                    \
     }                                                          \
   } while (0)
-// instantiate a row kernel for NC = ceil(d / 256) chunks per lane
-#define ROWK(NCV, ...)                                     \
-  switch (NCV) {                                           \
-    case 1: { constexpr int NC = 1; __VA_ARGS__; } break;  \
-    case 2: { constexpr int NC = 2; __VA_ARGS__; } break;  \
-    case 3: { constexpr int NC = 3; __VA_ARGS__; } break;  \
-    case 4: { constexpr int NC = 4; __VA_ARGS__; } break;  \
-    case 5: { constexpr int NC = 5; __VA_ARGS__; } break;  \
-    case 6: { constexpr int NC = 6; __VA_ARGS__; } break;  \
-    case 7: { constexpr int NC = 7; __VA_ARGS__; } break;  \
-    case 8: { constexpr int NC = 8; __VA_ARGS__; } break;  \
-    default: return GPTB_ERR_UNSUPPORTED;                  \
-  }
 #define TRY(x)                     \
   do {                             \
     int _r = (x);                  \
@@ -278,6 +266,13 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
   e.alpha = nullptr;
   e.amax_a = nullptr;
   e.amax_b = nullptr;
+  e.rope = nullptr;
+  e.rstd_qk = nullptr;
+  e.ve_table = nullptr;
+  e.idx = nullptr;
+  e.sg = nullptr;
+  e.T = e.H = e.Hkv = 0;
+  e.eps = 0.f;
   return e;
 }
 EpiParams epi8(EpiParams e, const float* amax_a, const float* amax_b) {
@@ -448,7 +443,7 @@ StackWs carve_stack(Carve& cv, const Dims& m) {
 int check_config(const gptb_config* c) {
   if (!c) return GPTB_ERR_INVALID_ARG;
   if (c->dtype != GPTB_F32 && c->dtype != GPTB_BF16 && c->dtype != GPTB_FP8_E4M3) return GPTB_ERR_UNSUPPORTED;
-  if (c->B < 1 || c->T < 1 || c->d < 8 || c->d % 8 || c->d > 8 * 32 * EW_MAXC) return GPTB_ERR_INVALID_ARG;
+  if (c->B < 1 || c->T < 1 || c->d < 8 || c->d % 8 || c->d > 8 * 32 * BR_MAX_WARPS) return GPTB_ERR_INVALID_ARG;
   if (c->n_head < 1 || c->n_kv_head < 1 || c->n_head % c->n_kv_head) return GPTB_ERR_INVALID_ARG;
   if (c->mlp_hidden < 8 || c->mlp_hidden % 8 || c->vocab < 8 || c->vocab % 8) return GPTB_ERR_INVALID_ARG;
   if (c->n_layer < 1 || c->n_layer > GPTB_MAX_LAYERS) return GPTB_ERR_INVALID_ARG;
@@ -467,6 +462,13 @@ int check_config(const gptb_config* c) {
   }
   if (((long long)c->B * c->T) > (1ll << 31) / 4) return GPTB_ERR_INVALID_ARG;
   return GPTB_OK;
+}
+
+// one CTA per token row: ceil(d/8) threads rounded up to whole warps
+int br_threads(int d) { return ((d / 8 + 31) / 32) * 32; }
+int br_grid(long long rows, int threads) {
+  const long long cap = (long long)dev_info().sms * (2048 / threads) * 2;
+  return (int)std::max<long long>(1, std::min(rows, cap));
 }
 
 int grid_rows(long long rows) {
@@ -530,29 +532,37 @@ template <class T>
 int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w, const T* x, const T* x0,
                    const int32_t* idx, T* x_out, const Saved& S, const Scratch& X, cudaStream_t st) {
   const Dims m = dims_of(c);
-  const int nc = (m.d + 255) / 256;
+  const int brt = br_threads(m.d);
+  const int brg = br_grid(m.N, brt);
   const bool ve = c.has_ve[layer] != 0;
   if (!w.w_qkv || !w.w_o || !w.w_fc || !w.w_proj || !w.lambdas || (ve && (!w.w_ve_gate || !w.ve_table)))
     return GPTB_ERR_INVALID_ARG;
-  const int gr = grid_rows(m.N);
-  ROWK(nc, mix_norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(x, x0, w.lambdas, (T*)X.xm, (T*)S.h, S.rstd1, m.N, m.d, c.norm_eps,
-                                                ve ? (const T*)w.w_ve_gate : nullptr, S.sg, m.Hkv, c.ve_gate_ch));
+  br_mix_norm_kernel<T><<<brg, brt, 0, st>>>(x, x0, w.lambdas, (T*)X.xm, (T*)S.h, S.rstd1, m.N, m.d, c.norm_eps,
+                                                ve ? (const T*)w.w_ve_gate : nullptr, S.sg, m.Hkv, c.ve_gate_ch);
   CKL();
   const long long Ho = (long long)m.H * m.hd;
-  TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, X.a8, S.amax + 0, true},
-              {w.w_qkv, m.d, false, (long long)m.Wq * m.d, S.wqkv8, S.amax + 4, true}, (int)m.N, m.Wq, m.d,
-              epi(EPI_STORE, c.dtype, S.qkv, m.Wq), st));
-  if constexpr (std::is_same<T, bf16>::value) {
-    // bf16 storage always has hd = 128: vectorised per-(token, head) kernel
-    qkv_post_h128_kernel<<<grid_rows(m.N * (m.NH + (ve ? m.Hkv : 0))), EW_THREADS, 0, st>>>(
-        (bf16*)S.qkv, m.Wq, S.rstd_qk, X.rope, m.T, m.N, m.H, m.Hkv, c.norm_eps,
-        ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg);
-  } else {
+  if (c.dtype == GPTB_F32) {
+    TRY(gemm(c.dtype, {S.h, m.d, false}, {w.w_qkv, m.d, false}, (int)m.N, m.Wq, m.d,
+             epi(EPI_STORE, c.dtype, S.qkv, m.Wq), st));
     qkv_post_kernel<T><<<grid_rows(m.N * (m.NH + (ve ? m.Hkv : 0))), EW_THREADS, 0, st>>>(
         (T*)S.qkv, m.Wq, S.rstd_qk, X.rope, m.T, m.N, m.H, m.Hkv, m.hd, c.norm_eps,
         ve ? (const T*)w.ve_table : nullptr, idx, S.sg);
+    CKL();
+  } else {
+    // tensor-core QKV projection with QK RMSNorm + RoPE + value embedding fused into its epilogue
+    EpiParams e = epi(EPI_QKV, c.dtype, S.qkv, m.Wq);
+    e.rope = X.rope;
+    e.rstd_qk = S.rstd_qk;
+    e.ve_table = ve ? (const bf16*)w.ve_table : nullptr;
+    e.idx = idx;
+    e.sg = S.sg;
+    e.T = m.T;
+    e.H = m.H;
+    e.Hkv = m.Hkv;
+    e.eps = c.norm_eps;
+    TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, X.a8, S.amax + 0, true},
+                {w.w_qkv, m.d, false, (long long)m.Wq * m.d, S.wqkv8, S.amax + 4, true}, (int)m.N, m.Wq, m.d, e, st));
   }
-  CKL();
   const int W = c.window[layer];
   if (c.dtype == GPTB_F32) {
     attn_fwd_simt_kernel<T><<<dim3(m.T, m.H, m.B), 128, 0, st>>>((const T*)S.qkv, m.Wq, (T*)S.o,
@@ -571,8 +581,8 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, X.a8, S.amax + 1, true},
               {w.w_o, Ho, false, m.d * Ho, S.wo8, S.amax + 5, true}, (int)m.N, m.d, (int)Ho,
               epi(EPI_RESID, c.dtype, X.x1, m.d, X.xm, m.d), st));
-  ROWK(nc, norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
-                                            c.norm_eps));
+  br_norm_kernel<T><<<brg, brt, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
+                                            c.norm_eps);
   CKL();
   TRY(proj<T>(c, {S.h2, m.d, false, m.N * m.d, X.a8, S.amax + 2, true},
               {w.w_fc, m.d, false, (long long)m.F * m.d, S.wfc8, S.amax + 6, true}, (int)m.N, m.F, m.d,
@@ -589,7 +599,8 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
                    const int32_t* idx, const Saved& S, const T* dx2, const T* dx_extra, T* dx, float* dx0_acc,
                    const gptb_block_grads& g, const Scratch& X, cudaStream_t st) {
   const Dims m = dims_of(c);
-  const int nc = (m.d + 255) / 256;
+  const int brt = br_threads(m.d);
+  const int brg = br_grid(m.N, brt);
   const bool ve = c.has_ve[layer] != 0;
   if (!g.w_qkv || !g.w_o || !g.w_fc || !g.w_proj || !g.lambdas || (ve && (!g.w_ve_gate || !g.ve_table)))
     return GPTB_ERR_INVALID_ARG;
@@ -608,8 +619,7 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
               m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
   TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, X.gamax, true}, {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false},
               N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
-  const int gr = grid_rows(m.N);
-  ROWK(nc, norm_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d));
+  br_norm_bwd_kernel<T><<<brg, brt, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d);
   CKL();
   // attention output projection
   TRY(proj<T>(c, {X.dx1, m.d, true, 0, nullptr, nullptr, false}, {S.o, Ho, true, 0, nullptr, nullptr, false}, m.d,
@@ -671,10 +681,10 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
                                                                      c.ve_gate_ch, g.w_ve_gate);
     CKL();
   }
-  ROWK(nc, mix_norm_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)X.dh, ve ? X.dz : nullptr,
+  br_mix_norm_bwd_kernel<T><<<brg, brt, 0, st>>>((const T*)X.dh, ve ? X.dz : nullptr,
                                                     ve ? (const T*)w.w_ve_gate : nullptr, m.Hkv, c.ve_gate_ch,
                                                     (const T*)S.h, S.rstd1, (const T*)X.dx1, x, x0, w.lambdas, dx_extra,
-                                                    dx, dx0_acc, g.lambdas, m.N, m.d));
+                                                    dx, dx0_acc, g.lambdas, m.N, m.d);
   CKL();
   return GPTB_OK;
 }
@@ -684,7 +694,8 @@ template <class T>
 int lm_head_impl(const gptb_config& c, const T* h, const T* w_lm, const int32_t* targets, float* loss_out, T* dh,
                  float* dw_lm, const LmWs& lw, cudaStream_t st) {
   const Dims m = dims_of(c);
-  const int nc = (m.d + 255) / 256;
+  const int brt = br_threads(m.d);
+  const int brg = br_grid(m.N, brt);
   const int dt = c.dtype == GPTB_FP8_E4M3 ? GPTB_BF16 : c.dtype;  // lm_head stays bf16
   for (long long c0 = 0; c0 < m.N; c0 += lw.chunk) {
     const int rows = (int)std::min<long long>(lw.chunk, m.N - c0);
@@ -707,15 +718,15 @@ template <class T>
 int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t* idx, const int32_t* targets,
                float* loss_out, const gptb_model_grads& g, const StackWs& S, cudaStream_t st) {
   const Dims m = dims_of(c);
-  const int nc = (m.d + 255) / 256;
+  const int brt = br_threads(m.d);
+  const int brg = br_grid(m.N, brt);
   if (!w.wte || !w.w_lm || !g.wte || !g.w_lm) return GPTB_ERR_INVALID_ARG;
   if (c.smear_ch > 0 && (!w.w_smear_gate || !w.smear_lambda || !g.w_smear_gate || !g.smear_lambda))
     return GPTB_ERR_INVALID_ARG;
   if (c.backout_layer >= 0 && (!w.backout_lambda || !g.backout_lambda)) return GPTB_ERR_INVALID_ARG;
   TRY(rope_init<T>(c, S.scr.rope, st));
-  const int gr = grid_rows(m.N);
-  ROWK(nc, embed_smear_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(idx, (const T*)w.wte, (const T*)w.w_smear_gate, w.smear_lambda,
-                                                   (T*)S.x_in[0], m.B, m.T, m.d, c.smear_ch));
+  br_embed_smear_kernel<T><<<brg, brt, 0, st>>>(idx, (const T*)w.wte, (const T*)w.w_smear_gate, w.smear_lambda,
+                                                   (T*)S.x_in[0], m.B, m.T, m.d, c.smear_ch);
   CKL();
   const T* x0 = (const T*)S.x_in[0];
   for (int i = 0; i < m.L; ++i) {
@@ -723,13 +734,13 @@ int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t*
     TRY(block_fwd_impl<T>(c, i, w.layers[i], (const T*)S.x_in[i], x0, idx, xo, S.saved[i], S.scr, st));
   }
   const T* x_bo = c.backout_layer >= 0 ? (const T*)S.x_in[c.backout_layer] : nullptr;
-  ROWK(nc, norm_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)S.xL, x_bo, w.backout_lambda, (T*)S.hf, S.rstd_f, m.N, m.d,
-                                            c.norm_eps));
+  br_norm_kernel<T><<<brg, brt, 0, st>>>((const T*)S.xL, x_bo, w.backout_lambda, (T*)S.hf, S.rstd_f, m.N, m.d,
+                                            c.norm_eps);
   CKL();
   TRY(lm_head_impl<T>(c, (const T*)S.hf, (const T*)w.w_lm, targets, loss_out, (T*)S.dhf, g.w_lm, S.lm, st));
-  ROWK(nc, final_norm_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>((const T*)S.dhf, (const T*)S.hf, S.rstd_f, x_bo,
+  br_final_norm_bwd_kernel<T><<<brg, brt, 0, st>>>((const T*)S.dhf, (const T*)S.hf, S.rstd_f, x_bo,
                                                       w.backout_lambda, (T*)S.dxA, (T*)S.dx_bo, g.backout_lambda,
-                                                      m.N, m.d));
+                                                      m.N, m.d);
   CKL();
   CK(cudaMemsetAsync(S.dx0, 0, m.N * m.d * 4, st));
   T* cur = (T*)S.dxA;
@@ -740,14 +751,31 @@ int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t*
                           g.layers[i], S.scr, st));
     std::swap(cur, nxt);
   }
-  ROWK(nc, smear_embed_bwd_kernel<T, NC><<<gr, EW_THREADS, 0, st>>>(cur, S.dx0, idx, (const T*)w.wte, (const T*)w.w_smear_gate,
+  br_smear_embed_bwd_kernel<T><<<brg, brt, 0, st>>>(cur, S.dx0, idx, (const T*)w.wte, (const T*)w.w_smear_gate,
                                                        w.smear_lambda, g.wte, g.w_smear_gate, g.smear_lambda, m.B, m.T,
-                                                       m.d, c.smear_ch));
+                                                       m.d, c.smear_ch);
   CKL();
   return GPTB_OK;
 }
 
 }  // namespace
+
+// ------------------------------------------------------ wait self-test ----
+// One CTA waits on an mbarrier that nothing arrives on.  The bounded wait
+// must expire, record ERRW_TIMEOUT_PROBE and let the kernel return.
+__device__ int g_probe_result = -1;
+__global__ void wait_probe_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait_warp(&bar, 0, &abort_flag, ERRW_TIMEOUT_PROBE);
+  if (threadIdx.x == 0) g_probe_result = ok ? 1 : 0;
+}
 
 // ================================================================ C ABI ====
 extern "C" {
@@ -849,6 +877,22 @@ int gptb_device_error(gptb_stream_t stream) {
     return GPTB_ERR_TIMEOUT;
   }
   return GPTB_OK;
+}
+
+int gptb_probe_bounded_wait(unsigned long long limit_ns, gptb_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned long long prev = 0;
+  if (cudaMemcpyFromSymbol(&prev, g_wait_limit_ns, sizeof(prev)) != cudaSuccess) return GPTB_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_wait_limit_ns, &limit_ns, sizeof(limit_ns)) != cudaSuccess) return GPTB_ERR_CUDA;
+  wait_probe_kernel<<<1, 32, 0, st>>>();
+  LAUNCHED();
+  const bool launched = cudaPeekAtLastError() == cudaSuccess;
+  const int rc = launched ? gptb_device_error(stream) : GPTB_ERR_CUDA;
+  cudaMemcpyToSymbol(g_wait_limit_ns, &prev, sizeof(prev));
+  int res = -1;
+  cudaMemcpyFromSymbol(&res, g_probe_result, sizeof(res));
+  if (rc == GPTB_ERR_TIMEOUT && res != 0) return GPTB_ERR_CUDA;  // the kernel must have seen the expiry
+  return rc;
 }
 
 int gptb_set_wait_limit_ns(unsigned long long ns) {

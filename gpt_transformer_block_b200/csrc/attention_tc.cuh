@@ -528,6 +528,22 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       const int tq = q0 + cb * 32;  // first query of this warp's columns
       const bool need_mask = (key > tq) || (k0 + AB2_BK - 1 > tq) || (tq + 32 > T) || (k0 + AB2_BK > T) ||
                              (window >= 0 && tq + 31 - k0 > window);
+      // P^T and dS^T for this warp's 32 queries, packed to bf16 in registers
+      uint32_t pu[16], du[16];
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        float pe[2], de[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int e = e2 * 2 + h2;
+          const int t = tq + e;
+          const bool vis = !need_mask || (t >= q_vis_lo && t <= q_vis_hi);
+          pe[h2] = vis ? fast_exp2(fmaf(__uint_as_float(sv[e]), sl2, -l2[e])) : 0.f;
+          de[h2] = pe[h2] * (__uint_as_float(dv[e]) - Dq[e]) * scale;
+        }
+        pu[e2] = pack_bf16(pe[0], pe[1]);
+        du[e2] = pack_bf16(de[0], de[1]);
+      }
       // the previous step's dV/dK/dQ MMAs must be done reading P^T / dS^T
       if (i > 0) {
         ok = mbar_wait_warp(ds_free, (i - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
@@ -537,24 +553,11 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       uint8_t* drow = sDS + r * 128;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pu[4], du[4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          float pe[2], de[2];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = c * 8 + e2 * 2 + h2;
-            const int t = tq + e;
-            const bool vis = !need_mask || (t >= q_vis_lo && t <= q_vis_hi);
-            pe[h2] = vis ? fast_exp2(fmaf(__uint_as_float(sv[e]), sl2, -l2[e])) : 0.f;
-            de[h2] = pe[h2] * (__uint_as_float(dv[e]) - Dq[e]) * scale;
-          }
-          pu[e2] = pack_bf16(pe[0], pe[1]);
-          du[e2] = pack_bf16(de[0], de[1]);
-        }
         const int cc = cb * 4 + c;  // 16-byte chunk (8 queries) within the 128-byte row
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
-        *reinterpret_cast<uint4*>(drow + ((cc ^ (r & 7)) << 4)) = make_uint4(du[0], du[1], du[2], du[3]);
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(pu[c * 4], pu[c * 4 + 1], pu[c * 4 + 2], pu[c * 4 + 3]);
+        *reinterpret_cast<uint4*>(drow + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(du[c * 4], du[c * 4 + 1], du[c * 4 + 2], du[c * 4 + 3]);
       }
       fence_proxy_async_smem();
       __syncwarp();

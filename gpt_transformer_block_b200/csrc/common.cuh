@@ -28,6 +28,7 @@ enum : int {
   ERRW_TIMEOUT_MMA = 0x102,
   ERRW_TIMEOUT_EPILOGUE = 0x103,
   ERRW_TIMEOUT_DRAIN = 0x104,
+  ERRW_TIMEOUT_PROBE = 0x105,
 };
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_error_word, 0, code); }

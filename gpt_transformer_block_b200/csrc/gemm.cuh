@@ -32,6 +32,8 @@ enum EpiKind : int {
   EPI_RELU2 = 2,      // out = u = alpha*acc, out2 = relu(u)^2 (MLP activation)
   EPI_DRELU2 = 3,     // out = alpha*acc * 2*relu(aux)         (aux = saved u)
   EPI_ACCUM_F32 = 4,  // out(f32) += alpha*acc, atomic          (weight grads)
+  EPI_QKV = 5,        // q,k heads: rope(rmsnorm(acc)) + saved rstd; v heads:
+                      // acc + 3*sigmoid(z) * VE[idx] (value-embedding layers)
 };
 
 struct EpiParams {
@@ -48,6 +50,14 @@ struct EpiParams {
   // (amax_a / 448) * (amax_b / 448), the inverse of the two quantisation scales
   const float* amax_a;
   const float* amax_b;
+  // EPI_QKV: per-head QK RMSNorm + RoPE and the value-embedding add
+  const float2* rope;     // [T, 64] (cos, sin)
+  float* rstd_qk;         // [M, H + Hkv]
+  const bf16* ve_table;   // [V, Hkv*128] or nullptr
+  const int32_t* idx;     // [M] token ids
+  const float* sg;        // [M, Hkv] sigmoid of the gate logits
+  int T, H, Hkv;
+  float eps;
 };
 
 __device__ __forceinline__ float epi_alpha(const EpiParams& ep) {
@@ -148,6 +158,86 @@ __device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, 
   const int r = t - g * per_group;
   tm = first_m + r % gsize;
   tn = r / gsize;
+}
+
+// EPI_QKV for one 128-column head of the tile (one TMEM lane quarter = 32
+// rows, thread = row): q/k heads get the per-head RMSNorm (rstd saved) and the
+// rotation of the pairs (j, j+64) by the row's position; v heads get
+// + 3*sigmoid(z)*VE[idx] on value-embedding layers.  Columns 0..63 go to
+// staging tile stg0, 64..127 to stg1 (32 rows x 128 bytes, 128-byte swizzle).
+__device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, uint32_t ta, uint8_t* stg0, uint8_t* stg1, int lane,
+                                             float alpha, int head, int grow, bool rv) {
+  const int swz = lane & 7;
+  uint8_t* p0 = stg0 + lane * 128;
+  uint8_t* p1 = stg1 + lane * 128;
+  if (head < ep.H + ep.Hkv) {
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(ta + c * 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x = __uint_as_float(v[i]) * alpha;
+        ss = fmaf(x, x, ss);
+      }
+    }
+    const float rr = rsqrtf(ss * (1.f / 128.f) + ep.eps);
+    const float sc = alpha * rr;
+    const float2* cs = ep.rope + (long long)(rv ? grow % ep.T : 0) * 64;
+#pragma unroll
+    for (int j0 = 0; j0 < 64; j0 += 32) {
+      uint32_t a1[32], a2[32];
+      tmem_ld_32x32b_x32(ta + j0, a1);
+      tmem_ld_32x32b_x32(ta + 64 + j0, a2);
+      tmem_ld_wait();
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float y1[8], y2[8];
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const float4 c2 = *reinterpret_cast<const float4*>(cs + j0 + g * 8 + k);  // (cos, sin) of two pairs
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float c = h ? c2.z : c2.x, sn = h ? c2.w : c2.y;
+            const float x1 = __uint_as_float(a1[g * 8 + k + h]) * sc, x2 = __uint_as_float(a2[g * 8 + k + h]) * sc;
+            y1[k + h] = x1 * c - x2 * sn;
+            y2[k + h] = x1 * sn + x2 * c;
+          }
+        }
+        const int chunk = (j0 >> 3) + g;
+        store8(reinterpret_cast<bf16*>(p0 + ((chunk ^ swz) << 4)), y1);
+        store8(reinterpret_cast<bf16*>(p1 + ((chunk ^ swz) << 4)), y2);
+      }
+    }
+    if (rv) ep.rstd_qk[(long long)grow * (ep.H + ep.Hkv) + head] = rr;
+  } else {
+    const int kv = head - ep.H - ep.Hkv;
+    const bool ve = ep.ve_table != nullptr && rv;
+    const float gate = ve ? 3.f * ep.sg[(long long)grow * ep.Hkv + kv] : 0.f;
+    const bf16* e = ve ? ep.ve_table + (long long)ep.idx[grow] * ep.Hkv * 128 + kv * 128 : nullptr;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(ta + c * 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[g * 8 + i]) * alpha;
+        if (ve) {
+          float ev[8];
+          load8(e + c * 32 + g * 8, ev);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[i] = fmaf(gate, ev[i], y[i]);
+        }
+        const int chunk = (c & 1) * 4 + g;
+        store8(reinterpret_cast<bf16*>((c < 2 ? p0 : p1) + ((chunk ^ swz) << 4)), y);
+      }
+    }
+  }
 }
 
 template <bool A_MN, bool B_MN, bool FP8>
@@ -336,8 +426,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
       const int row0 = tm * TC_BM + q * 32;
+      if (ep.kind == EPI_QKV) {
 #pragma unroll 1
-      for (int cc = 0; cc < TC_BN / 64; ++cc) {
+        for (int hb = 0; hb < TC_BN / 128; ++hb) {
+          const int col0 = tn * TC_BN + hb * 128;
+          if (col0 >= N) break;  // warp-uniform
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + hb * 128);
+          epi_qkv_head(ep, ta, stg0, stg1, lane, alpha, col0 / 128, row0 + lane, row0 + lane < M);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmO, stg0, col0, row0);
+            tma_store_2d(&tmO, stg1, col0 + 64, row0);
+            bulk_commit_group();
+          }
+        }
+      }
+#pragma unroll 1
+      for (int cc = 0; cc < (ep.kind == EPI_QKV ? 0 : TC_BN / 64); ++cc) {
         const int col0 = tn * TC_BN + cc * 64;
         if (col0 >= N) break;  // warp-uniform
         uint32_t r0[32], r1[32];

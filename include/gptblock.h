@@ -198,6 +198,13 @@ int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_
  * (the kernel recorded it, drained and returned), or GPTB_ERR_CUDA. */
 int gptb_device_error(gptb_stream_t stream);
 
+/* Self-test of the bounded waits: sets the wait limit to limit_ns, launches
+ * one CTA that waits on an mbarrier nothing ever arrives on, synchronises,
+ * restores the previous limit and returns the device status.  The expected
+ * result is GPTB_ERR_TIMEOUT: the wait expired, the kernel recorded it and
+ * returned, and the context stays usable.  No counterpart on the pages. */
+int gptb_probe_bounded_wait(unsigned long long limit_ns, gptb_stream_t stream);
+
 /* Wait limit (nanoseconds) of every bounded device wait; default 2 s.
  * Applies to kernels launched afterwards on the current device. */
 int gptb_set_wait_limit_ns(unsigned long long ns);

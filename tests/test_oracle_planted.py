@@ -1,0 +1,93 @@
+"""Planted mistakes: each test swaps one oracle function for a version with a
+plausible slip (wrong sign, dropped term, wrong index, wrong scale, wrong
+operand) and checks that at least one of the pins in test_oracle_pins.py /
+test_oracle_fd.py fails on it.  CPU only; nothing here touches the GPU."""
+import numpy as np
+import pytest
+
+from oracle import model as om
+import test_oracle_pins as pins
+import test_oracle_fd as fd
+
+
+def _fails(fn, *args):
+    with pytest.raises(AssertionError):
+        fn(*args)
+
+
+def test_rope_rotation_sign_is_caught(monkeypatch):
+    orig = om.rope
+    monkeypatch.setattr(om, "rope", lambda x, c, s: orig(x, c, -s))
+    _fails(pins.test_rope_head_dim_2_is_textbook_rotation_by_t_radians)
+    _fails(pins.test_block_matches_torch_library_build, 0)
+
+
+def test_rope_pairing_is_caught(monkeypatch):
+    def interleaved(x, cos, sin):  # pairs (2j, 2j+1) instead of (j, j + hd/2)
+        y = x.copy()
+        c, s = cos[None, :, None, :], sin[None, :, None, :]
+        x1, x2 = x[..., 0::2], x[..., 1::2]
+        y[..., 0::2] = x1 * c - x2 * s
+        y[..., 1::2] = x1 * s + x2 * c
+        return y
+    monkeypatch.setattr(om, "rope", interleaved)
+    _fails(pins.test_rope_frequencies_and_pairing)
+
+
+def test_rmsnorm_backward_dropped_term_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "rmsnorm_backward", lambda dy, y, r: r * dy)
+    _fails(pins.test_rmsnorm_backward_matches_torch_autograd)
+    _fails(fd.test_block_gradients_fd, 1)
+
+
+def test_gqa_head_mapping_is_caught(monkeypatch):
+    orig = om.attention_forward
+    # kv head h % Hkv instead of h // (H / Hkv): permute the query heads' kv source
+    def bad(q, k, v, window):
+        H, Hk = q.shape[2], k.shape[2]
+        G = H // Hk
+        perm = [(h % Hk) * G + h // Hk for h in range(H)]
+        o, lse = orig(q[:, :, perm], k, v, window)
+        inv = np.argsort(perm)
+        return o[:, :, inv], lse[:, inv]
+    monkeypatch.setattr(om, "attention_forward", bad)
+    _fails(pins.test_attention_matches_torch_sdpa, 4, 2, 3)
+
+
+def test_softmax_scale_is_caught(monkeypatch):
+    orig = om.attention_forward
+    monkeypatch.setattr(om, "attention_forward", lambda q, k, v, w: orig(q / np.sqrt(q.shape[-1]), k, v, w))
+    _fails(pins.test_attention_matches_torch_sdpa, 4, 4, -1)
+
+
+def test_window_off_by_one_is_caught(monkeypatch):
+    orig = om.visible_mask
+    monkeypatch.setattr(om, "visible_mask", lambda T, w: orig(T, w - 1 if w is not None and w > 0 else w))
+    _fails(pins.test_attention_matches_torch_sdpa, 4, 2, 3)
+
+
+def test_smear_uses_current_token_is_caught(monkeypatch):
+    def bad(x, w_gate, lam):
+        x = np.asarray(x, dtype=np.float64)
+        C = np.asarray(w_gate).shape[0]
+        sg = 1.0 / (1.0 + np.exp(-(x[..., :C] @ np.asarray(w_gate, dtype=np.float64))))
+        y = x.copy()
+        y[:, 1:, :] += lam * sg[:, 1:, None] * x[:, 1:, :]   # current token instead of the previous one
+        return y, sg
+    monkeypatch.setattr(om, "smear_forward", bad)
+    _fails(pins.test_smear_two_token_closed_form)
+
+
+def test_lm_head_transposed_weight_gradient_is_caught(monkeypatch):
+    orig = om.lm_head_xent
+    def bad(h, w, y):
+        loss, dh, dw = orig(h, w, y)
+        return loss, dh, dw[::-1]          # rows of dW_lm attached to the wrong vocabulary entries
+    monkeypatch.setattr(om, "lm_head_xent", bad)
+    _fails(pins.test_xent_closed_form_and_torch)
+
+
+def test_ve_gate_scale_is_caught(monkeypatch):
+    orig = om._sigmoid
+    monkeypatch.setattr(om, "_sigmoid", lambda z: 2.0 * orig(z) / 3.0)   # gate 2*sigmoid instead of 3*sigmoid
+    _fails(pins.test_block_special_cases)
