@@ -318,7 +318,7 @@ namespace gptb {
 //   dV  += P^T dO     (M=128, N=128, K=64 queries)   -> TMEM cols 128..255
 //   dK  += dS^T Q     (M=128, N=128, K=64)           -> TMEM cols   0..127
 //   dQ^T = K^T dS^T   (M=128 hd, N=64, K=128 keys)   -> TMEM cols 384..447
-// Warps: 0 TMA producer (K, V once; Q, dO, LSE, D per step in a 2-stage
+// Warps: 0 TMA producer (K, V once; Q, dO, LSE, D per step in a 3-stage
 // ring), 1 MMA issuer, 2-9 softmax backward (thread = key row, 32 of the 64
 // queries): P^T = exp2(S^T*scale*log2e - LSE*log2e), dS^T = P^T (dP^T - D)/sqrt(hd)
 // written as bf16 into swizzled smem tiles that are both the K-major A
@@ -332,7 +332,9 @@ constexpr int AB2_KV_TILE = 128 * 128 * 2;  // 32 KB
 constexpr int AB2_Q_TILE = 64 * 128 * 2;    // 16 KB
 constexpr int AB2_PS_TILE = 128 * 64 * 2;   // 16 KB
 constexpr int AB2_DQ_STAGE = 64 * 128 * 4;  // 32 KB
-constexpr int AB2_SMEM = 1024 + 2 * AB2_KV_TILE + 4 * AB2_Q_TILE + 2 * AB2_PS_TILE + AB2_DQ_STAGE + 256 + 2 * 2 * 64 * 4;
+constexpr int AB2_STAGES = 3;              // Q / dO / LSE / D ring
+constexpr int AB2_SMEM = 1024 + 2 * AB2_KV_TILE + 2 * AB2_STAGES * AB2_Q_TILE + 2 * AB2_PS_TILE + AB2_DQ_STAGE + 256 +
+                         AB2_STAGES * 2 * 64 * 4;
 
 __global__ void __launch_bounds__(AB2_THREADS, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
@@ -343,26 +345,26 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ab_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + AB2_KV_TILE;
-  uint8_t* sQ = sV + AB2_KV_TILE;        // 2 stages
-  uint8_t* sDO = sQ + 2 * AB2_Q_TILE;    // 2 stages
-  uint8_t* sP = sDO + 2 * AB2_Q_TILE;
+  uint8_t* sQ = sV + AB2_KV_TILE;                  // AB2_STAGES stages
+  uint8_t* sDO = sQ + AB2_STAGES * AB2_Q_TILE;     // AB2_STAGES stages
+  uint8_t* sP = sDO + AB2_STAGES * AB2_Q_TILE;
   uint8_t* sDS = sP + AB2_PS_TILE;
   float* sDQ = reinterpret_cast<float*>(sDS + AB2_PS_TILE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sDQ) + AB2_DQ_STAGE);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qdo_full = bars + 1;   // [2]
-  uint64_t* qdo_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_empty = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* ds_free = bars + 8;
-  uint64_t* dq_full = bars + 9;
-  uint64_t* dq_free = bars + 10;
-  uint64_t* acc_done = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* qdo_full = bars + 1;   // [AB2_STAGES] TMA bytes + one arrival after LSE / D are stored
+  uint64_t* qdo_empty = bars + 4;  // [AB2_STAGES]
+  uint64_t* s_full = bars + 7;
+  uint64_t* s_empty = bars + 8;
+  uint64_t* p_full = bars + 9;
+  uint64_t* ds_free = bars + 10;
+  uint64_t* dq_full = bars + 11;
+  uint64_t* dq_free = bars + 12;
+  uint64_t* acc_done = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* sLD = reinterpret_cast<float*>(bars + 32);  // [2 stages][lse*log2e 64 | D 64]
+  float* sLD = reinterpret_cast<float*>(bars + 32);  // [AB2_STAGES][lse*log2e 64 | D 64]
 
   const int kb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int G = H / Hkv;
@@ -376,8 +378,8 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&qdo_full[i], 1);
+    for (int i = 0; i < AB2_STAGES; ++i) {
+      mbar_init(&qdo_full[i], 2);
       mbar_init(&qdo_empty[i], 1);
     }
     mbar_init(s_full, 1);
@@ -412,19 +414,13 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     }
     bool ok = true;
     for (int i = 0; i < steps && ok; ++i) {
-      const int st = i & 1;
+      const int st = i % AB2_STAGES;
       const int hh = kvh * G + i / nq;
       const int q0 = (qt_lo + i % nq) * AB2_BQ;
-      ok = mbar_wait_warp(&qdo_empty[st], ((i >> 1) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_PRODUCER);
+      ok = mbar_wait_warp(&qdo_empty[st], ((i / AB2_STAGES) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_PRODUCER);
       if (!ok) break;
-      float* ld = sLD + st * 128;
-      for (int e = lane; e < 64; e += 32) {
-        const int t = q0 + e;
-        const long long li = ((long long)b * H + hh) * T + t;
-        ld[e] = (t < T) ? lse[li] * LOG2E : 0.f;
-        ld[64 + e] = (t < T) ? Dd[li] : 0.f;
-      }
-      __syncwarp();
+      // the tile loads go out first; LSE and D (plain loads, guarded at the
+      // sequence end) overlap them and complete the stage with a second arrival
       if (lane == 0) {
         mbar_arrive_expect_tx(&qdo_full[st], 2 * AB2_Q_TILE);
         uint8_t* q = sQ + st * AB2_Q_TILE;
@@ -434,7 +430,15 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
         tma_load_2d(d, &tm_do, &qdo_full[st], hh * 128, row_base + q0);
         tma_load_2d(d + 8192, &tm_do, &qdo_full[st], hh * 128 + 64, row_base + q0);
       }
+      float* ld = sLD + st * 128;
+      for (int e = lane; e < 64; e += 32) {
+        const int t = q0 + e;
+        const long long li = ((long long)b * H + hh) * T + t;
+        ld[e] = (t < T) ? lse[li] * LOG2E : 0.f;
+        ld[64 + e] = (t < T) ? Dd[li] : 0.f;
+      }
       __syncwarp();
+      if (lane == 0) mbar_arrive(&qdo_full[st]);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -445,7 +449,7 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP), aDS = smem_u32(sDS);
       bool ok = mbar_wait(kv_full, 0, abort_flag, ERRW_TIMEOUT_MMA);
       auto grads = [&](int i) -> bool {
-        const int st = i & 1;
+        const int st = i % AB2_STAGES;
         if (!mbar_wait(p_full, i & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
         tc_fence_after();
         const uint32_t aQ = smem_u32(sQ + st * AB2_Q_TILE), aDO = smem_u32(sDO + st * AB2_Q_TILE);
@@ -473,8 +477,8 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
         return true;
       };
       for (int i = 0; ok && i < steps; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(&qdo_full[st], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
+        const int st = i % AB2_STAGES;
+        if (!mbar_wait(&qdo_full[st], (i / AB2_STAGES) & 1, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
         if (!mbar_wait(s_empty, (i & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aQ = smem_u32(sQ + st * AB2_Q_TILE), aDO = smem_u32(sDO + st * AB2_Q_TILE);
@@ -511,7 +515,7 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     const int q_vis_hi = (key < T) ? ((window >= 0) ? min(T - 1, key + window) : T - 1) : -1;
     bool ok = true;
     for (int i = 0; i < steps && ok; ++i) {
-      const int st = i & 1;
+      const int st = i % AB2_STAGES;
       const int q0 = (qt_lo + i % nq) * AB2_BQ;
       ok = mbar_wait_warp(s_full, i & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
       if (!ok) break;

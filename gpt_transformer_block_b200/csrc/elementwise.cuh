@@ -303,7 +303,95 @@ __device__ __forceinline__ void st4(bf16* p, const float (&v)[4]) {
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-__global__ void __launch_bounds__(EW_THREADS)
+// one (token, head) item of the backward: its loads, issued before any compute
+struct QkvBwdItem {
+  long long n;
+  int hh;
+  bool valid;
+  float g[4], y[4], e[4];
+  float2 cs[4];
+  float r, s;
+};
+
+__device__ __forceinline__ void qkv_bwd_load(QkvBwdItem& it, long long item, long long total, int nh, int H, int Hkv,
+                                             int Tn, const bf16* qkv, long long ld, const float* rstd_qk,
+                                             const float2* rope, const float* dq, long long lddq, const float* dk,
+                                             const float* dv, long long lddkv, const bf16* ve_table,
+                                             const int32_t* idx, const float* sg, int lane) {
+  it.valid = item < total;
+  if (!it.valid) return;
+  it.n = item / nh;
+  it.hh = (int)(item - it.n * nh);
+  const long long n = it.n;
+  const int hh = it.hh;
+  if (hh < H + Hkv) {
+    const float* gp = (hh < H) ? dq + n * lddq + (long long)hh * 128 : dk + n * lddkv + (long long)(hh - H) * 128;
+    const float4 g4 = *reinterpret_cast<const float4*>(gp + lane * 4);
+    it.g[0] = g4.x; it.g[1] = g4.y; it.g[2] = g4.z; it.g[3] = g4.w;
+    ld4(qkv + n * ld + (long long)hh * 128 + lane * 4, it.y);
+    const int t = (int)(n % Tn);
+    const float4 c01 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4);
+    const float4 c23 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4 + 2);
+    it.cs[0] = make_float2(c01.x, c01.y);
+    it.cs[1] = make_float2(c01.z, c01.w);
+    it.cs[2] = make_float2(c23.x, c23.y);
+    it.cs[3] = make_float2(c23.z, c23.w);
+    it.r = rstd_qk[n * (H + Hkv) + hh];
+  } else {
+    const int kv = hh - H - Hkv;
+    const float4 g4 = *reinterpret_cast<const float4*>(dv + n * lddkv + (long long)kv * 128 + lane * 4);
+    it.g[0] = g4.x; it.g[1] = g4.y; it.g[2] = g4.z; it.g[3] = g4.w;
+    if (ve_table) {
+      ld4(ve_table + (long long)idx[n] * Hkv * 128 + (long long)kv * 128 + lane * 4, it.e);
+      it.s = sg[n * Hkv + kv];
+    }
+  }
+}
+
+__device__ __forceinline__ void qkv_bwd_compute(const QkvBwdItem& it, int H, int Hkv, bf16* dqkv, long long ld,
+                                                const bf16* ve_table, const int32_t* idx, float* dve_table,
+                                                float* dz, int lane) {
+  if (!it.valid) return;  // warp-uniform: every lane of the warp holds the same item
+  const long long n = it.n;
+  const int hh = it.hh;
+  bf16* out = dqkv + n * ld + (long long)hh * 128 + lane * 4;
+  const bool hi = lane >= 16;
+  if (hh < H + Hkv) {
+    // undo the rotation on the gradient and on the stored (rotated) output:
+    // first half: a1 c + a2 s ; second half: -a1 s + a2 c  (a1 = first-half value)
+    float gu[4], yu[4], dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float go = __shfl_xor_sync(0xffffffffu, it.g[e], 16);
+      const float yo = __shfl_xor_sync(0xffffffffu, it.y[e], 16);
+      const float c = it.cs[e].x, sn = it.cs[e].y;
+      gu[e] = hi ? (it.g[e] * c - go * sn) : (it.g[e] * c + go * sn);
+      yu[e] = hi ? (it.y[e] * c - yo * sn) : (it.y[e] * c + yo * sn);
+      dot = fmaf(gu[e], yu[e], dot);
+    }
+    const float m = warp_sum(dot) * (1.f / 128.f);
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = it.r * (gu[e] - yu[e] * m);
+    st4(out, o);
+  } else {
+    if (ve_table) {
+      const int kv = hh - H - Hkv;
+      const long long row = (long long)idx[n] * Hkv * 128 + (long long)kv * 128 + lane * 4;
+      const float gate = 3.f * it.s;
+      const float dg = warp_sum(it.g[0] * it.e[0] + it.g[1] * it.e[1] + it.g[2] * it.e[2] + it.g[3] * it.e[3]);
+      atomicAdd(reinterpret_cast<float4*>(dve_table + row),
+                make_float4(gate * it.g[0], gate * it.g[1], gate * it.g[2], gate * it.g[3]));
+      if (lane == 0) dz[n * Hkv + kv] = dg * 3.f * it.s * (1.f - it.s);
+    }
+    float o[4] = {it.g[0], it.g[1], it.g[2], it.g[3]};
+    st4(out, o);
+  }
+}
+
+// backward of q,k <- rope(rmsnorm(.)) and of the VE term for hd = 128: one
+// warp per (token, head) item, two items' loads in flight per warp
+__global__ void __launch_bounds__(EW_THREADS, 4)
     qkv_post_bwd_h128_kernel(const bf16* __restrict__ qkv, long long ld, const float* __restrict__ rstd_qk,
                              const float2* __restrict__ rope, const float* __restrict__ dq, long long lddq,
                              const float* __restrict__ dk, const float* __restrict__ dv, long long lddkv,
@@ -312,55 +400,17 @@ __global__ void __launch_bounds__(EW_THREADS)
                              const float* __restrict__ sg, float* __restrict__ dve_table, float* __restrict__ dz) {
   const int lane = threadIdx.x & 31;
   const int nh = H + 2 * Hkv;
-  const bool hi = lane >= 16;
-  const int j0 = (lane & 15) * 4;
-  for (RowLoop it(N * nh); it.row < it.nrows; it.row += it.stride) {
-    const long long n = it.row / nh;
-    const int hh = (int)(it.row - n * nh);
-    bf16* out = dqkv + n * ld + (long long)hh * 128 + lane * 4;
-    if (hh < H + Hkv) {
-      const float* gp = (hh < H) ? dq + n * lddq + (long long)hh * 128 : dk + n * lddkv + (long long)(hh - H) * 128;
-      const float4 g4 = *reinterpret_cast<const float4*>(gp + lane * 4);
-      const float g[4] = {g4.x, g4.y, g4.z, g4.w};
-      float y[4];
-      ld4(qkv + n * ld + (long long)hh * 128 + lane * 4, y);
-      const int t = (int)(n % Tn);
-      const float4 c01 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + j0);
-      const float4 c23 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + j0 + 2);
-      const float cs[4][2] = {{c01.x, c01.y}, {c01.z, c01.w}, {c23.x, c23.y}, {c23.z, c23.w}};
-      // undo the rotation on the gradient and on the stored (rotated) output:
-      // first half: a1 c + a2 s ; second half: -a1 s + a2 c  (a1 = first-half value)
-      float gu[4], yu[4], dot = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float go = __shfl_xor_sync(0xffffffffu, g[e], 16);
-        const float yo = __shfl_xor_sync(0xffffffffu, y[e], 16);
-        gu[e] = hi ? (g[e] * cs[e][0] - go * cs[e][1]) : (g[e] * cs[e][0] + go * cs[e][1]);
-        yu[e] = hi ? (y[e] * cs[e][0] - yo * cs[e][1]) : (y[e] * cs[e][0] + yo * cs[e][1]);
-        dot = fmaf(gu[e], yu[e], dot);
-      }
-      const float m = warp_sum(dot) * (1.f / 128.f);
-      const float r = rstd_qk[n * (H + Hkv) + hh];
-      float o[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = r * (gu[e] - yu[e] * m);
-      st4(out, o);
-    } else {
-      const int kv = hh - H - Hkv;
-      const float4 g4 = *reinterpret_cast<const float4*>(dv + n * lddkv + (long long)kv * 128 + lane * 4);
-      float g[4] = {g4.x, g4.y, g4.z, g4.w};
-      if (ve_table) {
-        const long long row = (long long)idx[n] * Hkv * 128 + (long long)kv * 128 + lane * 4;
-        const float s = sg[n * Hkv + kv];
-        const float gate = 3.f * s;
-        float e[4];
-        ld4(ve_table + row, e);
-        const float dg = warp_sum(g[0] * e[0] + g[1] * e[1] + g[2] * e[2] + g[3] * e[3]);
-        atomicAdd(reinterpret_cast<float4*>(dve_table + row), make_float4(gate * g[0], gate * g[1], gate * g[2], gate * g[3]));
-        if (lane == 0) dz[n * Hkv + kv] = dg * 3.f * s * (1.f - s);
-      }
-      st4(out, g);
-    }
+  const long long total = N * nh;
+  const long long wpb = blockDim.x >> 5;
+  const long long stride = gridDim.x * wpb;
+  for (long long base = blockIdx.x * wpb + (threadIdx.x >> 5); base < total; base += 2 * stride) {
+    QkvBwdItem a, b;
+    qkv_bwd_load(a, base, total, nh, H, Hkv, Tn, qkv, ld, rstd_qk, rope, dq, lddq, dk, dv, lddkv, ve_table, idx, sg,
+                 lane);
+    qkv_bwd_load(b, base + stride, total, nh, H, Hkv, Tn, qkv, ld, rstd_qk, rope, dq, lddq, dk, dv, lddkv, ve_table,
+                 idx, sg, lane);
+    qkv_bwd_compute(a, H, Hkv, dqkv, ld, ve_table, idx, dve_table, dz, lane);
+    qkv_bwd_compute(b, H, Hkv, dqkv, ld, ve_table, idx, dve_table, dz, lane);
   }
 }
 

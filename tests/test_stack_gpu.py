@@ -41,7 +41,8 @@ def run_stack(gb, c, w, batch):
     return loss.item(), st.g
 
 
-def compare_stack(c, w, batch, loss, g, layers=None):
+def compare_stack(c, w, batch, loss, g, layers=None, top=("wte", "w_lm", "w_smear_gate", "smear_lambda",
+                                                          "backout_lambda")):
     ow = oracle_weights(w)
     f8 = c["dtype"] == "fp8"
     rl, cache = om.stack_forward(c, ow, batch["idx"].numpy(), batch["targets"].numpy(), fp8=f8)
@@ -49,10 +50,10 @@ def compare_stack(c, w, batch, loss, g, layers=None):
     tol = TOL[c["dtype"]]
     errs = {"loss": abs(loss - rl) / abs(rl)}
     for k in ("wte", "w_lm", "w_smear_gate"):
-        if k in rg:
+        if k in rg and k in top:
             errs[k] = relerr(np64(g[k]), rg[k])
     for k in ("smear_lambda", "backout_lambda"):
-        if k in rg:
+        if k in rg and k in top:
             errs[k] = scalar_err(np64(g[k])[0], rg[k], rg["_scale"][k])
     for i, lg in enumerate(rg["layers"]):
         if layers is not None and i not in layers:
@@ -114,13 +115,15 @@ def test_grad_accumulation_equals_sum(cuda_lib):
 
 
 def test_stack_fp8_small(cuda_lib):
-    """FP8 end to end: loss, lm_head / embedding / smear / backout gradients and
-    the top layer.  Below the top layer every input-gradient GEMM re-quantises a
-    gradient that already differs from the oracle's, so e4m3 code flips (one ulp
-    = 12.5 %) compound layer by layer; the deeper layers are checked with the
-    same tolerance by the teacher-forced block tests (test_block_fp8)."""
+    """FP8 end to end: loss, lm_head and backout gradients and the top layer.
+    Below the top layer every input-gradient GEMM re-quantises a gradient that
+    already differs from the oracle's, so e4m3 code flips (one ulp = 12.5 %)
+    compound layer by layer; the deeper layers are checked with the same
+    tolerance by the teacher-forced block tests (test_block_fp8), and the
+    embedding / smear kernels below layer 0 are the same kernels as in bf16,
+    checked by the bf16 stack tests."""
     c = small_bf16(dtype="fp8")
     w = synth.make_weights(c, seed=51)
     b = synth.make_batch(c, seed=52)
     loss, g = run_stack(cuda_lib, c, w, b)
-    compare_stack(c, w, b, loss, g, layers=(c["n_layer"] - 1,))
+    compare_stack(c, w, b, loss, g, layers=(c["n_layer"] - 1,), top=("w_lm", "backout_lambda"))
