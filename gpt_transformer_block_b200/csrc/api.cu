@@ -134,6 +134,22 @@ bool make_tmap_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
   return r == CUDA_SUCCESS;
 }
 
+// fp32 [outer2][outer1][inner] view (row stride ld, plane stride ld*outer1), 128-byte swizzle;
+// a store box that runs past outer1 is clipped there (the sequence end)
+bool make_tmap_f32_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer1, uint64_t outer2, uint64_t ld,
+                      uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, outer1, outer2};
+  cuuint64_t strides[2] = {ld * 4, ld * 4 * outer1};
+  cuuint32_t box[3] = {box_inner, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // --------------------------------------------------------------- GEMM ----
@@ -647,16 +663,19 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     CKL();
   } else {
     // tcgen05 flash backward: K/V tiles (128 rows) and Q/dO tiles (64 rows) by
-    // TMA, dQ accumulated with TMA bulk reduce-add into the fp32 buffer
-    CUtensorMap tkv, tq, tdo, tdq;
+    // TMA, dQ accumulated with fp32 reductions at L2 into the zeroed buffer,
+    // dK / dV written whole by TMA stores (every key row of every tile)
+    CUtensorMap tkv, tq, tdo, tdk, tdv;
     bool okm = make_tmap(&tkv, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128);
     okm = okm && make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 64);
     okm = okm && make_tmap(&tdo, X.dO, false, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 64, 64);
-    okm = okm && make_tmap_f32(&tdq, X.dq, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 128, 64, false);
+    okm = okm && make_tmap_f32_3d(&tdk, X.dk, (uint64_t)Kv, (uint64_t)m.T, (uint64_t)m.B, (uint64_t)Kv, 32, 32);
+    okm = okm && make_tmap_f32_3d(&tdv, X.dv, (uint64_t)Kv, (uint64_t)m.T, (uint64_t)m.B, (uint64_t)Kv, 32, 32);
     if (!okm) return GPTB_ERR_CUDA;
     CK(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AB2_SMEM));
-    attn_bwd_tc_kernel<<<dim3((m.T + AB2_BK - 1) / AB2_BK, m.Hkv, m.B), AB2_THREADS, AB2_SMEM, st>>>(
-        tkv, tq, tdo, tdq, S.lse, X.D, X.dk, X.dv, Kv, m.T, m.H, m.Hkv, W);
+    const int nkb = (m.T + AB2_BK - 1) / AB2_BK;
+    attn_bwd_tc_kernel<<<nkb * m.Hkv * m.B, AB2_THREADS, AB2_SMEM, st>>>(tkv, tq, tdo, tdk, tdv, S.lse, X.D, X.dq, Ho,
+                                                                       m.T, m.H, m.Hkv, m.B, W);
     CKL();
   }
   if constexpr (std::is_same<T, bf16>::value) {

@@ -318,55 +318,62 @@ namespace gptb {
 //   dV  += P^T dO     (M=128, N=128, K=64 queries)   -> TMEM cols 128..255
 //   dK  += dS^T Q     (M=128, N=128, K=64)           -> TMEM cols   0..127
 //   dQ^T = K^T dS^T   (M=128 hd, N=64, K=128 keys)   -> TMEM cols 384..447
-// Warps: 0 TMA producer (K, V once; Q, dO, LSE, D per step in a 3-stage
+// Shared-memory bandwidth, not the tensor core, bounds this loop (the
+// N=64 products read 6 KB of operands per 32 MMA cycles), so operands that
+// can stay off shared memory do: P^T and dS^T go to TMEM as bf16 (cols
+// 448..479 and 480..511) and are the A operands of dV / dK, read from TMEM;
+// only dS^T is also written to smem, as the B operand of dQ^T; dQ leaves
+// TMEM straight to L2 as fp32 reductions, without a staging tile.
+// Warps: 0 TMA producer (K, V once; Q, dO, LSE, D per step in a 4-stage
 // ring), 1 MMA issuer, 2-9 softmax backward (thread = key row, 32 of the 64
-// queries): P^T = exp2(S^T*scale*log2e - LSE*log2e), dS^T = P^T (dP^T - D)/sqrt(hd)
-// written as bf16 into swizzled smem tiles that are both the K-major A
-// operand of dV/dK and the MN-major B operand of dQ^T; 10-13 dQ epilogue:
-// thread = hd lane, dQ^T row -> smem [64 q][128 hd] fp32 -> one TMA bulk
-// reduce-add into the fp32 dQ accumulator (no per-element atomics).
-// At the end the softmax warps write dK, dV (fp32) for the CTA's keys.
+// queries): P^T = exp2(S^T*scale*log2e - LSE*log2e), dS^T = P^T (dP^T - D)/sqrt(hd);
+// 10-13 dQ epilogue (thread = hd lane of dQ^T).  At the end the softmax warps
+// write dK, dV (fp32) through swizzled staging tiles in the then idle Q/dO
+// ring and TMA stores that clip at the sequence end.
+// CTAs are numbered key-tile-major so the tiles with the most query tiles
+// (the first ones under a causal mask) start first.
 constexpr int AB2_BK = 128, AB2_BQ = 64;
 constexpr int AB2_THREADS = 448;
 constexpr int AB2_KV_TILE = 128 * 128 * 2;  // 32 KB
 constexpr int AB2_Q_TILE = 64 * 128 * 2;    // 16 KB
 constexpr int AB2_PS_TILE = 128 * 64 * 2;   // 16 KB
-constexpr int AB2_DQ_STAGE = 64 * 128 * 4;  // 32 KB
-constexpr int AB2_STAGES = 3;              // Q / dO / LSE / D ring
-constexpr int AB2_SMEM = 1024 + 2 * AB2_KV_TILE + 2 * AB2_STAGES * AB2_Q_TILE + 2 * AB2_PS_TILE + AB2_DQ_STAGE + 256 +
+constexpr int AB2_STAGES = 4;              // Q / dO / LSE / D ring
+constexpr int AB2_SMEM = 1024 + 2 * AB2_KV_TILE + 2 * AB2_STAGES * AB2_Q_TILE + AB2_PS_TILE + 256 +
                          AB2_STAGES * 2 * 64 * 4;
+// the dK / dV staging (8 warps x 4 tiles of 32 rows x 128 bytes) fits in the Q / dO ring
+static_assert(8 * 4 * 4096 <= 2 * AB2_STAGES * AB2_Q_TILE, "dK/dV staging does not fit the ring");
 
 __global__ void __launch_bounds__(AB2_THREADS, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dq,
-                       const float* __restrict__ lse, const float* __restrict__ Dd, float* __restrict__ dk_out,
-                       float* __restrict__ dv_out, long long lddkv, int T, int H, int Hkv, int window) {
+                       const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dk,
+                       const __grid_constant__ CUtensorMap tm_dv, const float* __restrict__ lse,
+                       const float* __restrict__ Dd, float* __restrict__ dq, long long lddq, int T, int H, int Hkv,
+                       int Bsz, int window) {
   extern __shared__ uint8_t ab_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ab_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + AB2_KV_TILE;
   uint8_t* sQ = sV + AB2_KV_TILE;                  // AB2_STAGES stages
   uint8_t* sDO = sQ + AB2_STAGES * AB2_Q_TILE;     // AB2_STAGES stages
-  uint8_t* sP = sDO + AB2_STAGES * AB2_Q_TILE;
-  uint8_t* sDS = sP + AB2_PS_TILE;
-  float* sDQ = reinterpret_cast<float*>(sDS + AB2_PS_TILE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sDQ) + AB2_DQ_STAGE);
+  uint8_t* sDS = sDO + AB2_STAGES * AB2_Q_TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + AB2_PS_TILE);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qdo_full = bars + 1;   // [AB2_STAGES] TMA bytes + one arrival after LSE / D are stored
-  uint64_t* qdo_empty = bars + 4;  // [AB2_STAGES]
-  uint64_t* s_full = bars + 7;
-  uint64_t* s_empty = bars + 8;
-  uint64_t* p_full = bars + 9;
-  uint64_t* ds_free = bars + 10;
-  uint64_t* dq_full = bars + 11;
-  uint64_t* dq_free = bars + 12;
-  uint64_t* acc_done = bars + 13;
-  uint64_t* drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* qdo_full = bars + 1;                 // [AB2_STAGES] TMA bytes + one arrival after LSE / D are stored
+  uint64_t* qdo_empty = bars + 1 + AB2_STAGES;   // [AB2_STAGES]
+  uint64_t* s_full = bars + 1 + 2 * AB2_STAGES;
+  uint64_t* s_empty = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* ds_free = s_full + 3;
+  uint64_t* dq_full = s_full + 4;
+  uint64_t* dq_free = s_full + 5;
+  uint64_t* acc_done = s_full + 6;
+  uint64_t* drain = s_full + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sLD = reinterpret_cast<float*>(bars + 32);  // [AB2_STAGES][lse*log2e 64 | D 64]
 
-  const int kb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int nkv = Hkv * Bsz;
+  const int kb = blockIdx.x / nkv, kvh = blockIdx.x % Hkv, b = (blockIdx.x % nkv) / Hkv;
   const int G = H / Hkv;
   const int k0 = kb * AB2_BK;
   const int row_base = b * T;
@@ -395,7 +402,8 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     tma_prefetch_desc(&tm_kv);
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_do);
-    tma_prefetch_desc(&tm_dq);
+    tma_prefetch_desc(&tm_dk);
+    tma_prefetch_desc(&tm_dv);
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -444,9 +452,9 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_S = make_idesc(128, 64, false, false, false);   // S^T, dP^T
-      constexpr uint32_t ID_G = make_idesc(128, 128, false, true, false);   // dV, dK
+      constexpr uint32_t ID_G = make_idesc(128, 128, false, true, false);   // dV, dK (A from TMEM)
       constexpr uint32_t ID_Q = make_idesc(128, 64, true, true, false);     // dQ^T
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP), aDS = smem_u32(sDS);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS);
       bool ok = mbar_wait(kv_full, 0, abort_flag, ERRW_TIMEOUT_MMA);
       auto grads = [&](int i) -> bool {
         const int st = i % AB2_STAGES;
@@ -456,12 +464,10 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          // A: P^T / dS^T tile (128 key rows x 64 queries, K-major, one 128-byte K block)
+          // A: P^T / dS^T in TMEM (lane = key, 8 columns per 16 queries)
           // B: dO / Q as MN-major (hd halves 8 KB apart), K step = 16 query rows
-          mma_bf16_ss(tmem + 128, smem_desc_sw128(aP + k * 32, 16, 1024), smem_desc_sw128(aDO + k * 2048, 8192, 1024),
-                      ID_G, acc);
-          mma_bf16_ss(tmem + 0, smem_desc_sw128(aDS + k * 32, 16, 1024), smem_desc_sw128(aQ + k * 2048, 8192, 1024),
-                      ID_G, acc);
+          mma_bf16_ts(tmem + 128, tmem + 448 + k * 8, smem_desc_sw128(aDO + k * 2048, 8192, 1024), ID_G, acc);
+          mma_bf16_ts(tmem + 0, tmem + 480 + k * 8, smem_desc_sw128(aQ + k * 2048, 8192, 1024), ID_G, acc);
         }
         if (!mbar_wait(dq_free, (i & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) return false;
         tc_fence_after();
@@ -520,80 +526,110 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       ok = mbar_wait_warp(s_full, i & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[32], dv[32];
-      tmem_ld_32x32b_x32(lane_addr + 256 + cb * 32, sv);
-      tmem_ld_32x32b_x32(lane_addr + 320 + cb * 32, dv);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty);
-      const float* l2 = sLD + st * 128 + cb * 32;
-      const float* Dq = sLD + st * 128 + 64 + cb * 32;
       const int tq = q0 + cb * 32;  // first query of this warp's columns
       const bool need_mask = (key > tq) || (k0 + AB2_BK - 1 > tq) || (tq + 32 > T) || (k0 + AB2_BK > T) ||
                              (window >= 0 && tq + 31 - k0 > window);
-      // P^T and dS^T for this warp's 32 queries, packed to bf16 in registers
+      const float4* l2v = reinterpret_cast<const float4*>(sLD + st * 128 + cb * 32);
+      const float4* ddv = reinterpret_cast<const float4*>(sLD + st * 128 + 64 + cb * 32);
+      // P^T and dS^T for this warp's 32 queries, packed to bf16 pairs (query
+      // 2j in the low half), in two halves of 16 queries
       uint32_t pu[16], du[16];
 #pragma unroll
-      for (int e2 = 0; e2 < 16; ++e2) {
-        float pe[2], de[2];
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sv[16], dv[16];
+        tmem_ld_32x32b_x16(lane_addr + 256 + cb * 32 + hf * 16, sv);
+        tmem_ld_32x32b_x16(lane_addr + 320 + cb * 32 + hf * 16, dv);
+        float l2[16], dd[16];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int e = e2 * 2 + h2;
-          const int t = tq + e;
-          const bool vis = !need_mask || (t >= q_vis_lo && t <= q_vis_hi);
-          pe[h2] = vis ? fast_exp2(fmaf(__uint_as_float(sv[e]), sl2, -l2[e])) : 0.f;
-          de[h2] = pe[h2] * (__uint_as_float(dv[e]) - Dq[e]) * scale;
+        for (int g = 0; g < 4; ++g) {
+          const float4 a = l2v[hf * 4 + g], d = ddv[hf * 4 + g];
+          l2[g * 4] = a.x; l2[g * 4 + 1] = a.y; l2[g * 4 + 2] = a.z; l2[g * 4 + 3] = a.w;
+          dd[g * 4] = d.x; dd[g * 4 + 1] = d.y; dd[g * 4 + 2] = d.z; dd[g * 4 + 3] = d.w;
         }
-        pu[e2] = pack_bf16(pe[0], pe[1]);
-        du[e2] = pack_bf16(de[0], de[1]);
+        tmem_ld_wait();
+        if (hf == 1) {
+          // S^T / dP^T are in registers: the next step's products may overwrite them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_empty);
+        }
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          float pe[2], de[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = e2 * 2 + h2;
+            const int t = tq + hf * 16 + e;
+            const bool vis = !need_mask || (t >= q_vis_lo && t <= q_vis_hi);
+            pe[h2] = vis ? fast_exp2(fmaf(__uint_as_float(sv[e]), sl2, -l2[e])) : 0.f;
+            de[h2] = pe[h2] * (__uint_as_float(dv[e]) - dd[e]) * scale;
+          }
+          pu[hf * 8 + e2] = pack_bf16(pe[0], pe[1]);
+          du[hf * 8 + e2] = pack_bf16(de[0], de[1]);
+        }
       }
       // the previous step's dV/dK/dQ MMAs must be done reading P^T / dS^T
       if (i > 0) {
         ok = mbar_wait_warp(ds_free, (i - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
         if (!ok) break;
+        tc_fence_after();
       }
-      uint8_t* prow = sP + r * 128;
+      tmem_st_32x32b_x16(lane_addr + 448 + cb * 16, pu);
+      tmem_st_32x32b_x16(lane_addr + 480 + cb * 16, du);
       uint8_t* drow = sDS + r * 128;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int cc = cb * 4 + c;  // 16-byte chunk (8 queries) within the 128-byte row
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(pu[c * 4], pu[c * 4 + 1], pu[c * 4 + 2], pu[c * 4 + 3]);
         *reinterpret_cast<uint4*>(drow + ((cc ^ (r & 7)) << 4)) =
             make_uint4(du[c * 4], du[c * 4 + 1], du[c * 4 + 2], du[c * 4 + 3]);
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // dK, dV rows (fp32) for this CTA's keys: columns cb*64 .. cb*64+63
+    // dK, dV rows (fp32) for this CTA's keys, columns cb*64 .. cb*64+63, through
+    // four 32x32 swizzled staging tiles per warp in the (now idle) Q/dO ring
     if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(acc_done, 0, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
       tc_fence_after();
+      uint8_t* stg = sQ + (warp - 2) * 4 * 4096;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        float* dst = (which == 0 ? dk_out : dv_out) + ((long long)row_base + key) * lddkv + kvh * 128 + cb * 64;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(lane_addr + which * 128 + cb * 64 + c * 32, v);
           tmem_ld_wait();
-          if (key < T) {
+          uint8_t* prow = stg + (which * 2 + c) * 4096 + lane * 128;
 #pragma unroll
-            for (int g = 0; g < 8; ++g)
-              *reinterpret_cast<float4*>(dst + c * 32 + g * 4) =
-                  make_float4(__uint_as_float(v[g * 4]), __uint_as_float(v[g * 4 + 1]), __uint_as_float(v[g * 4 + 2]),
-                              __uint_as_float(v[g * 4 + 3]));
-          }
+          for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<float4*>(prow + ((g ^ (lane & 7)) << 4)) =
+                make_float4(__uint_as_float(v[g * 4]), __uint_as_float(v[g * 4 + 1]), __uint_as_float(v[g * 4 + 2]),
+                            __uint_as_float(v[g * 4 + 3]));
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && k0 + qw * 32 < T) {  // (a box wholly past the sequence end is not issued)
+#pragma unroll
+        for (int which = 0; which < 2; ++which)
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            tma_store_3d(which == 0 ? &tm_dk : &tm_dv, stg + (which * 2 + c) * 4096, kvh * 128 + cb * 64 + c * 32,
+                         k0 + qw * 32, b);
+        bulk_commit_group();
+        bulk_wait0();
+      }
+      __syncwarp();
     }
   } else {
     // ------------------------------------------------------- dQ epilogue
+    // thread = hd column of dQ; each of the 64 query rows is one coalesced
+    // 128-byte fp32 reduction per warp
     const int qw = warp & 3;
-    const int hdl = qw * 32 + lane;  // hd column this thread holds
+    const int hdl = qw * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
-    const bool issuer = (warp == 10 && lane == 0);
     bool ok = true;
     for (int i = 0; i < steps; ++i) {
       const int hh = kvh * G + i / nq;
@@ -609,23 +645,17 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
-      // staging buffer: the previous reduction must have finished reading it
-      if (issuer) bulk_wait_read0();
-      named_bar_sync(2, 128);
       if (ok) {
+        float* dst = dq + (long long)(row_base + q0) * lddq + hh * 128 + hdl;
+        const int nv = T - q0;  // query rows of this tile inside the sequence
 #pragma unroll
-        for (int q = 0; q < 32; ++q) sDQ[q * 128 + hdl] = __uint_as_float(v0[q]);
+        for (int q = 0; q < 32; ++q)
+          if (q < nv) red_add_f32(dst + (long long)q * lddq, __uint_as_float(v0[q]));
 #pragma unroll
-        for (int q = 0; q < 32; ++q) sDQ[(32 + q) * 128 + hdl] = __uint_as_float(v1[q]);
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(2, 128);
-      if (issuer && ok) {
-        tma_reduce_add_2d(&tm_dq, sDQ, hh * 128, row_base + q0);
-        bulk_commit_group();
+        for (int q = 0; q < 32; ++q)
+          if (32 + q < nv) red_add_f32(dst + (long long)(32 + q) * lddq, __uint_as_float(v1[q]));
       }
     }
-    if (issuer) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
