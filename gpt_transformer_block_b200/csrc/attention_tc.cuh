@@ -625,10 +625,12 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------- dQ epilogue
-    // thread = hd column of dQ; each of the 64 query rows is one coalesced
-    // 128-byte fp32 reduction per warp
+    // TMEM gives each thread one hd column of dQ^T (64 queries).  A 4x4
+    // transpose among each group of 4 lanes (two butterfly stages of
+    // shuffles) turns that into 4 consecutive hd values of one query, so one
+    // 16-byte fp32 reduction per thread covers 4 rows x 128 bytes per warp:
+    // a quarter of the reduction instructions of one-float-per-lane.
     const int qw = warp & 3;
-    const int hdl = qw * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
     bool ok = true;
     for (int i = 0; i < steps; ++i) {
@@ -646,14 +648,28 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
       if (ok) {
-        float* dst = dq + (long long)(row_base + q0) * lddq + hh * 128 + hdl;
+        const int m4 = lane & 3;
+        const bool b1 = (m4 & 2) != 0, b0 = (m4 & 1) != 0;
         const int nv = T - q0;  // query rows of this tile inside the sequence
+        float* dst = dq + (long long)(row_base + q0 + m4) * lddq + hh * 128 + qw * 32 + (lane & ~3);
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (q < nv) red_add_f32(dst + (long long)q * lddq, __uint_as_float(v0[q]));
+        for (int qb = 0; qb < 16; ++qb) {
+          // a[j]: query 4qb+j at this lane's hd  ->  a[j]: query 4qb+m4 at hd (lane&~3)+j
+          float a[4];
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (32 + q < nv) red_add_f32(dst + (long long)(32 + q) * lddq, __uint_as_float(v1[q]));
+          for (int j = 0; j < 4; ++j) a[j] = __uint_as_float(qb < 8 ? v0[qb * 4 + j] : v1[(qb - 8) * 4 + j]);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {  // swap the off-diagonal 2x2 blocks (lane bit 1)
+            const float y = __shfl_xor_sync(0xffffffffu, b1 ? a[t] : a[2 + t], 2);
+            if (b1) a[t] = y; else a[2 + t] = y;
+          }
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {  // transpose inside each 2x2 block (lane bit 0)
+            const float y = __shfl_xor_sync(0xffffffffu, b0 ? a[2 * t] : a[2 * t + 1], 1);
+            if (b0) a[2 * t] = y; else a[2 * t + 1] = y;
+          }
+          if (4 * qb + m4 < nv) red_add_v4_f32(dst + (long long)(4 * qb) * lddq, a[0], a[1], a[2], a[3]);
+        }
       }
     }
   }
