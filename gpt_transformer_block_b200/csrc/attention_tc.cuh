@@ -327,13 +327,15 @@ namespace gptb {
 // Warps: 0 TMA producer (K, V once; Q, dO, LSE, D per step in a 4-stage
 // ring), 1 MMA issuer, 2-9 softmax backward (thread = key row, 32 of the 64
 // queries): P^T = exp2(S^T*scale*log2e - LSE*log2e), dS^T = P^T (dP^T - D)/sqrt(hd);
-// 10-13 dQ epilogue (thread = hd lane of dQ^T).  At the end the softmax warps
+// 10-17 dQ epilogue (thread = hd lane of dQ^T, 32 of the 64 queries; two
+// warps per TMEM lane quarter, as the reductions are bound by how many
+// requests each warp keeps in flight).  At the end the softmax warps
 // write dK, dV (fp32) through swizzled staging tiles in the then idle Q/dO
 // ring and TMA stores that clip at the sequence end.
 // CTAs are numbered key-tile-major so the tiles with the most query tiles
 // (the first ones under a causal mask) start first.
 constexpr int AB2_BK = 128, AB2_BQ = 64;
-constexpr int AB2_THREADS = 448;
+constexpr int AB2_THREADS = 576;
 constexpr int AB2_KV_TILE = 128 * 128 * 2;  // 32 KB
 constexpr int AB2_Q_TILE = 64 * 128 * 2;    // 16 KB
 constexpr int AB2_PS_TILE = 128 * 64 * 2;   // 16 KB
@@ -394,7 +396,7 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     mbar_init(p_full, 8);
     mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 4);
+    mbar_init(dq_free, 8);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -631,17 +633,17 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
     // 16-byte fp32 reduction per thread covers 4 rows x 128 bytes per warp:
     // a quarter of the reduction instructions of one-float-per-lane.
     const int qw = warp & 3;
+    const int qh = (warp - 10) >> 2;  // queries qh*32 .. qh*32+31 of the tile
     const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
     bool ok = true;
     for (int i = 0; i < steps; ++i) {
       const int hh = kvh * G + i / nq;
       const int q0 = (qt_lo + i % nq) * AB2_BQ;
       ok = ok && mbar_wait_warp(dq_full, i & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
-      uint32_t v0[32], v1[32];
+      uint32_t v0[32];
       if (ok) {
         tc_fence_after();
-        tmem_ld_32x32b_x32(lane_addr + 384, v0);
-        tmem_ld_32x32b_x32(lane_addr + 416, v1);
+        tmem_ld_32x32b_x32(lane_addr + 384 + qh * 32, v0);
         tmem_ld_wait();
         tc_fence_before();
       }
@@ -650,14 +652,14 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       if (ok) {
         const int m4 = lane & 3;
         const bool b1 = (m4 & 2) != 0, b0 = (m4 & 1) != 0;
-        const int nv = T - q0;  // query rows of this tile inside the sequence
-        float* dst = dq + (long long)(row_base + q0 + m4) * lddq + hh * 128 + qw * 32 + (lane & ~3);
+        const int nv = T - q0 - qh * 32;  // query rows of this half inside the sequence
+        float* dst = dq + (long long)(row_base + q0 + qh * 32 + m4) * lddq + hh * 128 + qw * 32 + (lane & ~3);
 #pragma unroll
-        for (int qb = 0; qb < 16; ++qb) {
+        for (int qb = 0; qb < 8; ++qb) {
           // a[j]: query 4qb+j at this lane's hd  ->  a[j]: query 4qb+m4 at hd (lane&~3)+j
           float a[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) a[j] = __uint_as_float(qb < 8 ? v0[qb * 4 + j] : v1[(qb - 8) * 4 + j]);
+          for (int j = 0; j < 4; ++j) a[j] = __uint_as_float(v0[qb * 4 + j]);
 #pragma unroll
           for (int t = 0; t < 2; ++t) {  // swap the off-diagonal 2x2 blocks (lane bit 1)
             const float y = __shfl_xor_sync(0xffffffffu, b1 ? a[t] : a[2 + t], 2);
