@@ -9,8 +9,9 @@
 //   warp 1    TMEM owner + single-thread MMA issuer:
 //               S_j = Q K_j^T   (M=128, N=128, K=128) into one of two TMEM
 //                               score buffers (columns 0..127 / 128..255)
-//               O  += P_j V_j   (M=128, N=128, K=128; V as MN-major operand)
-//                               into TMEM columns 256..383
+//               O  += P_j V_j   (M=128, N=128, K=128; P read from TMEM,
+//                               V as MN-major smem operand) into TMEM
+//                               columns 256..383
 //             S_{j+1} is issued before O += P_j V_j so the scores of the next
 //             tile are ready when the softmax finishes the current one.
 //   warps 2-9 softmax: two warps per TMEM lane quarter; thread = one query
@@ -20,8 +21,10 @@
 //             rescales O in TMEM only when the max grows by more than 8 (a
 //             factor 256; P stays below 256 in bf16 and the final
 //             normalisation uses the same max, so the result is exact), writes
-//             P (bf16) into a swizzled smem tile for the PV MMA, and at the end
-//             normalises its half of O and writes o and the LSE.
+//             P (bf16 pairs) into one of two TMEM buffers (columns 384..447 /
+//             448..511), the A operand of the PV MMA, so P costs no shared-
+//             memory bandwidth, and at the end normalises its half of O and
+//             writes o and the LSE.
 // Only key tiles that intersect [q0 - W, q0 + 127] are visited.
 #pragma once
 #include "common.cuh"
@@ -32,7 +35,7 @@ constexpr int FA_BM = 128, FA_BN = 128;
 constexpr int FA_THREADS = 320;
 constexpr int FA_SOFTMAX_THREADS = 256;
 constexpr int FA_TILE = 128 * 128 * 2;  // one 128x128 bf16 tile: 32 KB (two 64-column swizzled halves)
-constexpr int FA_SMEM = 1024 /*align*/ + FA_TILE /*Q*/ + 4 * FA_TILE /*K,V x2*/ + FA_TILE /*P*/ + 256 /*barriers*/ +
+constexpr int FA_SMEM = 1024 /*align*/ + FA_TILE /*Q*/ + 4 * FA_TILE /*K,V x2*/ + 256 /*barriers*/ +
                         2 * 2 * 128 * 4 /*row max exchange, 2 tiles in flight*/ + 2 * 128 * 4 /*row sums*/;
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -58,19 +61,18 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + FA_TILE;          // 2 stages
   uint8_t* sV = sK + 2 * FA_TILE;      // 2 stages
-  uint8_t* sP = sV + 2 * FA_TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + FA_TILE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * FA_TILE);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]  K ring: a slot is free once S_j = Q K_j^T is done
   uint64_t* k_empty = bars + 3;   // [2]
   uint64_t* s_full = bars + 5;    // [2]
   uint64_t* s_empty = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* pv_done = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint64_t* v_full = bars + 12;   // [2]  V ring: a slot is free once O += P_j V_j is done
-  uint64_t* v_empty = bars + 14;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* p_full = bars + 9;    // [2]  P buffer j&1 written
+  uint64_t* pv_done = bars + 11;  // [2]  O += P_j V_j done (P buffer j&1 free again)
+  uint64_t* drain = bars + 13;
+  uint64_t* v_full = bars + 14;   // [2]  V ring: a slot is free once O += P_j V_j is done
+  uint64_t* v_empty = bars + 16;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xmax = reinterpret_cast<float*>(bars + 32);  // [2 tile parities][2 halves][128 rows] (after 256 B of barriers)
   float* xsum = xmax + 2 * 2 * 128;                   // [2 halves][128 rows]
@@ -95,9 +97,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 8);
+      mbar_init(&p_full[i], 8);
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_full, 8);
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -134,16 +136,19 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = make_idesc(128, 128, false, false, false);
       constexpr uint32_t IDESC_O = make_idesc(128, 128, false, true, false);
-      const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP);
+      const uint32_t aQ = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, abort_flag, ERRW_TIMEOUT_MMA);
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
-        if (!mbar_wait(p_full, i & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
         tc_fence_after();
         const uint32_t aV = smem_u32(sV + (i & 1) * FA_TILE);
+        // A = P_i from TMEM (lane = query row, 8 columns per 16 keys)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mma_bf16_ss(tmem + 256, fa_desc_k(aP, k), fa_desc_mn(aV, k), IDESC_O, (i > 0 || k > 0) ? 1u : 0u);
-        mma_commit(pv_done);
+        for (int k = 0; k < 8; ++k)
+          mma_bf16_ts(tmem + 256, tmem + 384 + (i & 1) * 64 + k * 8, fa_desc_mn(aV, k), IDESC_O,
+                      (i > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&pv_done[i & 1]);
         mma_commit(&v_empty[i & 1]);
         return true;
       };
@@ -216,8 +221,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       xm[hf * 128 + r] = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
       named_bar_sync(1, FA_SOFTMAX_THREADS);
       const float mx = fmaxf(xm[r], xm[128 + r]) * sl2;
-      // the previous PV product must be done before P is overwritten or O rescaled
-      if (j > 0) ok = ok && mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+      // P buffer j&1 was last read by the PV product of tile j-2
+      if (j > 1) ok = ok && mbar_wait_warp(&pv_done[sb], ((j >> 1) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_EPILOGUE);
       if (!ok) continue;
       // rescale decision is per row (identical in both halves) but the TMEM
       // accesses are warp-collective: the whole warp enters, rows that keep
@@ -226,6 +231,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       if (__any_sync(0xffffffffu, grow)) {
         const float corr = grow ? fast_exp2(m_used - mx) : 1.f;  // 0 when m_used is -inf
         if (j > 0) {
+          // O may only be rescaled once every issued PV product (up to tile j-1) is done
+          ok = mbar_wait_warp(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+          if (!ok) continue;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -244,36 +252,31 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      // pass 2: P = exp2(s*scale - m) (bf16) into K-block hf of the K-major
-      // swizzled P tile; 16-byte chunk cc of row r sits at cc ^ (r & 7)
-      uint8_t* prow = sP + hf * 16384 + r * 128;
+      // pass 2: P = exp2(s*scale - m) as bf16 pairs (key 2c in the low half)
+      // into TMEM columns 384 + 64*(j&1) + 32*hf .. +31 of this row's lane
+      uint32_t pk[32];
       float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = fast_exp2(fmaf(__uint_as_float(v[cc * 8 + e]), sl2, -mu));  // exp2(-inf) = 0 for masked keys
-          lp[e & 3] += p[e];
-        }
-        uint4 u;
-        u.x = pack_bf16(p[0], p[1]);
-        u.y = pack_bf16(p[2], p[3]);
-        u.z = pack_bf16(p[4], p[5]);
-        u.w = pack_bf16(p[6], p[7]);
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = u;
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * c]), sl2, -mu));  // exp2(-inf) = 0 for masked keys
+        const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * c + 1]), sl2, -mu));
+        lp[(2 * c) & 3] += p0;
+        lp[(2 * c + 1) & 3] += p1;
+        pk[c] = pack_bf16(p0, p1);
       }
       l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-      // P visible to the tensor core
-      fence_proxy_async_smem();
+      tmem_st_32x32b_x32(lane_addr + 384 + sb * 64 + hf * 32, pk);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[sb]);
     }
     // the two halves' sums share the same running max: add them
     xsum[hf * 128 + r] = l;
     named_bar_sync(1, FA_SOFTMAX_THREADS);
     const float lt = xsum[r] + xsum[128 + r];
-    if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(pv_done, (ntiles - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
+    if (__all_sync(0xffffffffu, ok) &&
+        mbar_wait_warp(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
       tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       bf16* orow = o + ((long long)b * T + t) * ldo + h * 128 + hf * 64;
