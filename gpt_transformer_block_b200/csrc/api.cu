@@ -225,8 +225,10 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
     const int align = f8 ? 16 : 8;  // row strides must be multiples of 16 bytes
     const uint32_t bk = f8 ? 128 : 64;
     const bool acc32 = ep.kind == EPI_ACCUM_F32;
-    const bool has_aux = ep.kind == EPI_RESID || ep.kind == EPI_DRELU2;
-    if (ep.out_f32 && !acc32) return GPTB_ERR_UNSUPPORTED;  // tensor-core outputs are bf16 or fp32 accumulations
+    const bool has_aux = ep.kind == EPI_RESID || ep.kind == EPI_DRELU2 || ep.kind == EPI_DOT;
+    if (ep.out_f32 && !acc32) return GPTB_ERR_UNSUPPORTED;
+    // a row's groups of 128 columns must lie inside one N tile
+    if (ep.kind == EPI_DOT && (N % 128 || !ep.rowdot || ep.T <= 0 || M % ep.T)) return GPTB_ERR_INVALID_ARG;  // tensor-core outputs are bf16 or fp32 accumulations
     if (!aligned16(A.p) || !aligned16(B.p) || !aligned16(ep.out) || (A.ld % align) || (B.ld % align) ||
         (ep.ldo % (acc32 ? 4 : 8)) || (N % 8))
       return GPTB_ERR_INVALID_ARG;
@@ -289,6 +291,7 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
   e.sg = nullptr;
   e.T = e.H = e.Hkv = 0;
   e.eps = 0.f;
+  e.rowdot = nullptr;
   return e;
 }
 EpiParams epi8(EpiParams e, const float* amax_a, const float* amax_b) {
@@ -640,18 +643,22 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   // attention output projection
   TRY(proj<T>(c, {X.dx1, m.d, true, 0, nullptr, nullptr, false}, {S.o, Ho, true, 0, nullptr, nullptr, false}, m.d,
               (int)Ho, N, epi(EPI_ACCUM_F32, dt, g.w_o, Ho), st));
-  TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
-              (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
-  // attention
+  // dO = dx1 Wo, and the attention backward's D = rowsum(dO * o) per head
   if constexpr (std::is_same<T, bf16>::value) {
-    attn_bwd_pre_h128_kernel<<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const bf16*)S.o, Ho, (const bf16*)X.dO, Ho,
-                                                                        X.D, m.T, m.N, m.H);
+    // bf16 / FP8 configurations: D comes out of the dO GEMM's epilogue (o read by TMA)
+    EpiParams ed = epi(EPI_DOT, dt, X.dO, Ho, S.o, Ho);
+    ed.rowdot = X.D;
+    ed.T = m.T;
+    ed.H = m.H;
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+                (int)Ho, m.d, ed, st));
   } else {
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+                (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
     attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
                                                                        m.B, m.T, m.H, m.hd);
-  
+    CKL();
   }
-  CKL();
   CK(cudaMemsetAsync(X.dq, 0, m.N * Ho * 4, st));
   const int W = c.window[layer];
   if (dt == GPTB_F32) {

@@ -416,26 +416,3 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
 
 }  // namespace gptb
 
-namespace gptb {
-
-// D[b,h,t] = sum_c dO[t,h,c] * o[t,h,c] for hd = 128: one warp per (token, head),
-// 8-byte loads per lane
-__global__ void __launch_bounds__(EW_THREADS)
-    attn_bwd_pre_h128_kernel(const bf16* __restrict__ o, long long ldo, const bf16* __restrict__ dO, long long lddo,
-                             float* __restrict__ D, int Tn, long long N, int H) {
-  const int lane = threadIdx.x & 31;
-  for (RowLoop it(N * H); it.row < it.nrows; it.row += it.stride) {
-    const long long n = it.row / H;
-    const int h = (int)(it.row - n * H);
-    float a[4], g[4];
-    ld4(o + n * ldo + (long long)h * 128 + lane * 4, a);
-    ld4(dO + n * lddo + (long long)h * 128 + lane * 4, g);
-    const float s = warp_sum(a[0] * g[0] + a[1] * g[1] + a[2] * g[2] + a[3] * g[3]);
-    if (lane == 0) {
-      const long long b = n / Tn, t = n - b * Tn;
-      D[(b * H + h) * Tn + t] = s;
-    }
-  }
-}
-
-}  // namespace gptb

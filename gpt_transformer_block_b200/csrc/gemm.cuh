@@ -34,6 +34,9 @@ enum EpiKind : int {
   EPI_ACCUM_F32 = 4,  // out(f32) += alpha*acc, atomic          (weight grads)
   EPI_QKV = 5,        // q,k heads: rope(rmsnorm(acc)) + saved rstd; v heads:
                       // acc + 3*sigmoid(z) * VE[idx] (value-embedding layers)
+  EPI_DOT = 6,        // out = alpha*acc (bf16) and, per row and 128-column
+                      // group h, rowdot[b, h, t] = sum(out * aux) (aux = the
+                      // attention output o, out = dO: the backward's D term)
 };
 
 struct EpiParams {
@@ -58,6 +61,7 @@ struct EpiParams {
   const float* sg;        // [M, Hkv] sigmoid of the gate logits
   int T, H, Hkv;
   float eps;
+  float* rowdot;          // EPI_DOT: [B, H, T] fp32
 };
 
 __device__ __forceinline__ float epi_alpha(const EpiParams& ep) {
@@ -413,7 +417,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint8_t* stg1 = stg0 + 4096;
     uint64_t* abar = &aux_bar[warp - 2];
     uint32_t aphase = 0;
-    const bool has_aux = (ep.kind == EPI_RESID || ep.kind == EPI_DRELU2);
+    const bool has_aux = (ep.kind == EPI_RESID || ep.kind == EPI_DRELU2 || ep.kind == EPI_DOT);
     const bool acc32 = (ep.kind == EPI_ACCUM_F32);
     const int swz = (lane & 7);  // 16-byte chunk swizzle of this lane's 128-byte staging row
     int acc = 0;
@@ -444,6 +448,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
       }
+      float dsum = 0.f;  // EPI_DOT: this row's running sum over the current 128-column group
 #pragma unroll 1
       for (int cc = 0; cc < (ep.kind == EPI_QKV ? 0 : TC_BN / 64); ++cc) {
         const int col0 = tn * TC_BN + cc * 64;
@@ -495,9 +500,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               if (ep.kind == EPI_RESID) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] += a[i];
-              } else {
+              } else if (ep.kind == EPI_DRELU2) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] *= 2.f * fmaxf(a[i], 0.f);
+              } else {
+                // the dot takes the values as stored (rounded to bf16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dsum = fmaf(__bfloat162float(__float2bfloat16_rn(v[i])), a[i], dsum);
               }
             }
             store8(reinterpret_cast<bf16*>(cp0), v);
@@ -510,6 +519,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               store8(reinterpret_cast<bf16*>(cp1), v);
             }
           }
+        }
+        if (ep.kind == EPI_DOT && (cc & 1)) {  // a 128-column group (one head) is complete
+          const int row = row0 + lane;
+          if (row < M) {
+            const int bb = row / ep.T, t = row - bb * ep.T;
+            ep.rowdot[((long long)bb * ep.H + col0 / 128) * ep.T + t] = dsum;
+          }
+          dsum = 0.f;
         }
         fence_proxy_async_smem();
         __syncwarp();

@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(256)
                        T* __restrict__ xm_out, T* __restrict__ h_out, float* __restrict__ rstd_out, long long N, int d,
                        float eps, const T* __restrict__ w_gate, float* __restrict__ sg_out, int Hkv, int Cg) {
   __shared__ float sh[2 * BR_MAX_WARPS];
+  __shared__ float hg[256];  // the gate's input channels of the current row
   const BRow r(d);
   const float a = lam[0], b = lam[1];
   for (long long n = blockIdx.x; n < N; n += gridDim.x) {
@@ -134,17 +135,21 @@ __global__ void __launch_bounds__(256)
     if (r.act) store8(h_out + n * d + r.c0, v);
     if (r.tid == 0) rstd_out[n] = rstd;
     if (w_gate != nullptr && r.warp == 0) {
-      // the first Cg channels live in warp 0
-      for (int k = 0; k < Hkv; ++k) {
-        float z = 0.f;
-        if (r.c0 < Cg) {
+      // the first Cg (<= 256) channels live in warp 0: gather them in shared
+      // memory, then lane k computes gate k on its own (no serial reductions)
+      if (r.c0 < Cg) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (r.c0 + e < Cg) z = fmaf(v[e], to_f(w_gate[(long long)k * Cg + r.c0 + e]), z);
-        }
-        z = warp_sum(z);
-        if (r.lane == 0) sg_out[n * Hkv + k] = sigmoidf_(z);
+        for (int e = 0; e < 8; ++e)
+          if (r.c0 + e < Cg) hg[r.c0 + e] = v[e];
       }
+      __syncwarp();
+      for (int k = r.lane; k < Hkv; k += 32) {
+        const T* wk = w_gate + (long long)k * Cg;
+        float z = 0.f;
+        for (int c = 0; c < Cg; ++c) z = fmaf(hg[c], to_f(wk[c]), z);
+        sg_out[n * Hkv + k] = sigmoidf_(z);
+      }
+      __syncwarp();  // hg is rewritten for the next row
     }
   }
 }
