@@ -686,7 +686,7 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     CKL();
   }
   if constexpr (std::is_same<T, bf16>::value) {
-    qkv_post_bwd_h128_kernel<<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(
+    qkv_post_bwd_h128_kernel<<<grid_rows(m.N), EW_THREADS, 0, st>>>(
         (const bf16*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (bf16*)X.dqkv, m.T, m.N, m.H, m.Hkv,
         ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz);
   } else {

@@ -303,94 +303,11 @@ __device__ __forceinline__ void st4(bf16* p, const float (&v)[4]) {
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-// one (token, head) item of the backward: its loads, issued before any compute
-struct QkvBwdItem {
-  long long n;
-  int hh;
-  bool valid;
-  float g[4], y[4], e[4];
-  float2 cs[4];
-  float r, s;
-};
-
-__device__ __forceinline__ void qkv_bwd_load(QkvBwdItem& it, long long item, long long total, int nh, int H, int Hkv,
-                                             int Tn, const bf16* qkv, long long ld, const float* rstd_qk,
-                                             const float2* rope, const float* dq, long long lddq, const float* dk,
-                                             const float* dv, long long lddkv, const bf16* ve_table,
-                                             const int32_t* idx, const float* sg, int lane) {
-  it.valid = item < total;
-  if (!it.valid) return;
-  it.n = item / nh;
-  it.hh = (int)(item - it.n * nh);
-  const long long n = it.n;
-  const int hh = it.hh;
-  if (hh < H + Hkv) {
-    const float* gp = (hh < H) ? dq + n * lddq + (long long)hh * 128 : dk + n * lddkv + (long long)(hh - H) * 128;
-    const float4 g4 = *reinterpret_cast<const float4*>(gp + lane * 4);
-    it.g[0] = g4.x; it.g[1] = g4.y; it.g[2] = g4.z; it.g[3] = g4.w;
-    ld4(qkv + n * ld + (long long)hh * 128 + lane * 4, it.y);
-    const int t = (int)(n % Tn);
-    const float4 c01 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4);
-    const float4 c23 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4 + 2);
-    it.cs[0] = make_float2(c01.x, c01.y);
-    it.cs[1] = make_float2(c01.z, c01.w);
-    it.cs[2] = make_float2(c23.x, c23.y);
-    it.cs[3] = make_float2(c23.z, c23.w);
-    it.r = rstd_qk[n * (H + Hkv) + hh];
-  } else {
-    const int kv = hh - H - Hkv;
-    const float4 g4 = *reinterpret_cast<const float4*>(dv + n * lddkv + (long long)kv * 128 + lane * 4);
-    it.g[0] = g4.x; it.g[1] = g4.y; it.g[2] = g4.z; it.g[3] = g4.w;
-    if (ve_table) {
-      ld4(ve_table + (long long)idx[n] * Hkv * 128 + (long long)kv * 128 + lane * 4, it.e);
-      it.s = sg[n * Hkv + kv];
-    }
-  }
-}
-
-__device__ __forceinline__ void qkv_bwd_compute(const QkvBwdItem& it, int H, int Hkv, bf16* dqkv, long long ld,
-                                                const bf16* ve_table, const int32_t* idx, float* dve_table,
-                                                float* dz, int lane) {
-  if (!it.valid) return;  // warp-uniform: every lane of the warp holds the same item
-  const long long n = it.n;
-  const int hh = it.hh;
-  bf16* out = dqkv + n * ld + (long long)hh * 128 + lane * 4;
-  const bool hi = lane >= 16;
-  if (hh < H + Hkv) {
-    // undo the rotation on the gradient and on the stored (rotated) output:
-    // first half: a1 c + a2 s ; second half: -a1 s + a2 c  (a1 = first-half value)
-    float gu[4], yu[4], dot = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float go = __shfl_xor_sync(0xffffffffu, it.g[e], 16);
-      const float yo = __shfl_xor_sync(0xffffffffu, it.y[e], 16);
-      const float c = it.cs[e].x, sn = it.cs[e].y;
-      gu[e] = hi ? (it.g[e] * c - go * sn) : (it.g[e] * c + go * sn);
-      yu[e] = hi ? (it.y[e] * c - yo * sn) : (it.y[e] * c + yo * sn);
-      dot = fmaf(gu[e], yu[e], dot);
-    }
-    const float m = warp_sum(dot) * (1.f / 128.f);
-    float o[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = it.r * (gu[e] - yu[e] * m);
-    st4(out, o);
-  } else {
-    if (ve_table) {
-      const int kv = hh - H - Hkv;
-      const long long row = (long long)idx[n] * Hkv * 128 + (long long)kv * 128 + lane * 4;
-      const float gate = 3.f * it.s;
-      const float dg = warp_sum(it.g[0] * it.e[0] + it.g[1] * it.e[1] + it.g[2] * it.e[2] + it.g[3] * it.e[3]);
-      atomicAdd(reinterpret_cast<float4*>(dve_table + row),
-                make_float4(gate * it.g[0], gate * it.g[1], gate * it.g[2], gate * it.g[3]));
-      if (lane == 0) dz[n * Hkv + kv] = dg * 3.f * it.s * (1.f - it.s);
-    }
-    float o[4] = {it.g[0], it.g[1], it.g[2], it.g[3]};
-    st4(out, o);
-  }
-}
-
 // backward of q,k <- rope(rmsnorm(.)) and of the VE term for hd = 128: one
-// warp per (token, head) item, two items' loads in flight per warp
+// warp per token.  The token's rotation row is loaded once; heads are taken
+// QKV_BWD_HEADS at a time with all of their loads issued before any compute,
+// so each warp keeps several kilobytes in flight.
+constexpr int QKV_BWD_HEADS = 2;
 __global__ void __launch_bounds__(EW_THREADS, 4)
     qkv_post_bwd_h128_kernel(const bf16* __restrict__ qkv, long long ld, const float* __restrict__ rstd_qk,
                              const float2* __restrict__ rope, const float* __restrict__ dq, long long lddq,
@@ -398,19 +315,102 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
                              bf16* __restrict__ dqkv, int Tn, long long N, int H, int Hkv,
                              const bf16* __restrict__ ve_table, const int32_t* __restrict__ idx,
                              const float* __restrict__ sg, float* __restrict__ dve_table, float* __restrict__ dz) {
+  constexpr int QB = QKV_BWD_HEADS;
   const int lane = threadIdx.x & 31;
-  const int nh = H + 2 * Hkv;
-  const long long total = N * nh;
+  const bool hi = lane >= 16;
+  const int nqk = H + Hkv;
   const long long wpb = blockDim.x >> 5;
-  const long long stride = gridDim.x * wpb;
-  for (long long base = blockIdx.x * wpb + (threadIdx.x >> 5); base < total; base += 2 * stride) {
-    QkvBwdItem a, b;
-    qkv_bwd_load(a, base, total, nh, H, Hkv, Tn, qkv, ld, rstd_qk, rope, dq, lddq, dk, dv, lddkv, ve_table, idx, sg,
-                 lane);
-    qkv_bwd_load(b, base + stride, total, nh, H, Hkv, Tn, qkv, ld, rstd_qk, rope, dq, lddq, dk, dv, lddkv, ve_table,
-                 idx, sg, lane);
-    qkv_bwd_compute(a, H, Hkv, dqkv, ld, ve_table, idx, dve_table, dz, lane);
-    qkv_bwd_compute(b, H, Hkv, dqkv, ld, ve_table, idx, dve_table, dz, lane);
+  for (long long n = blockIdx.x * wpb + (threadIdx.x >> 5); n < N; n += gridDim.x * wpb) {
+    const int t = (int)(n % Tn);
+    float2 cs[4];
+    {
+      const float4 c01 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4);
+      const float4 c23 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4 + 2);
+      cs[0] = make_float2(c01.x, c01.y);
+      cs[1] = make_float2(c01.z, c01.w);
+      cs[2] = make_float2(c23.x, c23.y);
+      cs[3] = make_float2(c23.z, c23.w);
+    }
+    const bf16* yrow = qkv + n * ld + lane * 4;
+    bf16* orow = dqkv + n * ld + lane * 4;
+    // q and k heads: undo the rotation on the gradient and on the stored
+    // (rotated, normalised) output, then the RMSNorm backward
+    for (int h0 = 0; h0 < nqk; h0 += QB) {
+      float4 g4[QB];
+      uint2 yb[QB];  // 4 bf16, converted at use
+      float r[QB];
+#pragma unroll
+      for (int b = 0; b < QB; ++b) {
+        const int hh = h0 + b;
+        if (hh < nqk) {
+          const float* gp = (hh < H) ? dq + n * lddq + (long long)hh * 128 : dk + n * lddkv + (long long)(hh - H) * 128;
+          g4[b] = *reinterpret_cast<const float4*>(gp + lane * 4);
+          yb[b] = *reinterpret_cast<const uint2*>(yrow + (long long)hh * 128);
+          r[b] = rstd_qk[n * nqk + hh];
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < QB; ++b) {
+        const int hh = h0 + b;
+        if (hh < nqk) {  // warp-uniform
+        const float g[4] = {g4[b].x, g4[b].y, g4[b].z, g4[b].w};
+        const float2 y01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yb[b].x));
+        const float2 y23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yb[b].y));
+        const float y[4] = {y01.x, y01.y, y23.x, y23.y};
+        // first half: a1 c + a2 s ; second half: -a1 s + a2 c  (a1 = first-half value)
+        float gu[4], yu[4], dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float go = __shfl_xor_sync(0xffffffffu, g[e], 16);
+          const float yo = __shfl_xor_sync(0xffffffffu, y[e], 16);
+          const float c = cs[e].x, sn = cs[e].y;
+          gu[e] = hi ? (g[e] * c - go * sn) : (g[e] * c + go * sn);
+          yu[e] = hi ? (y[e] * c - yo * sn) : (y[e] * c + yo * sn);
+          dot = fmaf(gu[e], yu[e], dot);
+        }
+        const float m = warp_sum(dot) * (1.f / 128.f);
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = r[b] * (gu[e] - yu[e] * m);
+        st4(orow + (long long)hh * 128, o);
+        }
+      }
+    }
+    // v heads: the gradient passes through; with value embeddings also the
+    // VE-table gradient (3*sigmoid(z) * dv, scattered by token id) and dz
+    const long long ve_row = ve_table ? (long long)idx[n] * Hkv * 128 + lane * 4 : 0;
+    for (int k0 = 0; k0 < Hkv; k0 += QB) {
+      float4 g4[QB];
+      uint2 eb[QB];
+      float sv[QB];
+#pragma unroll
+      for (int b = 0; b < QB; ++b) {
+        const int kv = k0 + b;
+        if (kv < Hkv) {
+          g4[b] = *reinterpret_cast<const float4*>(dv + n * lddkv + (long long)kv * 128 + lane * 4);
+          if (ve_table) {
+            eb[b] = *reinterpret_cast<const uint2*>(ve_table + ve_row + (long long)kv * 128);
+            sv[b] = sg[n * Hkv + kv];
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < QB; ++b) {
+        const int kv = k0 + b;
+        if (kv < Hkv) {  // warp-uniform
+        const float g[4] = {g4[b].x, g4[b].y, g4[b].z, g4[b].w};
+        if (ve_table) {
+          const float2 e01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&eb[b].x));
+          const float2 e23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&eb[b].y));
+          const float gate = 3.f * sv[b];
+          const float dg = warp_sum(g[0] * e01.x + g[1] * e01.y + g[2] * e23.x + g[3] * e23.y);
+          red_add_v4_f32(dve_table + ve_row + (long long)kv * 128, gate * g[0], gate * g[1], gate * g[2], gate * g[3]);
+          if (lane == 0) dz[n * Hkv + kv] = dg * 3.f * sv[b] * (1.f - sv[b]);
+        }
+        st4(orow + (long long)(nqk + kv) * 128, g);
+        }
+      }
+    }
   }
 }
 

@@ -381,8 +381,8 @@ __global__ void __launch_bounds__(256)
     }
     if (r.act) {
       float* dst = dwte + (long long)idx[n] * d + r.c0;
-      atomicAdd(reinterpret_cast<float4*>(dst), make_float4(g[0], g[1], g[2], g[3]));
-      atomicAdd(reinterpret_cast<float4*>(dst + 4), make_float4(g[4], g[5], g[6], g[7]));
+      red_add_v4_f32(dst, g[0], g[1], g[2], g[3]);
+      red_add_v4_f32(dst + 4, g[4], g[5], g[6], g[7]);
     }
   }
   if (C > 0) {
