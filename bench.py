@@ -144,13 +144,18 @@ def measured_peaks() -> dict:
 
 
 def profile_traffic(workload: str) -> float | None:
-    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", f"gemm_tc_{workload}.json")
-    if os.path.exists(p):
-        try:
-            return float(json.load(open(p))["dram_bytes_per_launch"])
-        except Exception:
-            return None
+    """Average DRAM bytes per GEMM launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary of this workload's step, if there is one: the
+    line 'dram bytes per GEMM launch: <value>' of profiles/gemm_tc_<workload>_traffic.md."""
+    p = os.path.join(ROOT, "profiles", f"gemm_tc_{workload}_traffic.md")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        if line.lower().startswith("dram bytes per gemm launch:"):
+            try:
+                return float(line.split(":", 1)[1].split()[0])
+            except ValueError:
+                return None
     return None
 
 

@@ -335,9 +335,13 @@ namespace gptb {
 // requests each warp keeps in flight).  At the end the softmax warps
 // write dK, dV (fp32) through swizzled staging tiles in the then idle Q/dO
 // ring and TMA stores that clip at the sequence end.
-// CTAs are numbered key-tile-major so the tiles with the most query tiles
-// (the first ones under a causal mask) start first.
+// CTA order: groups of AB2_GROUP (kv head, sequence) pairs, key-tile-major
+// inside a group, so the tiles with the most query tiles (the first ones
+// under a causal mask) start first while the CTAs in flight reduce into the
+// dQ rows of one or two groups only (a few MB that stay in L2, where a
+// whole-batch order would send every reduction to DRAM and back).
 constexpr int AB2_BK = 128, AB2_BQ = 64;
+constexpr int AB2_GROUP = 16;
 constexpr int AB2_THREADS = 576;
 constexpr int AB2_KV_TILE = 128 * 128 * 2;  // 32 KB
 constexpr int AB2_Q_TILE = 64 * 128 * 2;    // 16 KB
@@ -377,8 +381,14 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sLD = reinterpret_cast<float*>(bars + 32);  // [AB2_STAGES][lse*log2e 64 | D 64]
 
-  const int nkv = Hkv * Bsz;
-  const int kb = blockIdx.x / nkv, kvh = blockIdx.x % Hkv, b = (blockIdx.x % nkv) / Hkv;
+  const int nkb = (T + AB2_BK - 1) / AB2_BK;
+  const int npairs = Hkv * Bsz;
+  const int grp = blockIdx.x / (AB2_GROUP * nkb);
+  const int gsize = min(AB2_GROUP, npairs - grp * AB2_GROUP);  // the last group may be smaller
+  const int wg = blockIdx.x - grp * AB2_GROUP * nkb;
+  const int kb = wg / gsize;
+  const int pair = grp * AB2_GROUP + wg % gsize;
+  const int kvh = pair % Hkv, b = pair / Hkv;
   const int G = H / Hkv;
   const int k0 = kb * AB2_BK;
   const int row_base = b * T;
