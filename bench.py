@@ -232,11 +232,22 @@ def main():
     ap.add_argument("--workload", default="d24", choices=list(synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    # smaller footprints of the same workload for profiler captures; a line
+    # printed with either override is not the workload's measurement
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling only)")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
-    c = synth.config(args.workload)
+    over = {}
+    if args.batch:
+        over["B"] = args.batch
+    if args.layers:
+        over["n_layer"] = args.layers
+    c = synth.config(args.workload, **over)
+    if over:
+        c["name"] = c["name"] + "_profiling_" + "_".join(f"{k}{v}" for k, v in over.items())
     fl = flops_per_token(c)
     if args.impl == "reference":
         run_reference(args, c, fl)
