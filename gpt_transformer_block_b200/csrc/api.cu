@@ -727,8 +727,13 @@ int lm_head_impl(const gptb_config& c, const T* h, const T* w_lm, const int32_t*
     const int rows = (int)std::min<long long>(lw.chunk, m.N - c0);
     const T* hc = h + c0 * m.d;
     TRY(gemm(dt, {hc, m.d, false}, {w_lm, m.d, false}, rows, m.V, m.d, epi(EPI_STORE, dt, lw.logits, m.V), st));
-    xent_rows_kernel<T><<<rows, 512, 0, st>>>((T*)lw.logits, m.V, m.V, targets + c0, lw.row_loss + c0,
-                                              1.f / (float)m.N, rows);
+    if (std::is_same<T, bf16>::value && m.V <= XENT_REG_THREADS * 8 * XENT_REG_VEC) {
+      xent_rows_reg_kernel<<<rows, XENT_REG_THREADS, 0, st>>>((bf16*)lw.logits, m.V, m.V, targets + c0,
+                                                              lw.row_loss + c0, 1.f / (float)m.N, rows);
+    } else {
+      xent_rows_kernel<T><<<rows, 512, 0, st>>>((T*)lw.logits, m.V, m.V, targets + c0, lw.row_loss + c0,
+                                                1.f / (float)m.N, rows);
+    }
     CKL();
     TRY(gemm(dt, {lw.logits, m.V, false}, {w_lm, m.d, true}, rows, m.d, m.V, epi(EPI_STORE, dt, dh + c0 * m.d, m.d),
              st));

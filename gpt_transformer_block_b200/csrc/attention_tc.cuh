@@ -38,11 +38,6 @@ constexpr int FA_TILE = 128 * 128 * 2;  // one 128x128 bf16 tile: 32 KB (two 64-
 constexpr int FA_SMEM = 1024 /*align*/ + FA_TILE /*Q*/ + 4 * FA_TILE /*K,V x2*/ + 256 /*barriers*/ +
                         2 * 2 * 128 * 4 /*row max exchange, 2 tiles in flight*/ + 2 * 128 * 4 /*row sums*/;
 
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // K-major SW128 descriptor of a 128-row tile, k-th 16-element K step
 __device__ __forceinline__ uint64_t fa_desc_k(uint32_t tile, int k) {

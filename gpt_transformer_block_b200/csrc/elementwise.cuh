@@ -219,6 +219,75 @@ __global__ void __launch_bounds__(512)
   if (threadIdx.x == 0) row_loss[r] = lse - zy;
 }
 
+// bf16 rows of up to XENT_REG_THREADS * 8 * XENT_REG_VEC entries: one CTA per
+// row holds the whole row in registers (all 16-byte loads issued before any
+// use), takes the max, the sum of exp and then the gradient from the same
+// registers, so each logit is read once and written once.  exp by ex2 with the
+// log2(e) scale folded into one FMA.
+constexpr int XENT_REG_THREADS = 512, XENT_REG_VEC = 8;  // 32768 entries
+__global__ void __launch_bounds__(XENT_REG_THREADS, 2)
+    xent_rows_reg_kernel(bf16* __restrict__ logits, long long ld, int V, const int32_t* __restrict__ targets,
+                         float* __restrict__ row_loss, float inv_n, int nrows) {
+  __shared__ float red[XENT_REG_THREADS / 32];
+  const long long r = blockIdx.x;
+  if (r >= nrows) return;
+  bf16* z = logits + r * ld;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = XENT_REG_THREADS / 32;
+  uint4 u[XENT_REG_VEC];
+#pragma unroll
+  for (int j = 0; j < XENT_REG_VEC; ++j) {
+    const int c = (j * XENT_REG_THREADS + tid) * 8;
+    // past the vocabulary: -inf (bf16 0xff80), which adds nothing below
+    u[j] = (c < V) ? *reinterpret_cast<const uint4*>(z + c) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+  }
+  const int y = targets[r];
+  const float zy = __bfloat162float(z[y]);
+  auto val = [&](int j, int k) -> float {  // element k (0..7) of vector j
+    const uint32_t w = (k < 2) ? u[j].x : (k < 4) ? u[j].y : (k < 6) ? u[j].z : u[j].w;
+    return __uint_as_float((k & 1) ? (w & 0xffff0000u) : (w << 16));
+  };
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < XENT_REG_VEC; ++j)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, val(j, k));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  float M = red[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+  const float ml2 = M * LOG2E;
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < XENT_REG_VEC; ++j)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s += fast_exp2(fmaf(val(j, k), LOG2E, -ml2));
+  s = warp_sum(s);
+  if (lane == 0) red[warp] = s;
+  __syncthreads();
+  float S = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) S += red[w];
+  const float lse = M + logf(S);
+  const float ll2 = lse * LOG2E;
+  // gradient (softmax - onehot) / n over the same registers
+#pragma unroll
+  for (int j = 0; j < XENT_REG_VEC; ++j) {
+    const int c = (j * XENT_REG_THREADS + tid) * 8;
+    if (c < V) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = (fast_exp2(fmaf(val(j, k), LOG2E, -ll2)) - (c + k == y ? 1.f : 0.f)) * inv_n;
+      store8(z + c, v);
+    }
+  }
+  if (tid == 0) row_loss[r] = lse - zy;
+}
+
 // loss = mean of the row losses (single CTA, fixed order)
 __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ x, long long n, float* __restrict__ out) {
   __shared__ float sred[32];
