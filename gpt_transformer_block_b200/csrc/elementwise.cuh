@@ -1,12 +1,15 @@
 // Per-(token, head) and per-tensor kernels of the block (HBM-bound):
 //   - QK RMSNorm + RoPE and the value-embedding add: backward (one warp per
-//     (token, head), vectorised for hd = 128) and a generic forward and
-//     backward for the fp32 configuration (bf16/fp8 fuse the forward into
-//     the QKV GEMM epilogue);
-//   - the attention-backward preprocess D = rowsum(dO o o);
+//     token, vectorised for hd = 128) and a generic forward and backward for
+//     the fp32 configuration (bf16/fp8 fuse the forward into the QKV GEMM
+//     epilogue);
 //   - the value-embedding gate weight gradient;
-//   - cross-entropy over a chunk of logits rows and the loss mean;
+//   - cross-entropy over a chunk of logits rows (register-resident rows for
+//     bf16) and the loss mean;
 //   - FP8 (e4m3) per-tensor amax and quantisation.
+// (The attention-backward term D = rowsum(dO o o) comes out of the dO GEMM's
+// epilogue for bf16/fp8, and out of attn_bwd_pre_kernel in attention.cuh for
+// the fp32 configuration.)
 // The per-token-row kernels (norms, lambda mix, smear, backout) are in rows.cuh.
 #pragma once
 #include "common.cuh"
@@ -355,9 +358,9 @@ __global__ void __launch_bounds__(256)
 namespace gptb {
 
 // ------------------------------------------- vectorised hd = 128 variants --
-// One warp per (token, head).  Lane l holds elements 4l..4l+3 of the head:
-// lanes 0-15 the first half (rotation partner j), lanes 16-31 the second half
-// (j + 64); the partner value is one shuffle (lane ^ 16) away.
+// Lane l holds elements 4l..4l+3 of a head: lanes 0-15 the first half
+// (rotation partner j), lanes 16-31 the second half (j + 64); the partner
+// value is one shuffle (lane ^ 16) away.
 
 __device__ __forceinline__ void ld4(const bf16* p, float (&v)[4]) {
   const uint2 u = *reinterpret_cast<const uint2*>(p);
