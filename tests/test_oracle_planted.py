@@ -91,3 +91,51 @@ def test_ve_gate_scale_is_caught(monkeypatch):
     orig = om._sigmoid
     monkeypatch.setattr(om, "_sigmoid", lambda z: 2.0 * orig(z) / 3.0)   # gate 2*sigmoid instead of 3*sigmoid
     _fails(pins.test_block_special_cases)
+
+
+# ----------------------------------------------------------- optimizer oracle
+import numpy as np  # noqa: E402
+from oracle import optim as oo  # noqa: E402
+import test_oracle_optim as opins  # noqa: E402
+
+
+def _pe_variant(kind):
+    """polar_express with one slip: the roles of b and c swapped, or the a X
+    term dropped (a read as 1)."""
+    def pe(G, coeffs, ns_steps=None, eps=1e-7):
+        X = np.asarray(G, dtype=np.float64)
+        wide = X.shape[0] < X.shape[1]
+        X = X.T if wide else X
+        X = X / (np.linalg.norm(X) + eps)
+        for a, b, c in list(coeffs)[: (len(coeffs) if ns_steps is None else ns_steps)]:
+            A = X.T @ X
+            if kind == "swap_bc":
+                X = a * X + X @ (c * A + b * (A @ A))
+            else:
+                X = X + X @ (b * A + c * (A @ A))
+        return X.T if wide else X
+    return pe
+
+
+@pytest.mark.parametrize("kind", ["swap_bc", "drop_a"])
+def test_polar_express_slips_are_caught(monkeypatch, kind):
+    monkeypatch.setattr(oo, "polar_express", _pe_variant(kind))
+    _fails(opins.test_one_step_maps_singular_values_by_the_odd_polynomial, (12, 7), opins.PAGE_TUPLES[0])
+
+
+def test_adamw_without_bias_correction_is_caught(monkeypatch):
+    def bad(p, g, m, v, t, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0):
+        m = beta1 * m + (1 - beta1) * g
+        v = beta2 * v + (1 - beta2) * g * g
+        return p * (1 - lr * weight_decay) - lr * m / (np.sqrt(v) + eps), m, v
+    monkeypatch.setattr(oo, "adamw_step", bad)
+    _fails(opins.test_adamw_matches_torch_over_steps)
+    _fails(opins.test_adamw_first_step_closed_form)
+
+
+def test_adamw_coupled_weight_decay_is_caught(monkeypatch):
+    orig = oo.adamw_step
+    def bad(p, g, m, v, t, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0):
+        return orig(p, np.asarray(g) + weight_decay * np.asarray(p), m, v, t, lr, beta1, beta2, eps, 0.0)
+    monkeypatch.setattr(oo, "adamw_step", bad)
+    _fails(opins.test_adamw_matches_torch_over_steps)
