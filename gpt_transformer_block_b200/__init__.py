@@ -23,6 +23,7 @@ EXPORTS = [
     "gpt_stack_step", "gptb_gemm_bf16", "gptb_device_error", "gptb_set_wait_limit_ns",
     "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
     "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
+    "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express",
 ]
 
 _vp = ctypes.c_void_p
@@ -92,9 +93,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptb_gemm_timing.argtypes = [P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_longlong)]
     lib.gptb_error_string.argtypes = [ctypes.c_int]
     lib.gptb_error_string.restype = ctypes.c_char_p
+    lib.gptb_adamw_step.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, ctypes.c_float, ctypes.c_float,
+                                    ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int, _vp]
+    lib.gptb_polar_express_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.gptb_polar_express_workspace_bytes.restype = ctypes.c_size_t
+    lib.gptb_polar_express.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _fp, ctypes.c_int, _vp,
+                                       ctypes.c_size_t, _vp]
     for name in EXPORTS:
         if name not in ("gptb_workspace_bytes", "gptb_error_string", "gptb_reset_counters",
-                        "gptb_launch_count"):
+                        "gptb_launch_count", "gptb_polar_express_workspace_bytes"):
             getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -214,6 +221,28 @@ def gpt_stack_step(cfg, w: ModelWeights, idx, targets, loss_out, g: ModelGrads, 
 def gptb_gemm_bf16(A, a_mn, lda, B, b_mn, ldb, C, c_f32, ldc, M, N, K, stream=None):
     _check(load().gptb_gemm_bf16(ptr(A), int(a_mn), lda, ptr(B), int(b_mn), ldb, ptr(C), int(c_f32), ldc,
                                  M, N, K, _stream(stream)), "gptb_gemm_bf16")
+
+
+def gptb_adamw_step(p, g, m, v, p_bf16, n, lr, beta1, beta2, eps, weight_decay, step, stream=None):
+    """One AdamW step over n fp32 parameters in place (p, m, v); p_bf16 (or None)
+    receives the bf16 copy of the new parameters."""
+    _check(load().gptb_adamw_step(ptr(p), ptr(g), ptr(m), ptr(v), ptr(p_bf16) if p_bf16 is not None else None,
+                                  int(n), float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                                  int(step), _stream(stream)), "gptb_adamw_step")
+
+
+def gptb_polar_express_workspace_bytes(m: int, n: int, steps: int) -> int:
+    return int(load().gptb_polar_express_workspace_bytes(int(m), int(n), int(steps)))
+
+
+def gptb_polar_express(G, out, m, n, coeffs, workspace, stream=None):
+    """Polar Express orthogonalisation of the bf16 [m, n] matrix G into out;
+    coeffs: a host sequence of (a, b, c) tuples, one per step."""
+    flat = [float(x) for abc in coeffs for x in abc]
+    arr = (ctypes.c_float * len(flat))(*flat)
+    nbytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
+    _check(load().gptb_polar_express(ptr(G), ptr(out), int(m), int(n), arr, len(coeffs), ptr(workspace),
+                                     nbytes, _stream(stream)), "gptb_polar_express")
 
 
 def gptb_device_error(stream=None) -> int:

@@ -282,6 +282,7 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
   e.out2 = out2;
   e.ldo2 = ldo2;
   e.alpha = nullptr;
+  e.beta = nullptr;
   e.amax_a = nullptr;
   e.amax_b = nullptr;
   e.rope = nullptr;
@@ -896,6 +897,96 @@ int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_
   if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
   EpiParams e = epi(c_f32 ? EPI_ACCUM_F32 : EPI_STORE, GPTB_BF16, C, ldc);
   return gemm(GPTB_BF16, {A, lda, a_mn != 0}, {B, ldb, b_mn != 0}, M, N, K, e, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------ optimizer step --
+
+int gptb_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, long long n, float lr, float beta1,
+                    float beta2, float eps, float weight_decay, int step, gptb_stream_t stream) {
+  if (!p || !g || !m || !v || n < 0 || step < 1) return GPTB_ERR_INVALID_ARG;
+  if (n == 0) return GPTB_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const double bc1 = 1.0 - std::pow((double)beta1, step), bc2 = 1.0 - std::pow((double)beta2, step);
+  if (!(bc1 > 0.0) || !(bc2 > 0.0)) return GPTB_ERR_INVALID_ARG;  // beta1 or beta2 outside [0, 1)
+  const bool vec4 = (n % 4 == 0) && aligned16(p) && aligned16(g) && aligned16(m) && aligned16(v) &&
+                    (p_bf16 == nullptr || (reinterpret_cast<uintptr_t>(p_bf16) & 7u) == 0);
+  const long long items = vec4 ? n / 4 : n;
+  const int threads = 256;
+  const long long cap = (long long)dev_info().sms * 8;
+  const int grid = (int)std::max<long long>(1, std::min((items + threads - 1) / threads, cap));
+  adamw_kernel<<<grid, threads, 0, st>>>(p, g, m, v, reinterpret_cast<bf16*>(p_bf16), n, lr, beta1, beta2, eps,
+                                         1.f - lr * weight_decay, (float)(1.0 / bc1), (float)(1.0 / std::sqrt(bc2)),
+                                         vec4 ? 1 : 0);
+  CKL();
+  return GPTB_OK;
+}
+
+namespace {
+constexpr size_t PE_HEADER = 1024;  // sum of squares (4 B) at 0, coefficients (<= 64 x 3 floats) at 256
+size_t pe_align(size_t b) { return (b + 255) & ~size_t(255); }
+}  // namespace
+
+size_t gptb_polar_express_workspace_bytes(int m, int n, int steps) {
+  if (m <= 0 || n <= 0 || steps < 1 || steps > 64) return 0;
+  const size_t s = (size_t)std::min(m, n);
+  return PE_HEADER + 2 * pe_align((size_t)m * n * 2) + 2 * pe_align(s * s * 2);
+}
+
+int gptb_polar_express(const void* G, void* out, int m, int n, const float* coeffs, int steps, void* workspace,
+                       size_t workspace_bytes, gptb_stream_t stream) {
+  if (!G || !out || !coeffs || !workspace || m <= 0 || n <= 0 || m % 8 || n % 8 || steps < 1 || steps > 64)
+    return GPTB_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GPTB_ERR_INVALID_ARG;
+  const size_t ne = (size_t)m * n;
+  {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(G), b = reinterpret_cast<uintptr_t>(out);
+    if (a < b + ne * 2 && b < a + ne * 2) return GPTB_ERR_INVALID_ARG;  // out overlaps G
+  }
+  if (workspace_bytes < gptb_polar_express_workspace_bytes(m, n, steps)) return GPTB_ERR_WORKSPACE;
+  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  float* sumsq = reinterpret_cast<float*>(w);
+  float* cf = reinterpret_cast<float*>(w + 256);
+  bf16* X[2];
+  X[0] = reinterpret_cast<bf16*>(w + PE_HEADER);
+  X[1] = reinterpret_cast<bf16*>(w + PE_HEADER + pe_align(ne * 2));
+  const bool wide = m < n;
+  const int s = wide ? m : n;  // side of the Gram matrix
+  bf16* A = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(ne * 2));
+  bf16* Bm = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(ne * 2) + pe_align((size_t)s * s * 2));
+  // the coefficients go through the stream (the host array is read before this returns)
+  CK(cudaMemcpyAsync(cf, coeffs, sizeof(float) * 3 * steps, cudaMemcpyHostToDevice, st));
+  CK(cudaMemsetAsync(sumsq, 0, sizeof(float), st));
+  const int grid = (int)std::max<long long>(1, std::min<long long>(((long long)ne + 255) / 256, dev_info().sms * 8LL));
+  sumsq_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16*>(G), (long long)ne, sumsq);
+  CKL();
+  scale_by_norm_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16*>(G), X[0], (long long)ne, sumsq, 1e-7f);
+  CKL();
+  bf16* cur = X[0];
+  for (int t = 0; t < steps; ++t) {
+    const float* a = cf + 3 * t;
+    bf16* nxt = (t == steps - 1) ? static_cast<bf16*>(out) : X[(t + 1) & 1];
+    // A = Gram matrix of the smaller side (X^T X for a tall X, X X^T for a wide one)
+    if (!wide)
+      TRY(gemm(GPTB_BF16, {cur, n, true}, {cur, n, true}, n, n, m, epi(EPI_STORE, GPTB_BF16, A, n), st));
+    else
+      TRY(gemm(GPTB_BF16, {cur, n, false}, {cur, n, false}, m, m, n, epi(EPI_STORE, GPTB_BF16, A, m), st));
+    // B = b A + c A A   (A symmetric, so A A = A A^T)
+    EpiParams eb = epi(EPI_RESID, GPTB_BF16, Bm, s, A, s);
+    eb.alpha = a + 2;
+    eb.beta = a + 1;
+    TRY(gemm(GPTB_BF16, {A, s, false}, {A, s, false}, s, s, s, eb, st));
+    // X = a X + X B   (B symmetric); for a wide X the same update of X^T reads X = a X + B X
+    EpiParams ex = epi(EPI_RESID, GPTB_BF16, nxt, n, cur, n);
+    ex.beta = a;
+    if (!wide)
+      TRY(gemm(GPTB_BF16, {cur, n, false}, {Bm, s, false}, m, n, n, ex, st));
+    else
+      TRY(gemm(GPTB_BF16, {Bm, s, false}, {cur, n, true}, m, n, m, ex, st));
+    cur = nxt;
+  }
+  return GPTB_OK;
 }
 
 int gptb_device_error(gptb_stream_t stream) {

@@ -291,6 +291,73 @@ __global__ void __launch_bounds__(XENT_REG_THREADS, 2)
   if (tid == 0) row_loss[r] = lse - zy;
 }
 
+// ------------------------------------------------------ optimizer step --
+// AdamW over n fp32 parameters (decoupled weight decay, bias-corrected
+// moments; inv_bc1 = 1/(1-b1^t), inv_sqrt_bc2 = 1/sqrt(1-b2^t)), with an
+// optional bf16 copy of the new parameters.  vec4: all arrays hold whole
+// 16-byte groups (n % 4 == 0, aligned), else one element per thread.
+__device__ __forceinline__ void adamw_one(float& p, float g, float& m, float& v, float lr, float b1, float b2,
+                                          float eps, float decay, float inv_bc1, float inv_sqrt_bc2) {
+  m = fmaf(b1, m, (1.f - b1) * g);
+  v = fmaf(b2, v, (1.f - b2) * g * g);
+  p = p * decay - lr * (m * inv_bc1) / (sqrtf(v) * inv_sqrt_bc2 + eps);
+}
+__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                             float* __restrict__ v, bf16* __restrict__ pb, long long n, float lr, float b1, float b2,
+                             float eps, float decay, float inv_bc1, float inv_sqrt_bc2, int vec4) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  if (vec4) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n / 4; i += stride) {
+      float4 pp = reinterpret_cast<float4*>(p)[i], mm = reinterpret_cast<float4*>(m)[i],
+             vv = reinterpret_cast<float4*>(v)[i];
+      const float4 gg = reinterpret_cast<const float4*>(g)[i];
+      adamw_one(pp.x, gg.x, mm.x, vv.x, lr, b1, b2, eps, decay, inv_bc1, inv_sqrt_bc2);
+      adamw_one(pp.y, gg.y, mm.y, vv.y, lr, b1, b2, eps, decay, inv_bc1, inv_sqrt_bc2);
+      adamw_one(pp.z, gg.z, mm.z, vv.z, lr, b1, b2, eps, decay, inv_bc1, inv_sqrt_bc2);
+      adamw_one(pp.w, gg.w, mm.w, vv.w, lr, b1, b2, eps, decay, inv_bc1, inv_sqrt_bc2);
+      reinterpret_cast<float4*>(p)[i] = pp;
+      reinterpret_cast<float4*>(m)[i] = mm;
+      reinterpret_cast<float4*>(v)[i] = vv;
+      if (pb) reinterpret_cast<uint2*>(pb)[i] = make_uint2(pack_bf16(pp.x, pp.y), pack_bf16(pp.z, pp.w));
+    }
+  } else {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += stride) {
+      float pp = p[i], mm = m[i], vv = v[i];
+      adamw_one(pp, g[i], mm, vv, lr, b1, b2, eps, decay, inv_bc1, inv_sqrt_bc2);
+      p[i] = pp;
+      m[i] = mm;
+      v[i] = vv;
+      if (pb) pb[i] = __float2bfloat16_rn(pp);
+    }
+  }
+}
+
+// sum of squares of a bf16 array into *out (fp32, zeroed by the caller)
+__global__ void __launch_bounds__(256) sumsq_bf16_kernel(const bf16* __restrict__ x, long long n, float* __restrict__ out) {
+  __shared__ float sred[8];
+  float s = 0.f;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float t = __bfloat162float(x[i]);
+    s = fmaf(t, t, s);
+  }
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) sred[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sred[w];
+    atomicAdd(out, t);
+  }
+}
+
+// y = x / (sqrt(*sumsq) + eps), rounded to bf16
+__global__ void scale_by_norm_bf16_kernel(const bf16* __restrict__ x, bf16* __restrict__ y, long long n,
+                                          const float* __restrict__ sumsq, float eps) {
+  const float inv = 1.f / (sqrtf(*sumsq) + eps);
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    y[i] = __float2bfloat16_rn(__bfloat162float(x[i]) * inv);
+}
+
 // loss = mean of the row losses (single CTA, fixed order)
 __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ x, long long n, float* __restrict__ out) {
   __shared__ float sred[32];

@@ -28,7 +28,7 @@ namespace gptb {
 
 enum EpiKind : int {
   EPI_STORE = 0,      // out = alpha*acc
-  EPI_RESID = 1,      // out = aux + alpha*acc                (residual add)
+  EPI_RESID = 1,      // out = beta*aux + alpha*acc           (residual add)
   EPI_RELU2 = 2,      // out = u = alpha*acc, out2 = relu(u)^2 (MLP activation)
   EPI_DRELU2 = 3,     // out = alpha*acc * 2*relu(aux)         (aux = saved u)
   EPI_ACCUM_F32 = 4,  // out(f32) += alpha*acc, atomic          (weight grads)
@@ -49,6 +49,7 @@ struct EpiParams {
   void* out2;
   long long ldo2;
   const float* alpha;  // device scalar or nullptr (= 1)
+  const float* beta;   // EPI_RESID: device scale of aux, or nullptr (= 1)
   // e4m3 operands: per-tensor amax of A and B; the product is rescaled by
   // (amax_a / 448) * (amax_b / 448), the inverse of the two quantisation scales
   const float* amax_a;
@@ -64,6 +65,7 @@ struct EpiParams {
   float* rowdot;          // EPI_DOT: [B, H, T] fp32
 };
 
+__device__ __forceinline__ float epi_beta(const EpiParams& ep) { return ep.beta ? *ep.beta : 1.f; }
 __device__ __forceinline__ float epi_alpha(const EpiParams& ep) {
   float a = ep.alpha ? *ep.alpha : 1.f;
   if (ep.amax_a) a *= (fmaxf(*ep.amax_a, 1e-12f) / 448.f) * (fmaxf(*ep.amax_b, 1e-12f) / 448.f);
@@ -78,8 +80,9 @@ __device__ __forceinline__ void epi_store8_t(const EpiParams& ep, long long r, i
     case EPI_RESID: {
       float a[8];
       load8(reinterpret_cast<const T*>(ep.aux) + r * ep.ld_aux + c, a);
+      const float beta = epi_beta(ep);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] += a[i];
+      for (int i = 0; i < 8; ++i) v[i] = fmaf(beta, a[i], v[i]);
       store8(o, v);
     } break;
     case EPI_RELU2: {
@@ -120,7 +123,7 @@ template <class T>
 __device__ __forceinline__ void epi_scalar_t(const EpiParams& ep, long long r, int c, float v) {
   T* o = reinterpret_cast<T*>(ep.out) + r * ep.ldo + c;
   switch (ep.kind) {
-    case EPI_RESID: *o = from_f<T>(to_f(reinterpret_cast<const T*>(ep.aux)[r * ep.ld_aux + c]) + v); break;
+    case EPI_RESID: *o = from_f<T>(fmaf(epi_beta(ep), to_f(reinterpret_cast<const T*>(ep.aux)[r * ep.ld_aux + c]), v)); break;
     case EPI_RELU2: {
       *o = from_f<T>(v);
       float t = fmaxf(v, 0.f);
@@ -423,6 +426,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     const float alpha = epi_alpha(ep);
+    const float beta = epi_beta(ep);
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int tm, tn, split;
@@ -499,7 +503,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               load8(reinterpret_cast<const bf16*>(cp1), a);
               if (ep.kind == EPI_RESID) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] += a[i];
+                for (int i = 0; i < 8; ++i) v[i] = fmaf(beta, a[i], v[i]);
               } else if (ep.kind == EPI_DRELU2) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] *= 2.f * fmaxf(a[i], 0.f);

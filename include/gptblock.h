@@ -193,6 +193,42 @@ int gpt_stack_step(const gptb_config* cfg, const gptb_model_weights* w, const in
 int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, void* C,
                    int c_f32, long long ldc, int M, int N, int K, gptb_stream_t stream);
 
+/* ---------------------------------------------------- optimizer step ----
+ * The step after the training step (nanochat's mixed optimizer: AdamW for the
+ * embeddings, the lm_head and the scalar parameters; Muon, whose update is
+ * orthogonalised by the Polar Express iteration, for the 2-D matrices).
+ * Source: apidog.com/fr "Comment Entraîner Votre Propre ChatGPT Pour 50€ ?",
+ * § "Comment nanochat fonctionne" › 2 "L'optimiseur Muon"; dev.to/aakira
+ * "ChatGPTを50ドルでトレーニングする方法" § 2 (parameter groups). */
+
+/* One AdamW step over n fp32 parameters, in place:
+ *   m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
+ *   p = p (1 - lr wd) - lr (m / (1-b1^step)) / (sqrt(v / (1-b2^step)) + eps).
+ * p, m, v: device fp32 [n], updated; g: device fp32 [n], read.  p_bf16:
+ * device bf16 [n] that receives the new p rounded to nearest-even (the
+ * working copy the GEMMs read), or NULL.  step >= 1.  Errors:
+ * GPTB_ERR_INVALID_ARG for null arrays, n < 0 or step < 1 (nothing enqueued). */
+int gptb_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, long long n, float lr, float beta1,
+                    float beta2, float eps, float weight_decay, int step, gptb_stream_t stream);
+
+/* Device workspace in bytes of gptb_polar_express for an [m, n] matrix. */
+size_t gptb_polar_express_workspace_bytes(int m, int n, int steps);
+
+/* Polar Express orthogonalisation of a 2-D update G [m, n] (bf16, row-major,
+ * row stride n) into out [m, n] (bf16; must not overlap G): X = G / ||G||_F,
+ * then for each (a, b, c) of coeffs[0..steps-1]:
+ *   A = X^T X,  B = b A + c A A,  X = a X + X B
+ * with A the Gram matrix of the smaller side (a wide G runs the same loop on
+ * G^T, written back untransposed).  Every product is a tensor-core GEMM with
+ * bf16 operands and fp32 accumulation; A, B and X are stored in bf16.
+ * coeffs: HOST float [3*steps] (a, b, c per step; copied before return).
+ * workspace: device, gptb_polar_express_workspace_bytes(m, n, steps) bytes.
+ * Errors: GPTB_ERR_INVALID_ARG (m or n not a positive multiple of 8, steps
+ * < 1 or > 64, null pointers), GPTB_ERR_WORKSPACE (too small),
+ * GPTB_ERR_UNSUPPORTED (not an sm_100 device). */
+int gptb_polar_express(const void* G, void* out, int m, int n, const float* coeffs, int steps, void* workspace,
+                       size_t workspace_bytes, gptb_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word.
  * Returns GPTB_OK, GPTB_ERR_TIMEOUT if a bounded wait inside a kernel expired
  * (the kernel recorded it, drained and returned), or GPTB_ERR_CUDA. */

@@ -97,3 +97,29 @@ def test_unknown_dtype_unsupported(gb):
     w = gb.BlockWeights()
     assert lib.gpt_block_forward(ctypes.byref(cfg), 0, ctypes.byref(w), None, None, None, None, None, None,
                                  None) == gb.ERR_UNSUPPORTED
+
+
+def test_optimizer_entry_points_validate_on_the_host(gb):
+    lib = gb.load()
+    # workspace: 0 for bad shapes, grows with the matrix and the Gram side
+    assert gb.gptb_polar_express_workspace_bytes(0, 8, 2) == 0
+    assert gb.gptb_polar_express_workspace_bytes(8, 8, 0) == 0
+    assert gb.gptb_polar_express_workspace_bytes(8, 8, 65) == 0
+    small = gb.gptb_polar_express_workspace_bytes(64, 32, 5)
+    assert small >= 1024 + 2 * 64 * 32 * 2 + 2 * 32 * 32 * 2
+    assert gb.gptb_polar_express_workspace_bytes(32, 64, 5) == small  # wide: same buffers
+    coeffs = (ctypes.c_float * 3)(1.5, -0.5, 0.0)
+    # shapes that are not multiples of 8, bad step counts and null pointers are rejected before any CUDA call
+    for m, n, steps in ((12, 8, 1), (8, 12, 1), (8, 8, 0), (8, 8, 65)):
+        assert lib.gptb_polar_express(16, 4096, m, n, coeffs, steps, 256, 1 << 20, None) == gb.ERR_INVALID_ARG
+    assert lib.gptb_polar_express(None, 4096, 8, 8, coeffs, 1, 256, 1 << 20, None) == gb.ERR_INVALID_ARG
+    # out overlapping G
+    assert lib.gptb_polar_express(4096, 4096 + 64, 8, 8, coeffs, 1, 256, 1 << 20, None) == gb.ERR_INVALID_ARG
+    # too small a workspace
+    assert lib.gptb_polar_express(4096, 1 << 16, 8, 8, coeffs, 1, 256, 16, None) == gb.ERR_WORKSPACE
+    # AdamW: null arrays, negative n, step 0, beta outside [0, 1)
+    assert lib.gptb_adamw_step(None, 16, 32, 48, None, 4, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, None) == gb.ERR_INVALID_ARG
+    assert lib.gptb_adamw_step(16, 16, 32, 48, None, -1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, None) == gb.ERR_INVALID_ARG
+    assert lib.gptb_adamw_step(16, 16, 32, 48, None, 4, 1e-3, 0.9, 0.999, 1e-8, 0.0, 0, None) == gb.ERR_INVALID_ARG
+    assert lib.gptb_adamw_step(16, 16, 32, 48, None, 4, 1e-3, 1.0, 0.999, 1e-8, 0.0, 1, None) == gb.ERR_INVALID_ARG
+    assert lib.gptb_adamw_step(16, 16, 32, 48, None, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, None) == gb.OK

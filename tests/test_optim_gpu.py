@@ -1,0 +1,72 @@
+"""Optimizer-step kernels through the C ABI against the fp64 oracle
+(oracle/optim.py): AdamW (fp32, 1e-5) and the Polar Express
+orthogonalisation on the tensor-core GEMM (bf16 operands and stores, 2e-2)."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import TOL, relerr
+from oracle import optim as oo
+
+pytestmark = pytest.mark.gpu
+
+PAGE_TUPLES = [(8.156, -22.483, 15.879), (4.043, -2.809, 0.500)]
+
+
+@pytest.mark.parametrize("n", [4096, 4099, 1])
+def test_adamw_step_matches_oracle(cuda_lib, n):
+    gb = cuda_lib
+    rng = np.random.default_rng(11)
+    p0 = rng.standard_normal(n).astype(np.float32)
+    hp = dict(lr=2e-3, beta1=0.8, beta2=0.95, eps=1e-10, weight_decay=0.05)
+    p, m, v = (torch.tensor(x, device="cuda") for x in (p0, np.zeros(n, np.float32), np.zeros(n, np.float32)))
+    pb = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    rp, rm, rv = p0.astype(np.float64), np.zeros(n), np.zeros(n)
+    for t in range(1, 4):
+        g = rng.standard_normal(n).astype(np.float32)
+        gb.gptb_adamw_step(p, torch.tensor(g, device="cuda"), m, v, pb, n, hp["lr"], hp["beta1"], hp["beta2"],
+                           hp["eps"], hp["weight_decay"], t)
+        rp, rm, rv = oo.adamw_step(rp, g, rm, rv, t, hp["lr"], hp["beta1"], hp["beta2"], hp["eps"],
+                                   hp["weight_decay"])
+    torch.cuda.synchronize()
+    assert relerr(p.double().cpu().numpy() - p0, rp - p0) <= TOL["f32"] * 10  # the update itself, to 1e-4
+    assert relerr(p.double().cpu().numpy(), rp) <= TOL["f32"]
+    assert relerr(m.double().cpu().numpy(), rm) <= TOL["f32"]
+    assert relerr(v.double().cpu().numpy(), rv) <= TOL["f32"]
+    # the bf16 copy is the round-to-nearest of the fp32 result
+    assert torch.equal(pb, p.bfloat16())
+
+
+@pytest.mark.parametrize("shape", [(256, 128), (192, 192), (128, 384), (1536, 6144)])
+def test_polar_express_matches_oracle(cuda_lib, shape):
+    gb = cuda_lib
+    m, n = shape
+    g = torch.Generator().manual_seed(5)
+    G = (torch.randn(m, n, generator=g) * 0.02).bfloat16()
+    out = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(gb.gptb_polar_express_workspace_bytes(m, n, len(PAGE_TUPLES)), dtype=torch.uint8,
+                     device="cuda")
+    gb.gptb_polar_express(G.cuda(), out, m, n, PAGE_TUPLES, ws)
+    torch.cuda.synchronize()
+    assert gb.gptb_device_error() == 0
+    ref = oo.polar_express(G.double().numpy(), PAGE_TUPLES)
+    # bf16 stores of X, A and B in each step: a float model of that rounding gives 6e-3 for these sizes
+    assert relerr(out.double().cpu().numpy(), ref) <= TOL["bf16"]
+
+
+def test_polar_express_single_step_singular_values(cuda_lib):
+    """One step maps singular values by a s + b s^3 + c s^5 (property, any size)."""
+    gb = cuda_lib
+    m, n = 512, 256
+    g = torch.Generator().manual_seed(9)
+    G = (torch.randn(m, n, generator=g)).bfloat16()
+    out = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(gb.gptb_polar_express_workspace_bytes(m, n, 1), dtype=torch.uint8, device="cuda")
+    a, b, c = PAGE_TUPLES[1]
+    gb.gptb_polar_express(G.cuda(), out, m, n, [(a, b, c)], ws)
+    torch.cuda.synchronize()
+    X = G.double().numpy()
+    s = np.linalg.svd(X / np.linalg.norm(X), compute_uv=False)
+    want = np.sort(np.abs(a * s + b * s ** 3 + c * s ** 5))[::-1]
+    got = np.linalg.svd(out.double().cpu().numpy(), compute_uv=False)
+    assert np.max(np.abs(got - want)) / want.max() <= TOL["bf16"]
