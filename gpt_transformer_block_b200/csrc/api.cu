@@ -955,9 +955,11 @@ int gptb_polar_express(const void* G, void* out, int m, int n, const float* coef
   const int s = wide ? m : n;  // side of the Gram matrix
   bf16* A = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(ne * 2));
   bf16* Bm = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(ne * 2) + pe_align((size_t)s * s * 2));
-  // the coefficients go through the stream (the host array is read before this returns)
-  CK(cudaMemcpyAsync(cf, coeffs, sizeof(float) * 3 * steps, cudaMemcpyHostToDevice, st));
-  CK(cudaMemsetAsync(sumsq, 0, sizeof(float), st));
+  // the coefficients travel in the launch parameters (the host array is read here)
+  HostFloats192 hc;
+  std::memcpy(hc.v, coeffs, sizeof(float) * 3 * steps);
+  store_floats_kernel<<<1, 32, 0, st>>>(hc, 3 * steps, cf, sumsq);
+  CKL();
   const int grid = (int)std::max<long long>(1, std::min<long long>(((long long)ne + 255) / 256, dev_info().sms * 8LL));
   sumsq_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16*>(G), (long long)ne, sumsq);
   CKL();

@@ -332,6 +332,16 @@ __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
   }
 }
 
+// small host arrays (Polar Express coefficients) reach the device through the
+// launch parameters: no pageable host copy, nothing that waits on the host
+struct HostFloats192 {
+  float v[192];
+};
+__global__ void store_floats_kernel(HostFloats192 src, int n, float* __restrict__ dst, float* __restrict__ zero) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src.v[i];
+  if (threadIdx.x == 0 && zero) *zero = 0.f;
+}
+
 // sum of squares of a bf16 array into *out (fp32, zeroed by the caller)
 __global__ void __launch_bounds__(256) sumsq_bf16_kernel(const bf16* __restrict__ x, long long n, float* __restrict__ out) {
   __shared__ float sred[8];
