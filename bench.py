@@ -270,6 +270,41 @@ def run_optimizer(args, c: dict):
     print(json.dumps(line))
 
 
+def run_decode(args, c: dict):
+    """One decode step of attention over a full KV cache of the workload's
+    shape (B sequences of T cached tokens, every layer's heads; the newest token
+    of each sequence attends to all its keys).  Bound by reading the cache."""
+    import gpt_transformer_block_b200 as gb
+    gb.load()
+    B, T, H, Hk = c["B"], c["T"], c["n_head"], c["n_kv_head"]
+    g = torch.Generator(device="cuda").manual_seed(3)
+    q = torch.randn(B, H, 128, device="cuda", generator=g).bfloat16()
+    k = torch.randn(B, T, Hk, 128, device="cuda", generator=g).bfloat16()
+    v = torch.randn(B, T, Hk, 128, device="cuda", generator=g).bfloat16()
+    lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    o = torch.empty(B, H, 128, dtype=torch.bfloat16, device="cuda")
+    for _ in range(args.warmup):
+        gb.gptb_decode_attention(q, k, v, lens, o, None, B, H, Hk, T, -1)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        gb.gptb_decode_attention(q, k, v, lens, o, None, B, H, Hk, T, -1)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    nbytes = 2 * B * T * Hk * 128 * 2 + 2 * B * H * 128 * 2  # K and V caches, q and o
+    gbs = nbytes / (us * 1e-6) / 1e9
+    peak = measured_peaks()["hbm_gbs"]
+    print(json.dumps({"metric": "decode attention step time (one layer, full cache)", "value": us, "unit": "us",
+                      "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
+                      "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": c["name"] + "_decode", "batch": B, "cached_tokens": T, "heads": H,
+                                 "kv_heads": Hk},
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                                   "frac": gbs / peak, "bytes": nbytes}}))
+
+
 def run_reference(args, c: dict, fl: dict):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -311,6 +346,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
     ap.add_argument("--optimizer", action="store_true",
                     help="time the optimizer step (Polar Express + AdamW) instead of the training step")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one decode step of attention over a full KV cache instead of the training step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -327,9 +364,9 @@ def main():
     if args.impl == "reference":
         run_reference(args, c, fl)
         return
-    if args.optimizer:
+    if args.optimizer or args.decode:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        run_optimizer(args, c)
+        (run_optimizer if args.optimizer else run_decode)(args, c)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -23,7 +23,7 @@ EXPORTS = [
     "gpt_stack_step", "gptb_gemm_bf16", "gptb_device_error", "gptb_set_wait_limit_ns",
     "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
     "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
-    "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express",
+    "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express", "gptb_decode_attention",
 ]
 
 _vp = ctypes.c_void_p
@@ -99,6 +99,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptb_polar_express_workspace_bytes.restype = ctypes.c_size_t
     lib.gptb_polar_express.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _fp, ctypes.c_int, _vp,
                                        ctypes.c_size_t, _vp]
+    lib.gptb_decode_attention.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, _vp]
     for name in EXPORTS:
         if name not in ("gptb_workspace_bytes", "gptb_error_string", "gptb_reset_counters",
                         "gptb_launch_count", "gptb_polar_express_workspace_bytes"):
@@ -243,6 +245,13 @@ def gptb_polar_express(G, out, m, n, coeffs, workspace, stream=None):
     nbytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
     _check(load().gptb_polar_express(ptr(G), ptr(out), int(m), int(n), arr, len(coeffs), ptr(workspace),
                                      nbytes, _stream(stream)), "gptb_polar_express")
+
+
+def gptb_decode_attention(q, k_cache, v_cache, lens, o, lse, B, H, Hkv, T_max, window, stream=None):
+    """One decode step: attention of each sequence's newest token over its KV cache."""
+    _check(load().gptb_decode_attention(ptr(q), ptr(k_cache), ptr(v_cache), ptr(lens), ptr(o), ptr(lse), int(B),
+                                        int(H), int(Hkv), int(T_max), int(window), _stream(stream)),
+           "gptb_decode_attention")
 
 
 def gptb_device_error(stream=None) -> int:

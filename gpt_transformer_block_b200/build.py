@@ -13,7 +13,8 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libgptblock.so")
 SOURCES = ["api.cu"]
-DEPS = ["api.cu", "common.cuh", "gemm.cuh", "attention.cuh", "attention_tc.cuh", "elementwise.cuh", "rows.cuh"]
+DEPS = ["api.cu", "common.cuh", "gemm.cuh", "attention.cuh", "attention_tc.cuh", "elementwise.cuh", "rows.cuh",
+        "decode.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -16,6 +16,7 @@
 #include "attention.cuh"
 #include "attention_tc.cuh"
 #include "common.cuh"
+#include "decode.cuh"
 #include "elementwise.cuh"
 #include "rows.cuh"
 #include "gemm.cuh"
@@ -988,6 +989,27 @@ int gptb_polar_express(const void* G, void* out, int m, int n, const float* coef
       TRY(gemm(GPTB_BF16, {Bm, s, false}, {cur, n, true}, m, n, m, ex, st));
     cur = nxt;
   }
+  return GPTB_OK;
+}
+
+// --------------------------------------------------------------- decode --
+
+int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, void* o,
+                          float* lse, int B, int H, int Hkv, int T_max, int window, gptb_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !lens || !o || B < 0 || H <= 0 || Hkv <= 0 || H % Hkv || T_max <= 0)
+    return GPTB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return GPTB_ERR_INVALID_ARG;
+  if (B == 0) return GPTB_OK;
+  const int G = H / Hkv;
+  const size_t smem = decode_smem_bytes(G, T_max);
+  if (G > 16 || smem > 220 * 1024) return GPTB_ERR_UNSUPPORTED;  // scores of the whole cache stay in shared memory
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (smem > 48 * 1024)
+    CK(cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  decode_attn_kernel<<<B * Hkv, DEC_THREADS, smem, st>>>(
+      static_cast<const bf16*>(q), static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache), lens,
+      static_cast<bf16*>(o), lse, H, Hkv, T_max, window);
+  CKL();
   return GPTB_OK;
 }
 

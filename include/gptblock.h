@@ -229,7 +229,29 @@ size_t gptb_polar_express_workspace_bytes(int m, int n, int steps);
 int gptb_polar_express(const void* G, void* out, int m, int n, const float* coeffs, int steps, void* workspace,
                        size_t workspace_bytes, gptb_stream_t stream);
 
-/* Synchronises `stream`, then reads and clears the device error word.
+/* ---------------------------------------------------------- decode ----
+ * One generation step of the inference engine (apidog.com/fr "Comment
+ * Entraîner Votre Propre ChatGPT Pour 50€ ?", § 6 "Moteur d'inférence": a KV
+ * cache filled at prefill, one new token per sequence per step): attention of
+ * each sequence's newest token over its cache, with the training attention's
+ * causal window and grouped-query heads (kv head of q head h = h / (H/H_kv)),
+ * softmax scale 1/sqrt(128).
+ *   q:       device bf16 [B, H, 128], the new tokens' (normalised, rotated) queries
+ *   k_cache, v_cache: device bf16 [B, T_max, H_kv, 128] (row stride H_kv*128,
+ *            sequence stride T_max*H_kv*128) holding positions 0..lens[b]-1 of
+ *            sequence b, the new token's own k and v included
+ *   lens:    device int32 [B]; a sequence with lens[b] outside 1..T_max gets
+ *            o = 0 and lse = -inf
+ *   window:  -1 = every cached key; W >= 0 keeps keys lens[b]-1-W .. lens[b]-1
+ *   o:       device bf16 [B, H, 128]; lse: device fp32 [B, H] (natural log of
+ *            the softmax denominator incl. its max) or NULL
+ * Errors: GPTB_ERR_INVALID_ARG (null / misaligned pointers, H % H_kv != 0),
+ * GPTB_ERR_UNSUPPORTED (more than 16 query heads per kv head, or a cache too
+ * long for the per-CTA score buffer: (H/H_kv) * (T_max + 128) floats <= 220 KB). */
+int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, void* o,
+                          float* lse, int B, int H, int Hkv, int T_max, int window, gptb_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word./* Synchronises `stream`, then reads and clears the device error word.
  * Returns GPTB_OK, GPTB_ERR_TIMEOUT if a bounded wait inside a kernel expired
  * (the kernel recorded it, drained and returned), or GPTB_ERR_CUDA. */
 int gptb_device_error(gptb_stream_t stream);
