@@ -305,6 +305,17 @@ def run_decode(args, c: dict):
                                    "frac": gbs / peak, "bytes": nbytes}}))
 
 
+METRIC = "training tokens/sec (fwd+bwd) on 1 B200 and MFU vs bf16/FP8 tensor peak"
+
+
+def step_config(c: dict, world: int) -> dict:
+    """The `config` object of the training-step line (both arms)."""
+    return {"workload": c["name"], "global_batch": c["B"] * world, "seq_len": c["T"],
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "n_layer": c["n_layer"], "d_model": c["d"], "vocab": c["vocab"],
+            "l2": "working set (~40 GB of saved activations) far larger than L2; no flush"}
+
+
 def run_reference(args, c: dict, fl: dict):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -317,10 +328,10 @@ def run_reference(args, c: dict, fl: dict):
             vals.append(info["tok_per_s"])
     v = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": "training tokens/sec (fwd+bwd)", "value": v, "unit": "tokens/s",
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": c["name"], "global_batch": c["B"], "seq_len": c["T"], "parallelism": "cpu"},
+        "config": step_config(c, 1),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
                          "sample": info["sample"]},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -450,14 +461,12 @@ def main():
     gemm_tflops = gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     peak_t = peaks["bf16_tflops_sustained"]
     line = {
-        "metric": "training tokens/sec (fwd+bwd) on 1 B200 and MFU vs bf16 tensor peak",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": c["name"], "global_batch": c["B"] * world, "seq_len": c["T"],
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "n_layer": c["n_layer"], "d_model": c["d"], "vocab": c["vocab"],
-                   "l2": "working set (~40 GB of saved activations) far larger than L2; no flush"},
+        "dtype": "bf16" if c["dtype"] != "fp8" else "fp8 e4m3 (forward and input-gradient GEMMs) / bf16",
+        "data": "synthetic",
+        "config": step_config(c, world),
         "mfu": {"algorithmic_flops_per_token": fl["algorithmic"],
                 "pages_flops_per_token": fl["pages_convention"],
                 "vs_nominal_2250": flops_s / 2.25e15,
