@@ -464,7 +464,7 @@ def main():
         "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if c["dtype"] != "fp8" else "fp8 e4m3 (forward and input-gradient GEMMs) / bf16",
+        "dtype": {"bf16": "bf16", "fp8": "e4m3/bf16", "f32": "f32"}[c["dtype"]],
         "data": "synthetic",
         "config": step_config(c, world),
         "mfu": {"algorithmic_flops_per_token": fl["algorithmic"],
