@@ -48,3 +48,41 @@ def fp8_matmul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     qa, sa = quantize_e4m3(a)
     qb, sb = quantize_e4m3(b)
     return (qa @ qb) / (sa * sb)
+
+
+# ------------------------------------------------------------ e5m2 (NEXT-4)
+# The gradient variant of the FP8 recipe: e5m2 (1 sign, 5 exponent bits with
+# bias 15, 2 mantissa bits; largest finite 57344, smallest normal 2^-14,
+# subnormal spacing 2^-16) for the gradient operand of the input-gradient
+# GEMMs, the weight operand staying e4m3.  Reading (the pages name FP8 with
+# per-tensor scaling only): scale 57344 / amax, round to nearest (ties to
+# even), saturate at the largest finite value.
+
+E5M2_MAX = 57344.0
+
+
+def e5m2_round(x: np.ndarray) -> np.ndarray:
+    """Nearest e5m2 value to each element (ties to even), saturating to ±57344."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.maximum(a, 2.0 ** -14))
+    e = ex.astype(np.float64) - 1.0
+    ulp = np.exp2(e - 2)
+    y = np.minimum(np.round(a / ulp) * ulp, E5M2_MAX)
+    return np.copysign(y, x)
+
+
+def quantize_e5m2(t: np.ndarray) -> tuple[np.ndarray, float]:
+    """Return (codes as fp64 values, scale) with t ~= codes / scale, scale = 57344 / amax."""
+    t = np.asarray(t, dtype=np.float64)
+    amax = float(np.max(np.abs(t))) if t.size else 0.0
+    s = E5M2_MAX / max(amax, 1e-12)
+    return e5m2_round(t * s), s
+
+
+def fp8_matmul_grad(g: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """g @ w with the gradient g quantised per tensor to e5m2 and the weight w to
+    e4m3, fp64 accumulate (an input-gradient GEMM of the e5m2 variant)."""
+    qg, sg = quantize_e5m2(g)
+    qw, sw = quantize_e4m3(w)
+    return (qg @ qw) / (sg * sw)

@@ -369,3 +369,30 @@ def test_stack_backout_and_smear_switches():
     l_c, _ = om.stack_forward(c, w1, idx, tg)
     l_d, _ = om.stack_forward(dict(c, smear_ch=0), w1, idx, tg)
     assert l_c == l_d
+
+
+# ---------------------------------------------------------------- e5m2 -------
+def test_e5m2_all_codes_are_fixed_points():
+    codes = torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).double().numpy()
+    finite = codes[np.isfinite(codes)]
+    np.testing.assert_array_equal(of.e5m2_round(finite), finite)
+
+
+def test_e5m2_midpoints_and_random_match_torch():
+    codes = torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).double().numpy()
+    grid = np.unique(codes[np.isfinite(codes)])
+    mids = (grid[:-1] + grid[1:]) / 2.0              # exact ties: round half to even
+    x = np.concatenate([mids, RNG.uniform(-57344, 57344, 20000), RNG.standard_normal(20000) * 1e-3])
+    ref = torch.from_numpy(x).to(torch.float8_e5m2).double().numpy()
+    np.testing.assert_array_equal(of.e5m2_round(x), ref)
+
+
+def test_e5m2_saturates_and_mixed_matmul():
+    np.testing.assert_array_equal(of.e5m2_round(np.array([60000.0, 1e9, -70000.0])),
+                                  np.array([57344.0, 57344.0, -57344.0]))
+    # operands on their grids with amax at the format maxima have scale 1: the product is exact
+    g = of.e5m2_round(RNG.uniform(-57344, 57344, (4, 6)))
+    g[0, 0] = 57344.0
+    w = of.e4m3_round(RNG.uniform(-448, 448, (6, 3)))
+    w[0, 0] = 448.0
+    np.testing.assert_allclose(of.fp8_matmul_grad(g, w), g @ w, rtol=0, atol=0)
