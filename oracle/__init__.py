@@ -35,9 +35,10 @@ window W keeps keys t-W..t; kv head of q head h is h // (H/H_kv); the VE gate
 reads the first 32 channels of the normed block input; smear adds the previous
 token's embedding, gated from the current token's first 24 channels; backout
 subtracts the residual entering layer L/2 after the last layer; the loss is the
-mean next-token cross-entropy over all B*T positions; FP8 quantises each GEMM
-operand of the forward and input-gradient GEMMs per tensor with scale
-448/amax, round-to-nearest-even, saturating (weight-gradient GEMMs exact).
+mean next-token cross-entropy over all B*T positions; FP8 quantises each
+operand of every product of the four block GEMMs (forward, input gradient,
+weight gradient), taken as the bf16 tensor it is in the model, per tensor
+with scale 448/amax, round-to-nearest-even, saturating.
 
 Parity status: every function here is pinned by the "not gpu" tests in
 tests/test_oracle_*.py (finite differences, closed forms, invariants, and
@@ -49,4 +50,4 @@ from .model import (  # noqa: F401
     block_forward, block_backward, stack_forward, stack_backward,
     lm_head_xent, smear_forward, smear_backward,
 )
-from .fp8 import e4m3_round, quantize_e4m3, fp8_scale  # noqa: F401
+from .fp8 import bf16_round, e4m3_round, quantize_e4m3, fp8_scale, fp8_matmul  # noqa: F401

@@ -7,6 +7,10 @@ rounded to the nearest e4m3fn value (ties to even) and saturated at ±448.
 
 e4m3fn: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no
 infinities; largest finite 448; smallest normal 2^-6; subnormal spacing 2^-9.
+
+bfloat16 (the activation dtype of the bf16 and FP8 configurations, [AP-lin]):
+1 sign bit, 8 exponent bits (bias 127), 7 stored mantissa bits; largest finite
+(2 - 2^-7) * 2^127; smallest normal 2^-126; subnormal spacing 2^-133.
 """
 from __future__ import annotations
 
@@ -28,6 +32,21 @@ def e4m3_round(x: np.ndarray) -> np.ndarray:
     ulp = np.exp2(e - _MANT_BITS)
     y = np.round(a / ulp) * ulp          # numpy rounds halves to even
     y = np.minimum(y, E4M3_MAX)
+    return np.copysign(y, x)
+
+
+BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Nearest bfloat16 value to each element (ties to even); beyond the
+    largest finite value the result is +-inf (round-to-nearest overflow)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.maximum(a, 2.0 ** -126))
+    ulp = np.exp2(ex.astype(np.float64) - 1.0 - 7.0)
+    y = np.round(a / ulp) * ulp          # numpy rounds halves to even
+    y = np.where(y > BF16_MAX, np.inf, y)
     return np.copysign(y, x)
 
 

@@ -5,20 +5,21 @@ and the readings taken where the pages are silent).
 
 Shapes: activations are [B, T, ...] row-major; weights follow nn.Linear,
 [out, in], and every projection is y = x @ W^T (the Linear of [AP-lin]).
-All arithmetic is float64.  ``fp8=True`` replaces the forward and
-input-gradient products of the four block GEMMs (qkv, attention output, MLP
-fc, MLP proj) by their per-tensor e4m3 emulation from ``fp8.py``; the
-weight-gradient products stay exact.  (Reading of [AP-lin]: "most layers" in
-FP8 with per-tensor scaling.  With e4m3 gradients in the weight-gradient
-products, one-ulp (12.5 %) code flips between two evaluations of the same
-gradient already exceed the 6e-2 bound set for this configuration, so those
-products keep high-precision operands.)
+All arithmetic is float64.  ``fp8=True`` replaces every product of the four
+block GEMMs (qkv, attention output, MLP fc, MLP proj) -- forward, input
+gradient and weight gradient -- by its per-tensor e4m3 emulation from
+``fp8.py``.  Reading of [AP-lin] ("most layers" become FP8 linears with
+per-tensor scaling; the model's activations are bf16, the Linear casting its
+weight to the activation dtype): an FP8 linear quantises the bf16 tensors it
+is given, so each operand is first rounded to bf16 and then scaled by
+448/amax and rounded to e4m3; the products accumulate exactly and are
+rescaled.  The lm_head and the small gate linears stay exact.
 """
 from __future__ import annotations
 
 import numpy as np
 
-from .fp8 import fp8_matmul
+from .fp8 import bf16_round, fp8_matmul
 
 
 def _f64(a) -> np.ndarray:
@@ -30,8 +31,10 @@ def _sigmoid(z):
 
 
 def _mm(a, b, fp8: bool):
-    """Plain matrix product of 2-D operands (optionally e4m3-emulated)."""
-    return fp8_matmul(a, b) if fp8 else a @ b
+    """Plain matrix product of 2-D operands.  FP8: the e4m3 product of the
+    operands as bf16 tensors (each rounded to bf16, then quantised per
+    tensor), accumulated exactly."""
+    return fp8_matmul(bf16_round(a), bf16_round(b)) if fp8 else a @ b
 
 
 def _linear(x, w, fp8=False):
@@ -48,9 +51,9 @@ def _linear_dgrad(dy, w, fp8=False):
     return dx.reshape(*lead, w.shape[1])
 
 
-def _linear_wgrad(dy, x):
+def _linear_wgrad(dy, x, fp8=False):
     """Weight gradient of y = x @ w^T: dw = dy^T @ x, summed over tokens."""
-    return dy.reshape(-1, dy.shape[-1]).T @ x.reshape(-1, x.shape[-1])
+    return _mm(dy.reshape(-1, dy.shape[-1]).T, x.reshape(-1, x.shape[-1]), fp8)
 
 
 # ---------------------------------------------------------------------------
@@ -221,14 +224,14 @@ def block_backward(c, lw, cache, dx2, idx, layer, fp8=False):
     dx2 = _f64(dx2)
     g = {}
     # MLP
-    g["w_proj"] = _linear_wgrad(dx2, cache["act"])
+    g["w_proj"] = _linear_wgrad(dx2, cache["act"], fp8)
     dact = _linear_dgrad(dx2, _f64(lw["w_proj"]), fp8)
     du = dact * 2.0 * np.maximum(cache["u"], 0.0)
-    g["w_fc"] = _linear_wgrad(du, cache["h2"])
+    g["w_fc"] = _linear_wgrad(du, cache["h2"], fp8)
     dh2 = _linear_dgrad(du, _f64(lw["w_fc"]), fp8)
     dx1 = dx2 + rmsnorm_backward(dh2, cache["h2"], cache["r2"])
     # attention output projection
-    g["w_o"] = _linear_wgrad(dx1, cache["o"])
+    g["w_o"] = _linear_wgrad(dx1, cache["o"], fp8)
     do = _linear_dgrad(dx1, _f64(lw["w_o"]), fp8).reshape(B, T, H, hd)
     dxm = dx1.copy()
     dqr, dkr, dv = attention_backward(cache["qr"], cache["kr"], cache["v"], do,
@@ -252,7 +255,7 @@ def block_backward(c, lw, cache, dx2, idx, layer, fp8=False):
         g["ve_table"] = dtab
     dqkv = np.concatenate([dq.reshape(B, T, H * hd), dk.reshape(B, T, Hk * hd),
                            dv.reshape(B, T, Hk * hd)], axis=-1)
-    g["w_qkv"] = _linear_wgrad(dqkv, cache["h"])
+    g["w_qkv"] = _linear_wgrad(dqkv, cache["h"], fp8)
     dh = dh + _linear_dgrad(dqkv, _f64(lw["w_qkv"]), fp8)
     dxm = dxm + rmsnorm_backward(dh, cache["h"], cache["r1"])
     a, b = float(lw["resid_lambda"]), float(lw["x0_lambda"])

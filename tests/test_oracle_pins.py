@@ -55,6 +55,77 @@ def test_fp8_matmul_exact_on_representable_operands():
     np.testing.assert_allclose(of.fp8_matmul(a, b), a @ b, rtol=0, atol=0)
 
 
+def test_fp8_matmul_closed_forms_at_non_unit_scales():
+    # 1x1: the single element is its own amax, so it maps to 448 exactly and back
+    np.testing.assert_array_equal(of.fp8_matmul(np.array([[3.0]]), np.array([[5.0]])), [[15.0]])
+    # 2x2 by hand: amax(a) = 2, scale 224; 0.3 * 224 = 67.2 lies between the e4m3
+    # neighbours 64 and 72 (spacing 8 in [64, 128)) and rounds to 64, i.e. 2/7;
+    # 1*224, 0.5*224 and 2*224 are on the grid.  b = [[1, 3], [2, 0.75]] has
+    # amax 3, scale 448/3: 1 -> 149.33 -> 144 (spacing 16 in [128, 256)), i.e.
+    # 144*3/448 = 27/28; 2 -> 298.67 -> 288, i.e. 27/14; 3 -> 448 exactly;
+    # 0.75 -> 112 exactly.
+    a = np.array([[1.0, 0.3], [0.5, 2.0]])
+    b = np.array([[1.0, 3.0], [2.0, 0.75]])
+    qa = np.array([[1.0, 2.0 / 7.0], [0.5, 2.0]])
+    qb = np.array([[27.0 / 28.0, 3.0], [27.0 / 14.0, 0.75]])
+    np.testing.assert_allclose(of.fp8_matmul(a, b), qa @ qb, rtol=1e-15, atol=0)
+    q, s = of.quantize_e4m3(a)
+    assert s == 224.0
+    np.testing.assert_array_equal(q, [[224.0, 64.0], [112.0, 448.0]])
+
+
+def test_fp8_matmul_power_of_two_scaling_is_exact():
+    # scaling an operand by 2^k scales its amax by 2^k and its scale by 2^-k:
+    # the codes are unchanged and the product scales by exactly 2^k
+    a, b = rnd(6, 9), rnd(9, 4, scale=0.03)
+    base = of.fp8_matmul(a, b)
+    for k, m in ((3, 0), (-5, 2), (7, -9)):
+        np.testing.assert_array_equal(of.fp8_matmul(a * 2.0 ** k, b * 2.0 ** m), base * 2.0 ** (k + m))
+
+
+def test_fp8_matmul_error_bound_and_torch_casts():
+    # per element: |fp8(a) fp8(b) - ab| <= sum_k |a||b| ((1+u)^2 - 1) + subnormal terms,
+    # u = 2^-4 the unit roundoff of e4m3 (3 mantissa bits); codes below 2^-6 carry an
+    # absolute error of at most 2^-10 before rescaling
+    a, b = rnd(12, 40), rnd(40, 7, scale=5.0)
+    a[3, 4] = 1e-5  # lands in the subnormal range after scaling
+    sa, sb = of.fp8_scale(a), of.fp8_scale(b)
+    u = 2.0 ** -4
+    ea = np.abs(a) * u + 2.0 ** -10 / sa
+    eb = np.abs(b) * u + 2.0 ** -10 / sb
+    bound = np.abs(a) @ eb + ea @ np.abs(b) + ea @ eb
+    err = np.abs(of.fp8_matmul(a, b) - a @ b)
+    assert np.all(err <= bound * (1 + 1e-12))
+    # the same product from torch's own e4m3 casts of the scaled operands
+    ta = (torch.from_numpy(a) * sa).float().to(torch.float8_e4m3fn).double()
+    tb = (torch.from_numpy(b) * sb).float().to(torch.float8_e4m3fn).double()
+    np.testing.assert_allclose(of.fp8_matmul(a, b), ((ta @ tb) / (sa * sb)).numpy(), rtol=1e-13, atol=0)
+
+
+def test_bf16_round_matches_torch():
+    bits = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    codes = bits.double().numpy()
+    finite = codes[np.isfinite(codes)]
+    np.testing.assert_array_equal(of.bf16_round(finite), finite)
+    pos = np.unique(finite[finite > 0])
+    mids = (pos[1:] + pos[:-1]) / 2                     # exact ties: round to even
+    x = np.concatenate([mids, -mids, RNG.standard_normal(20000) * 3.0, RNG.standard_normal(2000) * 1e-39])
+    ref = torch.from_numpy(x).float().to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(of.bf16_round(x), ref)
+    assert np.isinf(of.bf16_round(np.array([3.4e38]))[0])
+
+
+def test_fp8_block_product_quantises_bf16_tensors():
+    # the FP8 product of the model acts on bf16 tensors: x = 0.265625 + 2^-12
+    # rounds to 0.265625 in bf16 (spacing 2^-9 in [0.25, 0.5)); with amax 1.75
+    # the scale is 256, so the bf16 value maps to 68, the e4m3 tie between 64
+    # and 72, which goes to 64 (even).  Unrounded, 68.0625 would go to 72.
+    a = np.array([[1.75, 0.265625 + 2.0 ** -12]])
+    ones = np.array([[1.0], [1.0]])
+    np.testing.assert_array_equal(om._mm(a, ones, True), [[1.75 + 64.0 / 256.0]])
+    np.testing.assert_array_equal(of.fp8_matmul(a, ones), [[1.75 + 72.0 / 256.0]])
+
+
 # ------------------------------------------------------------- RMSNorm -------
 
 def test_rmsnorm_matches_torch_and_unit_rms():

@@ -93,6 +93,35 @@ def test_ve_gate_scale_is_caught(monkeypatch):
     _fails(pins.test_block_special_cases)
 
 
+def test_fp8_inverted_scale_is_caught(monkeypatch):
+    from oracle import fp8 as of
+
+    def bad(a, b):  # multiplies by the scales instead of dividing by them
+        qa, sa = of.quantize_e4m3(a)
+        qb, sb = of.quantize_e4m3(b)
+        return (qa @ qb) * (sa * sb)
+    monkeypatch.setattr(of, "fp8_matmul", bad)
+    _fails(pins.test_fp8_matmul_closed_forms_at_non_unit_scales)
+    _fails(pins.test_fp8_matmul_error_bound_and_torch_casts)
+
+
+def test_fp8_one_scale_for_both_operands_is_caught(monkeypatch):
+    from oracle import fp8 as of
+
+    def bad(a, b):  # b quantised with a's scale
+        qa, sa = of.quantize_e4m3(a)
+        qb = of.e4m3_round(np.asarray(b, dtype=np.float64) * sa)
+        return (qa @ qb) / (sa * sa)
+    monkeypatch.setattr(of, "fp8_matmul", bad)
+    _fails(pins.test_fp8_matmul_closed_forms_at_non_unit_scales)
+
+
+def test_fp8_missing_bf16_rounding_is_caught(monkeypatch):
+    from oracle import fp8 as of
+    monkeypatch.setattr(om, "_mm", lambda a, b, fp8: of.fp8_matmul(a, b) if fp8 else a @ b)
+    _fails(pins.test_fp8_block_product_quantises_bf16_tensors)
+
+
 # ----------------------------------------------------------- optimizer oracle
 import numpy as np  # noqa: E402
 from oracle import optim as oo  # noqa: E402
