@@ -168,3 +168,33 @@ def test_adamw_coupled_weight_decay_is_caught(monkeypatch):
         return orig(p, np.asarray(g) + weight_decay * np.asarray(p), m, v, t, lr, beta1, beta2, eps, 0.0)
     monkeypatch.setattr(oo, "adamw_step", bad)
     _fails(opins.test_adamw_matches_torch_over_steps)
+
+
+def test_normuon_reduction_axis_is_caught(monkeypatch):
+    def bad(o, v, beta2, eps=1e-10):  # per-column statistics instead of per-row (neuron)
+        o = np.asarray(o, dtype=np.float64)
+        v_mean = np.mean(o * o, axis=0)
+        v_norm = np.sqrt(np.sum(v_mean))
+        v = beta2 * np.resize(np.asarray(v, dtype=np.float64), v_mean.shape) + (1.0 - beta2) * v_mean
+        step = 1.0 / np.sqrt(np.maximum(v, eps))
+        new = np.sqrt(np.sum(v_mean * step ** 2))
+        return o * (step * v_norm / max(new, eps))[None, :], v
+    monkeypatch.setattr(oo, "normuon_scale", bad)
+    with pytest.raises((AssertionError, ValueError)):  # wrong shapes or wrong values
+        opins.test_normuon_keeps_the_norm_and_equalises_rows()
+
+
+def test_muon_without_nesterov_is_caught(monkeypatch):
+    def bad(g, buf, mu):
+        buf = mu * np.asarray(buf, dtype=np.float64) + np.asarray(g, dtype=np.float64)
+        return buf, buf
+    monkeypatch.setattr(oo, "muon_momentum", bad)
+    _fails(opins.test_muon_nesterov_momentum_closed_form)
+
+
+def test_polar_express_coefficient_typo_is_caught(monkeypatch):
+    bad = list(oo.POLAR_EXPRESS_COEFFS)
+    a, b, c = bad[3]
+    bad[3] = (a + 0.05, b, c)
+    monkeypatch.setattr(oo, "POLAR_EXPRESS_COEFFS", bad)
+    _fails(opins.test_coefficients_follow_the_greedy_minimax_construction)
