@@ -105,3 +105,11 @@ def fp8_matmul_grad(g: np.ndarray, w: np.ndarray) -> np.ndarray:
     qg, sg = quantize_e5m2(g)
     qw, sw = quantize_e4m3(w)
     return (qg @ qw) / (sg * sw)
+
+
+# ------------------------------------------------- fixed-scale quantisation
+def quantize_fixed(t: np.ndarray, scale: float, fmt: str = "e4m3") -> np.ndarray:
+    """Codes (as fp64 values) of t * scale rounded to e4m3 or e5m2, for a tensor
+    whose per-tensor scale is known in advance rather than measured."""
+    r = e4m3_round if fmt == "e4m3" else e5m2_round
+    return r(np.asarray(t, dtype=np.float64) * scale)

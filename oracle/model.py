@@ -13,13 +13,23 @@ per-tensor scaling; the model's activations are bf16, the Linear casting its
 weight to the activation dtype): an FP8 linear quantises the bf16 tensors it
 is given, so each operand is first rounded to bf16 and then scaled by
 448/amax and rounded to e4m3; the products accumulate exactly and are
-rescaled.  The lm_head and the small gate linears stay exact.
+rescaled.  The small gate linears stay exact.
+
+Variants (NEXT rows of the same reading): ``fp8="e5m2"`` quantises the
+gradient operand of the input-gradient and weight-gradient products to e5m2
+(scale 57344/amax) instead of e4m3; a config with ``fp8_lm_head`` also runs
+the lm_head products in FP8: the logits from e4m3 casts of hf and W_lm, and
+the two gradient products from the logits gradient dz, whose entries
+(softmax - onehot)/n lie in [-1/n, 1/n], quantised with the per-tensor
+scale that bound fixes (448 n, or 57344 n for e5m2), so that splitting the
+rows into chunks does not change the product.  Without ``fp8_lm_head`` the
+lm_head stays exact.
 """
 from __future__ import annotations
 
 import numpy as np
 
-from .fp8 import bf16_round, fp8_matmul
+from .fp8 import E4M3_MAX, E5M2_MAX, bf16_round, fp8_matmul, fp8_matmul_grad, quantize_e4m3, quantize_fixed
 
 
 def _f64(a) -> np.ndarray:
@@ -30,11 +40,16 @@ def _sigmoid(z):
     return 1.0 / (1.0 + np.exp(-z))
 
 
-def _mm(a, b, fp8: bool):
+def _mm(a, b, fp8, grad=False):
     """Plain matrix product of 2-D operands.  FP8: the e4m3 product of the
     operands as bf16 tensors (each rounded to bf16, then quantised per
-    tensor), accumulated exactly."""
-    return fp8_matmul(bf16_round(a), bf16_round(b)) if fp8 else a @ b
+    tensor), accumulated exactly; with fp8 == "e5m2" a gradient operand a
+    (grad=True) is quantised to e5m2 instead."""
+    if not fp8:
+        return a @ b
+    if grad and fp8 == "e5m2":
+        return fp8_matmul_grad(bf16_round(a), bf16_round(b))
+    return fp8_matmul(bf16_round(a), bf16_round(b))
 
 
 def _linear(x, w, fp8=False):
@@ -47,13 +62,13 @@ def _linear(x, w, fp8=False):
 def _linear_dgrad(dy, w, fp8=False):
     """Input gradient of y = x @ w^T: dx = dy @ w."""
     lead = dy.shape[:-1]
-    dx = _mm(dy.reshape(-1, dy.shape[-1]), w, fp8)
+    dx = _mm(dy.reshape(-1, dy.shape[-1]), w, fp8, grad=True)
     return dx.reshape(*lead, w.shape[1])
 
 
 def _linear_wgrad(dy, x, fp8=False):
     """Weight gradient of y = x @ w^T: dw = dy^T @ x, summed over tokens."""
-    return _mm(dy.reshape(-1, dy.shape[-1]).T, x.reshape(-1, x.shape[-1]), fp8)
+    return _mm(dy.reshape(-1, dy.shape[-1]).T, x.reshape(-1, x.shape[-1]), fp8, grad=True)
 
 
 # ---------------------------------------------------------------------------
@@ -302,13 +317,14 @@ def smear_backward(dy, x, sg, w_gate, lam):
 # [JA-tok] vocabulary 32768).  Reading: mean over all B*T positions.
 # ---------------------------------------------------------------------------
 
-def lm_head_xent(h, w_lm, targets):
-    """Returns (loss, dh, dw_lm) for loss = mean_t(logsumexp(z_t) - z_t[y_t])."""
+def lm_head_xent(h, w_lm, targets, fp8=False):
+    """Returns (loss, dh, dw_lm) for loss = mean_t(logsumexp(z_t) - z_t[y_t]).
+    fp8 (True or "e5m2"): the FP8 lm_head of the module docstring."""
     h = _f64(h)
     w = _f64(w_lm)
     hf = h.reshape(-1, h.shape[-1])
     y = np.asarray(targets).reshape(-1)
-    z = hf @ w.T
+    z = _mm(hf, w.T, fp8)
     m = z.max(axis=1, keepdims=True)
     e = np.exp(z - m)
     zs = e.sum(axis=1, keepdims=True)
@@ -318,7 +334,15 @@ def lm_head_xent(h, w_lm, targets):
     dz = e / zs
     dz[np.arange(n), y] -= 1.0
     dz /= n
-    return loss, (dz @ w).reshape(h.shape), dz.T @ hf
+    if not fp8:
+        return loss, (dz @ w).reshape(h.shape), dz.T @ hf
+    # |dz| <= 1/n fixes the per-tensor scale of the logits gradient
+    fmt = "e5m2" if fp8 == "e5m2" else "e4m3"
+    s_dz = (E5M2_MAX if fmt == "e5m2" else E4M3_MAX) * n
+    qdz = quantize_fixed(bf16_round(dz), s_dz, fmt)
+    qw, sw = quantize_e4m3(bf16_round(w))
+    qh, sh = quantize_e4m3(bf16_round(hf))
+    return loss, ((qdz @ qw) / (s_dz * sw)).reshape(h.shape), (qdz.T @ qh) / (s_dz * sh)
 
 
 # ---------------------------------------------------------------------------
@@ -349,7 +373,7 @@ def stack_forward(c, w, idx, targets, fp8=False):
     else:
         xf = x
     hf, rf = rmsnorm(xf, c["norm_eps"])
-    loss, dhf, dw_lm = lm_head_xent(hf, w["w_lm"], targets)
+    loss, dhf, dw_lm = lm_head_xent(hf, w["w_lm"], targets, fp8 if c.get("fp8_lm_head") else False)
     cache.update(x0=x0, blocks=blocks, x_bo=x_bo, xL=x, xf=xf, hf=hf, rf=rf,
                  dhf=dhf, dw_lm=dw_lm)
     return loss, cache

@@ -467,3 +467,65 @@ def test_e5m2_saturates_and_mixed_matmul():
     w = of.e4m3_round(RNG.uniform(-448, 448, (6, 3)))
     w[0, 0] = 448.0
     np.testing.assert_allclose(of.fp8_matmul_grad(g, w), g @ w, rtol=0, atol=0)
+
+
+# ------------------------------------------------- FP8 variants (NEXT rows) --
+def test_fp8_matmul_grad_at_non_unit_scales():
+    # 1x1: each operand is its own amax and maps to the format maximum exactly
+    np.testing.assert_allclose(of.fp8_matmul_grad(np.array([[0.3]]), np.array([[7.0]])), [[2.1]], rtol=1e-15)
+    # exact power-of-two scaling, as for e4m3
+    g, w = rnd(5, 8), rnd(8, 3, scale=0.1)
+    base = of.fp8_matmul_grad(g, w)
+    np.testing.assert_array_equal(of.fp8_matmul_grad(g * 2.0 ** -7, w * 8.0), base * 2.0 ** -4)
+    # error bound: e5m2 has unit roundoff 2^-3, e4m3 2^-4 (subnormals absolute)
+    sg, sw = 57344.0 / np.max(np.abs(g)), 448.0 / np.max(np.abs(w))
+    eg = np.abs(g) * 2.0 ** -3 + 2.0 ** -17 / sg
+    ew = np.abs(w) * 2.0 ** -4 + 2.0 ** -10 / sw
+    bound = np.abs(g) @ ew + eg @ np.abs(w) + eg @ ew
+    assert np.all(np.abs(base - g @ w) <= bound * (1 + 1e-12))
+    # against torch's own e5m2 / e4m3 casts of the scaled operands
+    tg = (torch.from_numpy(g) * sg).float().to(torch.float8_e5m2).double()
+    tw = (torch.from_numpy(w) * sw).float().to(torch.float8_e4m3fn).double()
+    np.testing.assert_allclose(base, ((tg @ tw) / (sg * sw)).numpy(), rtol=1e-13, atol=0)
+
+
+def test_fp8_e5m2_mode_quantises_only_gradient_operands():
+    # 0.65 with amax 1: e4m3 scale 448 -> 291.2 -> 288 (spacing 32 in [256, 512));
+    # e5m2 scale 57344 -> 37273.6 -> 40960 (spacing 8192 in [32768, 65536))
+    a = np.array([[1.0, 0.65]])
+    ones = np.array([[1.0], [1.0]])
+    np.testing.assert_allclose(om._mm(a, ones, True, grad=True), [[1.0 + 288.0 / 448.0]], rtol=1e-15)
+    np.testing.assert_allclose(om._mm(a, ones, "e5m2", grad=True), [[1.0 + 40960.0 / 57344.0]], rtol=1e-15)
+    np.testing.assert_allclose(om._mm(a, ones, "e5m2", grad=False), [[1.0 + 288.0 / 448.0]], rtol=1e-15)
+
+
+@pytest.mark.parametrize("mode", [True, "e5m2"])
+def test_fp8_lm_head_matches_torch_casts_and_bound(mode):
+    rng = np.random.default_rng(21)
+    n, d, V = 12, 16, 40
+    h = of.bf16_round(rng.standard_normal((n, d)))
+    w = of.bf16_round(rng.standard_normal((V, d)) * 0.3)
+    y = rng.integers(0, V, n)
+    loss, dh, dw = om.lm_head_xent(h, w, y, fp8=mode)
+    # the same steps from torch: e4m3 casts of h and W with their amax scales,
+    # fp64 softmax of the dequantised product, dz = (softmax - onehot)/n cast
+    # to bf16 and then to the gradient format with the fixed scale qmax * n
+    th, tw = torch.from_numpy(h), torch.from_numpy(w)
+    sh, sw = 448.0 / th.abs().max(), 448.0 / tw.abs().max()
+    qh = (th * sh).float().to(torch.float8_e4m3fn).double()
+    qw = (tw * sw).float().to(torch.float8_e4m3fn).double()
+    z = (qh @ qw.T) / (sh * sw)
+    lse = torch.logsumexp(z, 1)
+    assert abs(loss - float(torch.mean(lse - z[torch.arange(n), torch.from_numpy(y)]))) < 1e-12
+    dz = torch.softmax(z, 1)
+    dz[torch.arange(n), torch.from_numpy(y)] -= 1.0
+    dz = (dz / n).to(torch.bfloat16).double()
+    assert float(dz.abs().max()) <= 1.0 / n
+    fdt, qmax = (torch.float8_e5m2, 57344.0) if mode == "e5m2" else (torch.float8_e4m3fn, 448.0)
+    sdz = qmax * n
+    qdz = (dz * sdz).float().to(fdt).double()
+    np.testing.assert_allclose(dh, ((qdz @ qw) / (sdz * sw)).numpy(), rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(dw, ((qdz.T @ qh) / (sdz * sh)).numpy(), rtol=1e-12, atol=1e-18)
+    # and close to the exact head (FP8 rounding only)
+    l0, dh0, dw0 = om.lm_head_xent(h, w, y)
+    assert abs(loss - l0) < 0.05 * abs(l0)

@@ -198,3 +198,22 @@ def test_polar_express_coefficient_typo_is_caught(monkeypatch):
     bad[3] = (a + 0.05, b, c)
     monkeypatch.setattr(oo, "POLAR_EXPRESS_COEFFS", bad)
     _fails(opins.test_coefficients_follow_the_greedy_minimax_construction)
+
+
+
+def test_fp8_lm_head_dynamic_gradient_scale_is_caught(monkeypatch):
+    from oracle import fp8 as of
+    orig = of.quantize_fixed
+
+    def dynamic(t, scale, fmt="e4m3"):  # the measured amax instead of the 1/n bound
+        t = np.asarray(t, dtype=np.float64)
+        qmax = 448.0 if fmt == "e4m3" else 57344.0
+        return orig(t, qmax / np.max(np.abs(t)), fmt) * (scale / (qmax / np.max(np.abs(t))))
+    monkeypatch.setattr(om, "quantize_fixed", dynamic)
+    _fails(pins.test_fp8_lm_head_matches_torch_casts_and_bound, True)
+
+
+def test_fp8_e5m2_on_the_weight_operand_is_caught(monkeypatch):
+    from oracle import fp8 as of
+    monkeypatch.setattr(om, "fp8_matmul_grad", lambda g, w: of.fp8_matmul_grad(w.T, g.T).T)
+    _fails(pins.test_fp8_e5m2_mode_quantises_only_gradient_operands)
