@@ -13,8 +13,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgptblock.so")
 MAX_LAYERS = 64
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_BAD_INPUT = 0, -1, -2, -3, -4, -5, -6
 F32, BF16, FP8_E4M3 = 0, 1, 2
+FP8_GRAD_E5M2, FP8_LM_HEAD = 1, 2
 WS_BLOCK_SAVED, WS_BLOCK_SCRATCH, WS_LM_HEAD, WS_STACK = 0, 1, 2, 3
 DTYPES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3}
 
@@ -24,6 +25,7 @@ EXPORTS = [
     "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
     "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
     "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express", "gptb_decode_attention",
+    "gptb_muon_workspace_bytes", "gptb_muon_step",
 ]
 
 _vp = ctypes.c_void_p
@@ -38,6 +40,7 @@ class Config(ctypes.Structure):
         ("window", ctypes.c_int * MAX_LAYERS), ("has_ve", ctypes.c_int * MAX_LAYERS),
         ("ve_gate_ch", ctypes.c_int), ("smear_ch", ctypes.c_int), ("backout_layer", ctypes.c_int),
         ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float), ("dtype", ctypes.c_int),
+        ("fp8_flags", ctypes.c_int),
     ]
 
 
@@ -90,7 +93,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptb_reset_counters.restype = None
     lib.gptb_launch_count.restype = ctypes.c_longlong
     lib.gptb_set_gemm_timing.argtypes = [ctypes.c_int]
-    lib.gptb_gemm_timing.argtypes = [P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_longlong)]
+    lib.gptb_gemm_timing.argtypes = [P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_double),
+                                     P(ctypes.c_longlong)]
     lib.gptb_error_string.argtypes = [ctypes.c_int]
     lib.gptb_error_string.restype = ctypes.c_char_p
     lib.gptb_adamw_step.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, ctypes.c_float, ctypes.c_float,
@@ -101,9 +105,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        ctypes.c_size_t, _vp]
     lib.gptb_decode_attention.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, _vp]
+    lib.gptb_muon_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.gptb_muon_workspace_bytes.restype = ctypes.c_size_t
+    lib.gptb_muon_step.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _fp, ctypes.c_int,
+                                   ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp,
+                                   ctypes.c_size_t, _vp]
     for name in EXPORTS:
         if name not in ("gptb_workspace_bytes", "gptb_error_string", "gptb_reset_counters",
-                        "gptb_launch_count", "gptb_polar_express_workspace_bytes"):
+                        "gptb_launch_count", "gptb_polar_express_workspace_bytes", "gptb_muon_workspace_bytes"):
             getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -150,6 +159,7 @@ def make_config(c: dict) -> Config:
     cfg.rope_base = float(c["rope_base"])
     cfg.norm_eps = float(c["norm_eps"])
     cfg.dtype = DTYPES[c["dtype"]] if isinstance(c["dtype"], str) else int(c["dtype"])
+    cfg.fp8_flags = (FP8_GRAD_E5M2 if c.get("fp8_grad") == "e5m2" else 0) | (FP8_LM_HEAD if c.get("fp8_lm_head") else 0)
     return cfg
 
 
@@ -247,6 +257,20 @@ def gptb_polar_express(G, out, m, n, coeffs, workspace, stream=None):
                                      nbytes, _stream(stream)), "gptb_polar_express")
 
 
+def gptb_muon_workspace_bytes(m: int, n: int, steps: int) -> int:
+    return int(load().gptb_muon_workspace_bytes(int(m), int(n), int(steps)))
+
+
+def gptb_muon_step(w, w_bf16, g, buf, v, m, n, coeffs, lr, mu, beta2, weight_decay, workspace, stream=None):
+    """One Muon step (momentum, Polar Express, NorMuon, decoupled decay) on the fp32 [m, n] weight w."""
+    flat = [float(x) for abc in coeffs for x in abc]
+    arr = (ctypes.c_float * len(flat))(*flat)
+    nbytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
+    _check(load().gptb_muon_step(ptr(w), ptr(w_bf16), ptr(g), ptr(buf), ptr(v), int(m), int(n), arr, len(coeffs),
+                                 float(lr), float(mu), float(beta2), float(weight_decay), ptr(workspace), nbytes,
+                                 _stream(stream)), "gptb_muon_step")
+
+
 def gptb_decode_attention(q, k_cache, v_cache, lens, o, lse, B, H, Hkv, T_max, window, stream=None):
     """One decode step: attention of each sequence's newest token over its KV cache."""
     _check(load().gptb_decode_attention(ptr(q), ptr(k_cache), ptr(v_cache), ptr(lens), ptr(o), ptr(lse), int(B),
@@ -280,9 +304,12 @@ def gptb_set_gemm_timing(enable: bool):
 
 
 def gptb_gemm_timing():
-    ms, fl, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_longlong()
-    _check(load().gptb_gemm_timing(ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(n)), "gptb_gemm_timing")
-    return ms.value, fl.value, n.value
+    """(ms, flops, ms of e4m3 GEMMs, flops of e4m3 GEMMs, launches) since the last reset."""
+    ms, fl, ms8, fl8, n = (ctypes.c_double(), ctypes.c_double(), ctypes.c_double(), ctypes.c_double(),
+                           ctypes.c_longlong())
+    _check(load().gptb_gemm_timing(ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(ms8), ctypes.byref(fl8),
+                                   ctypes.byref(n)), "gptb_gemm_timing")
+    return ms.value, fl.value, ms8.value, fl8.value, n.value
 
 
 from .model import GPTStack, BlockRunner, to_device_weights  # noqa: E402,F401

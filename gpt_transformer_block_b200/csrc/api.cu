@@ -32,6 +32,7 @@ bool g_timing = false;
 struct TimedLaunch {
   cudaEvent_t a, b;
   double flops;
+  bool fp8;  // e4m3 operands
 };
 std::vector<TimedLaunch> g_timed;
 std::vector<cudaEvent_t> g_event_pool;
@@ -177,18 +178,79 @@ int plan_splits(int tiles, int kb_total, int sms) {
   return best;
 }
 
-template <bool AM, bool BM, bool F8>
+// Largest number of two-CTA clusters of a pair-form GEMM kernel that fit on
+// the device at once (one CTA per SM); a persistent grid larger than this
+// would leave clusters waiting for others to finish.
+template <class K>
+int max_pair_clusters(K kern, int smem) {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  int& c = cache[dev & 63];
+  if (c == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (dev_info().sms / 2));
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = dev_info().sms / 2;
+    }
+    c = std::min(n, dev_info().sms / 2);
+  }
+  return c;
+}
+
+template <bool AM, bool BM, bool F8, bool PAIR>
 int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const CUtensorMap& to2,
-              const CUtensorMap& tx, int M, int N, int K, int splits, const EpiParams& ep, cudaStream_t st, int sms) {
-  auto kern = gemm_tc_kernel<AM, BM, F8>;
-  const int smem = tc_smem_bytes();
+              const CUtensorMap& tx, int M, int N, int K, int splits, const EpiParams& ep, cudaStream_t st) {
+  auto kern = gemm_tc_kernel<AM, BM, F8, PAIR>;
+  const int smem = TcShape<PAIR>::SMEM;
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  const long long units = (long long)((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN) * splits;
-  const int grid = (int)std::min<long long>(units, sms);
-  kern<<<grid, TC_THREADS, smem, st>>>(ta, tb, to, to2, tx, M, N, K, splits, ep);
+  const long long units = (long long)((M + TcShape<PAIR>::TILE_M - 1) / TcShape<PAIR>::TILE_M) *
+                          ((N + TC_BN - 1) / TC_BN) * splits;
+  if (!PAIR) {
+    const int grid = (int)std::min<long long>(units, dev_info().sms);
+    kern<<<grid, TC_THREADS, smem, st>>>(ta, tb, to, to2, tx, M, N, K, splits, ep);
+  } else {
+    const int clusters = (int)std::min<long long>(units, max_pair_clusters(kern, smem));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, to2, tx, M, N, K, splits, ep) != cudaSuccess) {
+      cudaGetLastError();
+      LAUNCHED();
+      return GPTB_ERR_CUDA;
+    }
+  }
   CKL();
   return GPTB_OK;
 }
+
+// GEMMs with at least this many rows run in the pair form (two CTAs, M = 256
+// per tile); smaller ones in the single-CTA form.
+#ifndef GPTB_PAIR_MIN_M
+#define GPTB_PAIR_MIN_M 256
+#endif
 
 int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t st) {
   if (M <= 0 || N <= 0) return GPTB_OK;
@@ -206,6 +268,7 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
   if (timed) cudaEventRecord(ea, st);
   int rc = GPTB_OK;
   if (dtype == GPTB_F32) {
+    if (ep.kind == EPI_XENT || ep.kind == EPI_QKV || ep.kind == EPI_DOT) return GPTB_ERR_UNSUPPORTED;
     dim3 grid((N + 63) / 64, (M + 63) / 64);
     const float* a = static_cast<const float*>(A.p);
     const float* b = static_cast<const float*>(B.p);
@@ -230,14 +293,18 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
     if (ep.out_f32 && !acc32) return GPTB_ERR_UNSUPPORTED;
     // a row's groups of 128 columns must lie inside one N tile
     if (ep.kind == EPI_DOT && (N % 128 || !ep.rowdot || ep.T <= 0 || M % ep.T)) return GPTB_ERR_INVALID_ARG;  // tensor-core outputs are bf16 or fp32 accumulations
+    if (ep.kind == EPI_XENT && (!ep.xent_part || !ep.targets || !ep.xent_zy || ep.xent_nt < (N + TC_BN - 1) / TC_BN))
+      return GPTB_ERR_INVALID_ARG;
     if (!aligned16(A.p) || !aligned16(B.p) || !aligned16(ep.out) || (A.ld % align) || (B.ld % align) ||
         (ep.ldo % (acc32 ? 4 : 8)) || (N % 8))
       return GPTB_ERR_INVALID_ARG;
     if (has_aux && (!aligned16(ep.aux) || ep.ld_aux % 8)) return GPTB_ERR_INVALID_ARG;
     if (ep.kind == EPI_RELU2 && (!aligned16(ep.out2) || ep.ldo2 % 8)) return GPTB_ERR_INVALID_ARG;
+    const bool pair = M >= GPTB_PAIR_MIN_M;
+    const int b_rows = pair ? TcShape<true>::B_ROWS : TcShape<false>::B_ROWS;  // rows of B one CTA stages
     CUtensorMap ta, tb, to, to2, tx;
     bool ok = A.mn ? make_tmap(&ta, A.p, f8, M, K, A.ld, bk, bk) : make_tmap(&ta, A.p, f8, K, M, A.ld, bk, TC_BM);
-    ok = ok && (B.mn ? make_tmap(&tb, B.p, f8, N, K, B.ld, bk, bk) : make_tmap(&tb, B.p, f8, K, N, B.ld, bk, TC_BN));
+    ok = ok && (B.mn ? make_tmap(&tb, B.p, f8, N, K, B.ld, bk, bk) : make_tmap(&tb, B.p, f8, K, N, B.ld, bk, b_rows));
     // epilogue maps: 32-row boxes of 64 bf16 / 32 fp32 columns, 128-byte swizzle
     ok = ok && (acc32 ? make_tmap_f32(&to, ep.out, N, M, ep.ldo, 32, 32, true)
                       : make_tmap(&to, ep.out, false, N, M, ep.ldo, 64, 32));
@@ -248,25 +315,33 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
     if (!ok) return GPTB_ERR_CUDA;
     int splits = 1;
     if (ep.kind == EPI_ACCUM_F32) {
-      const int tiles = ((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN);
-      splits = plan_splits(tiles, (K + (int)bk - 1) / (int)bk, di.sms);
+      const int tile_m = pair ? TcShape<true>::TILE_M : TcShape<false>::TILE_M;
+      const int tiles = ((M + tile_m - 1) / tile_m) * ((N + TC_BN - 1) / TC_BN);
+      splits = plan_splits(tiles, (K + (int)bk - 1) / (int)bk, pair ? di.sms / 2 : di.sms);
     }
-    const int sel = (A.mn ? 1 : 0) | (B.mn ? 2 : 0) | (f8 ? 4 : 0);
+    const int sel = (A.mn ? 1 : 0) | (B.mn ? 2 : 0) | (f8 ? 4 : 0) | (pair ? 8 : 0);
     switch (sel) {
-      case 0: rc = launch_tc<false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
-      case 1: rc = launch_tc<true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
-      case 2: rc = launch_tc<false, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
-      case 3: rc = launch_tc<true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
-      case 4: rc = launch_tc<false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
-      case 6: rc = launch_tc<false, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
-      case 7: rc = launch_tc<true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st, di.sms); break;
+      case 0: rc = launch_tc<false, false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 1: rc = launch_tc<true, false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 2: rc = launch_tc<false, true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 3: rc = launch_tc<true, true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 4: rc = launch_tc<false, false, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 6: rc = launch_tc<false, true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 7: rc = launch_tc<true, true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 8: rc = launch_tc<false, false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 9: rc = launch_tc<true, false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 10: rc = launch_tc<false, true, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 11: rc = launch_tc<true, true, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 12: rc = launch_tc<false, false, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 14: rc = launch_tc<false, true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 15: rc = launch_tc<true, true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
       default: rc = GPTB_ERR_UNSUPPORTED;  // e4m3 with A M-major and B K-major: not used
     }
   }
   if (timed) {
     cudaEventRecord(eb, st);
     std::lock_guard<std::mutex> lk(g_timing_mu);
-    g_timed.push_back({ea, eb, 2.0 * M * (double)N * K});
+    g_timed.push_back({ea, eb, 2.0 * M * (double)N * K, dtype == GPTB_FP8_E4M3});
   }
   return rc;
 }
@@ -286,6 +361,7 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
   e.beta = nullptr;
   e.amax_a = nullptr;
   e.amax_b = nullptr;
+  e.a_e5m2 = 0;
   e.rope = nullptr;
   e.rstd_qk = nullptr;
   e.ve_table = nullptr;
@@ -294,11 +370,16 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
   e.T = e.H = e.Hkv = 0;
   e.eps = 0.f;
   e.rowdot = nullptr;
+  e.xent_part = nullptr;
+  e.xent_nt = 0;
+  e.targets = nullptr;
+  e.xent_zy = nullptr;
   return e;
 }
-EpiParams epi8(EpiParams e, const float* amax_a, const float* amax_b) {
+EpiParams epi8(EpiParams e, const float* amax_a, const float* amax_b, bool a_e5m2 = false) {
   e.amax_a = amax_a;
   e.amax_b = amax_b;
+  e.a_e5m2 = a_e5m2 ? 1 : 0;
   return e;
 }
 
@@ -319,6 +400,8 @@ struct Dims {
   long long N;
   int B, T, d, H, Hkv, hd, F, V, L, Wq, NH, esz;
   bool fp8;
+  bool grad_e5m2;  // FP8: gradient operands in e5m2
+  bool fp8_lm;     // FP8: the lm_head GEMMs in FP8 as well
 };
 Dims dims_of(const gptb_config& c) {
   Dims m;
@@ -336,6 +419,8 @@ Dims dims_of(const gptb_config& c) {
   m.NH = c.n_head + c.n_kv_head;
   m.esz = c.dtype == GPTB_F32 ? 4 : 2;
   m.fp8 = c.dtype == GPTB_FP8_E4M3;
+  m.grad_e5m2 = m.fp8 && (c.fp8_flags & GPTB_FP8_GRAD_E5M2);
+  m.fp8_lm = m.fp8 && (c.fp8_flags & GPTB_FP8_LM_HEAD);
   return m;
 }
 
@@ -343,8 +428,10 @@ struct Saved {
   void *h, *qkv, *o, *h2, *u, *act;
   float *rstd1, *sg, *rstd_qk, *lse, *rstd2;
   // FP8 only: e4m3 copies of the four weights (reused by the input-gradient
-  // GEMMs) and the amax of the four GEMM activations and four weights
+  // GEMMs) and of the four GEMM activations (reused by the weight-gradient
+  // GEMMs), and the amax of each
   uint8_t *wqkv8, *wo8, *wfc8, *wproj8;
+  uint8_t *h8, *o8, *h2_8, *act8;
   float* amax;  // [h, o, h2, act, wqkv, wo, wfc, wproj]
 };
 Saved carve_saved(Carve& cv, const Dims& m) {
@@ -362,6 +449,7 @@ Saved carve_saved(Carve& cv, const Dims& m) {
   s.u = cv.take(m.N * m.F * e);
   s.act = cv.take(m.N * m.F * e);
   s.wqkv8 = s.wo8 = s.wfc8 = s.wproj8 = nullptr;
+  s.h8 = s.o8 = s.h2_8 = s.act8 = nullptr;
   s.amax = nullptr;
   if (m.fp8) {
     const long long Ho = (long long)m.H * m.hd;
@@ -369,6 +457,10 @@ Saved carve_saved(Carve& cv, const Dims& m) {
     s.wo8 = (uint8_t*)cv.take((size_t)m.d * Ho);
     s.wfc8 = (uint8_t*)cv.take((size_t)m.F * m.d);
     s.wproj8 = (uint8_t*)cv.take((size_t)m.d * m.F);
+    s.h8 = (uint8_t*)cv.take((size_t)(m.N * m.d));
+    s.o8 = (uint8_t*)cv.take((size_t)(m.N * Ho));
+    s.h2_8 = (uint8_t*)cv.take((size_t)(m.N * m.d));
+    s.act8 = (uint8_t*)cv.take((size_t)(m.N * m.F));
     s.amax = (float*)cv.take(8 * 4);
   }
   return s;
@@ -378,7 +470,6 @@ struct Scratch {
   float2* rope;
   // forward
   void *xm, *x1;
-  uint8_t* a8;  // FP8: e4m3 copy of the activation feeding a forward GEMM
   // backward
   void *du, *dh2, *dx1, *dO, *dqkv, *dh;
   float *D, *dq, *dk, *dv, *dz;
@@ -392,11 +483,6 @@ Scratch carve_scratch(Carve& cv, const Dims& m) {
   const size_t start = cv.off;
   s.xm = cv.take(m.N * m.d * e);
   s.x1 = cv.take(m.N * m.d * e);
-  s.a8 = nullptr;
-  if (m.fp8) {
-    const long long w = std::max<long long>(std::max<long long>(m.d, m.F), (long long)m.H * m.hd);
-    s.a8 = (uint8_t*)cv.take(m.N * w);
-  }
   const size_t fwd_end = cv.off;
   cv.off = start;  // backward temporaries reuse the forward's space
   s.du = cv.take(m.N * m.F * e);
@@ -421,16 +507,39 @@ Scratch carve_scratch(Carve& cv, const Dims& m) {
   return s;
 }
 
+// lm_head temporaries: one row chunk of logits (overwritten by their
+// gradient), the chunk's per-(row, 256-column tile) softmax statistics from
+// the logits GEMM, z at the target and the log-sum-exp of each row, and the
+// loss of every row.
 struct LmWs {
   void* logits;
+  float2* part;
+  float* zy;
+  float* lse;
   float* row_loss;
   int chunk;
+  // FP8 lm_head: e4m3 copies of hf [N, d] and W_lm [V, d], the chunk's FP8
+  // logits gradient, and the amax slots [hf, W_lm, bound of dz]
+  uint8_t *h8, *w8, *dz8;
+  float* amx;
 };
+int lm_tiles(int V) { return (V + TC_BN - 1) / TC_BN; }
 LmWs carve_lm(Carve& cv, const Dims& m) {
   LmWs l;
   l.chunk = (int)std::min<long long>(m.N, 8192);
   l.logits = cv.take((size_t)l.chunk * m.V * m.esz);
+  l.part = (float2*)cv.take((size_t)l.chunk * lm_tiles(m.V) * sizeof(float2));
+  l.zy = (float*)cv.take((size_t)l.chunk * 4);
+  l.lse = (float*)cv.take((size_t)l.chunk * 4);
   l.row_loss = (float*)cv.take(m.N * 4);
+  l.h8 = l.w8 = l.dz8 = nullptr;
+  l.amx = nullptr;
+  if (m.fp8_lm) {
+    l.h8 = (uint8_t*)cv.take((size_t)(m.N * m.d));
+    l.w8 = (uint8_t*)cv.take((size_t)m.V * m.d);
+    l.dz8 = (uint8_t*)cv.take((size_t)l.chunk * m.V);
+    l.amx = (float*)cv.take(4 * 4);
+  }
   return l;
 }
 
@@ -464,6 +573,9 @@ StackWs carve_stack(Carve& cv, const Dims& m) {
 int check_config(const gptb_config* c) {
   if (!c) return GPTB_ERR_INVALID_ARG;
   if (c->dtype != GPTB_F32 && c->dtype != GPTB_BF16 && c->dtype != GPTB_FP8_E4M3) return GPTB_ERR_UNSUPPORTED;
+  if (c->fp8_flags & ~(GPTB_FP8_GRAD_E5M2 | GPTB_FP8_LM_HEAD)) return GPTB_ERR_INVALID_ARG;
+  if (c->fp8_flags && c->dtype != GPTB_FP8_E4M3) return GPTB_ERR_INVALID_ARG;
+  if ((c->fp8_flags & GPTB_FP8_LM_HEAD) && (c->d % 16 || c->vocab % 16)) return GPTB_ERR_INVALID_ARG;
   if (c->B < 1 || c->T < 1 || c->d < 8 || c->d % 8 || c->d > 8 * 32 * BR_MAX_WARPS) return GPTB_ERR_INVALID_ARG;
   if (c->n_head < 1 || c->n_kv_head < 1 || c->n_head % c->n_kv_head) return GPTB_ERR_INVALID_ARG;
   if (c->mlp_hidden < 8 || c->mlp_hidden % 8 || c->vocab < 8 || c->vocab % 8) return GPTB_ERR_INVALID_ARG;
@@ -509,15 +621,16 @@ int rope_init(const gptb_config& c, float2* tab, cudaStream_t st) {
 }
 
 
-// per-tensor e4m3 quantisation: amax (fp32 bits, atomicMax) then codes
+// per-tensor FP8 quantisation: amax (fp32 bits, atomicMax) then codes, e4m3
+// (scale 448/amax) or e5m2 (57344/amax)
 template <class T>
-int quant(const T* x, long long n, uint8_t* out, float* amax, cudaStream_t st) {
+int quant(const T* x, long long n, uint8_t* out, float* amax, bool e5m2, cudaStream_t st) {
   CK(cudaMemsetAsync(amax, 0, sizeof(float), st));
   const long long n8 = n / 8;
   const int grid = (int)std::max<long long>(1, std::min<long long>((n8 + 255) / 256, (long long)dev_info().sms * 8));
   amax_kernel<T><<<grid, 256, 0, st>>>(x, n8, reinterpret_cast<unsigned int*>(amax));
   CKL();
-  quantize_e4m3_kernel<T><<<grid, 256, 0, st>>>(x, n8, amax, out);
+  quantize_fp8_kernel<T><<<grid, 256, 0, st>>>(x, n8, amax, e5m2 ? 1 : 0, out);
   CKL();
   return GPTB_OK;
 }
@@ -532,20 +645,21 @@ struct Operand {
   uint8_t* q;
   float* amax;
   bool quant;
+  bool e5m2;  // FP8 copy in e5m2 (gradient operands of the e5m2 variant)
 };
 
 // A projection GEMM of the block in the config's arithmetic: f32 (SIMT) or
-// bf16 (tcgen05) operands as stored, or per-tensor e4m3 operands (FP8).  In
-// FP8 configs an operand without an e4m3 slot (q == nullptr) selects the bf16
-// GEMM: the weight-gradient products keep high-precision operands.
+// bf16 (tcgen05) operands as stored, or per-tensor e4m3 operands (FP8: every
+// product of the four block GEMMs -- forward, input gradient and weight
+// gradient -- takes the e4m3 copies of its two bf16 operands).
 template <class T>
 int proj(const gptb_config& c, const Operand& A, const Operand& B, int M, int N, int K, const EpiParams& e,
          cudaStream_t st) {
   if (c.dtype != GPTB_FP8_E4M3) return gemm(c.dtype, {A.p, A.ld, A.mn}, {B.p, B.ld, B.mn}, M, N, K, e, st);
-  if (!A.q) return gemm(GPTB_BF16, {A.p, A.ld, A.mn}, {B.p, B.ld, B.mn}, M, N, K, e, st);  // high-precision GEMM
-  if (A.quant) TRY(quant<T>((const T*)A.p, A.elems, A.q, A.amax, st));
-  if (B.quant) TRY(quant<T>((const T*)B.p, B.elems, B.q, B.amax, st));
-  return gemm(GPTB_FP8_E4M3, {A.q, A.ld, A.mn}, {B.q, B.ld, B.mn}, M, N, K, epi8(e, A.amax, B.amax), st);
+  if (!A.q || !B.q || !A.amax || !B.amax || B.e5m2) return GPTB_ERR_INVALID_ARG;
+  if (A.quant) TRY(quant<T>((const T*)A.p, A.elems, A.q, A.amax, A.e5m2, st));
+  if (B.quant) TRY(quant<T>((const T*)B.p, B.elems, B.q, B.amax, false, st));
+  return gemm(GPTB_FP8_E4M3, {A.q, A.ld, A.mn}, {B.q, B.ld, B.mn}, M, N, K, epi8(e, A.amax, B.amax, A.e5m2), st);
 }
 
 // ------------------------------------------------------ block forward -----
@@ -581,7 +695,7 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     e.H = m.H;
     e.Hkv = m.Hkv;
     e.eps = c.norm_eps;
-    TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, X.a8, S.amax + 0, true},
+    TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, S.h8, S.amax + 0, true},
                 {w.w_qkv, m.d, false, (long long)m.Wq * m.d, S.wqkv8, S.amax + 4, true}, (int)m.N, m.Wq, m.d, e, st));
   }
   const int W = c.window[layer];
@@ -599,16 +713,16 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
         tq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W);
     CKL();
   }
-  TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, X.a8, S.amax + 1, true},
+  TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, S.o8, S.amax + 1, true},
               {w.w_o, Ho, false, m.d * Ho, S.wo8, S.amax + 5, true}, (int)m.N, m.d, (int)Ho,
               epi(EPI_RESID, c.dtype, X.x1, m.d, X.xm, m.d), st));
   br_norm_kernel<T><<<brg, brt, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
                                             c.norm_eps);
   CKL();
-  TRY(proj<T>(c, {S.h2, m.d, false, m.N * m.d, X.a8, S.amax + 2, true},
+  TRY(proj<T>(c, {S.h2, m.d, false, m.N * m.d, S.h2_8, S.amax + 2, true},
               {w.w_fc, m.d, false, (long long)m.F * m.d, S.wfc8, S.amax + 6, true}, (int)m.N, m.F, m.d,
               epi(EPI_RELU2, c.dtype, S.u, m.F, nullptr, 0, S.act, m.F), st));
-  TRY(proj<T>(c, {S.act, m.F, false, m.N * m.F, X.a8, S.amax + 3, true},
+  TRY(proj<T>(c, {S.act, m.F, false, m.N * m.F, S.act8, S.amax + 3, true},
               {w.w_proj, m.F, false, (long long)m.d * m.F, S.wproj8, S.amax + 7, true}, (int)m.N, m.d, m.F,
               epi(EPI_RESID, c.dtype, x_out, m.d, X.x1, m.d), st));
   return GPTB_OK;
@@ -629,21 +743,22 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   const int N = (int)m.N;
   const long long Ho = (long long)m.H * m.hd, Kv = (long long)m.Hkv * m.hd;
   // MLP
-  // (FP8: the input-gradient GEMMs quantise the gradient and reuse the
-  // forward's e4m3 weights; the weight-gradient GEMMs run on the bf16 tensors)
+  // (FP8: the weight-gradient GEMM quantises the gradient, whose e4m3 copy the
+  // input-gradient GEMM then reuses with the forward's e4m3 weight; the other
+  // weight-gradient operand is the forward's saved e4m3 activation)
   const long long Nd = m.N * m.d;
-  TRY(proj<T>(c, {dx2, m.d, true, Nd, nullptr, nullptr, false}, {S.act, m.F, true, 0, nullptr, nullptr, false}, m.d,
+  TRY(proj<T>(c, {dx2, m.d, true, Nd, X.g8, X.gamax, true, m.grad_e5m2}, {S.act, m.F, true, 0, S.act8, S.amax + 3, false}, m.d,
               m.F, N, epi(EPI_ACCUM_F32, dt, g.w_proj, m.F), st));
-  TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false},
+  TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false},
               N, m.F, m.d, epi(EPI_DRELU2, dt, X.du, m.F, S.u, m.F), st));
-  TRY(proj<T>(c, {X.du, m.F, true, 0, nullptr, nullptr, false}, {S.h2, m.d, true, 0, nullptr, nullptr, false}, m.F,
-              m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
-  TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, X.gamax, true}, {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false},
+  TRY(proj<T>(c, {X.du, m.F, true, m.N * m.F, X.g8, X.gamax, true, m.grad_e5m2}, {S.h2, m.d, true, 0, S.h2_8, S.amax + 2, false},
+              m.F, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
+  TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false},
               N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
   br_norm_bwd_kernel<T><<<brg, brt, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d);
   CKL();
   // attention output projection
-  TRY(proj<T>(c, {X.dx1, m.d, true, 0, nullptr, nullptr, false}, {S.o, Ho, true, 0, nullptr, nullptr, false}, m.d,
+  TRY(proj<T>(c, {X.dx1, m.d, true, Nd, X.g8, X.gamax, true, m.grad_e5m2}, {S.o, Ho, true, 0, S.o8, S.amax + 1, false}, m.d,
               (int)Ho, N, epi(EPI_ACCUM_F32, dt, g.w_o, Ho), st));
   // dO = dx1 Wo, and the attention backward's D = rowsum(dO * o) per head
   if constexpr (std::is_same<T, bf16>::value) {
@@ -652,10 +767,10 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     ed.rowdot = X.D;
     ed.T = m.T;
     ed.H = m.H;
-    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
                 (int)Ho, m.d, ed, st));
   } else {
-    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true, m.grad_e5m2}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
                 (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
     attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
                                                                        m.B, m.T, m.H, m.hd);
@@ -698,9 +813,9 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   }
   CKL();
   // QKV projection
-  TRY(proj<T>(c, {X.dqkv, m.Wq, true, 0, nullptr, nullptr, false}, {S.h, m.d, true, 0, nullptr, nullptr, false},
+  TRY(proj<T>(c, {X.dqkv, m.Wq, true, m.N * m.Wq, X.g8, X.gamax, true, m.grad_e5m2}, {S.h, m.d, true, 0, S.h8, S.amax + 0, false},
               m.Wq, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_qkv, m.d), st));
-  TRY(proj<T>(c, {X.dqkv, m.Wq, false, m.N * m.Wq, X.g8, X.gamax, true},
+  TRY(proj<T>(c, {X.dqkv, m.Wq, false, m.N * m.Wq, X.g8, X.gamax, false, m.grad_e5m2},
               {w.w_qkv, m.d, true, 0, S.wqkv8, S.amax + 4, false}, N, m.d, m.Wq, epi(EPI_STORE, dt, X.dh, m.d), st));
   if (ve) {
     const int nthreads = ((m.Hkv * c.ve_gate_ch + 31) / 32) * 32;
@@ -724,15 +839,51 @@ int lm_head_impl(const gptb_config& c, const T* h, const T* w_lm, const int32_t*
   const Dims m = dims_of(c);
   const int brt = br_threads(m.d);
   const int brg = br_grid(m.N, brt);
-  const int dt = c.dtype == GPTB_FP8_E4M3 ? GPTB_BF16 : c.dtype;  // lm_head stays bf16
+  const int dt = c.dtype == GPTB_FP8_E4M3 ? GPTB_BF16 : c.dtype;  // lm_head bf16 unless GPTB_FP8_LM_HEAD
+  if constexpr (std::is_same<T, bf16>::value) {
+    if (m.fp8_lm) {
+      // FP8 lm_head: e4m3 copies of the whole hf and of W_lm (per-tensor scales)
+      if (!lw.h8 || !lw.w8 || !lw.dz8 || !lw.amx) return GPTB_ERR_UNSUPPORTED;
+      TRY(quant<bf16>(h, m.N * m.d, lw.h8, lw.amx + 0, false, st));
+      TRY(quant<bf16>(w_lm, (long long)m.V * m.d, lw.w8, lw.amx + 1, false, st));
+    }
+  }
   for (long long c0 = 0; c0 < m.N; c0 += lw.chunk) {
     const int rows = (int)std::min<long long>(lw.chunk, m.N - c0);
     const T* hc = h + c0 * m.d;
-    TRY(gemm(dt, {hc, m.d, false}, {w_lm, m.d, false}, rows, m.V, m.d, epi(EPI_STORE, dt, lw.logits, m.V), st));
-    if (std::is_same<T, bf16>::value && m.V <= XENT_REG_THREADS * 8 * XENT_REG_VEC) {
-      xent_rows_reg_kernel<<<rows, XENT_REG_THREADS, 0, st>>>((bf16*)lw.logits, m.V, m.V, targets + c0,
-                                                              lw.row_loss + c0, 1.f / (float)m.N, rows);
+    if constexpr (std::is_same<T, bf16>::value) {
+      // logits GEMM whose epilogue also emits the per-tile softmax statistics
+      // and z at the target; then the row log-sum-exp and the logits gradient
+      EpiParams e = epi(EPI_XENT, dt, lw.logits, m.V);
+      e.xent_part = lw.part;
+      e.xent_nt = lm_tiles(m.V);
+      e.targets = targets + c0;
+      e.xent_zy = lw.zy;
+      if (m.fp8_lm)
+        TRY(gemm(GPTB_FP8_E4M3, {lw.h8 + c0 * m.d, m.d, false}, {lw.w8, m.d, false}, rows, m.V, m.d,
+                 epi8(e, lw.amx + 0, lw.amx + 1), st));
+      else
+        TRY(gemm(dt, {hc, m.d, false}, {w_lm, m.d, false}, rows, m.V, m.d, e, st));
+      xent_lse_kernel<<<grid_rows(rows), EW_THREADS, 0, st>>>(lw.part, lm_tiles(m.V), lw.zy, targets + c0, m.V,
+                                                               lw.lse, lw.row_loss + c0, rows);
+      CKL();
+      if (m.fp8_lm) {
+        // the logits gradient as FP8 codes with the scale its bound 1/N fixes,
+        // then the two gradient GEMMs on FP8 operands
+        xent_grad_fp8_kernel<<<rows, XENT_GRAD_THREADS, 0, st>>>((const bf16*)lw.logits, m.V, m.V, targets + c0,
+                                                                  lw.lse, 1.f / (float)m.N, m.grad_e5m2 ? 1 : 0,
+                                                                  lw.dz8, m.V, lw.amx + 2, rows);
+        CKL();
+        TRY(gemm(GPTB_FP8_E4M3, {lw.dz8, m.V, false}, {lw.w8, m.d, true}, rows, m.d, m.V,
+                 epi8(epi(EPI_STORE, dt, dh + c0 * m.d, m.d), lw.amx + 2, lw.amx + 1, m.grad_e5m2), st));
+        TRY(gemm(GPTB_FP8_E4M3, {lw.dz8, m.V, true}, {lw.h8 + c0 * m.d, m.d, true}, m.V, m.d, rows,
+                 epi8(epi(EPI_ACCUM_F32, dt, dw_lm, m.d), lw.amx + 2, lw.amx + 0, m.grad_e5m2), st));
+        continue;
+      }
+      xent_grad_kernel<<<rows, XENT_GRAD_THREADS, 0, st>>>((bf16*)lw.logits, m.V, m.V, targets + c0, lw.lse,
+                                                            1.f / (float)m.N, rows);
     } else {
+      TRY(gemm(dt, {hc, m.d, false}, {w_lm, m.d, false}, rows, m.V, m.d, epi(EPI_STORE, dt, lw.logits, m.V), st));
       xent_rows_kernel<T><<<rows, 512, 0, st>>>((T*)lw.logits, m.V, m.V, targets + c0, lw.row_loss + c0,
                                                 1.f / (float)m.N, rows);
     }
@@ -933,20 +1084,14 @@ size_t gptb_polar_express_workspace_bytes(int m, int n, int steps) {
   return PE_HEADER + 2 * pe_align((size_t)m * n * 2) + 2 * pe_align(s * s * 2);
 }
 
-int gptb_polar_express(const void* G, void* out, int m, int n, const float* coeffs, int steps, void* workspace,
-                       size_t workspace_bytes, gptb_stream_t stream) {
-  if (!G || !out || !coeffs || !workspace || m <= 0 || n <= 0 || m % 8 || n % 8 || steps < 1 || steps > 64)
-    return GPTB_ERR_INVALID_ARG;
-  if (!aligned16(G) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GPTB_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+// The Polar Express loop on a bf16 [m, n] matrix into out (workspace laid out
+// as gptb_polar_express_workspace_bytes describes; arguments already checked).
+int polar_express_impl(const void* G, void* out, int m, int n, const float* coeffs, int steps, uint8_t* w,
+                       cudaStream_t st) {
   const size_t ne = (size_t)m * n;
-  {
-    const uintptr_t a = reinterpret_cast<uintptr_t>(G), b = reinterpret_cast<uintptr_t>(out);
-    if (a < b + ne * 2 && b < a + ne * 2) return GPTB_ERR_INVALID_ARG;  // out overlaps G
-  }
-  if (workspace_bytes < gptb_polar_express_workspace_bytes(m, n, steps)) return GPTB_ERR_WORKSPACE;
-  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* w = static_cast<uint8_t*>(workspace);
   float* sumsq = reinterpret_cast<float*>(w);
   float* cf = reinterpret_cast<float*>(w + 256);
   bf16* X[2];
@@ -991,6 +1136,65 @@ int gptb_polar_express(const void* G, void* out, int m, int n, const float* coef
   }
   return GPTB_OK;
 }
+}  // namespace
+
+extern "C" {
+
+int gptb_polar_express(const void* G, void* out, int m, int n, const float* coeffs, int steps, void* workspace,
+                       size_t workspace_bytes, gptb_stream_t stream) {
+  if (!G || !out || !coeffs || !workspace || m <= 0 || n <= 0 || m % 8 || n % 8 || steps < 1 || steps > 64)
+    return GPTB_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GPTB_ERR_INVALID_ARG;
+  const size_t ne = (size_t)m * n;
+  {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(G), b = reinterpret_cast<uintptr_t>(out);
+    if (a < b + ne * 2 && b < a + ne * 2) return GPTB_ERR_INVALID_ARG;  // out overlaps G
+  }
+  if (workspace_bytes < gptb_polar_express_workspace_bytes(m, n, steps)) return GPTB_ERR_WORKSPACE;
+  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  return polar_express_impl(G, out, m, n, coeffs, steps, static_cast<uint8_t*>(workspace),
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t gptb_muon_workspace_bytes(int m, int n, int steps) {
+  const size_t pe = gptb_polar_express_workspace_bytes(m, n, steps);
+  if (pe == 0) return 0;
+  // Polar Express workspace, the bf16 input u and output o, per-row step sizes, two sums
+  return pe + 2 * pe_align((size_t)m * n * 2) + pe_align((size_t)m * 4) + 256;
+}
+
+int gptb_muon_step(float* w, void* w_bf16, const float* g, float* buf, float* v, int m, int n, const float* coeffs,
+                   int steps, float lr, float mu, float beta2, float weight_decay, void* workspace,
+                   size_t workspace_bytes, gptb_stream_t stream) {
+  if (!w || !g || !buf || !v || !coeffs || !workspace || m <= 0 || n <= 0 || m % 8 || n % 8 || steps < 1 ||
+      steps > 64)
+    return GPTB_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(g) || !aligned16(buf) || (w_bf16 && (reinterpret_cast<uintptr_t>(w_bf16) & 7u)) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GPTB_ERR_INVALID_ARG;
+  if (workspace_bytes < gptb_muon_workspace_bytes(m, n, steps)) return GPTB_ERR_WORKSPACE;
+  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t ne = (size_t)m * n;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t pe = gptb_polar_express_workspace_bytes(m, n, steps);
+  bf16* u = reinterpret_cast<bf16*>(ws + pe);
+  bf16* o = reinterpret_cast<bf16*>(ws + pe + pe_align(ne * 2));
+  float* step = reinterpret_cast<float*>(ws + pe + 2 * pe_align(ne * 2));
+  float* sums = reinterpret_cast<float*>(ws + pe + 2 * pe_align(ne * 2) + pe_align((size_t)m * 4));
+  const long long n4 = (long long)ne / 4;  // m, n multiples of 8
+  const int grid = (int)std::max<long long>(1, std::min<long long>((n4 + 255) / 256, dev_info().sms * 8LL));
+  // momentum (Nesterov): buf = mu buf + g, u = g + mu buf (bf16)
+  muon_momentum_kernel<<<grid, 256, 0, st>>>(g, buf, u, n4, mu, sums);
+  CKL();
+  TRY(polar_express_impl(u, o, m, n, coeffs, steps, ws, st));
+  // NorMuon: per-row second moment and step size, then the norm-keeping scale and the update
+  normuon_rows_kernel<<<grid_rows(m), EW_THREADS, 0, st>>>(o, m, n, v, beta2, step, sums);
+  CKL();
+  muon_apply_kernel<<<grid, 256, 0, st>>>(w, static_cast<bf16*>(w_bf16), o, step, sums, m, n, lr, weight_decay);
+  CKL();
+  return GPTB_OK;
+}
 
 // --------------------------------------------------------------- decode --
 
@@ -1020,7 +1224,7 @@ int gptb_device_error(gptb_stream_t stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return GPTB_ERR_CUDA;
-    return GPTB_ERR_TIMEOUT;
+    return (v & 0xf00) == 0x200 ? GPTB_ERR_BAD_INPUT : GPTB_ERR_TIMEOUT;
   }
   return GPTB_OK;
 }
@@ -1063,18 +1267,24 @@ int gptb_set_gemm_timing(int enable) {
   return GPTB_OK;
 }
 
-int gptb_gemm_timing(double* ms, double* flops, long long* launches) {
+int gptb_gemm_timing(double* ms, double* flops, double* ms_fp8, double* flops_fp8, long long* launches) {
   std::lock_guard<std::mutex> lk(g_timing_mu);
-  double tms = 0, tf = 0;
+  double tms = 0, tf = 0, tms8 = 0, tf8 = 0;
   for (auto& t : g_timed) {
     if (cudaEventSynchronize(t.b) != cudaSuccess) return GPTB_ERR_CUDA;
     float e = 0.f;
     if (cudaEventElapsedTime(&e, t.a, t.b) != cudaSuccess) return GPTB_ERR_CUDA;
     tms += e;
     tf += t.flops;
+    if (t.fp8) {
+      tms8 += e;
+      tf8 += t.flops;
+    }
   }
   if (ms) *ms = tms;
   if (flops) *flops = tf;
+  if (ms_fp8) *ms_fp8 = tms8;
+  if (flops_fp8) *flops_fp8 = tf8;
   if (launches) *launches = (long long)g_timed.size();
   return GPTB_OK;
 }
@@ -1087,6 +1297,7 @@ const char* gptb_error_string(int code) {
     case GPTB_ERR_CUDA: return "CUDA error";
     case GPTB_ERR_TIMEOUT: return "bounded device wait expired";
     case GPTB_ERR_WORKSPACE: return "workspace too small";
+    case GPTB_ERR_BAD_INPUT: return "invalid input data found on the device (a target outside [0, vocab))";
     default: return "unknown error";
   }
 }
@@ -1095,32 +1306,29 @@ const char* gptb_error_string(int code) {
 
 // ======================================================= no-alloc lm_head ==
 // lm_head_xent for callers that cannot allocate device memory: its scratch
-// (one chunk of logits and the per-row losses) lives in this file-scope
-// device array instead of a caller-provided workspace.  Every GPU that loads
-// the library holds the array until the process exits.
+// (one chunk of logits, the chunk's softmax statistics, and the per-row
+// losses) lives in this file-scope device array instead of a caller-provided
+// workspace.  Every GPU that loads the library holds the array until the
+// process exits.
 namespace {
 
 constexpr size_t NOALLOC_LOGITS_BYTES = size_t(8) << 20;  // logits of one row chunk
-constexpr long long NOALLOC_MAX_ROWS = 65536;             // B*T limit (row losses)
-static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_LOGITS_BYTES + NOALLOC_MAX_ROWS * 4];
+constexpr size_t NOALLOC_PART_BYTES = size_t(1) << 20;    // per-(row, tile) statistics of the chunk
+constexpr long long NOALLOC_MAX_ROWS = 65536;             // B*T limit (row losses; z at the target and
+                                                          // the log-sum-exp of a chunk's rows)
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[NOALLOC_LOGITS_BYTES + NOALLOC_PART_BYTES + 3 * NOALLOC_MAX_ROWS * 4];
 
-// Device address of g_noalloc_scratch, looked up once per device with that
-// device current (host code only sees a host-side stand-in under the name).
+// Device address of g_noalloc_scratch on the current device (host code only
+// sees a host-side stand-in under the name).  Looked up on every call, so a
+// module reloaded at another address after a context teardown is still found.
 int noalloc_scratch(unsigned char** out) {
-  static std::mutex mu;
-  static unsigned char* addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTB_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
-      cudaGetLastError();
-      return GPTB_ERR_CUDA;
-    }
-    addr[dev] = static_cast<unsigned char*>(p);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+    cudaGetLastError();
+    return GPTB_ERR_CUDA;
   }
-  *out = addr[dev];
+  *out = static_cast<unsigned char*>(p);
   return GPTB_OK;
 }
 
@@ -1131,15 +1339,22 @@ extern "C" int lm_head_xent_noalloc(const gptb_config* cfg, const void* h, const
   TRY(check_config(cfg));
   if (!h || !w_lm || !targets || !loss_out || !dh || !dw_lm) return GPTB_ERR_INVALID_ARG;
   const Dims m = dims_of(*cfg);
+  if (m.fp8_lm) return GPTB_ERR_UNSUPPORTED;  // its FP8 copies of hf and W_lm need a workspace
   if (m.N > NOALLOC_MAX_ROWS) return GPTB_ERR_WORKSPACE;
-  const long long rows = (long long)(NOALLOC_LOGITS_BYTES / ((size_t)m.V * m.esz));
+  long long rows = (long long)(NOALLOC_LOGITS_BYTES / ((size_t)m.V * m.esz));
+  rows = std::min<long long>(rows, (long long)(NOALLOC_PART_BYTES / (lm_tiles(m.V) * sizeof(float2))));
   if (rows < 1) return GPTB_ERR_WORKSPACE;
   unsigned char* base = nullptr;
   TRY(noalloc_scratch(&base));
   LmWs lw;
   lw.logits = base;
-  lw.row_loss = reinterpret_cast<float*>(base + NOALLOC_LOGITS_BYTES);
+  lw.part = reinterpret_cast<float2*>(base + NOALLOC_LOGITS_BYTES);
+  lw.row_loss = reinterpret_cast<float*>(base + NOALLOC_LOGITS_BYTES + NOALLOC_PART_BYTES);
+  lw.zy = lw.row_loss + NOALLOC_MAX_ROWS;
+  lw.lse = lw.zy + NOALLOC_MAX_ROWS;
   lw.chunk = (int)std::min<long long>(rows, m.N);
+  lw.h8 = lw.w8 = lw.dz8 = nullptr;
+  lw.amx = nullptr;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cfg->dtype == GPTB_F32)
     return lm_head_impl<float>(*cfg, (const float*)h, (const float*)w_lm, targets, loss_out, (float*)dh, dw_lm, lw, st);

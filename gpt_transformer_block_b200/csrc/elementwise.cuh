@@ -4,8 +4,9 @@
 //     the fp32 configuration (bf16/fp8 fuse the forward into the QKV GEMM
 //     epilogue);
 //   - the value-embedding gate weight gradient;
-//   - cross-entropy over a chunk of logits rows (register-resident rows for
-//     bf16) and the loss mean;
+//   - cross-entropy: the row log-sum-exp from the logits GEMM's per-tile
+//     statistics and the logits gradient (bf16), a two-pass row kernel (fp32),
+//     and the loss mean;
 //   - FP8 (e4m3) per-tensor amax and quantisation.
 // (The attention-backward term D = rowsum(dO o o) comes out of the dO GEMM's
 // epilogue for bf16/fp8, and out of attn_bwd_pre_kernel in attention.cuh for
@@ -17,6 +18,19 @@
 namespace gptb {
 
 constexpr int EW_THREADS = 256;
+
+constexpr float E4M3_MAXF = 448.f, E5M2_MAXF = 57344.f;
+
+// 8 floats times s -> 8 FP8 codes (RNE, saturating), e4m3 or e5m2
+__device__ __forceinline__ uint2 to_fp8x8(const float (&v)[8], float s, bool e5m2) {
+  __nv_fp8x2_storage_t p[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    p[k] = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * k] * s, v[2 * k + 1] * s), __NV_SATFINITE,
+                                    e5m2 ? __NV_E5M2 : __NV_E4M3);
+  return make_uint2((uint32_t)p[0] | ((uint32_t)p[1] << 16), (uint32_t)p[2] | ((uint32_t)p[3] << 16));
+}
+
 
 struct RowLoop {
   long long row, nrows, stride;
@@ -158,8 +172,9 @@ __global__ void ve_gate_wgrad_kernel(const float* __restrict__ dz, const T* __re
 }
 
 // ------------------------------------------------------ cross-entropy ----
-// One CTA per logits row (bf16, V wide): lse, row loss, and the gradient
-// (softmax - onehot) * inv_n written back over the logits in bf16.
+// fp32 logits (SIMT path): one CTA per logits row computes the lse (online
+// max / sum over the row), the row loss, and the gradient
+// (softmax - onehot) * inv_n written back over the logits.
 __device__ __forceinline__ void lse_combine(float& m, float& s, float m2, float s2) {
   if (m2 == -INFINITY) return;
   if (m == -INFINITY) {
@@ -210,7 +225,8 @@ __global__ void __launch_bounds__(512)
   for (int w = 1; w < nw; ++w) lse_combine(M, S, sm[w], ss[w]);
   const float lse = M + logf(S);
   const int y = targets[r];
-  const float zy = to_f(z[y]);
+  const bool y_ok = y >= 0 && y < V;  // an out-of-range target is reported, never read
+  const float zy = y_ok ? to_f(z[y]) : 0.f;
   __syncthreads();
   for (int c = threadIdx.x * 8; c < V; c += blockDim.x * 8) {
     float v[8];
@@ -219,76 +235,134 @@ __global__ void __launch_bounds__(512)
     for (int k = 0; k < 8; ++k) v[k] = (expf(v[k] - lse) - (c + k == y ? 1.f : 0.f)) * inv_n;
     store8(z + c, v);
   }
-  if (threadIdx.x == 0) row_loss[r] = lse - zy;
+  if (threadIdx.x == 0) {
+    if (!y_ok) record_error(ERRW_BAD_TARGET);
+    row_loss[r] = y_ok ? lse - zy : 0.f;
+  }
 }
 
-// bf16 rows of up to XENT_REG_THREADS * 8 * XENT_REG_VEC entries: one CTA per
-// row holds the whole row in registers (all 16-byte loads issued before any
-// use), takes the max, the sum of exp and then the gradient from the same
-// registers, so each logit is read once and written once.  exp by ex2 with the
-// log2(e) scale folded into one FMA.
-constexpr int XENT_REG_THREADS = 512, XENT_REG_VEC = 8;  // 32768 entries
-__global__ void __launch_bounds__(XENT_REG_THREADS, 2)
-    xent_rows_reg_kernel(bf16* __restrict__ logits, long long ld, int V, const int32_t* __restrict__ targets,
-                         float* __restrict__ row_loss, float inv_n, int nrows) {
-  __shared__ float red[XENT_REG_THREADS / 32];
-  const long long r = blockIdx.x;
-  if (r >= nrows) return;
-  bf16* z = logits + r * ld;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = XENT_REG_THREADS / 32;
-  uint4 u[XENT_REG_VEC];
+// bf16 logits (tensor-core path): the row statistics come out of the logits
+// GEMM's epilogue (EPI_XENT: per 256-column tile the max and the sum of
+// exp(z - max), and z at the target), so no kernel reduces over a stored row.
+// xent_lse_kernel: one warp per row combines the row's tile statistics into
+// the log-sum-exp and the row loss lse - z[y].
+__global__ void __launch_bounds__(256)
+    xent_lse_kernel(const float2* __restrict__ part, int nt, const float* __restrict__ zy,
+                    const int32_t* __restrict__ targets, int V, float* __restrict__ lse_l2,
+                    float* __restrict__ row_loss, int rows) {
+  const int lane = threadIdx.x & 31;
+  const long long wpb = blockDim.x >> 5;
+  for (long long r = blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += gridDim.x * wpb) {
+    float m = -INFINITY, sm = 0.f;
+    for (int t = lane; t < nt; t += 32) {
+      const float2 p = part[r * nt + t];
+      lse_combine(m, sm, p.x, p.y);
+    }
 #pragma unroll
-  for (int j = 0; j < XENT_REG_VEC; ++j) {
-    const int c = (j * XENT_REG_THREADS + tid) * 8;
-    // past the vocabulary: -inf (bf16 0xff80), which adds nothing below
-    u[j] = (c < V) ? *reinterpret_cast<const uint4*>(z + c) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
-  }
-  const int y = targets[r];
-  const float zy = __bfloat162float(z[y]);
-  auto val = [&](int j, int k) -> float {  // element k (0..7) of vector j
-    const uint32_t w = (k < 2) ? u[j].x : (k < 4) ? u[j].y : (k < 6) ? u[j].z : u[j].w;
-    return __uint_as_float((k & 1) ? (w & 0xffff0000u) : (w << 16));
-  };
-  float m = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < XENT_REG_VEC; ++j)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) m = fmaxf(m, val(j, k));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[warp] = m;
-  __syncthreads();
-  float M = red[0];
-#pragma unroll
-  for (int w = 1; w < NW; ++w) M = fmaxf(M, red[w]);
-  __syncthreads();
-  const float ml2 = M * LOG2E;
-  float s = 0.f;
-#pragma unroll
-  for (int j = 0; j < XENT_REG_VEC; ++j)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) s += fast_exp2(fmaf(val(j, k), LOG2E, -ml2));
-  s = warp_sum(s);
-  if (lane == 0) red[warp] = s;
-  __syncthreads();
-  float S = 0.f;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) S += red[w];
-  const float lse = M + logf(S);
-  const float ll2 = lse * LOG2E;
-  // gradient (softmax - onehot) / n over the same registers
-#pragma unroll
-  for (int j = 0; j < XENT_REG_VEC; ++j) {
-    const int c = (j * XENT_REG_THREADS + tid) * 8;
-    if (c < V) {
-      float v[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = (fast_exp2(fmaf(val(j, k), LOG2E, -ll2)) - (c + k == y ? 1.f : 0.f)) * inv_n;
-      store8(z + c, v);
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sm, o);
+      lse_combine(m, sm, m2, s2);
+    }
+    if (lane == 0) {
+      const float lse = m + logf(sm);
+      lse_l2[r] = lse * LOG2E;
+      const int y = targets[r];
+      if (y < 0 || y >= V) {
+        record_error(ERRW_BAD_TARGET);  // no z[y]: the row adds nothing to the loss
+        row_loss[r] = 0.f;
+      } else {
+        row_loss[r] = lse - zy[r];
+      }
     }
   }
-  if (tid == 0) row_loss[r] = lse - zy;
+}
+
+// The gradient of the mean loss with respect to the logits, (softmax - onehot)
+// / n, written in bf16 over the logits: one CTA per row, a pure stream (each
+// thread issues XENT_GRAD_VEC 16-byte loads before using any of them).  An
+// out-of-range target drops the one-hot term (and was reported above).
+constexpr int XENT_GRAD_THREADS = 256, XENT_GRAD_VEC = 8;
+__global__ void __launch_bounds__(XENT_GRAD_THREADS)
+    xent_grad_kernel(bf16* __restrict__ z, long long ld, int V, const int32_t* __restrict__ targets,
+                     const float* __restrict__ lse_l2, float inv_n, int rows) {
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  bf16* zr = z + (long long)r * ld;
+  const float l2 = lse_l2[r];
+  const int y = targets[r];
+  const int nvec = V / 8;
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += XENT_GRAD_THREADS * XENT_GRAD_VEC) {
+    uint4 u[XENT_GRAD_VEC];
+#pragma unroll
+    for (int j = 0; j < XENT_GRAD_VEC; ++j) {
+      const int vi = v0 + j * XENT_GRAD_THREADS;
+      if (vi < nvec) u[j] = *reinterpret_cast<const uint4*>(zr + (long long)vi * 8);
+    }
+#pragma unroll
+    for (int j = 0; j < XENT_GRAD_VEC; ++j) {
+      const int vi = v0 + j * XENT_GRAD_THREADS;
+      if (vi < nvec) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h[k]);
+          v[2 * k] = f.x;
+          v[2 * k + 1] = f.y;
+        }
+        const int c = vi * 8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = (fast_exp2(fmaf(v[k], LOG2E, -l2)) - (c + k == y ? 1.f : 0.f)) * inv_n;
+        store8(zr + c, v);
+      }
+    }
+  }
+}
+
+// The FP8 lm_head variant: the same gradient (softmax - onehot)/n, rounded to
+// bf16 (the tensor the FP8 cast applies to) and written as FP8 codes with the
+// fixed scale qmax * n that |dz| <= 1/n allows, into a separate [rows, V]
+// byte buffer; block 0 also stores the bound 1/n, the dequantisation amax.
+__global__ void __launch_bounds__(XENT_GRAD_THREADS)
+    xent_grad_fp8_kernel(const bf16* __restrict__ z, long long ld, int V, const int32_t* __restrict__ targets,
+                         const float* __restrict__ lse_l2, float inv_n, int e5m2, uint8_t* __restrict__ out,
+                         long long ldo, float* __restrict__ bound, int rows) {
+  const int r = blockIdx.x;
+  if (r == 0 && threadIdx.x == 0) *bound = inv_n;
+  if (r >= rows) return;
+  const bf16* zr = z + (long long)r * ld;
+  uint8_t* orow = out + (long long)r * ldo;
+  const float l2 = lse_l2[r];
+  const int y = targets[r];
+  const float s = (e5m2 ? E5M2_MAXF : E4M3_MAXF) / inv_n;
+  const int nvec = V / 8;
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += XENT_GRAD_THREADS * XENT_GRAD_VEC) {
+    uint4 u[XENT_GRAD_VEC];
+#pragma unroll
+    for (int j = 0; j < XENT_GRAD_VEC; ++j) {
+      const int vi = v0 + j * XENT_GRAD_THREADS;
+      if (vi < nvec) u[j] = *reinterpret_cast<const uint4*>(zr + (long long)vi * 8);
+    }
+#pragma unroll
+    for (int j = 0; j < XENT_GRAD_VEC; ++j) {
+      const int vi = v0 + j * XENT_GRAD_THREADS;
+      if (vi < nvec) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h[k]);
+          v[2 * k] = f.x;
+          v[2 * k + 1] = f.y;
+        }
+        const int c = vi * 8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          v[k] = __bfloat162float(__float2bfloat16_rn((fast_exp2(fmaf(v[k], LOG2E, -l2)) - (c + k == y ? 1.f : 0.f)) * inv_n));
+        *reinterpret_cast<uint2*>(orow + c) = to_fp8x8(v, s, e5m2 != 0);
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------ optimizer step --
@@ -368,6 +442,84 @@ __global__ void scale_by_norm_bf16_kernel(const bf16* __restrict__ x, bf16* __re
     y[i] = __float2bfloat16_rn(__bfloat162float(x[i]) * inv);
 }
 
+// Muon momentum (Nesterov form): buf = mu buf + g; u = g + mu buf in bf16,
+// the input of the orthogonalisation.  Four elements per thread step.  Also
+// zeroes the two NorMuon sums used later in the step.
+__global__ void muon_momentum_kernel(const float* __restrict__ g, float* __restrict__ buf, bf16* __restrict__ u,
+                                     long long n4, float mu, float* __restrict__ sums) {
+  if (blockIdx.x == 0 && threadIdx.x < 2) sums[threadIdx.x] = 0.f;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 gg = reinterpret_cast<const float4*>(g)[i];
+    float4 b = reinterpret_cast<float4*>(buf)[i];
+    b.x = fmaf(mu, b.x, gg.x);
+    b.y = fmaf(mu, b.y, gg.y);
+    b.z = fmaf(mu, b.z, gg.z);
+    b.w = fmaf(mu, b.w, gg.w);
+    reinterpret_cast<float4*>(buf)[i] = b;
+    reinterpret_cast<uint2*>(u)[i] =
+        make_uint2(pack_bf16(fmaf(mu, b.x, gg.x), fmaf(mu, b.y, gg.y)), pack_bf16(fmaf(mu, b.z, gg.z), fmaf(mu, b.w, gg.w)));
+  }
+}
+
+// NorMuon statistics, one warp per row (neuron) of the orthogonalised update
+// o [m, n]: v_mean = mean(o^2) over the row, v = beta2 v + (1-beta2) v_mean,
+// step = 1/sqrt(max(v, 1e-10)); sums[0] += v_mean, sums[1] += v_mean step^2.
+__global__ void __launch_bounds__(256)
+    normuon_rows_kernel(const bf16* __restrict__ o, int m, int n, float* __restrict__ v, float beta2,
+                        float* __restrict__ step, float* __restrict__ sums) {
+  const int lane = threadIdx.x & 31;
+  const long long wpb = blockDim.x >> 5;
+  float s1 = 0.f, s2 = 0.f;  // this warp's share of the two sums (lane 0)
+  for (long long r = blockIdx.x * wpb + (threadIdx.x >> 5); r < m; r += gridDim.x * wpb) {
+    const bf16* row = o + r * n;
+    float ss = 0.f;
+    for (int c = lane * 8; c < n; c += 256) {
+      float x[8];
+      load8(row + c, x);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ss = fmaf(x[k], x[k], ss);
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) {
+      const float vm = ss / (float)n;
+      const float vv = fmaf(beta2, v[r], (1.f - beta2) * vm);
+      v[r] = vv;
+      const float st = rsqrtf(fmaxf(vv, 1e-10f));
+      step[r] = st;
+      s1 += vm;
+      s2 += vm * st * st;
+    }
+  }
+  if (lane == 0) {
+    atomicAdd(&sums[0], s1);
+    atomicAdd(&sums[1], s2);
+  }
+}
+
+// w = w (1 - lr wd) - lr o step[row] sqrt(sums[0]) / max(sqrt(sums[1]), 1e-10),
+// and the bf16 working copy (if any).  Four elements per thread step.
+__global__ void muon_apply_kernel(float* __restrict__ w, bf16* __restrict__ wb, const bf16* __restrict__ o,
+                                  const float* __restrict__ step, const float* __restrict__ sums, int m, int n,
+                                  float lr, float wd) {
+  const float ratio = sqrtf(sums[0]) / fmaxf(sqrtf(sums[1]), 1e-10f);
+  const float decay = 1.f - lr * wd;
+  const long long n4 = (long long)m * n / 4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = (i * 4) / n;
+    const float sc = lr * step[r] * ratio;
+    const uint2 ou = reinterpret_cast<const uint2*>(o)[i];
+    const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ou.x));
+    const float2 o23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ou.y));
+    float4 ww = reinterpret_cast<float4*>(w)[i];
+    ww.x = fmaf(ww.x, decay, -sc * o01.x);
+    ww.y = fmaf(ww.y, decay, -sc * o01.y);
+    ww.z = fmaf(ww.z, decay, -sc * o23.x);
+    ww.w = fmaf(ww.w, decay, -sc * o23.y);
+    reinterpret_cast<float4*>(w)[i] = ww;
+    if (wb) reinterpret_cast<uint2*>(wb)[i] = make_uint2(pack_bf16(ww.x, ww.y), pack_bf16(ww.z, ww.w));
+  }
+}
+
 // loss = mean of the row losses (single CTA, fixed order)
 __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ x, long long n, float* __restrict__ out) {
   __shared__ float sred[32];
@@ -410,23 +562,16 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, long
   }
 }
 
-__device__ __forceinline__ float fp8_inv_scale(const float* amax) { return fmaxf(*amax, 1e-12f) / 448.f; }
-
+// codes = RNE-satfinite(x * qmax / amax), qmax = 448 (e4m3) or 57344 (e5m2)
 template <class T>
 __global__ void __launch_bounds__(256)
-    quantize_e4m3_kernel(const T* __restrict__ x, long long n8, const float* __restrict__ amax, uint8_t* __restrict__ out) {
-  const float s = 448.f / fmaxf(*amax, 1e-12f);
+    quantize_fp8_kernel(const T* __restrict__ x, long long n8, const float* __restrict__ amax, int e5m2,
+                        uint8_t* __restrict__ out) {
+  const float s = (e5m2 ? E5M2_MAXF : E4M3_MAXF) / fmaxf(*amax, 1e-12f);
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
     float v[8];
     load8(x + i * 8, v);
-    uint2 o;
-    __nv_fp8x2_storage_t p[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      p[k] = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * k] * s, v[2 * k + 1] * s), __NV_SATFINITE, __NV_E4M3);
-    o.x = (uint32_t)p[0] | ((uint32_t)p[1] << 16);
-    o.y = (uint32_t)p[2] | ((uint32_t)p[3] << 16);
-    *reinterpret_cast<uint2*>(out + i * 8) = o;
+    *reinterpret_cast<uint2*>(out + i * 8) = to_fp8x8(v, s, e5m2 != 0);
   }
 }
 

@@ -14,10 +14,14 @@
 //             elementwise op into a swizzled per-warp smem tile, written by
 //             TMA bulk stores (bf16) or TMA bulk reduce-add (fp32 weight
 //             gradients); residual / saved-u inputs arrive by TMA loads
-//   Tile 128 x 256, two TMEM accumulators (2 x 256 columns) so the epilogue
-//   of tile i overlaps the MMAs of tile i+1.  Split-K over the K blocks is
-//   used for weight gradients (long K, few tiles); partial sums meet in the
-//   fp32 gradient through vector atomics.
+//   Tile 128 x 256 per CTA, two TMEM accumulators (2 x 256 columns) so the
+//   epilogue of tile i overlaps the MMAs of tile i+1.  Pair form: a cluster
+//   of two CTAs runs M = 256 tcgen05.mma (cta_group::2) on a 256 x 256 tile,
+//   each CTA staging half of A and half of B (loads without multicast; the
+//   odd CTA's loads complete on the even CTA's barriers), so each SM reads a
+//   third less operand data per FLOP.  Split-K over the K blocks is used for
+//   weight gradients (long K, few tiles); partial sums meet in the fp32
+//   gradient through TMA reduce-adds.
 // fp32 path (SIMT, FFMA): a plain tiled kernel with the same epilogues, for
 //   the fp32 configuration whose 1e-5 tolerance tensor-core fp32 (tf32)
 //   inputs cannot meet.
@@ -37,6 +41,10 @@ enum EpiKind : int {
   EPI_DOT = 6,        // out = alpha*acc (bf16) and, per row and 128-column
                       // group h, rowdot[b, h, t] = sum(out * aux) (aux = the
                       // attention output o, out = dO: the backward's D term)
+  EPI_XENT = 7,       // out = z = alpha*acc (bf16 logits) and, per row and
+                      // 256-column tile n, the softmax statistics of the
+                      // tile: xent_part[row, n] = (max z, sum exp(z - max));
+                      // xent_zy[row] = z[row, targets[row]] (fp32)
 };
 
 struct EpiParams {
@@ -54,6 +62,7 @@ struct EpiParams {
   // (amax_a / 448) * (amax_b / 448), the inverse of the two quantisation scales
   const float* amax_a;
   const float* amax_b;
+  int a_e5m2;  // A operand in e5m2 (its scale 57344/amax; B is always e4m3, 448/amax)
   // EPI_QKV: per-head QK RMSNorm + RoPE and the value-embedding add
   const float2* rope;     // [T, 64] (cos, sin)
   float* rstd_qk;         // [M, H + Hkv]
@@ -63,12 +72,18 @@ struct EpiParams {
   int T, H, Hkv;
   float eps;
   float* rowdot;          // EPI_DOT: [B, H, T] fp32
+  // EPI_XENT: per-(row, 256-column tile) statistics, row stride xent_nt
+  float2* xent_part;
+  int xent_nt;
+  const int32_t* targets;  // [M] class ids; ids outside [0, N) match no column
+  float* xent_zy;          // [M]
 };
 
 __device__ __forceinline__ float epi_beta(const EpiParams& ep) { return ep.beta ? *ep.beta : 1.f; }
 __device__ __forceinline__ float epi_alpha(const EpiParams& ep) {
   float a = ep.alpha ? *ep.alpha : 1.f;
-  if (ep.amax_a) a *= (fmaxf(*ep.amax_a, 1e-12f) / 448.f) * (fmaxf(*ep.amax_b, 1e-12f) / 448.f);
+  if (ep.amax_a)
+    a *= (fmaxf(*ep.amax_a, 1e-12f) / (ep.a_e5m2 ? 57344.f : 448.f)) * (fmaxf(*ep.amax_b, 1e-12f) / 448.f);
   return a;
 }
 
@@ -142,17 +157,28 @@ __device__ __forceinline__ void epi_apply1(const EpiParams& ep, long long r, int
 }
 
 // ------------------------------------------------------ tcgen05 kernel ----
-constexpr int TC_BM = 128;
-constexpr int TC_BN = 256;
-constexpr int TC_STAGES = 4;
+constexpr int TC_BM = 128;   // rows of A (and TMEM lanes of D) per CTA
+constexpr int TC_BN = 256;   // columns of D per CTA (one TMEM accumulator)
 constexpr int TC_THREADS = 192;
 constexpr int TC_GROUP_M = 8;
 
 constexpr int TC_EPI_BYTES = 4 * 8192;  // per epilogue warp: two 32-row x 128-byte staging tiles
-__host__ __device__ constexpr int tc_smem_bytes() {
-  // stages * (A 16 KB + B 32 KB) + epilogue staging + barriers + 1 KB alignment slack
-  return TC_STAGES * (TC_BM * 128 + TC_BN * 128) + TC_EPI_BYTES + 256 + 1024;
-}
+
+// Tile shape of the two kernel forms.
+//   single: one CTA computes a 128 x 256 tile (A 128 rows, B 256 rows per stage)
+//   pair:   a cluster of two CTAs computes a 256 x 256 tile with M = 256
+//           tcgen05.mma issued by the even CTA; each CTA stages its own 128
+//           rows of A and 128 rows of B (so each SM reads 32 KB of operands
+//           per 64-deep K block instead of 48 KB) and holds its 128 rows of D
+template <bool PAIR> struct TcShape {
+  static constexpr int TILE_M = PAIR ? 256 : 128;
+  static constexpr int B_ROWS = PAIR ? 128 : 256;
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int A_BYTES = TC_BM * 128;
+  static constexpr int B_BYTES = B_ROWS * 128;
+  // stages * (A + B) + epilogue staging + barriers + 1 KB alignment slack
+  static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES) + TC_EPI_BYTES + 256 + 1024;
+};
 
 __device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, int& tm, int& tn, int& split) {
   const int tiles = tiles_m * tiles_n;
@@ -247,28 +273,33 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, uint32_t ta, u
   }
 }
 
-template <bool A_MN, bool B_MN, bool FP8>
+template <bool A_MN, bool B_MN, bool FP8, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                    const __grid_constant__ CUtensorMap tmX, int M, int N, int K, int splits, EpiParams ep) {
+  using SH = TcShape<PAIR>;
+  constexpr int STAGES = SH::STAGES;
   constexpr int ELEM = FP8 ? 1 : 2;
   constexpr int BK = 128 / ELEM;      // one 128-byte swizzle row of K (64 bf16 / 128 e4m3)
   constexpr int MMA_K = 32 / ELEM;    // K per tcgen05.mma (16 bf16 / 32 e4m3)
   constexpr int ATOM = BK;            // MN extent of one swizzle atom for MN-major operands
-  constexpr int A_BYTES = TC_BM * 128;
-  constexpr int B_BYTES = TC_BN * 128;
-  constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
-  constexpr uint32_t IDESC = make_idesc(TC_BM, TC_BN, A_MN, B_MN, FP8);
+  constexpr int A_BYTES = SH::A_BYTES;
+  constexpr int B_BYTES = SH::B_BYTES;
+  constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;             // bytes landing in one CTA per stage
+  constexpr uint32_t FULL_TX = PAIR ? 2 * STAGE_TX : STAGE_TX;  // bytes a stage's full barrier waits for
+  constexpr uint32_t IDESC0 = make_idesc(SH::TILE_M, TC_BN, A_MN, B_MN, FP8);
+  // kind::f8f6f4 A format (bits 7-9): 0 = e4m3, 1 = e5m2
+  const uint32_t IDESC = IDESC0 | ((FP8 && ep.a_e5m2) ? (1u << 7) : 0u);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + TC_STAGES * A_BYTES;
-  uint8_t* sEpi = sB + TC_STAGES * B_BYTES;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint8_t* sEpi = sB + STAGES * B_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + TC_EPI_BYTES);
-  uint64_t* empty = full + TC_STAGES;
-  uint64_t* tfull = empty + TC_STAGES;
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* aux_bar = drain + 1;  // [4] one per epilogue warp
@@ -276,19 +307,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_m = (M + TC_BM - 1) / TC_BM, tiles_n = (N + TC_BN - 1) / TC_BN;
+  // pair: both CTAs of a cluster walk the same units; the even CTA (rank 0)
+  // issues the MMAs and owns the stage and accumulator-drain barriers
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int ustep = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
+  const int tiles_m = (M + SH::TILE_M - 1) / SH::TILE_M, tiles_n = (N + TC_BN - 1) / TC_BN;
   const int units = tiles_m * tiles_n * splits;
   const int kb_total = (K + BK - 1) / BK;
   const int kb_per = (kb_total + splits - 1) / splits;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], PAIR ? 8 : 4);  // the epilogue warps of both CTAs drain an accumulator
     }
     mbar_init(drain, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&aux_bar[i], 1);
@@ -297,9 +333,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 1) {
+    if (PAIR) tmem_alloc_pair(tmem_slot, 512);
+    else tmem_alloc(tmem_slot, 512);
+  }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -309,63 +349,80 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;  // stages with a load in flight, and the phase they complete
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = unit0; u < units && ok; u += ustep) {
         int tm, tn, split;
         tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
         const int kb0 = split * kb_per, kb1 = min(kb_total, kb0 + kb_per);
+        const int arow = tm * SH::TILE_M + (int)rank * TC_BM;      // this CTA's rows of A
+        const int brow = tn * TC_BN + (int)rank * SH::B_ROWS;      // this CTA's rows of B
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, ERRW_TIMEOUT_PRODUCER)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], STAGE_TX);
+          // the even CTA arms its stage barrier for both CTAs' bytes; the odd
+          // CTA's loads count down the same barrier (a count that goes below
+          // zero before the arming is allowed: the phase needs the arrival)
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], FULL_TX);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           uint8_t* a = sA + stage * A_BYTES;
           uint8_t* b = sB + stage * B_BYTES;
           const int k0 = kb * BK;
+          auto load = [&](void* dst, const CUtensorMap* m, int c0, int c1) {
+            if (PAIR) tma_load_2d_pair(dst, m, map_shared_rank(&full[stage], 0), c0, c1);
+            else tma_load_2d(dst, m, &full[stage], c0, c1);
+          };
           if (!A_MN) {
-            tma_load_2d(a, &tmA, &full[stage], k0, tm * TC_BM);
+            load(a, &tmA, k0, arow);
           } else {
 #pragma unroll
-            for (int i = 0; i < TC_BM / ATOM; ++i) tma_load_2d(a + i * BK * 128, &tmA, &full[stage], tm * TC_BM + i * ATOM, k0);
+            for (int i = 0; i < TC_BM / ATOM; ++i) load(a + i * BK * 128, &tmA, arow + i * ATOM, k0);
           }
           if (!B_MN) {
-            tma_load_2d(b, &tmB, &full[stage], k0, tn * TC_BN);
+            load(b, &tmB, k0, brow);
           } else {
 #pragma unroll
-            for (int i = 0; i < TC_BN / ATOM; ++i) tma_load_2d(b + i * BK * 128, &tmB, &full[stage], tn * TC_BN + i * ATOM, k0);
+            for (int i = 0; i < SH::B_ROWS / ATOM; ++i) load(b + i * BK * 128, &tmB, brow + i * ATOM, k0);
           }
-          if (++stage == TC_STAGES) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       // after an abort, wait (bounded) for the loads this thread issued to land
-      // before the CTA exits; a consumed stage's phase has already completed
+      // before the CTA exits; a consumed stage's phase has already completed.
+      // The odd CTA of a pair cannot wait on the even CTA's barriers: it gives
+      // its loads a fixed 1 ms.
       if (!ok) {
-        for (int s2 = 0; s2 < TC_STAGES; ++s2) {
-          if (!(armed & (1u << s2))) continue;
-          const uint32_t par = (armed_par >> s2) & 1u;
+        if (PAIR && rank != 0) {
           const unsigned long long t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full[s2], par)) {
-            if (globaltimer_ns() - t0 > 100000000ull) {
-              record_error(ERRW_TIMEOUT_DRAIN);
-              break;
+          while (globaltimer_ns() - t0 < 1000000ull) {
+          }
+        } else {
+          for (int s2 = 0; s2 < STAGES; ++s2) {
+            if (!(armed & (1u << s2))) continue;
+            const uint32_t par = (armed_par >> s2) & 1u;
+            const unsigned long long t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[s2], par)) {
+              if (globaltimer_ns() - t0 > 100000000ull) {
+                record_error(ERRW_TIMEOUT_DRAIN);
+                break;
+              }
             }
           }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = unit0; u < units && ok; u += ustep) {
         int tm, tn, split;
         tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
         const int kb0 = split * kb_per, kb1 = min(kb_total, kb0 + kb_per);
@@ -388,23 +445,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + k * MMA_K * 128, BK * 128, 1024)
                                      : smem_desc_sw128(b_addr + k * 32, 16, 1024);
             const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
-            if (FP8) mma_f8_ss(d_tmem, ad, bd, IDESC, accum);
-            else mma_bf16_ss(d_tmem, ad, bd, IDESC, accum);
+            if (PAIR) {
+              if (FP8) mma_f8_ss_pair(d_tmem, ad, bd, IDESC, accum);
+              else mma_bf16_ss_pair(d_tmem, ad, bd, IDESC, accum);
+            } else {
+              if (FP8) mma_f8_ss(d_tmem, ad, bd, IDESC, accum);
+              else mma_bf16_ss(d_tmem, ad, bd, IDESC, accum);
+            }
           }
-          mma_commit(&empty[stage]);
-          if (++stage == TC_STAGES) {
+          // the stage is free again in both CTAs once these MMAs have read it
+          if (PAIR) mma_commit_pair_both(&empty[stage]);
+          else mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull[acc]);
+        if (PAIR) mma_commit_pair_both(&tfull[acc]);
+        else mma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       if (*abort_flag) {
         // let every MMA this thread issued finish before TMEM is released
-        mma_commit(drain);
+        if (PAIR) mma_commit_pair_local(drain);
+        else mma_commit(drain);
         const unsigned long long t0 = globaltimer_ns();
         while (!mbar_try_wait(drain, 0)) {
           if (globaltimer_ns() - t0 > 100000000ull) {
@@ -428,12 +494,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const float alpha = epi_alpha(ep);
     const float beta = epi_beta(ep);
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = unit0; u < units && ok; u += ustep) {
       int tm, tn, split;
       tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
       if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const int row0 = tm * TC_BM + q * 32;
+      const int row0 = tm * SH::TILE_M + (int)rank * TC_BM + q * 32;
       if (ep.kind == EPI_QKV) {
 #pragma unroll 1
         for (int hb = 0; hb < TC_BN / 128; ++hb) {
@@ -453,6 +519,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       float dsum = 0.f;  // EPI_DOT: this row's running sum over the current 128-column group
+      // EPI_XENT: this row's running max and sum of exp2((z - max) * log2 e) over the tile
+      float xm = -INFINITY, xs = 0.f;
+      const int xy = (ep.kind == EPI_XENT && row0 + lane < M) ? ep.targets[row0 + lane] : -1;
 #pragma unroll 1
       for (int cc = 0; cc < (ep.kind == EPI_QKV ? 0 : TC_BN / 64); ++cc) {
         const int col0 = tn * TC_BN + cc * 64;
@@ -478,6 +547,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         uint8_t* p0 = stg0 + lane * 128;
         uint8_t* p1 = stg1 + lane * 128;
+        float xml2 = 0.f;  // EPI_XENT: running max * log2 e after this chunk
+        if (ep.kind == EPI_XENT) {
+          float cm = xm;
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (col0 + i < N) cm = fmaxf(cm, __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
+          if (cm > xm) {  // rescale the sum to the new max (0 while the max was -inf)
+            xs = (xm == -INFINITY) ? 0.f : xs * fast_exp2((xm - cm) * LOG2E);
+            xm = cm;
+          }
+          xml2 = xm * LOG2E;
+        }
         if (acc32) {
           // fp32: columns 0..31 -> tile 0, 32..63 -> tile 1 (32 x 128-byte rows each)
 #pragma unroll
@@ -513,6 +594,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int i = 0; i < 8; ++i) dsum = fmaf(__bfloat162float(__float2bfloat16_rn(v[i])), a[i], dsum);
               }
             }
+            if (ep.kind == EPI_XENT) {
+              // columns past N (the last tile's tail) do not take part
+              const int c8 = col0 + g * 8;
+              float acc = 0.f;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc += (c8 + i < N) ? fast_exp2(fmaf(v[i], LOG2E, -xml2)) : 0.f;
+              xs += acc;
+              if (xy >= c8 && xy < c8 + 8) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  if (xy == c8 + i) ep.xent_zy[row0 + lane] = v[i];
+              }
+            }
             store8(reinterpret_cast<bf16*>(cp0), v);
             if (ep.kind == EPI_RELU2) {
 #pragma unroll
@@ -545,18 +639,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           bulk_commit_group();
         }
       }
+      // (a tile cut short by the N tail still covers at least one chunk)
+      if (ep.kind == EPI_XENT && ok && row0 + lane < M)
+        ep.xent_part[(long long)(row0 + lane) * ep.xent_nt + tn] = make_float2(xm, xs);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(map_shared_rank(&tempty[acc], 0));
+        else mbar_arrive(&tempty[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
     if (lane == 0) bulk_wait0();
   }
+  tc_fence_before();
   __syncthreads();
+  // pair: neither CTA leaves (or frees its tensor memory) while the other may
+  // still arrive on its barriers
+  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    if (PAIR) tmem_dealloc_pair(tmem_base, 512);
+    else tmem_dealloc(tmem_base, 512);
   }
 }
 

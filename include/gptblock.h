@@ -45,7 +45,10 @@ enum {
   GPTB_ERR_UNSUPPORTED = -2, /* dtype, head_dim or device not supported      */
   GPTB_ERR_CUDA = -3,        /* a CUDA call or kernel launch failed          */
   GPTB_ERR_TIMEOUT = -4,     /* a bounded device wait expired (see below)    */
-  GPTB_ERR_WORKSPACE = -5    /* workspace too small                          */
+  GPTB_ERR_WORKSPACE = -5,   /* workspace too small                          */
+  GPTB_ERR_BAD_INPUT = -6    /* a device-side check found invalid input data
+                                (a target id outside [0, vocab)); reported by
+                                gptb_device_error()                          */
 };
 
 enum { GPTB_F32 = 0, GPTB_BF16 = 1, GPTB_FP8_E4M3 = 2 };
@@ -70,7 +73,16 @@ typedef struct {
   float rope_base;     /* 10000                                                   */
   float norm_eps;      /* RMSNorm epsilon inside the rsqrt (1e-6)                 */
   int dtype;           /* GPTB_F32 | GPTB_BF16 | GPTB_FP8_E4M3                    */
+  int fp8_flags;       /* GPTB_FP8_E4M3 configs only (0 otherwise), bits:
+                          GPTB_FP8_GRAD_E5M2: gradient operands of the input- and
+                            weight-gradient GEMMs in e5m2 (scale 57344/amax);
+                          GPTB_FP8_LM_HEAD: the lm_head GEMMs in FP8 too (logits
+                            from e4m3 hf and W_lm; the logits gradient, whose
+                            entries lie in [-1/N, 1/N], with the fixed scale
+                            qmax*N, in e5m2 with GPTB_FP8_GRAD_E5M2)          */
 } gptb_config;
+
+enum { GPTB_FP8_GRAD_E5M2 = 1, GPTB_FP8_LM_HEAD = 2 };
 
 /* Weights of one block (storage dtype).  w_ve_gate / ve_table only on
  * value-embedding layers (NULL elsewhere). */
@@ -148,12 +160,28 @@ int gpt_block_backward(const gptb_config* cfg, int layer, const gptb_block_weigh
 
 /* Untied lm_head + mean next-token cross-entropy over N = B*T rows without
  * materialising the full [N, V] logits (row chunks of at most 8192 tokens).
+ * Source: the same page, § 1 feature list (untied embedding and output
+ * projection); dev.to/aakira "ChatGPTを50ドルでトレーニングする方法", table of
+ * what nanochat covers (BPE vocabulary 32,768).
  *   h [N,d] (normed final hidden state), w_lm [V,d], targets [N] int32
  *   loss_out: device fp32 scalar (written, the mean over N)
  *   dh [N,d] storage dtype (written); dw_lm [V,d] fp32 (accumulated)
- *   ws: GPTB_WS_LM_HEAD bytes.  bf16/fp8 configs only. */
+ *   ws: GPTB_WS_LM_HEAD bytes.
+ * bf16 and FP8 configs (the lm_head stays bf16 in FP8 configs): the logits
+ * GEMM's epilogue emits each row's softmax statistics per 256-column tile and
+ * z at the target, a warp per row combines them into the log-sum-exp, and one
+ * streaming pass writes the gradient (softmax - onehot)/N over the chunk's
+ * logits, which the dh and dW GEMMs read.  fp32 configs: SIMT GEMMs and a
+ * two-pass row kernel.
+ * targets must lie in [0, vocab).  A target outside that range is never read
+ * as an index: its row's loss term is 0 and its gradient lacks the one-hot
+ * term, and gptb_device_error() returns GPTB_ERR_BAD_INPUT afterwards (the
+ * call's results are then not meaningful). */
 int lm_head_xent(const gptb_config* cfg, const void* h, const void* w_lm, const int32_t* targets, float* loss_out,
                  void* dh, float* dw_lm, void* ws, gptb_stream_t stream);
+
+/* (GPTB_FP8_LM_HEAD configs: lm_head_xent_noalloc returns GPTB_ERR_UNSUPPORTED,
+ * since the FP8 copies of hf and W_lm need the workspace.) */
 
 /* lm_head_xent without a workspace, for callers that cannot allocate device
  * memory themselves: for example a plugin or C caller that is handed tensors
@@ -161,18 +189,21 @@ int lm_head_xent(const gptb_config* cfg, const void* h, const void* w_lm, const 
  * a latency-critical path that must not call cudaMalloc (which can
  * synchronise the device).  No counterpart on the source pages: this is a
  * convenience of this library.
- *   Same arguments, results and accumulation (+= into dw_lm) as lm_head_xent,
- *   minus `ws`.  Its scratch is one file-scope device array of 8 MiB of
- *   logits plus 256 KiB of row losses, held by every GPU that loads the
- *   library until the process exits.  Limits: B*T <= 65536 and
- *   vocab * element size <= 8 MiB (otherwise GPTB_ERR_WORKSPACE, nothing
- *   enqueued).  Rows are processed in chunks of 8 MiB / (vocab * element
- *   size) rows (128 rows for vocab 32768 in bf16).
- *   The first call on a device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
- *   Nothing is allocated or freed.  All calls share the one array and every
- *   call overwrites it: calls that overlap on the GPU (other streams, other
- *   threads) race and give wrong results; serialise them. */
+ *   Same arguments, results, target rule and accumulation (+= into dw_lm) as
+ *   lm_head_xent, minus `ws`.  Its scratch is one file-scope device array of
+ *   8 MiB of logits, 1 MiB of per-tile softmax statistics and 768 KiB of
+ *   per-row values (losses, z at the target, log-sum-exp), held by every GPU
+ *   that loads the library until the process exits.  Limits: B*T <= 65536
+ *   and vocab * element size <= 8 MiB (otherwise GPTB_ERR_WORKSPACE, nothing
+ *   enqueued).  Rows are processed in chunks of
+ *   min(8 MiB / (vocab * element size), 1 MiB / (8 * ceil(vocab / 256)))
+ *   rows (128 rows for vocab 32768 in bf16).
+ *   Every call looks up the array's device address on the current device;
+ *   the first call on a device also loads the library's kernels there, so
+ *   make that first call before any stream capture.  Nothing is allocated or
+ *   freed.  All calls share the one array and every call overwrites it:
+ *   calls that overlap on the GPU (other streams, other threads) race and
+ *   give wrong results; serialise them. */
 int lm_head_xent_noalloc(const gptb_config* cfg, const void* h, const void* w_lm, const int32_t* targets,
                          float* loss_out, void* dh, float* dw_lm, gptb_stream_t stream);
 
@@ -229,6 +260,32 @@ size_t gptb_polar_express_workspace_bytes(int m, int n, int steps);
 int gptb_polar_express(const void* G, void* out, int m, int n, const float* coeffs, int steps, void* workspace,
                        size_t workspace_bytes, gptb_stream_t stream);
 
+/* Device workspace in bytes of gptb_muon_step for an [m, n] matrix. */
+size_t gptb_muon_workspace_bytes(int m, int n, int steps);
+
+/* One Muon step on a 2-D weight W [m, n] (rows = output neurons), in place.
+ * Sources: the same page, § 2 (the Polar Express loop, two of its five
+ * coefficient tuples, the NorMuon lines); K. Jordan et al., "Muon: An
+ * optimizer for hidden layers in neural networks" (2024) for the Nesterov
+ * momentum; N. Amsel et al., "The Polar Express" (2025) for the five tuples;
+ * Z. Li et al., "NorMuon" (2025) for the per-neuron second moment.
+ *   buf = mu buf + g;  u = g + mu buf                       (momentum, Nesterov)
+ *   o = Polar Express of u over coeffs[0..steps-1]          (as gptb_polar_express)
+ *   v = beta2 v + (1-beta2) mean_row(o^2);  step = 1/sqrt(max(v, 1e-10))
+ *   scale_row = step_row * sqrt(sum mean_row(o^2)) / max(sqrt(sum mean_row(o^2) step_row^2), 1e-10)
+ *   w = w (1 - lr wd) - lr o scale_row;  w_bf16 = bf16(w)   (the update keeps the norm of o)
+ * w: device fp32 [m, n] (updated); w_bf16: device bf16 [m, n] receiving the
+ * new weight rounded to nearest-even, or NULL; g: device fp32 [m, n] (read);
+ * buf: device fp32 [m, n] momentum (updated); v: device fp32 [m] second
+ * moment (updated).  coeffs: HOST float [3*steps].  workspace: device,
+ * gptb_muon_workspace_bytes(m, n, steps) bytes, 256-byte aligned.  Errors:
+ * GPTB_ERR_INVALID_ARG (m or n not a positive multiple of 8, steps outside
+ * 1..64, null or misaligned pointers), GPTB_ERR_WORKSPACE, GPTB_ERR_UNSUPPORTED
+ * (not an sm_100 device). */
+int gptb_muon_step(float* w, void* w_bf16, const float* g, float* buf, float* v, int m, int n, const float* coeffs,
+                   int steps, float lr, float mu, float beta2, float weight_decay, void* workspace,
+                   size_t workspace_bytes, gptb_stream_t stream);
+
 /* ---------------------------------------------------------- decode ----
  * One generation step of the inference engine (apidog.com/fr "Comment
  * Entraîner Votre Propre ChatGPT Pour 50€ ?", § 6 "Moteur d'inférence": a KV
@@ -251,9 +308,11 @@ int gptb_polar_express(const void* G, void* out, int m, int n, const float* coef
 int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, void* o,
                           float* lse, int B, int H, int Hkv, int T_max, int window, gptb_stream_t stream);
 
-/* Synchronises `stream`, then reads and clears the device error word./* Synchronises `stream`, then reads and clears the device error word.
+/* Synchronises `stream`, then reads and clears the device error word.
  * Returns GPTB_OK, GPTB_ERR_TIMEOUT if a bounded wait inside a kernel expired
- * (the kernel recorded it, drained and returned), or GPTB_ERR_CUDA. */
+ * (the kernel recorded it, drained and returned), GPTB_ERR_BAD_INPUT if a
+ * kernel found invalid input data (a cross-entropy target outside
+ * [0, vocab)), or GPTB_ERR_CUDA. */
 int gptb_device_error(gptb_stream_t stream);
 
 /* Self-test of the bounded waits: sets the wait limit to limit_ns, launches
@@ -273,8 +332,10 @@ int gptb_set_wait_limit_ns(unsigned long long ns);
 void gptb_reset_counters(void);
 long long gptb_launch_count(void);
 int gptb_set_gemm_timing(int enable);
-/* Sum of GEMM device milliseconds and FLOPs since the last reset (syncs). */
-int gptb_gemm_timing(double* ms, double* flops, long long* launches);
+/* Sum of GEMM device milliseconds and FLOPs since the last reset (syncs);
+ * ms_fp8 / flops_fp8: the part of those from GEMMs with e4m3 operands.  Any
+ * output pointer may be NULL. */
+int gptb_gemm_timing(double* ms, double* flops, double* ms_fp8, double* flops_fp8, long long* launches);
 
 /* Human-readable text for a return code. */
 const char* gptb_error_string(int code);

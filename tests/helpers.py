@@ -25,6 +25,14 @@ def scalar_err(gpu: float, ref: float, scale: float) -> float:
     return abs(float(gpu) - float(ref)) / max(float(scale), 1e-300)
 
 
+def fp8_mode(c: dict):
+    """The oracle's fp8 argument for a config: False, True (e4m3 operands) or
+    "e5m2" (e5m2 gradient operands)."""
+    if c["dtype"] != "fp8":
+        return False
+    return "e5m2" if c.get("fp8_grad") == "e5m2" else True
+
+
 def np64(t) -> np.ndarray:
     if isinstance(t, torch.Tensor):
         return t.detach().float().cpu().double().numpy()

@@ -9,7 +9,7 @@ import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, np64, oracle_layer, relerr, scalar_err, small_bf16
+from helpers import TOL, fp8_mode, np64, oracle_layer, relerr, scalar_err, small_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -40,7 +40,7 @@ def check_block(gb, c, layer, seed=1, x_std=1.0, exact_keys=()):
     inp = synth.make_block_inputs(c, seed=seed + 1, x_std=x_std)
     x_out, dx, dx0, g = run_block(gb, c, w, inp, layer)
     lw = oracle_layer(w, layer)
-    f8 = c["dtype"] == "fp8"
+    f8 = fp8_mode(c)
     y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), inp["idx"].numpy(), layer, fp8=f8)
     rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), inp["idx"].numpy(), layer, fp8=f8)
     tol = TOL[c["dtype"]]
@@ -82,8 +82,10 @@ def test_block_fp32_all_terms(cuda_lib):
 
 
 @pytest.mark.parametrize("layer", [0, 1])
-def test_block_fp8(cuda_lib, layer):
+@pytest.mark.parametrize("grad", ["e4m3", "e5m2"])
+def test_block_fp8(cuda_lib, layer, grad):
     # e4m3 operands with per-tensor scales on the four block GEMMs (fwd, dgrad,
-    # wgrad); the oracle quantises the same operands the same way
-    c = small_bf16(dtype="fp8", n_layer=2, window=[-1, 48], has_ve=[0, 1])
+    # wgrad), or e5m2 gradient operands (the variant); the oracle quantises the
+    # same bf16 tensors the same way
+    c = small_bf16(dtype="fp8", n_layer=2, window=[-1, 48], has_ve=[0, 1], fp8_grad=grad)
     check_block(cuda_lib, c, layer)

@@ -1,28 +1,28 @@
-"""Full-size parity at the benchmark's shapes (B=16, T=2048): one block forward
-and backward through the C ABI; sampled batch rows are checked against the
-fp64 oracle run on those rows alone (rows of the batch are independent in the
-forward and in dx / dx0).  Weight gradients sum over all rows and are covered
-at smaller sizes by test_block_gpu.py."""
+"""Full-size parity at the configurations' widths and sequence length (T=2048).
+
+1. One block at full width (B=1, or B=2 for FP8 so that the per-tensor scales
+   see more than one batch row), forward and backward through the C ABI,
+   against the fp64 oracle: the block output, dx, dx0 and EVERY gradient
+   (w_qkv, w_o, w_fc, w_proj, w_ve_gate, ve_table and both lambdas).  Both
+   window kinds of d20_gqa (window 1024 on even layers, full on odd ones) are
+   covered, and value-embedding layers of every config.
+2. The benchmark's launch configuration (B=16, T=2048): sampled batch rows
+   of the block output, dx and dx0 checked against the oracle run on those
+   rows alone (rows are independent in the forward and in dx / dx0; bf16
+   only, since FP8's per-tensor scales depend on every row)."""
 import numpy as np
 import pytest
 import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, np64, oracle_layer, relerr
+from helpers import TOL, fp8_mode, np64, oracle_layer, relerr, scalar_err
 
 pytestmark = pytest.mark.gpu
 
 
-# (FP8 is left out here: its per-tensor scales depend on every row of the batch,
-# so one row alone is not the same computation; FP8 parity is in the block and
-# stack tests)
-@pytest.mark.parametrize("name,layer,rows", [("d24", 23, (0, 15)), ("d20_gqa", 0, (7,)), ("d12", 11, (3,))])
-def test_block_full_size_sampled_rows(cuda_lib, name, layer, rows):
+def _run_block(c, w, inp, layer):
     from gpt_transformer_block_b200.model import BlockRunner, to_device_weights, zero_grads_like
-    c = synth.config(name)
-    w = synth.make_weights(c, seed=101)
-    inp = synth.make_block_inputs(c, seed=102)
     dw = to_device_weights(c, w)
     lw = dw["layers"][layer]
     x = inp["x"].to("cuda", torch.bfloat16)
@@ -37,16 +37,49 @@ def test_block_full_size_sampled_rows(cuda_lib, name, layer, rows):
     dx0 = torch.zeros(x.shape, dtype=torch.float32, device="cuda")
     r.backward(layer, lw, x, x0, idx, dy, dx, dx0, g)
     torch.cuda.synchronize()
+    return x_out, dx, dx0, g
+
+
+@pytest.mark.parametrize("name,layer,B", [("d12", 11, 1), ("d12", 10, 1), ("d20_gqa", 18, 1), ("d20_gqa", 19, 1),
+                                          ("d24", 23, 1), ("d24", 12, 1), ("d26_fp8", 25, 2), ("d26_fp8", 0, 2)])
+def test_block_full_width_every_gradient(cuda_lib, name, layer, B):
+    c = synth.config(name, B=B)
+    w = synth.make_weights(c, seed=201 + layer)
+    inp = synth.make_block_inputs(c, seed=202 + layer)
+    x_out, dx, dx0, g = _run_block(c, w, inp, layer)
+    assert cuda_lib.gptb_device_error() == 0
+    lw = oracle_layer(w, layer)
+    f8 = fp8_mode(c)
+    idx = inp["idx"].numpy()
+    y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), idx, layer, fp8=f8)
+    rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), idx, layer, fp8=f8)
+    errs = {"x_out": relerr(np64(x_out), y), "dx": relerr(np64(dx), rdx), "dx0": relerr(np64(dx0), rdx0)}
+    for k in ("w_qkv", "w_o", "w_fc", "w_proj", "w_ve_gate", "ve_table"):
+        if k in rg:
+            errs[k] = relerr(np64(g[k]), rg[k])
+    lam = np64(g["lambdas"])
+    errs["resid_lambda"] = scalar_err(lam[0], rg["resid_lambda"], rg["_scale"]["resid_lambda"])
+    errs["x0_lambda"] = scalar_err(lam[1], rg["x0_lambda"], rg["_scale"]["x0_lambda"])
+    assert ("ve_table" in errs) == bool(c["has_ve"][layer])
+    tol = TOL[c["dtype"]]
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("name,layer,rows", [("d24", 23, (0, 15)), ("d20_gqa", 0, (7,)), ("d12", 11, (3,))])
+def test_block_bench_shape_sampled_rows(cuda_lib, name, layer, rows):
+    c = synth.config(name)
+    w = synth.make_weights(c, seed=101)
+    inp = synth.make_block_inputs(c, seed=102)
+    x_out, dx, dx0, _ = _run_block(c, w, inp, layer)
     assert cuda_lib.gptb_device_error() == 0
     olw = oracle_layer(w, layer)
-    f8 = False
     tol = TOL[c["dtype"]]
     for b in rows:
         c1 = dict(c, B=1)
         sl = slice(b, b + 1)
-        y, cache = om.block_forward(c1, olw, np64(inp["x"][sl]), np64(inp["x0"][sl]), inp["idx"][sl].numpy(), layer,
-                                    fp8=f8)
-        rdx, rdx0, _ = om.block_backward(c1, olw, cache, np64(inp["dy"][sl]), inp["idx"][sl].numpy(), layer, fp8=f8)
+        y, cache = om.block_forward(c1, olw, np64(inp["x"][sl]), np64(inp["x0"][sl]), inp["idx"][sl].numpy(), layer)
+        rdx, rdx0, _ = om.block_backward(c1, olw, cache, np64(inp["dy"][sl]), inp["idx"][sl].numpy(), layer)
         errs = {"x_out": relerr(np64(x_out[sl]), y), "dx": relerr(np64(dx[sl]), rdx),
                 "dx0": relerr(np64(dx0[sl]), rdx0)}
         assert all(v <= tol for v in errs.values()), (b, errs)

@@ -70,3 +70,41 @@ def test_polar_express_single_step_singular_values(cuda_lib):
     want = np.sort(np.abs(a * s + b * s ** 3 + c * s ** 5))[::-1]
     got = np.linalg.svd(out.double().cpu().numpy(), compute_uv=False)
     assert np.max(np.abs(got - want)) / want.max() <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("shape", [(256, 128), (128, 384), (768, 768)])
+def test_muon_step_matches_oracle(cuda_lib, shape):
+    """Two Muon steps (momentum, the five Polar Express tuples, NorMuon, decay)
+    against oracle.optim.muon_step: the weight update, the momentum buffer and
+    the second moment (bf16 orthogonalisation: 2e-2; fp32 momentum: 1e-5)."""
+    gb = cuda_lib
+    m, n = shape
+    rng = np.random.default_rng(m + n)
+    w0 = rng.standard_normal((m, n)).astype(np.float32) * 0.02
+    hp = dict(lr=0.02, mu=0.95, beta2=0.95, weight_decay=0.1)
+    w = torch.tensor(w0, device="cuda")
+    buf = torch.zeros(m, n, device="cuda")
+    v = torch.zeros(m, device="cuda")
+    wb = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(gb.gptb_muon_workspace_bytes(m, n, 5), dtype=torch.uint8, device="cuda")
+    rw, rbuf, rv = w0.astype(np.float64), np.zeros((m, n)), np.zeros(m)
+    for _ in range(2):
+        g = rng.standard_normal((m, n)).astype(np.float32)
+        gb.gptb_muon_step(w, wb, torch.tensor(g, device="cuda"), buf, v, m, n, oo.POLAR_EXPRESS_COEFFS, hp["lr"],
+                          hp["mu"], hp["beta2"], hp["weight_decay"], ws)
+        rw, rbuf, rv = oo.muon_step(rw, g, rbuf, rv, hp["lr"], hp["mu"], hp["beta2"], hp["weight_decay"])
+    torch.cuda.synchronize()
+    assert gb.gptb_device_error() == 0
+    got = w.double().cpu().numpy()
+    assert relerr(got - w0, rw - w0) <= TOL["bf16"]
+    assert relerr(buf.double().cpu().numpy(), rbuf) <= TOL["f32"]
+    assert relerr(v.double().cpu().numpy(), rv) <= TOL["bf16"]
+    assert torch.equal(wb, w.bfloat16())
+
+
+def test_muon_step_rejects_bad_shapes(cuda_lib):
+    gb = cuda_lib
+    t = torch.zeros(64, device="cuda")
+    with pytest.raises(gb.GPTBError) as e:
+        gb.gptb_muon_step(t, None, t, t, t, 12, 8, oo.POLAR_EXPRESS_COEFFS, 0.1, 0.9, 0.9, 0.0, t)
+    assert e.value.code == gb.ERR_INVALID_ARG

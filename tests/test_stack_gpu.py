@@ -6,16 +6,20 @@ import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, np64, oracle_weights, relerr, scalar_err, small_bf16
+from helpers import TOL, fp8_mode, np64, oracle_weights, relerr, scalar_err, small_bf16
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_lm_head_xent(cuda_lib, dtype):
+@pytest.mark.parametrize("dtype,N,V", [("bf16", 300, 1024), ("f32", 300, 1024), ("bf16", 300, 1000),
+                                       ("bf16", 9192, 32768)])
+def test_lm_head_xent(cuda_lib, dtype, N, V):
+    """N=9192 at the vocabulary of every stack config: two row chunks (8192 +
+    a ragged 1000), dW_lm accumulated across them; V=1000 leaves the last
+    256-column tile of the logits GEMM partly outside the vocabulary."""
     from gpt_transformer_block_b200.model import lm_head
     g = torch.Generator().manual_seed(3)
-    N, d, V = 300, 256, 1024
+    d = 256
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     h = torch.randn(N, d, generator=g).to(tdt)
     w = (torch.randn(V, d, generator=g) * 0.05).to(tdt)
@@ -25,6 +29,7 @@ def test_lm_head_xent(cuda_lib, dtype):
     dw = torch.zeros(V, d, dtype=torch.float32, device="cuda")
     loss = lm_head(c, h.cuda(), w.cuda(), y.cuda(), dh, dw)
     torch.cuda.synchronize()
+    assert cuda_lib.gptb_device_error() == 0
     rl, rdh, rdw = om.lm_head_xent(np64(h), np64(w), y.numpy())
     tol = TOL[dtype]
     assert abs(loss.item() - rl) / abs(rl) <= tol
@@ -44,7 +49,7 @@ def run_stack(gb, c, w, batch):
 def compare_stack(c, w, batch, loss, g, layers=None, top=("wte", "w_lm", "w_smear_gate", "smear_lambda",
                                                           "backout_lambda")):
     ow = oracle_weights(w)
-    f8 = c["dtype"] == "fp8"
+    f8 = fp8_mode(c)
     rl, cache = om.stack_forward(c, ow, batch["idx"].numpy(), batch["targets"].numpy(), fp8=f8)
     rg = om.stack_backward(c, ow, cache, batch["idx"].numpy(), fp8=f8)
     tol = TOL[c["dtype"]]
@@ -115,15 +120,70 @@ def test_grad_accumulation_equals_sum(cuda_lib):
 
 
 def test_stack_fp8_small(cuda_lib):
-    """FP8 end to end: loss, lm_head and backout gradients and the top layer.
-    Below the top layer every input-gradient GEMM re-quantises a gradient that
-    already differs from the oracle's, so e4m3 code flips (one ulp = 12.5 %)
-    compound layer by layer; the deeper layers are checked with the same
-    tolerance by the teacher-forced block tests (test_block_fp8), and the
-    embedding / smear kernels below layer 0 are the same kernels as in bf16,
-    checked by the bf16 stack tests."""
+    """FP8 end to end (every GEMM product of every block in e4m3): the loss and
+    every gradient of every layer, the embedding and the smear / backout terms."""
     c = small_bf16(dtype="fp8")
     w = synth.make_weights(c, seed=51)
     b = synth.make_batch(c, seed=52)
     loss, g = run_stack(cuda_lib, c, w, b)
-    compare_stack(c, w, b, loss, g, layers=(c["n_layer"] - 1,), top=("w_lm", "backout_lambda"))
+    compare_stack(c, w, b, loss, g)
+
+
+def test_stack_fp8_variant_small(cuda_lib):
+    """The FP8 variant end to end: e5m2 gradient operands in every block's
+    backward GEMMs and the lm_head in FP8 (e4m3 logits, FP8 logits gradient
+    with its fixed scale): the loss and every gradient of every layer."""
+    c = small_bf16(dtype="fp8", fp8_grad="e5m2", fp8_lm_head=True)
+    w = synth.make_weights(c, seed=53)
+    b = synth.make_batch(c, seed=54)
+    loss, g = run_stack(cuda_lib, c, w, b)
+    compare_stack(c, w, b, loss, g)
+
+
+@pytest.mark.parametrize("grad", ["e4m3", "e5m2"])
+def test_lm_head_fp8(cuda_lib, grad):
+    """FP8 lm_head at the stack configs' vocabulary over two row chunks (8192 +
+    a ragged 1000): e4m3 hf and W_lm, the logits gradient with the fixed scale
+    of its 1/N bound in e4m3 or e5m2; against the oracle's FP8 lm_head."""
+    from gpt_transformer_block_b200.model import lm_head
+    g = torch.Generator().manual_seed(13)
+    N, d, V = 9192, 256, 32768
+    h = torch.randn(N, d, generator=g).to(torch.bfloat16)
+    w = (torch.randn(V, d, generator=g) * 0.05).to(torch.bfloat16)
+    y = torch.randint(0, V, (N,), generator=g, dtype=torch.int32)
+    c = small_bf16(B=1, T=N, vocab=V, dtype="fp8", fp8_grad=grad, fp8_lm_head=True)
+    dh = torch.empty(N, d, dtype=torch.bfloat16, device="cuda")
+    dw = torch.zeros(V, d, dtype=torch.float32, device="cuda")
+    loss = lm_head(c, h.cuda(), w.cuda(), y.cuda(), dh, dw)
+    torch.cuda.synchronize()
+    assert cuda_lib.gptb_device_error() == 0
+    rl, rdh, rdw = om.lm_head_xent(np64(h), np64(w), y.numpy(), fp8=fp8_mode(c))
+    tol = TOL["fp8"]
+    assert abs(loss.item() - rl) / abs(rl) <= tol
+    assert relerr(np64(dh), rdh) <= tol
+    assert relerr(np64(dw), rdw) <= tol
+
+
+def test_lm_head_out_of_range_targets_are_reported(cuda_lib):
+    """Targets -1 and V are never used as indices: the call completes, the
+    device error check reports GPTB_ERR_BAD_INPUT, and the other rows' loss
+    terms are unchanged (the bad rows add 0 to the mean)."""
+    from gpt_transformer_block_b200.model import lm_head
+    g = torch.Generator().manual_seed(9)
+    N, d, V = 64, 256, 1024
+    for dtype in ("bf16", "f32"):
+        tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        h = torch.randn(N, d, generator=g).to(tdt)
+        w = (torch.randn(V, d, generator=g) * 0.05).to(tdt)
+        y = torch.randint(0, V, (N,), generator=g, dtype=torch.int32)
+        y[5], y[40] = -1, V
+        c = small_bf16(B=1, T=N, vocab=V, dtype=dtype, head_dim=128 if dtype == "bf16" else 64)
+        dh = torch.empty(N, d, dtype=tdt, device="cuda")
+        dw = torch.zeros(V, d, dtype=torch.float32, device="cuda")
+        loss = lm_head(c, h.cuda(), w.cuda(), y.cuda(), dh, dw)
+        assert cuda_lib.gptb_device_error() == cuda_lib.ERR_BAD_INPUT
+        assert cuda_lib.gptb_device_error() == 0  # the error word was cleared
+        keep = np.ones(N, dtype=bool)
+        keep[[5, 40]] = False
+        rl, _, _ = om.lm_head_xent(np64(h)[keep], np64(w), y.numpy()[keep])
+        assert abs(loss.item() - rl * keep.sum() / N) <= TOL[dtype] * abs(rl)
