@@ -25,8 +25,11 @@ EXPORTS = [
     "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
     "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
     "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express", "gptb_decode_attention",
-    "gptb_muon_workspace_bytes", "gptb_muon_step",
+    "gptb_muon_workspace_bytes", "gptb_muon_step", "gpt_stack_step_hooked", "gptb_cast_f32_bf16",
+    "gptb_cast_bf16_f32",
 ]
+
+GRADS_READY_FN = ctypes.CFUNCTYPE(None, ctypes.c_int, ctypes.c_void_p)
 
 _vp = ctypes.c_void_p
 _fp = ctypes.POINTER(ctypes.c_float)
@@ -105,6 +108,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        ctypes.c_size_t, _vp]
     lib.gptb_decode_attention.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, _vp]
+    lib.gpt_stack_step_hooked.argtypes = [P(Config), P(ModelWeights), _vp, _vp, _vp, P(ModelGrads), _vp, _vp,
+                                          GRADS_READY_FN, _vp]
+    lib.gptb_cast_f32_bf16.argtypes = [_vp, _vp, ctypes.c_longlong, ctypes.c_float, _vp]
+    lib.gptb_cast_bf16_f32.argtypes = [_vp, _vp, ctypes.c_longlong, ctypes.c_float, _vp]
     lib.gptb_muon_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.gptb_muon_workspace_bytes.restype = ctypes.c_size_t
     lib.gptb_muon_step.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _fp, ctypes.c_int,
@@ -228,6 +235,32 @@ def lm_head_xent_noalloc(cfg, h, w_lm, targets, loss_out, dh, dw_lm, stream=None
 def gpt_stack_step(cfg, w: ModelWeights, idx, targets, loss_out, g: ModelGrads, ws, stream=None):
     _check(load().gpt_stack_step(ctypes.byref(cfg), ctypes.byref(w), ptr(idx), ptr(targets), ptr(loss_out),
                                  ctypes.byref(g), ptr(ws), _stream(stream)), "gpt_stack_step")
+
+
+def gpt_stack_step_hooked(cfg, w: ModelWeights, idx, targets, loss_out, g: ModelGrads, ws, ready, stream=None):
+    """gpt_stack_step with ready(layer) called on this thread as each layer's
+    gradients are enqueued (L-1 .. 0, then -1 for the embedding / lm_head ones)."""
+    err = []
+
+    def _cb(layer, _user):
+        try:
+            ready(int(layer))
+        except BaseException as e:  # exceptions cannot cross the C frame: re-raised below
+            err.append(e)
+    cb = GRADS_READY_FN(_cb)
+    rc = load().gpt_stack_step_hooked(ctypes.byref(cfg), ctypes.byref(w), ptr(idx), ptr(targets), ptr(loss_out),
+                                      ctypes.byref(g), ptr(ws), _stream(stream), cb, None)
+    if err:
+        raise err[0]
+    _check(rc, "gpt_stack_step_hooked")
+
+
+def gptb_cast_f32_bf16(x, y, n, scale=1.0, stream=None):
+    _check(load().gptb_cast_f32_bf16(ptr(x), ptr(y), int(n), float(scale), _stream(stream)), "gptb_cast_f32_bf16")
+
+
+def gptb_cast_bf16_f32(x, y, n, scale=1.0, stream=None):
+    _check(load().gptb_cast_bf16_f32(ptr(x), ptr(y), int(n), float(scale), _stream(stream)), "gptb_cast_bf16_f32")
 
 
 def gptb_gemm_bf16(A, a_mn, lda, B, b_mn, ldb, C, c_f32, ldc, M, N, K, stream=None):

@@ -900,7 +900,8 @@ int lm_head_impl(const gptb_config& c, const T* h, const T* w_lm, const int32_t*
 // --------------------------------------------------------------- stack ----
 template <class T>
 int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t* idx, const int32_t* targets,
-               float* loss_out, const gptb_model_grads& g, const StackWs& S, cudaStream_t st) {
+               float* loss_out, const gptb_model_grads& g, const StackWs& S, cudaStream_t st,
+               gptb_grads_ready_fn ready = nullptr, void* user = nullptr) {
   const Dims m = dims_of(c);
   const int brt = br_threads(m.d);
   const int brg = br_grid(m.N, brt);
@@ -933,12 +934,14 @@ int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t*
     const T* extra = (i == c.backout_layer) ? (const T*)S.dx_bo : nullptr;
     TRY(block_bwd_impl<T>(c, i, w.layers[i], (const T*)S.x_in[i], x0, idx, S.saved[i], cur, extra, nxt, S.dx0,
                           g.layers[i], S.scr, st));
+    if (ready) ready(i, user);  // layer i's weight gradients are complete once this point of the stream is
     std::swap(cur, nxt);
   }
   br_smear_embed_bwd_kernel<T><<<brg, brt, 0, st>>>(cur, S.dx0, idx, (const T*)w.wte, (const T*)w.w_smear_gate,
                                                        w.smear_lambda, g.wte, g.w_smear_gate, g.smear_lambda, m.B, m.T,
                                                        m.d, c.smear_ch);
   CKL();
+  if (ready) ready(-1, user);  // the embedding, lm_head, smear and backout gradients
   return GPTB_OK;
 }
 
@@ -1041,6 +1044,19 @@ int gpt_stack_step(const gptb_config* cfg, const gptb_model_weights* w, const in
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cfg->dtype == GPTB_F32) return stack_impl<float>(*cfg, *w, idx, targets, loss_out, *g, S, st);
   return stack_impl<bf16>(*cfg, *w, idx, targets, loss_out, *g, S, st);
+}
+
+int gpt_stack_step_hooked(const gptb_config* cfg, const gptb_model_weights* w, const int32_t* idx,
+                          const int32_t* targets, float* loss_out, gptb_model_grads* g, void* ws, gptb_stream_t stream,
+                          gptb_grads_ready_fn ready, void* user) {
+  TRY(check_config(cfg));
+  if (!w || !idx || !targets || !loss_out || !g || !ws || !ready) return GPTB_ERR_INVALID_ARG;
+  const Dims m = dims_of(*cfg);
+  Carve cv(ws);
+  const StackWs S = carve_stack(cv, m);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == GPTB_F32) return stack_impl<float>(*cfg, *w, idx, targets, loss_out, *g, S, st, ready, user);
+  return stack_impl<bf16>(*cfg, *w, idx, targets, loss_out, *g, S, st, ready, user);
 }
 
 int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, void* C, int c_f32,
@@ -1213,6 +1229,25 @@ int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cach
   decode_attn_kernel<<<B * Hkv, DEC_THREADS, smem, st>>>(
       static_cast<const bf16*>(q), static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache), lens,
       static_cast<bf16*>(o), lse, H, Hkv, T_max, window);
+  CKL();
+  return GPTB_OK;
+}
+
+int gptb_cast_f32_bf16(const float* x, void* y, long long n, float scale, gptb_stream_t stream) {
+  if (!x || !y || n < 0) return GPTB_ERR_INVALID_ARG;
+  if (n == 0) return GPTB_OK;
+  const int grid = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, dev_info().sms * 8LL));
+  cast_f32_bf16_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, static_cast<bf16*>(y), n, scale);
+  CKL();
+  return GPTB_OK;
+}
+
+int gptb_cast_bf16_f32(const void* x, float* y, long long n, float scale, gptb_stream_t stream) {
+  if (!x || !y || n < 0) return GPTB_ERR_INVALID_ARG;
+  if (n == 0) return GPTB_OK;
+  const int grid = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, dev_info().sms * 8LL));
+  cast_bf16_f32_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<const bf16*>(x), y, n,
+                                                                                  scale);
   CKL();
   return GPTB_OK;
 }

@@ -520,6 +520,17 @@ __global__ void muon_apply_kernel(float* __restrict__ w, bf16* __restrict__ wb, 
   }
 }
 
+// y = bf16(x * scale) and x = float(y) * scale over n elements: gradient
+// buckets travel between ranks in bf16 (half the bytes of the fp32 gradients)
+__global__ void cast_f32_bf16_kernel(const float* __restrict__ x, bf16* __restrict__ y, long long n, float scale) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    y[i] = __float2bfloat16_rn(x[i] * scale);
+}
+__global__ void cast_bf16_f32_kernel(const bf16* __restrict__ x, float* __restrict__ y, long long n, float scale) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    y[i] = __bfloat162float(x[i]) * scale;
+}
+
 // loss = mean of the row losses (single CTA, fixed order)
 __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ x, long long n, float* __restrict__ out) {
   __shared__ float sred[32];

@@ -214,6 +214,23 @@ int lm_head_xent_noalloc(const gptb_config* cfg, const void* h, const void* w_lm
 int gpt_stack_step(const gptb_config* cfg, const gptb_model_weights* w, const int32_t* idx, const int32_t* targets,
                    float* loss_out, gptb_model_grads* g, void* ws, gptb_stream_t stream);
 
+/* gpt_stack_step for data-parallel training: identical work, plus a host
+ * callback ready(layer, user) made on the calling thread while the step is
+ * being enqueued, right after the last kernel that writes block `layer`'s
+ * weight gradients has been put on `stream` (layers in backward order,
+ * L-1 down to 0), and once more with layer = -1 after the embedding / smear /
+ * backout / lm_head gradients.  Work the callback enqueues on `stream`, or on
+ * another stream after an event recorded on `stream`, runs once those
+ * gradients are complete: the caller launches that layer's gradient
+ * reduction there, overlapping the rest of the backward (the ZeRO-2 phase 1
+ * of the page's "Entraînement distribué" section, bucketed per layer).  The
+ * callback must not call back into this library.  No counterpart on the
+ * pages beyond that section. */
+typedef void (*gptb_grads_ready_fn)(int layer, void* user);
+int gpt_stack_step_hooked(const gptb_config* cfg, const gptb_model_weights* w, const int32_t* idx,
+                          const int32_t* targets, float* loss_out, gptb_model_grads* g, void* ws, gptb_stream_t stream,
+                          gptb_grads_ready_fn ready, void* user);
+
 /* Plain GEMM entry point used by the tests of the tensor-core kernel:
  * C[M,N] (+)= A[M,K] B[N,K]^T (bf16 operands, fp32 accumulate).
  *   a_mn / b_mn: 0 = operand stored K-major (row-major [M,K] / [N,K]),
@@ -307,6 +324,13 @@ int gptb_muon_step(float* w, void* w_bf16, const float* g, float* buf, float* v,
  * long for the per-CTA score buffer: (H/H_kv) * (T_max + 128) floats <= 220 KB). */
 int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, void* o,
                           float* lse, int B, int H, int Hkv, int T_max, int window, gptb_stream_t stream);
+
+/* Element casts for data-parallel gradient buckets (bf16 on the wire):
+ * y[i] = bf16(x[i] * scale) and y[i] = float(x[i]) * scale, n elements,
+ * device pointers, round to nearest-even.  GPTB_ERR_INVALID_ARG for null
+ * pointers or n < 0. */
+int gptb_cast_f32_bf16(const float* x, void* y, long long n, float scale, gptb_stream_t stream);
+int gptb_cast_bf16_f32(const void* x, float* y, long long n, float scale, gptb_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word.
  * Returns GPTB_OK, GPTB_ERR_TIMEOUT if a bounded wait inside a kernel expired

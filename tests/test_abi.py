@@ -24,6 +24,7 @@ def gb():
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "gptblock.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"^\s*typedef[^;]*;", "", text, flags=re.M)  # callback types are not functions
     names = re.findall(r"^\s*(?:const\s+)?(?:long\s+long|unsigned\s+long\s+long|[A-Za-z_]\w*)\s*\*?\s*"
                        r"([A-Za-z_]\w*)\s*\(", text, flags=re.M)
     return sorted(set(n for n in names if n not in ("if", "while")))
@@ -44,7 +45,7 @@ def test_library_exports_every_declared_symbol(gb):
 
 def test_error_strings(gb):
     lib = gb.load()
-    for code in (0, -1, -2, -3, -4, -5):
+    for code in (0, -1, -2, -3, -4, -5, -6):
         assert lib.gptb_error_string(code)
 
 
