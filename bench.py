@@ -161,6 +161,18 @@ def profile_traffic(workload: str) -> float | None:
 
 # -------------------------------------------------------------- oracle arm -
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), for the CPU baseline."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def oracle_sample(c: dict, seed: int = 7) -> dict:
     """Time the fp64 oracle on one block slice (B=1, full T) forward+backward
     plus the lm_head on 512 tokens, and extrapolate to one full step."""
@@ -192,29 +204,39 @@ def oracle_sample(c: dict, seed: int = 7) -> dict:
     om.lm_head_xent(h, wl, y)
     t_lm = (time.perf_counter() - t0) * (cs["T"] / n_lm)
     t_step_row = cs["n_layer"] * t_block + t_lm   # one batch row of T tokens
-    return {"tok_per_s": cs["T"] / t_step_row, "cores": cores, "t_block_s": t_block, "t_lm_s": t_lm,
+    return {"tok_per_s": cs["T"] / t_step_row, "cores": cores, "cpu": cpu_model(), "t_block_s": t_block, "t_lm_s": t_lm,
             "sample": f"one block fwd+bwd at B=1,T={cs['T']},d={cs['d']} (layer {layer}) x {cs['n_layer']} layers "
                       f"+ lm_head fwd+bwd on {n_lm} tokens scaled to {cs['T']}; fp64 numpy"}
 
 
 def run_optimizer(args, c: dict):
     """The optimizer step after the training step, on the workload's parameters:
-    the Polar Express orthogonalisation (the two coefficient tuples the pages
-    print) of every block projection matrix (4 per layer; the tiny VE / smear
-    gate matrices are left out) and AdamW over the embedding, lm_head and VE
-    tables (fp32 masters with the bf16 copy written).  Inputs resident in HBM;
-    one JSON line, time-like metric (lower is better)."""
+    a whole Muon step (Nesterov momentum, the Polar Express orthogonalisation
+    with its five coefficient tuples, NorMuon scaling, decoupled decay, the bf16
+    working copy written) for every block projection matrix (4 per layer) and
+    AdamW over the embedding, lm_head and VE tables (fp32 masters with the bf16
+    copy written).  Inputs resident in HBM; one JSON line, time-like metric
+    (lower is better)."""
     import gpt_transformer_block_b200 as gb
     gb.load()
-    coeffs = [(8.156, -22.483, 15.879), (4.043, -2.809, 0.500)]
+    # the five Polar Express tuples (the pages print the first two; the Polar
+    # Express paper, Amsel et al. 2025, gives all five)
+    coeffs = [(8.156554524902461, -22.48329292557795, 15.878769915207462),
+              (4.042929935166739, -2.808917465908714, 0.5000178451051316),
+              (3.8916678022926607, -2.772484153217685, 0.5060648178503393),
+              (3.285753657755655, -2.3681294933425376, 0.46449024233003106),
+              (2.3465413258596377, -1.7097828382687081, 0.42323551169305323)]
     d, F, L = c["d"], c["mlp_hidden"], c["n_layer"]
     qkv = (c["n_head"] + 2 * c["n_kv_head"]) * c["head_dim"]
     ho = c["n_head"] * c["head_dim"]
     shapes = [(qkv, d), (d, ho), (F, d), (d, F)] * L
     g = torch.Generator(device="cuda").manual_seed(5)
-    mats = [torch.randn(m, n, device="cuda", generator=g).mul_(0.02).bfloat16() for m, n in shapes]
-    outs = [torch.empty_like(x) for x in mats]
-    ws = torch.empty(max(gb.gptb_polar_express_workspace_bytes(m, n, len(coeffs)) for m, n in shapes),
+    mats = []
+    for m, n in shapes:
+        w = torch.randn(m, n, device="cuda", generator=g).mul_(0.02)
+        mats.append(dict(w=w, wb=w.bfloat16(), g=torch.randn(m, n, device="cuda", generator=g),
+                         buf=torch.zeros(m, n, device="cuda"), v=torch.zeros(m, device="cuda"), m=m, n=n))
+    ws = torch.empty(max(gb.gptb_muon_workspace_bytes(m, n, len(coeffs)) for m, n in shapes),
                      dtype=torch.uint8, device="cuda")
     n_adam = c["vocab"] * d * 2 + sum(c["has_ve"]) * c["vocab"] * c["n_kv_head"] * c["head_dim"]
     p = torch.randn(n_adam, device="cuda", generator=g)
@@ -222,49 +244,53 @@ def run_optimizer(args, c: dict):
     m1, m2 = torch.zeros_like(p), torch.zeros_like(p)
     pb = torch.empty(n_adam, dtype=torch.bfloat16, device="cuda")
 
-    def pe_all():
-        for x, o in zip(mats, outs):
-            gb.gptb_polar_express(x, o, x.shape[0], x.shape[1], coeffs, ws)
+    def muon_all():
+        for x in mats:
+            gb.gptb_muon_step(x["w"], x["wb"], x["g"], x["buf"], x["v"], x["m"], x["n"], coeffs, 0.02, 0.95, 0.95,
+                              0.0, ws)
 
     def adam(t):
         gb.gptb_adamw_step(p, gr, m1, m2, pb, n_adam, 1e-3, 0.8, 0.95, 1e-10, 0.0, t)
 
     for t in range(1, args.warmup + 1):
-        pe_all()
+        muon_all()
         adam(t)
     torch.cuda.synchronize()
     if gb.gptb_device_error() != 0:
         raise RuntimeError("device error during warm-up")
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    t_pe = t_ad = 0.0
+    t_mu = t_ad = 0.0
     for k in range(args.steps):
         ev[0].record()
-        pe_all()
+        muon_all()
         ev[1].record()
         adam(args.warmup + 1 + k)
         ev[2].record()
         torch.cuda.synchronize()
-        t_pe += ev[0].elapsed_time(ev[1])
+        t_mu += ev[0].elapsed_time(ev[1])
         t_ad += ev[1].elapsed_time(ev[2])
-    t_pe /= args.steps
+    t_mu /= args.steps
     t_ad /= args.steps
     flops = 0.0
     for m, n in shapes:
-        s, lg = min(m, n), max(m, n)
-        flops += len(coeffs) * (4.0 * s * s * lg + 2.0 * s ** 3)
+        s_, lg = min(m, n), max(m, n)
+        flops += len(coeffs) * (4.0 * s_ * s_ * lg + 2.0 * s_ ** 3)
+    # Muon's elementwise passes: momentum (read g, buf; write buf, u bf16), the
+    # Polar Express input scaling (read u twice, write X), NorMuon (read o
+    # twice), the update (read w; write w, the bf16 copy)
+    muon_bytes = sum(m * n * (8 + 4 + 2 + 2 * 2 + 2 + 2 * 2 + 4 + 4 + 2) for m, n in shapes)
     adam_bytes = n_adam * (16 + 12 + 2)  # read p g m v, write p m v, write the bf16 copy
     peaks = measured_peaks()
-    tf = flops / (t_pe * 1e-3) / 1e12
+    tf = flops / (t_mu * 1e-3) / 1e12
     gbs = adam_bytes / (t_ad * 1e-3) / 1e9
-    line = {"metric": "optimizer step time (Polar Express on the block matrices + AdamW on embeddings, lm_head, "
-                      "VE tables)",
-            "value": t_pe + t_ad, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-            "higher_is_better": False, "dtype": "bf16 GEMMs / f32 AdamW", "data": "synthetic",
+    line = {"metric": "optimizer step time (Muon on the block matrices + AdamW on embeddings, lm_head, VE tables)",
+            "value": t_mu + t_ad, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": False, "dtype": "bf16 GEMMs / f32 elementwise", "data": "synthetic",
             "config": {"workload": c["name"] + "_optimizer", "matrices": len(shapes), "ns_steps": len(coeffs),
                        "adamw_params": n_adam},
-            "polar_express": {"ms": t_pe, "flops": flops, "achieved": tf, "unit": "TFLOP/s",
-                              "peak": peaks["bf16_tflops"], "frac": tf / peaks["bf16_tflops"],
-                              "peak_source": "measured bf16 burst"},
+            "muon": {"ms": t_mu, "polar_express_flops": flops, "achieved": tf, "unit": "TFLOP/s",
+                     "peak": peaks["bf16_tflops"], "frac": tf / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks['source']} bf16 burst", "elementwise_bytes": muon_bytes},
             "adamw": {"ms": t_ad, "bytes": adam_bytes, "achieved": gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                       "frac": gbs / peaks["hbm_gbs"]}}
     print(json.dumps(line))
@@ -332,7 +358,7 @@ def run_reference(args, c: dict, fl: dict):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": step_config(c, 1),
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": info["cores"], "cpu": info["cpu"], "kind": "oracle",
                          "sample": info["sample"]},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "mfu_algorithmic": None, "flops_per_token": fl,
@@ -356,7 +382,7 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling only)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
     ap.add_argument("--optimizer", action="store_true",
-                    help="time the optimizer step (Polar Express + AdamW) instead of the training step")
+                    help="time the optimizer step (Muon + AdamW) instead of the training step")
     ap.add_argument("--decode", action="store_true",
                     help="time one decode step of attention over a full KV cache instead of the training step")
     args = ap.parse_args()
@@ -489,6 +515,8 @@ def main():
                      "frac": (gemm_tflops / peak_t) if gemm_tflops else None,
                      "peak_source": peak_src,
                      "traffic": profile_traffic(c["name"]),
+                     "traffic_source": "committed ncu summary profiles/gemm_tc_<workload>_traffic.md (not "
+                                       "measured in this run; null when absent)",
                      "share_of_step": gemm_ms / ms if ms > 0 else None, "launches": gemm_n},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": 2 * tokens_per_step * 4,
                 "d2h_bytes_per_step": 4},
@@ -499,7 +527,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         info = oracle_sample(c)
         line["cpu_baseline"] = {"value": info["tok_per_s"], "unit": "tokens/s", "cores": info["cores"],
-                                "kind": "oracle", "sample": info["sample"]}
+                                "cpu": info["cpu"], "kind": "oracle", "sample": info["sample"]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del model
