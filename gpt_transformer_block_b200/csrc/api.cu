@@ -299,7 +299,6 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
         (ep.ldo % (acc32 ? 4 : 8)) || (N % 8))
       return GPTB_ERR_INVALID_ARG;
     if (has_aux && (!aligned16(ep.aux) || ep.ld_aux % 8)) return GPTB_ERR_INVALID_ARG;
-    if (ep.kind == EPI_RELU2 && (!aligned16(ep.out2) || ep.ldo2 % 8)) return GPTB_ERR_INVALID_ARG;
     const bool pair = M >= GPTB_PAIR_MIN_M;
     const int b_rows = pair ? TcShape<true>::B_ROWS : TcShape<false>::B_ROWS;  // rows of B one CTA stages
     CUtensorMap ta, tb, to, to2, tx;
@@ -310,7 +309,6 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
                       : make_tmap(&to, ep.out, false, N, M, ep.ldo, 64, 32));
     to2 = to;
     tx = to;
-    if (ok && ep.kind == EPI_RELU2) ok = make_tmap(&to2, ep.out2, false, N, M, ep.ldo2, 64, 32);
     if (ok && has_aux) ok = make_tmap(&tx, ep.aux, false, N, M, ep.ld_aux, 64, 32);
     if (!ok) return GPTB_ERR_CUDA;
     int splits = 1;
@@ -425,7 +423,7 @@ Dims dims_of(const gptb_config& c) {
 }
 
 struct Saved {
-  void *h, *qkv, *o, *h2, *u, *act;
+  void *h, *qkv, *o, *h2, *act;
   float *rstd1, *sg, *rstd_qk, *lse, *rstd2;
   // FP8 only: e4m3 copies of the four weights (reused by the input-gradient
   // GEMMs) and of the four GEMM activations (reused by the weight-gradient
@@ -446,7 +444,6 @@ Saved carve_saved(Carve& cv, const Dims& m) {
   s.lse = (float*)cv.take((size_t)m.B * m.H * m.T * 4);
   s.h2 = cv.take(m.N * m.d * e);
   s.rstd2 = (float*)cv.take(m.N * 4);
-  s.u = cv.take(m.N * m.F * e);
   s.act = cv.take(m.N * m.F * e);
   s.wqkv8 = s.wo8 = s.wfc8 = s.wproj8 = nullptr;
   s.h8 = s.o8 = s.h2_8 = s.act8 = nullptr;
@@ -721,7 +718,7 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   CKL();
   TRY(proj<T>(c, {S.h2, m.d, false, m.N * m.d, S.h2_8, S.amax + 2, true},
               {w.w_fc, m.d, false, (long long)m.F * m.d, S.wfc8, S.amax + 6, true}, (int)m.N, m.F, m.d,
-              epi(EPI_RELU2, c.dtype, S.u, m.F, nullptr, 0, S.act, m.F), st));
+              epi(EPI_RELU2, c.dtype, S.act, m.F), st));
   TRY(proj<T>(c, {S.act, m.F, false, m.N * m.F, S.act8, S.amax + 3, true},
               {w.w_proj, m.F, false, (long long)m.d * m.F, S.wproj8, S.amax + 7, true}, (int)m.N, m.d, m.F,
               epi(EPI_RESID, c.dtype, x_out, m.d, X.x1, m.d), st));
@@ -750,7 +747,7 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   TRY(proj<T>(c, {dx2, m.d, true, Nd, X.g8, X.gamax, true, m.grad_e5m2}, {S.act, m.F, true, 0, S.act8, S.amax + 3, false}, m.d,
               m.F, N, epi(EPI_ACCUM_F32, dt, g.w_proj, m.F), st));
   TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false},
-              N, m.F, m.d, epi(EPI_DRELU2, dt, X.du, m.F, S.u, m.F), st));
+              N, m.F, m.d, epi(EPI_DRELU2, dt, X.du, m.F, S.act, m.F), st));
   TRY(proj<T>(c, {X.du, m.F, true, m.N * m.F, X.g8, X.gamax, true, m.grad_e5m2}, {S.h2, m.d, true, 0, S.h2_8, S.amax + 2, false},
               m.F, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
   TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false},

@@ -33,8 +33,10 @@ namespace gptb {
 enum EpiKind : int {
   EPI_STORE = 0,      // out = alpha*acc
   EPI_RESID = 1,      // out = beta*aux + alpha*acc           (residual add)
-  EPI_RELU2 = 2,      // out = u = alpha*acc, out2 = relu(u)^2 (MLP activation)
-  EPI_DRELU2 = 3,     // out = alpha*acc * 2*relu(aux)         (aux = saved u)
+  EPI_RELU2 = 2,      // out = relu(alpha*acc)^2              (MLP activation)
+  EPI_DRELU2 = 3,     // out = alpha*acc * 2*sqrt(aux)          (aux = saved relu(u)^2:
+                      //   d relu(u)^2 / du = 2 relu(u) = 2 sqrt(relu(u)^2), so u
+                      //   itself need not be kept)
   EPI_ACCUM_F32 = 4,  // out(f32) += alpha*acc, atomic          (weight grads)
   EPI_QKV = 5,        // q,k heads: rope(rmsnorm(acc)) + saved rstd; v heads:
                       // acc + 3*sigmoid(z) * VE[idx] (value-embedding layers)
@@ -101,20 +103,18 @@ __device__ __forceinline__ void epi_store8_t(const EpiParams& ep, long long r, i
       store8(o, v);
     } break;
     case EPI_RELU2: {
-      float a[8];
-      store8(o, v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        float t = fmaxf(v[i], 0.f);
-        a[i] = t * t;
+        const float t = fmaxf(v[i], 0.f);
+        v[i] = t * t;
       }
-      store8(reinterpret_cast<T*>(ep.out2) + r * ep.ldo2 + c, a);
+      store8(o, v);
     } break;
     case EPI_DRELU2: {
-      float u[8];
-      load8(reinterpret_cast<const T*>(ep.aux) + r * ep.ld_aux + c, u);
+      float a[8];
+      load8(reinterpret_cast<const T*>(ep.aux) + r * ep.ld_aux + c, a);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] *= 2.f * fmaxf(u[i], 0.f);
+      for (int i = 0; i < 8; ++i) v[i] *= 2.f * sqrtf(fmaxf(a[i], 0.f));
       store8(o, v);
     } break;
     default:
@@ -140,12 +140,11 @@ __device__ __forceinline__ void epi_scalar_t(const EpiParams& ep, long long r, i
   switch (ep.kind) {
     case EPI_RESID: *o = from_f<T>(fmaf(epi_beta(ep), to_f(reinterpret_cast<const T*>(ep.aux)[r * ep.ld_aux + c]), v)); break;
     case EPI_RELU2: {
-      *o = from_f<T>(v);
-      float t = fmaxf(v, 0.f);
-      reinterpret_cast<T*>(ep.out2)[r * ep.ldo2 + c] = from_f<T>(t * t);
+      const float t = fmaxf(v, 0.f);
+      *o = from_f<T>(t * t);
     } break;
     case EPI_DRELU2:
-      *o = from_f<T>(v * 2.f * fmaxf(to_f(reinterpret_cast<const T*>(ep.aux)[r * ep.ld_aux + c]), 0.f));
+      *o = from_f<T>(v * 2.f * sqrtf(fmaxf(to_f(reinterpret_cast<const T*>(ep.aux)[r * ep.ld_aux + c]), 0.f)));
       break;
     default: *o = from_f<T>(v);
   }
@@ -587,7 +586,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int i = 0; i < 8; ++i) v[i] = fmaf(beta, a[i], v[i]);
               } else if (ep.kind == EPI_DRELU2) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= 2.f * fmaxf(a[i], 0.f);
+                for (int i = 0; i < 8; ++i) v[i] *= 2.f * sqrtf(fmaxf(a[i], 0.f));
               } else {
                 // the dot takes the values as stored (rounded to bf16)
 #pragma unroll
@@ -607,15 +606,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                   if (xy == c8 + i) ep.xent_zy[row0 + lane] = v[i];
               }
             }
-            store8(reinterpret_cast<bf16*>(cp0), v);
             if (ep.kind == EPI_RELU2) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const float t = fmaxf(v[i], 0.f);
                 v[i] = t * t;
               }
-              store8(reinterpret_cast<bf16*>(cp1), v);
             }
+            store8(reinterpret_cast<bf16*>(cp0), v);
           }
         }
         if (ep.kind == EPI_DOT && (cc & 1)) {  // a 128-column group (one head) is complete
@@ -634,7 +632,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tma_reduce_add_2d(&tmO, stg1, col0 + 32, row0);
           } else {
             tma_store_2d(&tmO, stg0, col0, row0);
-            if (ep.kind == EPI_RELU2) tma_store_2d(&tmO2, stg1, col0, row0);
           }
           bulk_commit_group();
         }
