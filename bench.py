@@ -309,13 +309,14 @@ def run_decode(args, c: dict):
     v = torch.randn(B, T, Hk, 128, device="cuda", generator=g).bfloat16()
     lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
     o = torch.empty(B, H, 128, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(gb.gptb_decode_workspace_bytes(B, H, T), dtype=torch.uint8, device="cuda")
     for _ in range(args.warmup):
-        gb.gptb_decode_attention(q, k, v, lens, o, None, B, H, Hk, T, -1)
+        gb.gptb_decode_attention(q, k, v, lens, o, None, B, H, Hk, T, -1, ws)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        gb.gptb_decode_attention(q, k, v, lens, o, None, B, H, Hk, T, -1)
+        gb.gptb_decode_attention(q, k, v, lens, o, None, B, H, Hk, T, -1, ws)
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / args.steps

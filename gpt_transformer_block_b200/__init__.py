@@ -26,7 +26,7 @@ EXPORTS = [
     "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
     "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express", "gptb_decode_attention",
     "gptb_muon_workspace_bytes", "gptb_muon_step", "gpt_stack_step_hooked", "gptb_cast_f32_bf16",
-    "gptb_cast_bf16_f32",
+    "gptb_cast_bf16_f32", "gptb_decode_workspace_bytes",
 ]
 
 GRADS_READY_FN = ctypes.CFUNCTYPE(None, ctypes.c_int, ctypes.c_void_p)
@@ -107,7 +107,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptb_polar_express.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _fp, ctypes.c_int, _vp,
                                        ctypes.c_size_t, _vp]
     lib.gptb_decode_attention.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                          ctypes.c_int, ctypes.c_int, _vp]
+                                          ctypes.c_int, ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    lib.gptb_decode_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.gptb_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.gpt_stack_step_hooked.argtypes = [P(Config), P(ModelWeights), _vp, _vp, _vp, P(ModelGrads), _vp, _vp,
                                           GRADS_READY_FN, _vp]
     lib.gptb_cast_f32_bf16.argtypes = [_vp, _vp, ctypes.c_longlong, ctypes.c_float, _vp]
@@ -119,7 +121,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                    ctypes.c_size_t, _vp]
     for name in EXPORTS:
         if name not in ("gptb_workspace_bytes", "gptb_error_string", "gptb_reset_counters",
-                        "gptb_launch_count", "gptb_polar_express_workspace_bytes", "gptb_muon_workspace_bytes"):
+                        "gptb_launch_count", "gptb_polar_express_workspace_bytes", "gptb_muon_workspace_bytes",
+                        "gptb_decode_workspace_bytes"):
             getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -304,11 +307,16 @@ def gptb_muon_step(w, w_bf16, g, buf, v, m, n, coeffs, lr, mu, beta2, weight_dec
                                  _stream(stream)), "gptb_muon_step")
 
 
-def gptb_decode_attention(q, k_cache, v_cache, lens, o, lse, B, H, Hkv, T_max, window, stream=None):
+def gptb_decode_workspace_bytes(B: int, H: int, T_max: int) -> int:
+    return int(load().gptb_decode_workspace_bytes(int(B), int(H), int(T_max)))
+
+
+def gptb_decode_attention(q, k_cache, v_cache, lens, o, lse, B, H, Hkv, T_max, window, workspace, stream=None):
     """One decode step: attention of each sequence's newest token over its KV cache."""
+    nbytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
     _check(load().gptb_decode_attention(ptr(q), ptr(k_cache), ptr(v_cache), ptr(lens), ptr(o), ptr(lse), int(B),
-                                        int(H), int(Hkv), int(T_max), int(window), _stream(stream)),
-           "gptb_decode_attention")
+                                        int(H), int(Hkv), int(T_max), int(window), ptr(workspace), nbytes,
+                                        _stream(stream)), "gptb_decode_attention")
 
 
 def gptb_device_error(stream=None) -> int:

@@ -1211,21 +1211,28 @@ int gptb_muon_step(float* w, void* w_bf16, const float* g, float* buf, float* v,
 
 // --------------------------------------------------------------- decode --
 
+size_t gptb_decode_workspace_bytes(int B, int H, int T_max) {
+  if (B < 0 || H <= 0 || T_max <= 0) return 0;
+  return (size_t)B * H * decode_pieces(T_max) * DEC_PART * sizeof(float) + 256;
+}
+
 int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, void* o,
-                          float* lse, int B, int H, int Hkv, int T_max, int window, gptb_stream_t stream) {
+                          float* lse, int B, int H, int Hkv, int T_max, int window, void* workspace,
+                          size_t workspace_bytes, gptb_stream_t stream) {
   if (!q || !k_cache || !v_cache || !lens || !o || B < 0 || H <= 0 || Hkv <= 0 || H % Hkv || T_max <= 0)
     return GPTB_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return GPTB_ERR_INVALID_ARG;
   if (B == 0) return GPTB_OK;
-  const int G = H / Hkv;
-  const size_t smem = decode_smem_bytes(G, T_max);
-  if (G > 16 || smem > 220 * 1024) return GPTB_ERR_UNSUPPORTED;  // scores of the whole cache stay in shared memory
+  if (H / Hkv > DEC_MAX_G) return GPTB_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace)) return GPTB_ERR_INVALID_ARG;
+  if (workspace_bytes < gptb_decode_workspace_bytes(B, H, T_max)) return GPTB_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (smem > 48 * 1024)
-    CK(cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  decode_attn_kernel<<<B * Hkv, DEC_THREADS, smem, st>>>(
-      static_cast<const bf16*>(q), static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache), lens,
-      static_cast<bf16*>(o), lse, H, Hkv, T_max, window);
+  float* part = static_cast<float*>(workspace);
+  decode_split_kernel<<<B * Hkv * decode_pieces(T_max), DEC_THREADS, 0, st>>>(
+      static_cast<const bf16*>(q), static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache), lens, part,
+      H, Hkv, T_max, window);
+  CKL();
+  decode_combine_kernel<<<B * H, DEC_HD, 0, st>>>(part, lens, static_cast<bf16*>(o), lse, H, T_max);
   CKL();
   return GPTB_OK;
 }

@@ -319,11 +319,17 @@ int gptb_muon_step(float* w, void* w_bf16, const float* g, float* buf, float* v,
  *   window:  -1 = every cached key; W >= 0 keeps keys lens[b]-1-W .. lens[b]-1
  *   o:       device bf16 [B, H, 128]; lse: device fp32 [B, H] (natural log of
  *            the softmax denominator incl. its max) or NULL
+ *   workspace: device, gptb_decode_workspace_bytes(B, H, T_max) bytes, 16-byte
+ *            aligned (partial softmax sums of the key pieces; the keys of a
+ *            sequence are split into pieces of 256 handled in parallel, then
+ *            combined)
  * Errors: GPTB_ERR_INVALID_ARG (null / misaligned pointers, H % H_kv != 0),
- * GPTB_ERR_UNSUPPORTED (more than 16 query heads per kv head, or a cache too
- * long for the per-CTA score buffer: (H/H_kv) * (T_max + 128) floats <= 220 KB). */
+ * GPTB_ERR_WORKSPACE (workspace too small), GPTB_ERR_UNSUPPORTED (more than
+ * 16 query heads per kv head). */
+size_t gptb_decode_workspace_bytes(int B, int H, int T_max);
 int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, void* o,
-                          float* lse, int B, int H, int Hkv, int T_max, int window, gptb_stream_t stream);
+                          float* lse, int B, int H, int Hkv, int T_max, int window, void* workspace,
+                          size_t workspace_bytes, gptb_stream_t stream);
 
 /* Element casts for data-parallel gradient buckets (bf16 on the wire):
  * y[i] = bf16(x[i] * scale) and y[i] = float(x[i]) * scale, n elements,

@@ -20,15 +20,16 @@ def _run(gb, B, H, Hk, Tmax, lens, window, seed=0):
     ln = torch.tensor(lens, dtype=torch.int32)
     o = torch.empty(B, H, 128, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
-    gb.gptb_decode_attention(q.cuda(), k.cuda(), v.cuda(), ln.cuda(), o, lse, B, H, Hk, Tmax, window)
+    ws = torch.empty(gb.gptb_decode_workspace_bytes(B, H, Tmax), dtype=torch.uint8, device="cuda")
+    gb.gptb_decode_attention(q.cuda(), k.cuda(), v.cuda(), ln.cuda(), o, lse, B, H, Hk, Tmax, window, ws)
     torch.cuda.synchronize()
     return q, k, v, ln, o.cpu(), lse.cpu()
 
 
 @pytest.mark.parametrize("window", [-1, 0, 37])
 def test_decode_gqa_ragged(cuda_lib, window):
-    B, H, Hk, Tmax = 5, 4, 2, 300
-    lens = [300, 1, 129, 64, 257]
+    B, H, Hk, Tmax = 6, 4, 2, 600
+    lens = [600, 1, 129, 64, 257, 513]  # several key pieces of 256, ragged last pieces
     q, k, v, ln, o, lse = _run(cuda_lib, B, H, Hk, Tmax, lens, window)
     ro, rl = od.decode_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(), lens, window)
     assert relerr(o.double().numpy(), ro) <= TOL["bf16"]
