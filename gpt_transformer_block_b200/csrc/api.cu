@@ -372,6 +372,7 @@ EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = n
   e.xent_nt = 0;
   e.targets = nullptr;
   e.xent_zy = nullptr;
+  e.amax_out = nullptr;
   return e;
 }
 EpiParams epi8(EpiParams e, const float* amax_a, const float* amax_b, bool a_e5m2 = false) {
@@ -471,7 +472,7 @@ struct Scratch {
   void *du, *dh2, *dx1, *dO, *dqkv, *dh;
   float *D, *dq, *dk, *dv, *dz;
   uint8_t* g8;   // FP8: e4m3 copy of the gradient feeding a GEMM pair
-  float* gamax;  // FP8: its amax
+  float* gamax;  // FP8: amax of the gradients [dx_out, du, dx1, dqkv]
 };
 Scratch carve_scratch(Carve& cv, const Dims& m) {
   Scratch s;
@@ -498,7 +499,7 @@ Scratch carve_scratch(Carve& cv, const Dims& m) {
   if (m.fp8) {
     const long long w = std::max<long long>(std::max<long long>(m.Wq, m.F), std::max<long long>(m.d, (long long)m.H * m.hd));
     s.g8 = (uint8_t*)cv.take(m.N * w);
-    s.gamax = (float*)cv.take(4);
+    s.gamax = (float*)cv.take(4 * 4);  // [block input gradient, du, dx1, dqkv]
   }
   cv.off = std::max(cv.off, fwd_end);
   return s;
@@ -620,13 +621,16 @@ int rope_init(const gptb_config& c, float2* tab, cudaStream_t st) {
 
 // per-tensor FP8 quantisation: amax (fp32 bits, atomicMax) then codes, e4m3
 // (scale 448/amax) or e5m2 (57344/amax)
+// (amax_ready: the producer of x already published its amax into *amax)
 template <class T>
-int quant(const T* x, long long n, uint8_t* out, float* amax, bool e5m2, cudaStream_t st) {
-  CK(cudaMemsetAsync(amax, 0, sizeof(float), st));
+int quant(const T* x, long long n, uint8_t* out, float* amax, bool e5m2, cudaStream_t st, bool amax_ready = false) {
   const long long n8 = n / 8;
   const int grid = (int)std::max<long long>(1, std::min<long long>((n8 + 255) / 256, (long long)dev_info().sms * 8));
-  amax_kernel<T><<<grid, 256, 0, st>>>(x, n8, reinterpret_cast<unsigned int*>(amax));
-  CKL();
+  if (!amax_ready) {
+    CK(cudaMemsetAsync(amax, 0, sizeof(float), st));
+    amax_kernel<T><<<grid, 256, 0, st>>>(x, n8, reinterpret_cast<unsigned int*>(amax));
+    CKL();
+  }
   quantize_fp8_kernel<T><<<grid, 256, 0, st>>>(x, n8, amax, e5m2 ? 1 : 0, out);
   CKL();
   return GPTB_OK;
@@ -642,7 +646,8 @@ struct Operand {
   uint8_t* q;
   float* amax;
   bool quant;
-  bool e5m2;  // FP8 copy in e5m2 (gradient operands of the e5m2 variant)
+  bool e5m2;        // FP8 copy in e5m2 (gradient operands of the e5m2 variant)
+  bool amax_ready;  // FP8: the producer of p already wrote its amax (no amax pass)
 };
 
 // A projection GEMM of the block in the config's arithmetic: f32 (SIMT) or
@@ -654,8 +659,8 @@ int proj(const gptb_config& c, const Operand& A, const Operand& B, int M, int N,
          cudaStream_t st) {
   if (c.dtype != GPTB_FP8_E4M3) return gemm(c.dtype, {A.p, A.ld, A.mn}, {B.p, B.ld, B.mn}, M, N, K, e, st);
   if (!A.q || !B.q || !A.amax || !B.amax || B.e5m2) return GPTB_ERR_INVALID_ARG;
-  if (A.quant) TRY(quant<T>((const T*)A.p, A.elems, A.q, A.amax, A.e5m2, st));
-  if (B.quant) TRY(quant<T>((const T*)B.p, B.elems, B.q, B.amax, false, st));
+  if (A.quant) TRY(quant<T>((const T*)A.p, A.elems, A.q, A.amax, A.e5m2, st, A.amax_ready));
+  if (B.quant) TRY(quant<T>((const T*)B.p, B.elems, B.q, B.amax, false, st, B.amax_ready));
   return gemm(GPTB_FP8_E4M3, {A.q, A.ld, A.mn}, {B.q, B.ld, B.mn}, M, N, K, epi8(e, A.amax, B.amax, A.e5m2), st);
 }
 
@@ -669,8 +674,12 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   const bool ve = c.has_ve[layer] != 0;
   if (!w.w_qkv || !w.w_o || !w.w_fc || !w.w_proj || !w.lambdas || (ve && (!w.w_ve_gate || !w.ve_table)))
     return GPTB_ERR_INVALID_ARG;
+  // FP8: the producers of the four GEMM activations publish their amax into S.amax[0..3]
+  unsigned int* am = m.fp8 ? reinterpret_cast<unsigned int*>(S.amax) : nullptr;
+  if (m.fp8) CK(cudaMemsetAsync(S.amax, 0, 4 * sizeof(float), st));
   br_mix_norm_kernel<T><<<brg, brt, 0, st>>>(x, x0, w.lambdas, (T*)X.xm, (T*)S.h, S.rstd1, m.N, m.d, c.norm_eps,
-                                                ve ? (const T*)w.w_ve_gate : nullptr, S.sg, m.Hkv, c.ve_gate_ch);
+                                                ve ? (const T*)w.w_ve_gate : nullptr, S.sg, m.Hkv, c.ve_gate_ch,
+                                                am ? am + 0 : nullptr);
   CKL();
   const long long Ho = (long long)m.H * m.hd;
   if (c.dtype == GPTB_F32) {
@@ -692,7 +701,7 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     e.H = m.H;
     e.Hkv = m.Hkv;
     e.eps = c.norm_eps;
-    TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, S.h8, S.amax + 0, true},
+    TRY(proj<T>(c, {S.h, m.d, false, m.N * m.d, S.h8, S.amax + 0, true, false, true},
                 {w.w_qkv, m.d, false, (long long)m.Wq * m.d, S.wqkv8, S.amax + 4, true}, (int)m.N, m.Wq, m.d, e, st));
   }
   const int W = c.window[layer];
@@ -707,19 +716,20 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     if (!make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128)) return GPTB_ERR_CUDA;
     CK(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM));
     attn_fwd_tc_kernel<<<dim3((m.T + FA_BM - 1) / FA_BM, m.H, m.B), FA_THREADS, FA_SMEM, st>>>(
-        tq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W);
+        tq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W, am ? am + 1 : nullptr);
     CKL();
   }
-  TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, S.o8, S.amax + 1, true},
+  TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, S.o8, S.amax + 1, true, false, true},
               {w.w_o, Ho, false, m.d * Ho, S.wo8, S.amax + 5, true}, (int)m.N, m.d, (int)Ho,
               epi(EPI_RESID, c.dtype, X.x1, m.d, X.xm, m.d), st));
   br_norm_kernel<T><<<brg, brt, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
-                                            c.norm_eps);
+                                            c.norm_eps, am ? am + 2 : nullptr);
   CKL();
-  TRY(proj<T>(c, {S.h2, m.d, false, m.N * m.d, S.h2_8, S.amax + 2, true},
-              {w.w_fc, m.d, false, (long long)m.F * m.d, S.wfc8, S.amax + 6, true}, (int)m.N, m.F, m.d,
-              epi(EPI_RELU2, c.dtype, S.act, m.F), st));
-  TRY(proj<T>(c, {S.act, m.F, false, m.N * m.F, S.act8, S.amax + 3, true},
+  EpiParams erelu = epi(EPI_RELU2, c.dtype, S.act, m.F);
+  erelu.amax_out = am ? am + 3 : nullptr;
+  TRY(proj<T>(c, {S.h2, m.d, false, m.N * m.d, S.h2_8, S.amax + 2, true, false, true},
+              {w.w_fc, m.d, false, (long long)m.F * m.d, S.wfc8, S.amax + 6, true}, (int)m.N, m.F, m.d, erelu, st));
+  TRY(proj<T>(c, {S.act, m.F, false, m.N * m.F, S.act8, S.amax + 3, true, false, true},
               {w.w_proj, m.F, false, (long long)m.d * m.F, S.wproj8, S.amax + 7, true}, (int)m.N, m.d, m.F,
               epi(EPI_RESID, c.dtype, x_out, m.d, X.x1, m.d), st));
   return GPTB_OK;
@@ -744,18 +754,33 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   // input-gradient GEMM then reuses with the forward's e4m3 weight; the other
   // weight-gradient operand is the forward's saved e4m3 activation)
   const long long Nd = m.N * m.d;
-  TRY(proj<T>(c, {dx2, m.d, true, Nd, X.g8, X.gamax, true, m.grad_e5m2}, {S.act, m.F, true, 0, S.act8, S.amax + 3, false}, m.d,
+  // FP8: amax slots of the four gradients [block input, du, dx1, dqkv]; the
+  // producers of the last three publish theirs (no separate amax pass)
+  float* ga[4] = {nullptr, nullptr, nullptr, nullptr};
+  unsigned int* gam[4] = {nullptr, nullptr, nullptr, nullptr};
+  if (m.fp8) {
+    for (int i = 0; i < 4; ++i) {
+      ga[i] = X.gamax + i;
+      gam[i] = reinterpret_cast<unsigned int*>(X.gamax + i);
+    }
+    CK(cudaMemsetAsync(X.gamax + 1, 0, 3 * sizeof(float), st));
+  }
+  const bool e5 = m.grad_e5m2;
+  TRY(proj<T>(c, {dx2, m.d, true, Nd, X.g8, ga[0], true, e5}, {S.act, m.F, true, 0, S.act8, S.amax + 3, false}, m.d,
               m.F, N, epi(EPI_ACCUM_F32, dt, g.w_proj, m.F), st));
-  TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false},
-              N, m.F, m.d, epi(EPI_DRELU2, dt, X.du, m.F, S.act, m.F), st));
-  TRY(proj<T>(c, {X.du, m.F, true, m.N * m.F, X.g8, X.gamax, true, m.grad_e5m2}, {S.h2, m.d, true, 0, S.h2_8, S.amax + 2, false},
+  EpiParams edr = epi(EPI_DRELU2, dt, X.du, m.F, S.act, m.F);
+  edr.amax_out = gam[1];
+  TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, ga[0], false, e5}, {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false},
+              N, m.F, m.d, edr, st));
+  TRY(proj<T>(c, {X.du, m.F, true, m.N * m.F, X.g8, ga[1], true, e5, true}, {S.h2, m.d, true, 0, S.h2_8, S.amax + 2, false},
               m.F, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d), st));
-  TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false},
+  TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, ga[1], false, e5}, {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false},
               N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
-  br_norm_bwd_kernel<T><<<brg, brt, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d);
+  br_norm_bwd_kernel<T><<<brg, brt, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d,
+                                                gam[2]);
   CKL();
   // attention output projection
-  TRY(proj<T>(c, {X.dx1, m.d, true, Nd, X.g8, X.gamax, true, m.grad_e5m2}, {S.o, Ho, true, 0, S.o8, S.amax + 1, false}, m.d,
+  TRY(proj<T>(c, {X.dx1, m.d, true, Nd, X.g8, ga[2], true, e5, true}, {S.o, Ho, true, 0, S.o8, S.amax + 1, false}, m.d,
               (int)Ho, N, epi(EPI_ACCUM_F32, dt, g.w_o, Ho), st));
   // dO = dx1 Wo, and the attention backward's D = rowsum(dO * o) per head
   if constexpr (std::is_same<T, bf16>::value) {
@@ -764,10 +789,10 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     ed.rowdot = X.D;
     ed.T = m.T;
     ed.H = m.H;
-    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, false, m.grad_e5m2}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, ga[2], false, e5}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
                 (int)Ho, m.d, ed, st));
   } else {
-    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, X.gamax, true, m.grad_e5m2}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, ga[2], true, e5}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
                 (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
     attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
                                                                        m.B, m.T, m.H, m.hd);
@@ -802,7 +827,7 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   if constexpr (std::is_same<T, bf16>::value) {
     qkv_post_bwd_h128_kernel<<<grid_rows(m.N), EW_THREADS, 0, st>>>(
         (const bf16*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (bf16*)X.dqkv, m.T, m.N, m.H, m.Hkv,
-        ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz);
+        ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz, gam[3]);
   } else {
     qkv_post_bwd_kernel<T><<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(
         (const T*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (T*)X.dqkv, m.T, m.N, m.H, m.Hkv, m.hd,
@@ -810,9 +835,9 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   }
   CKL();
   // QKV projection
-  TRY(proj<T>(c, {X.dqkv, m.Wq, true, m.N * m.Wq, X.g8, X.gamax, true, m.grad_e5m2}, {S.h, m.d, true, 0, S.h8, S.amax + 0, false},
+  TRY(proj<T>(c, {X.dqkv, m.Wq, true, m.N * m.Wq, X.g8, ga[3], true, e5, true}, {S.h, m.d, true, 0, S.h8, S.amax + 0, false},
               m.Wq, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_qkv, m.d), st));
-  TRY(proj<T>(c, {X.dqkv, m.Wq, false, m.N * m.Wq, X.g8, X.gamax, false, m.grad_e5m2},
+  TRY(proj<T>(c, {X.dqkv, m.Wq, false, m.N * m.Wq, X.g8, ga[3], false, e5},
               {w.w_qkv, m.d, true, 0, S.wqkv8, S.amax + 4, false}, N, m.d, m.Wq, epi(EPI_STORE, dt, X.dh, m.d), st));
   if (ve) {
     const int nthreads = ((m.Hkv * c.ve_gate_ch + 31) / 32) * 32;
@@ -917,7 +942,7 @@ int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t*
   }
   const T* x_bo = c.backout_layer >= 0 ? (const T*)S.x_in[c.backout_layer] : nullptr;
   br_norm_kernel<T><<<brg, brt, 0, st>>>((const T*)S.xL, x_bo, w.backout_lambda, (T*)S.hf, S.rstd_f, m.N, m.d,
-                                            c.norm_eps);
+                                            c.norm_eps, nullptr);
   CKL();
   TRY(lm_head_impl<T>(c, (const T*)S.hf, (const T*)w.w_lm, targets, loss_out, (T*)S.dhf, g.w_lm, S.lm, st));
   br_final_norm_bwd_kernel<T><<<brg, brt, 0, st>>>((const T*)S.dhf, (const T*)S.hf, S.rstd_f, x_bo,

@@ -50,7 +50,7 @@ __device__ __forceinline__ uint64_t fa_desc_mn(uint32_t tile, int k) {
 
 __global__ void __launch_bounds__(FA_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ o, long long ldo,
-                       float* __restrict__ lse, int T, int H, int Hkv, int window) {
+                       float* __restrict__ lse, int T, int H, int Hkv, int window, unsigned int* __restrict__ amax_o) {
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const int t = q0 + r;          // query position
     const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
     const float sl2 = LOG2E / sqrtf(128.f);
+    float oam = 0.f;  // max |o| this thread stores (FP8 amax)
     // keys visible from query t: [t - W, t] (or [0, t]) clipped to the sequence
     const int kv_lo = (window >= 0) ? t - window : 0;
     const int kv_hi = min(t, T - 1);
@@ -281,6 +282,10 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         tmem_ld_32x32b_x32(lane_addr + 256 + hf * 64 + c * 32, v);
         tmem_ld_wait();
         if (t < T) {
+          if (amax_o) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) oam = fmaxf(oam, fabsf(__uint_as_float(v[i]) * inv));
+          }
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             uint4 u;
@@ -293,6 +298,17 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
       }
       if (t < T && hf == 0) lse[((long long)b * H + h) * T + t] = (m_used + log2f(lt)) * LN2;
+    }
+    if (amax_o) {  // the softmax warps' max |o| (FP8 amax): one atomic per CTA
+      oam = warp_max(oam);
+      named_bar_sync(1, FA_SOFTMAX_THREADS);
+      if (lane == 0) xsum[warp - 2] = oam;  // xsum is free once every row's sum has been read
+      named_bar_sync(1, FA_SOFTMAX_THREADS);
+      if (warp == 2 && lane == 0) {
+        float mm = 0.f;
+        for (int w = 0; w < FA_SOFTMAX_THREADS / 32; ++w) mm = fmaxf(mm, xsum[w]);
+        atomicMax(amax_o, __float_as_uint(stored_abs_max_bf16(mm)));
+      }
     }
   }
   tc_fence_before();

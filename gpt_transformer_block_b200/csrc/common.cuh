@@ -385,6 +385,26 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// Per-tensor max |x| of values a kernel stores (the FP8 quantiser's amax):
+// the largest magnitude of the stored bf16 values equals the bf16 rounding of
+// the largest fp32 magnitude (rounding is monotone), so a thread keeps the
+// fp32 maximum and one thread per CTA publishes the CTA's maximum with an
+// atomicMax on the (non-negative) float's bits.
+__device__ __forceinline__ float stored_abs_max_bf16(float m) { return __bfloat162float(__float2bfloat16_rn(m)); }
+// block-wide max of v (all threads of the CTA must call it), then one atomic
+__device__ __forceinline__ void block_amax_publish(float v, unsigned int* amax, float* sh32) {
+  v = warp_max(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  __syncthreads();
+  if (lane == 0) sh32[warp] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int w = 0; w < nw; ++w) m = fmaxf(m, sh32[w]);
+    atomicMax(amax, __float_as_uint(stored_abs_max_bf16(m)));
+  }
+}
+
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 

@@ -619,8 +619,11 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
                              const float* __restrict__ dk, const float* __restrict__ dv, long long lddkv,
                              bf16* __restrict__ dqkv, int Tn, long long N, int H, int Hkv,
                              const bf16* __restrict__ ve_table, const int32_t* __restrict__ idx,
-                             const float* __restrict__ sg, float* __restrict__ dve_table, float* __restrict__ dz) {
+                             const float* __restrict__ sg, float* __restrict__ dve_table, float* __restrict__ dz,
+                             unsigned int* __restrict__ amax_out) {
   constexpr int QB = QKV_BWD_HEADS;
+  __shared__ float sa[32];
+  float am = 0.f;  // max |dqkv| this lane stores (FP8 amax)
   const int lane = threadIdx.x & 31;
   const bool hi = lane >= 16;
   const int nqk = H + Hkv;
@@ -676,7 +679,10 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
         const float m = warp_sum(dot) * (1.f / 128.f);
         float o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = r[b] * (gu[e] - yu[e] * m);
+        for (int e = 0; e < 4; ++e) {
+          o[e] = r[b] * (gu[e] - yu[e] * m);
+          am = fmaxf(am, fabsf(o[e]));
+        }
         st4(orow + (long long)hh * 128, o);
         }
       }
@@ -712,11 +718,14 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
           red_add_v4_f32(dve_table + ve_row + (long long)kv * 128, gate * g[0], gate * g[1], gate * g[2], gate * g[3]);
           if (lane == 0) dz[n * Hkv + kv] = dg * 3.f * sv[b] * (1.f - sv[b]);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(g[e]));
         st4(orow + (long long)(nqk + kv) * 128, g);
         }
       }
     }
   }
+  if (amax_out) block_amax_publish(am, amax_out, sa);
 }
 
 }  // namespace gptb

@@ -79,6 +79,8 @@ struct EpiParams {
   int xent_nt;
   const int32_t* targets;  // [M] class ids; ids outside [0, N) match no column
   float* xent_zy;          // [M]
+  // EPI_RELU2 / EPI_DRELU2: max |out| of the stored values (FP8 amax), or nullptr
+  unsigned int* amax_out;
 };
 
 __device__ __forceinline__ float epi_beta(const EpiParams& ep) { return ep.beta ? *ep.beta : 1.f; }
@@ -492,6 +494,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint32_t acc_phase = 0;
     const float alpha = epi_alpha(ep);
     const float beta = epi_beta(ep);
+    float oam = 0.f;  // max |out| stored by this thread (FP8 amax of EPI_RELU2 / EPI_DRELU2 outputs)
     bool ok = true;
     for (int u = unit0; u < units && ok; u += ustep) {
       int tm, tn, split;
@@ -613,6 +616,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 v[i] = t * t;
               }
             }
+            if (ep.amax_out && row0 + lane < M) {
+              const int c8 = col0 + g * 8;
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (c8 + i < N) oam = fmaxf(oam, fabsf(v[i]));
+            }
             store8(reinterpret_cast<bf16*>(cp0), v);
           }
         }
@@ -649,6 +658,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (acc == 0) acc_phase ^= 1u;
     }
     if (lane == 0) bulk_wait0();
+    if (ep.amax_out) {
+      oam = warp_max(oam);
+      if (lane == 0) atomicMax(ep.amax_out, __float_as_uint(stored_abs_max_bf16(oam)));
+    }
   }
   tc_fence_before();
   __syncthreads();

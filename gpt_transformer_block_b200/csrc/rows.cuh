@@ -111,11 +111,14 @@ template <class T>
 __global__ void __launch_bounds__(256)
     br_mix_norm_kernel(const T* __restrict__ x, const T* __restrict__ x0, const float* __restrict__ lam,
                        T* __restrict__ xm_out, T* __restrict__ h_out, float* __restrict__ rstd_out, long long N, int d,
-                       float eps, const T* __restrict__ w_gate, float* __restrict__ sg_out, int Hkv, int Cg) {
+                       float eps, const T* __restrict__ w_gate, float* __restrict__ sg_out, int Hkv, int Cg,
+                       unsigned int* __restrict__ amax_h) {
   __shared__ float sh[2 * BR_MAX_WARPS];
   __shared__ float hg[256];  // the gate's input channels of the current row
+  __shared__ float sa[32];
   const BRow r(d);
   const float a = lam[0], b = lam[1];
+  float am = 0.f;  // max |h| stored by this thread (FP8 amax)
   for (long long n = blockIdx.x; n < N; n += gridDim.x) {
     float v[8] = {}, v0[8] = {};
     if (r.act) {
@@ -131,7 +134,10 @@ __global__ void __launch_bounds__(256)
     if (r.act) store8(xm_out + n * d + r.c0, v);
     const float rstd = rsqrtf(br_sum(ss, sh, r) / d + eps);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] *= rstd;
+    for (int k = 0; k < 8; ++k) {
+      v[k] *= rstd;
+      am = fmaxf(am, fabsf(v[k]));
+    }
     if (r.act) store8(h_out + n * d + r.c0, v);
     if (r.tid == 0) rstd_out[n] = rstd;
     if (w_gate != nullptr && r.warp == 0) {
@@ -152,16 +158,20 @@ __global__ void __launch_bounds__(256)
       __syncwarp();  // hg is rewritten for the next row
     }
   }
+  if (amax_h) block_amax_publish(am, amax_h, sa);
 }
 
 // h = rmsnorm(x - lam_bo * x_bo)   (backout + final norm when x_bo != null)
 template <class T>
 __global__ void __launch_bounds__(256)
     br_norm_kernel(const T* __restrict__ x, const T* __restrict__ x_bo, const float* __restrict__ lam_bo,
-                   T* __restrict__ h_out, float* __restrict__ rstd_out, long long N, int d, float eps) {
+                   T* __restrict__ h_out, float* __restrict__ rstd_out, long long N, int d, float eps,
+                   unsigned int* __restrict__ amax_h) {
   __shared__ float sh[2 * BR_MAX_WARPS];
+  __shared__ float sa[32];
   const BRow r(d);
   const float lb = x_bo ? *lam_bo : 0.f;
+  float am = 0.f;
   for (long long n = blockIdx.x; n < N; n += gridDim.x) {
     float v[8] = {}, w[8] = {};
     if (r.act) {
@@ -176,10 +186,14 @@ __global__ void __launch_bounds__(256)
     }
     const float rstd = rsqrtf(br_sum(ss, sh, r) / d + eps);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] *= rstd;
+    for (int k = 0; k < 8; ++k) {
+      v[k] *= rstd;
+      am = fmaxf(am, fabsf(v[k]));
+    }
     if (r.act) store8(h_out + n * d + r.c0, v);
     if (r.tid == 0) rstd_out[n] = rstd;
   }
+  if (amax_h) block_amax_publish(am, amax_h, sa);
 }
 
 }  // namespace gptb
@@ -192,9 +206,12 @@ namespace gptb {
 template <class T>
 __global__ void __launch_bounds__(256)
     br_norm_bwd_kernel(const T* __restrict__ dres, const T* __restrict__ dh, const T* __restrict__ h,
-                       const float* __restrict__ rstd, T* __restrict__ out, long long N, int d) {
+                       const float* __restrict__ rstd, T* __restrict__ out, long long N, int d,
+                       unsigned int* __restrict__ amax_out) {
   __shared__ float sh[2 * BR_MAX_WARPS];
+  __shared__ float sa[32];
   const BRow r(d);
+  float am = 0.f;
   for (long long n = blockIdx.x; n < N; n += gridDim.x) {
     float g[8] = {}, y[8] = {}, o[8] = {};
     if (r.act) {
@@ -208,9 +225,13 @@ __global__ void __launch_bounds__(256)
     for (int k = 0; k < 8; ++k) dot = fmaf(g[k], y[k], dot);
     const float m = br_sum(dot, sh, r) / d;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) o[k] += rs * (g[k] - y[k] * m);
+    for (int k = 0; k < 8; ++k) {
+      o[k] += rs * (g[k] - y[k] * m);
+      am = fmaxf(am, fabsf(o[k]));
+    }
     if (r.act) store8(out + n * d + r.c0, o);
   }
+  if (amax_out) block_amax_publish(am, amax_out, sa);
 }
 
 // Block-input backward: dh (+ dz Wg on the first Cg channels) through the
