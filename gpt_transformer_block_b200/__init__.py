@@ -26,7 +26,7 @@ EXPORTS = [
     "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
     "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express", "gptb_decode_attention",
     "gptb_muon_workspace_bytes", "gptb_muon_step", "gpt_stack_step_hooked", "gptb_cast_f32_bf16",
-    "gptb_cast_bf16_f32", "gptb_decode_workspace_bytes",
+    "gptb_cast_bf16_f32", "gptb_decode_workspace_bytes", "gptb_gemm_fp8_workspace_bytes", "gptb_gemm_fp8",
 ]
 
 GRADS_READY_FN = ctypes.CFUNCTYPE(None, ctypes.c_int, ctypes.c_void_p)
@@ -108,6 +108,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        ctypes.c_size_t, _vp]
     lib.gptb_decode_attention.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    lib.gptb_gemm_fp8_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.gptb_gemm_fp8_workspace_bytes.restype = ctypes.c_size_t
+    lib.gptb_gemm_fp8.argtypes = [_vp, ctypes.c_int, ctypes.c_longlong, _vp, ctypes.c_int, ctypes.c_longlong, _vp,
+                                  ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp,
+                                  ctypes.c_size_t, _vp]
     lib.gptb_decode_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.gptb_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.gpt_stack_step_hooked.argtypes = [P(Config), P(ModelWeights), _vp, _vp, _vp, P(ModelGrads), _vp, _vp,
@@ -122,7 +127,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in EXPORTS:
         if name not in ("gptb_workspace_bytes", "gptb_error_string", "gptb_reset_counters",
                         "gptb_launch_count", "gptb_polar_express_workspace_bytes", "gptb_muon_workspace_bytes",
-                        "gptb_decode_workspace_bytes"):
+                        "gptb_decode_workspace_bytes", "gptb_gemm_fp8_workspace_bytes"):
             getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -264,6 +269,16 @@ def gptb_cast_f32_bf16(x, y, n, scale=1.0, stream=None):
 
 def gptb_cast_bf16_f32(x, y, n, scale=1.0, stream=None):
     _check(load().gptb_cast_bf16_f32(ptr(x), ptr(y), int(n), float(scale), _stream(stream)), "gptb_cast_bf16_f32")
+
+
+def gptb_gemm_fp8(A, a_mn, lda, B, b_mn, ldb, C, ldc, M, N, K, a_e5m2=False, stream=None):
+    """C += dequant(q(A) q(B)^T) with per-tensor FP8 casts of the bf16 operands (test entry point)."""
+    import torch
+    ws = torch.empty(int(load().gptb_gemm_fp8_workspace_bytes(int(M), int(N), int(K))), dtype=torch.uint8,
+                     device=C.device)
+    _check(load().gptb_gemm_fp8(ptr(A), int(a_mn), int(lda), ptr(B), int(b_mn), int(ldb), ptr(C), int(ldc), int(M),
+                                int(N), int(K), 1 if a_e5m2 else 0, ptr(ws), ws.numel(), _stream(stream)),
+           "gptb_gemm_fp8")
 
 
 def gptb_gemm_bf16(A, a_mn, lda, B, b_mn, ldb, C, c_f32, ldc, M, N, K, stream=None):

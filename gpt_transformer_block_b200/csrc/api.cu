@@ -1089,6 +1089,33 @@ int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_
   return gemm(GPTB_BF16, {A, lda, a_mn != 0}, {B, ldb, b_mn != 0}, M, N, K, e, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t gptb_gemm_fp8_workspace_bytes(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return ((size_t)M * K + 255) / 256 * 256 + ((size_t)N * K + 255) / 256 * 256 + 256;
+}
+
+int gptb_gemm_fp8(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, float* C,
+                  long long ldc, int M, int N, int K, int a_e5m2, void* workspace, size_t workspace_bytes,
+                  gptb_stream_t stream) {
+  if (!A || !B || !C || !workspace || M <= 0 || N <= 0 || K <= 0) return GPTB_ERR_INVALID_ARG;
+  if (a_mn && !b_mn) return GPTB_ERR_UNSUPPORTED;  // the one layout the block never uses
+  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  if (workspace_bytes < gptb_gemm_fp8_workspace_bytes(M, N, K) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GPTB_ERR_WORKSPACE;
+  // the stored matrices must be dense (row stride = the inner extent) for the per-tensor cast
+  if (lda != (a_mn ? M : K) || ldb != (b_mn ? N : K)) return GPTB_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  uint8_t* a8 = w;
+  uint8_t* b8 = w + ((size_t)M * K + 255) / 256 * 256;
+  float* amax = reinterpret_cast<float*>(b8 + ((size_t)N * K + 255) / 256 * 256);
+  if (((long long)M * K) % 8 || ((long long)N * K) % 8) return GPTB_ERR_INVALID_ARG;
+  TRY(quant<bf16>(static_cast<const bf16*>(A), (long long)M * K, a8, amax + 0, a_e5m2 != 0, st));
+  TRY(quant<bf16>(static_cast<const bf16*>(B), (long long)N * K, b8, amax + 1, false, st));
+  return gemm(GPTB_FP8_E4M3, {a8, lda, a_mn != 0}, {b8, ldb, b_mn != 0}, M, N, K,
+              epi8(epi(EPI_ACCUM_F32, GPTB_FP8_E4M3, C, ldc), amax + 0, amax + 1, a_e5m2 != 0), st);
+}
+
 // ------------------------------------------------------ optimizer step --
 
 int gptb_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, long long n, float lr, float beta1,

@@ -241,6 +241,18 @@ int gpt_stack_step_hooked(const gptb_config* cfg, const gptb_model_weights* w, c
 int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, void* C,
                    int c_f32, long long ldc, int M, int N, int K, gptb_stream_t stream);
 
+/* FP8 GEMM entry point used by the tests of the e4m3 / e5m2 tensor-core path:
+ * C[M,N] += dequant(q(A) q(B)^T), fp32 accumulate, where q casts the bf16
+ * operand to FP8 per tensor (A: e4m3 with scale 448/amax, or e5m2 with
+ * 57344/amax when a_e5m2; B: e4m3), RNE, saturating.  Layout flags as in
+ * gptb_gemm_bf16 (a_mn = 1 with b_mn = 0 is not supported); the operands must
+ * be dense (lda, ldb = their inner extents, multiples of 16).  workspace:
+ * device, gptb_gemm_fp8_workspace_bytes(M, N, K) bytes, 256-byte aligned. */
+size_t gptb_gemm_fp8_workspace_bytes(int M, int N, int K);
+int gptb_gemm_fp8(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, float* C,
+                  long long ldc, int M, int N, int K, int a_e5m2, void* workspace, size_t workspace_bytes,
+                  gptb_stream_t stream);
+
 /* ---------------------------------------------------- optimizer step ----
  * The step after the training step (nanochat's mixed optimizer: AdamW for the
  * embeddings, the lm_head and the scalar parameters; Muon, whose update is

@@ -61,3 +61,29 @@ def small_bf16(**kw) -> dict:
                 window=[-1, 48, -1], has_ve=[0, 1, 0], backout_layer=1)
     base.update(kw)
     return synth.config("d24", **base)
+
+
+# FP8 parity.  An FP8 product quantises bf16 tensors; the GPU and the
+# FP8-emulating oracle reach those tensors by different roundings (fp32 vs
+# fp64 upstream), so an e4m3 code near a rounding boundary can differ (one
+# code = 12.5 %).  Quantities made mostly of FP8 products (weight gradients,
+# gradients that crossed several FP8 layers) therefore differ from the
+# oracle's by the FP8 noise itself.  Such a quantity passes when it is within
+# the tolerance of the FP8 oracle, or when it is as close to the exact
+# (non-FP8) result as the FP8 oracle's own value is (within FP8_ENVELOPE
+# times that distance): a valid FP8 evaluation of the same inputs.  A wrong
+# scale, operand or index fails both.
+FP8_ENVELOPE = 1.5
+
+
+def judge(errs: dict, tol: float, gpu_exact: dict | None = None, ref_exact: dict | None = None) -> dict:
+    """The entries of errs (GPU vs the reference of its configuration) above
+    tol that, for FP8, are also outside the envelope; {} when all pass."""
+    bad = {}
+    for k, e in errs.items():
+        if e <= tol:
+            continue
+        if gpu_exact is not None and gpu_exact[k] <= FP8_ENVELOPE * ref_exact[k]:
+            continue
+        bad[k] = (e, gpu_exact.get(k) if gpu_exact else None, ref_exact.get(k) if ref_exact else None)
+    return bad

@@ -9,7 +9,7 @@ import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, fp8_mode, np64, oracle_layer, relerr, scalar_err, small_bf16
+from helpers import TOL, fp8_mode, judge, np64, oracle_layer, relerr, scalar_err, small_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -35,15 +35,8 @@ def run_block(gb, c, w, inp, layer):
     return x_out, dx, dx0, g
 
 
-def check_block(gb, c, layer, seed=1, x_std=1.0, exact_keys=()):
-    w = synth.make_weights(c, seed=seed)
-    inp = synth.make_block_inputs(c, seed=seed + 1, x_std=x_std)
-    x_out, dx, dx0, g = run_block(gb, c, w, inp, layer)
-    lw = oracle_layer(w, layer)
-    f8 = fp8_mode(c)
-    y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), inp["idx"].numpy(), layer, fp8=f8)
-    rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), inp["idx"].numpy(), layer, fp8=f8)
-    tol = TOL[c["dtype"]]
+def block_errors(x_out, dx, dx0, g, y, rdx, rdx0, rg):
+    """Per-output errors of a block's results against one oracle evaluation."""
     errs = {"x_out": relerr(np64(x_out), y), "dx": relerr(np64(dx), rdx), "dx0": relerr(np64(dx0), rdx0)}
     for k in ("w_qkv", "w_o", "w_fc", "w_proj", "w_ve_gate", "ve_table"):
         if k in rg:
@@ -51,7 +44,32 @@ def check_block(gb, c, layer, seed=1, x_std=1.0, exact_keys=()):
     lam = np64(g["lambdas"])
     errs["resid_lambda"] = scalar_err(lam[0], rg["resid_lambda"], rg["_scale"]["resid_lambda"])
     errs["x0_lambda"] = scalar_err(lam[1], rg["x0_lambda"], rg["_scale"]["x0_lambda"])
-    bad = {k: v for k, v in errs.items() if not v <= tol}
+    return errs
+
+
+def oracle_block(c, lw, inp, layer, f8):
+    idx = inp["idx"].numpy()
+    y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), idx, layer, fp8=f8)
+    rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), idx, layer, fp8=f8)
+    return y, rdx, rdx0, rg
+
+
+def check_block(gb, c, layer, seed=1, x_std=1.0):
+    w = synth.make_weights(c, seed=seed)
+    inp = synth.make_block_inputs(c, seed=seed + 1, x_std=x_std)
+    x_out, dx, dx0, g = run_block(gb, c, w, inp, layer)
+    lw = oracle_layer(w, layer)
+    f8 = fp8_mode(c)
+    ref = oracle_block(c, lw, inp, layer, f8)
+    errs = block_errors(x_out, dx, dx0, g, *ref)
+    gpu_exact = ref_exact = None
+    if f8:  # the FP8 envelope: distances to the exact (non-FP8) block
+        exact = oracle_block(c, lw, inp, layer, False)
+        gpu_exact = block_errors(x_out, dx, dx0, g, *exact)
+        y, rdx, rdx0, rg = ref
+        ref_exact = block_errors(y, rdx, rdx0, {k: v for k, v in rg.items() if k != "_scale"} | {"lambdas": [
+            rg["resid_lambda"], rg["x0_lambda"]]}, *exact)
+    bad = judge(errs, TOL[c["dtype"]], gpu_exact, ref_exact)
     assert not bad, (bad, errs)
     return errs
 

@@ -14,7 +14,7 @@ import torch
 import torch.distributed as dist
 
 import synth
-from helpers import small_bf16
+from helpers import TOL, relerr, small_bf16
 from oracle import optim as oo
 
 pytestmark = pytest.mark.gpu
@@ -40,6 +40,7 @@ def test_zero2_trainer_world1_matches_direct_updates(cuda_lib):
 
     # direct route: one plain step, then each parameter's update on the whole tensor
     ref = GPTStack(c, w)
+    w0 = {s.name: _get(ref.w, s.name).double().cpu() for s in stack_param_specs(c)}  # weights before the step
     ref.step(idx, tg)
     torch.cuda.synchronize()
     expect = {}
@@ -72,13 +73,14 @@ def test_zero2_trainer_world1_matches_direct_updates(cuda_lib):
         assert gb.gptb_device_error() == 0
         assert order == [1, 0, -1]
         assert abs(loss.item() - loss_ref) <= 1e-6 * abs(loss_ref)
+        # the two routes see the same gradients up to the order of the fp32
+        # atomics in the split-K and scatter reductions (and NorMuon's sums), so
+        # the updates (new - old weight) agree to the bf16 tolerance
         for s in stack_param_specs(c):
-            got, want = tr.param(s.name).float(), expect[s.name].float()
-            if s.kind == "adamw":
-                assert torch.equal(got, want), s.name
-            else:  # NorMuon's two sums use float atomics: the order may differ
-                assert torch.allclose(got, want, rtol=1e-2, atol=1e-6), s.name
-                assert (got - want).abs().max() <= 2 ** -8 * want.abs().max(), s.name
+            got, want = tr.param(s.name).double().cpu(), expect[s.name].double().cpu()
+            base = w0[s.name]
+            err = relerr((got - base).numpy(), (want - base).numpy())
+            assert err <= TOL["bf16"], (s.name, err)
     finally:
         dist.destroy_process_group()
 

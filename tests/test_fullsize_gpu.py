@@ -16,7 +16,7 @@ import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, fp8_mode, np64, oracle_layer, relerr, scalar_err
+from helpers import TOL, fp8_mode, judge, np64, oracle_layer, relerr
 
 pytestmark = pytest.mark.gpu
 
@@ -48,21 +48,20 @@ def test_block_full_width_every_gradient(cuda_lib, name, layer, B):
     inp = synth.make_block_inputs(c, seed=202 + layer)
     x_out, dx, dx0, g = _run_block(c, w, inp, layer)
     assert cuda_lib.gptb_device_error() == 0
+    from test_block_gpu import block_errors, oracle_block
     lw = oracle_layer(w, layer)
     f8 = fp8_mode(c)
-    idx = inp["idx"].numpy()
-    y, cache = om.block_forward(c, lw, np64(inp["x"]), np64(inp["x0"]), idx, layer, fp8=f8)
-    rdx, rdx0, rg = om.block_backward(c, lw, cache, np64(inp["dy"]), idx, layer, fp8=f8)
-    errs = {"x_out": relerr(np64(x_out), y), "dx": relerr(np64(dx), rdx), "dx0": relerr(np64(dx0), rdx0)}
-    for k in ("w_qkv", "w_o", "w_fc", "w_proj", "w_ve_gate", "ve_table"):
-        if k in rg:
-            errs[k] = relerr(np64(g[k]), rg[k])
-    lam = np64(g["lambdas"])
-    errs["resid_lambda"] = scalar_err(lam[0], rg["resid_lambda"], rg["_scale"]["resid_lambda"])
-    errs["x0_lambda"] = scalar_err(lam[1], rg["x0_lambda"], rg["_scale"]["x0_lambda"])
+    ref = oracle_block(c, lw, inp, layer, f8)
+    errs = block_errors(x_out, dx, dx0, g, *ref)
     assert ("ve_table" in errs) == bool(c["has_ve"][layer])
-    tol = TOL[c["dtype"]]
-    bad = {k: v for k, v in errs.items() if not v <= tol}
+    gpu_exact = ref_exact = None
+    if f8:  # the FP8 envelope (tests/helpers.py): distances to the exact block
+        exact = oracle_block(c, lw, inp, layer, False)
+        gpu_exact = block_errors(x_out, dx, dx0, g, *exact)
+        y, rdx, rdx0, rg = ref
+        ref_exact = block_errors(y, rdx, rdx0, {k: v for k, v in rg.items() if k != "_scale"} | {"lambdas": [
+            rg["resid_lambda"], rg["x0_lambda"]]}, *exact)
+    bad = judge(errs, TOL[c["dtype"]], gpu_exact, ref_exact)
     assert not bad, (bad, errs)
 
 

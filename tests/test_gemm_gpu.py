@@ -60,3 +60,27 @@ def test_gemm_rejects_misaligned(cuda_lib):
     C = torch.zeros(64, 64, dtype=torch.float32, device="cuda")
     with pytest.raises(gb.GPTBError):
         gb.gptb_gemm_bf16(A, 0, 100 - 1, A, 0, 100, C, 1, 64, 64, 64, 96)
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (304, 272, 208), (1008, 528, 1536)])
+@pytest.mark.parametrize("e5m2", [False, True])
+def test_gemm_fp8_matches_oracle_product(cuda_lib, a_mn, b_mn, M, N, K, e5m2):
+    """The FP8 tensor-core GEMM (single-CTA and CTA-pair forms, every layout
+    the block uses, e4m3 or e5m2 A) against the oracle's quantised product of
+    the same bf16 operands: identical codes, so only the fp32 accumulation
+    order differs."""
+    from oracle import fp8 as of
+    gb = cuda_lib
+    g = torch.Generator().manual_seed(M + N + K + (7 if e5m2 else 0))
+    A = _mk((M, K), g)
+    B = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    a, b = A.double().numpy(), B.double().numpy()
+    ref = of.fp8_matmul_grad(a, b.T) if e5m2 else of.fp8_matmul(a, b.T)
+    As = (A.t().contiguous() if a_mn else A).cuda()
+    Bs = (B.t().contiguous() if b_mn else B).cuda()
+    C = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    gb.gptb_gemm_fp8(As, a_mn, M if a_mn else K, Bs, b_mn, N if b_mn else K, C, N, M, N, K, e5m2)
+    torch.cuda.synchronize()
+    assert gb.gptb_device_error() == 0
+    assert relerr(C.cpu().double().numpy(), ref) < 1e-5

@@ -6,7 +6,7 @@ import torch
 
 import synth
 from oracle import model as om
-from helpers import TOL, fp8_mode, np64, oracle_weights, relerr, scalar_err, small_bf16
+from helpers import TOL, fp8_mode, judge, np64, oracle_weights, relerr, scalar_err, small_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -46,13 +46,8 @@ def run_stack(gb, c, w, batch):
     return loss.item(), st.g
 
 
-def compare_stack(c, w, batch, loss, g, layers=None, top=("wte", "w_lm", "w_smear_gate", "smear_lambda",
-                                                          "backout_lambda")):
-    ow = oracle_weights(w)
-    f8 = fp8_mode(c)
-    rl, cache = om.stack_forward(c, ow, batch["idx"].numpy(), batch["targets"].numpy(), fp8=f8)
-    rg = om.stack_backward(c, ow, cache, batch["idx"].numpy(), fp8=f8)
-    tol = TOL[c["dtype"]]
+def stack_errors(loss, g, rl, rg, top, layers):
+    """Per-output errors of a stack step's results against one oracle evaluation."""
     errs = {"loss": abs(loss - rl) / abs(rl)}
     for k in ("wte", "w_lm", "w_smear_gate"):
         if k in rg and k in top:
@@ -71,7 +66,33 @@ def compare_stack(c, w, batch, loss, g, layers=None, top=("wte", "w_lm", "w_smea
                 errs[f"L{i}.{k}"] = scalar_err(lam[0 if k == "resid_lambda" else 1], v, lg["_scale"][k])
             else:
                 errs[f"L{i}.{k}"] = relerr(np64(g["layers"][i][k]), v)
-    bad = {k: v for k, v in errs.items() if not v <= tol}
+    return errs
+
+
+def _as_grads(rg):
+    """An oracle gradient tree in the layout of the GPU's (lambdas as pairs)."""
+    g = {k: (np.array([v]) if isinstance(v, float) else v) for k, v in rg.items() if k not in ("layers", "_scale")}
+    g["layers"] = [dict({k: v for k, v in lg.items() if k not in ("_scale", "resid_lambda", "x0_lambda")},
+                        lambdas=np.array([lg["resid_lambda"], lg["x0_lambda"]])) for lg in rg["layers"]]
+    return g
+
+
+def compare_stack(c, w, batch, loss, g, layers=None, top=("wte", "w_lm", "w_smear_gate", "smear_lambda",
+                                                          "backout_lambda")):
+    ow = oracle_weights(w)
+    f8 = fp8_mode(c)
+    idx, tg = batch["idx"].numpy(), batch["targets"].numpy()
+    rl, cache = om.stack_forward(c, ow, idx, tg, fp8=f8)
+    rg = om.stack_backward(c, ow, cache, idx, fp8=f8)
+    errs = stack_errors(loss, g, rl, rg, top, layers)
+    gpu_exact = ref_exact = None
+    if f8:  # the FP8 envelope: distances to the exact (non-FP8) stack
+        c0 = dict(c, fp8_lm_head=False)
+        rl0, cache0 = om.stack_forward(c0, ow, idx, tg, fp8=False)
+        rg0 = om.stack_backward(c0, ow, cache0, idx, fp8=False)
+        gpu_exact = stack_errors(loss, g, rl0, rg0, top, layers)
+        ref_exact = stack_errors(rl, _as_grads(rg), rl0, rg0, top, layers)
+    bad = judge(errs, TOL[c["dtype"]], gpu_exact, ref_exact)
     assert not bad, (bad, errs)
     return errs
 
@@ -158,10 +179,12 @@ def test_lm_head_fp8(cuda_lib, grad):
     torch.cuda.synchronize()
     assert cuda_lib.gptb_device_error() == 0
     rl, rdh, rdw = om.lm_head_xent(np64(h), np64(w), y.numpy(), fp8=fp8_mode(c))
-    tol = TOL["fp8"]
-    assert abs(loss.item() - rl) / abs(rl) <= tol
-    assert relerr(np64(dh), rdh) <= tol
-    assert relerr(np64(dw), rdw) <= tol
+    l0, dh0, dw0 = om.lm_head_xent(np64(h), np64(w), y.numpy())
+    errs = {"loss": abs(loss.item() - rl) / abs(rl), "dh": relerr(np64(dh), rdh), "dw": relerr(np64(dw), rdw)}
+    gpu_exact = {"loss": abs(loss.item() - l0) / abs(l0), "dh": relerr(np64(dh), dh0), "dw": relerr(np64(dw), dw0)}
+    ref_exact = {"loss": abs(rl - l0) / abs(l0), "dh": relerr(rdh, dh0), "dw": relerr(rdw, dw0)}
+    bad = judge(errs, TOL["fp8"], gpu_exact, ref_exact)
+    assert not bad, (bad, errs)
 
 
 def test_lm_head_out_of_range_targets_are_reported(cuda_lib):
