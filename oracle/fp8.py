@@ -50,16 +50,33 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     return np.copysign(y, x)
 
 
-def fp8_scale(t: np.ndarray) -> float:
-    """Per-tensor scale: 448 / max|t| (a floor keeps an all-zero tensor finite)."""
-    amax = float(np.max(np.abs(t))) if t.size else 0.0
-    return E4M3_MAX / max(amax, 1e-12)
+# Where floating point decides an FP8 code, the decision is taken in single
+# precision, the precision of the quantising kernel: the tensor's values and
+# amax in fp32, the scale qmax / amax as one correctly rounded fp32 division,
+# each product value * scale rounded to fp32, and that fp32 value rounded to
+# the FP8 format.  (A value exactly on an FP8 midpoint otherwise rounds one way
+# in fp32 and the other in fp64.)  Dequantisation and accumulation stay fp64.
+
+def _f32(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float32)
+
+
+def fp8_scale(t: np.ndarray, qmax: float = E4M3_MAX) -> float:
+    """Per-tensor scale qmax / max|t| in fp32 (a floor keeps an all-zero tensor finite)."""
+    t32 = _f32(t)
+    amax = np.float32(np.max(np.abs(t32))) if t32.size else np.float32(0.0)
+    return float(np.float32(qmax) / np.maximum(amax, np.float32(1e-12)))
+
+
+def _scaled(t: np.ndarray, s: float) -> np.ndarray:
+    """fp32 products t * s (s an fp32 value), as fp64."""
+    return (_f32(t) * np.float32(s)).astype(np.float64)
 
 
 def quantize_e4m3(t: np.ndarray) -> tuple[np.ndarray, float]:
     """Return (codes as fp64 values, scale) with t ~= codes / scale."""
     s = fp8_scale(t)
-    return e4m3_round(np.asarray(t, dtype=np.float64) * s), s
+    return e4m3_round(_scaled(t, s)), s
 
 
 def fp8_matmul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
@@ -92,11 +109,9 @@ def e5m2_round(x: np.ndarray) -> np.ndarray:
 
 
 def quantize_e5m2(t: np.ndarray) -> tuple[np.ndarray, float]:
-    """Return (codes as fp64 values, scale) with t ~= codes / scale, scale = 57344 / amax."""
-    t = np.asarray(t, dtype=np.float64)
-    amax = float(np.max(np.abs(t))) if t.size else 0.0
-    s = E5M2_MAX / max(amax, 1e-12)
-    return e5m2_round(t * s), s
+    """Return (codes as fp64 values, scale) with t ~= codes / scale, scale = 57344 / amax (fp32)."""
+    s = fp8_scale(t, E5M2_MAX)
+    return e5m2_round(_scaled(t, s)), s
 
 
 def fp8_matmul_grad(g: np.ndarray, w: np.ndarray) -> np.ndarray:
@@ -110,6 +125,14 @@ def fp8_matmul_grad(g: np.ndarray, w: np.ndarray) -> np.ndarray:
 # ------------------------------------------------- fixed-scale quantisation
 def quantize_fixed(t: np.ndarray, scale: float, fmt: str = "e4m3") -> np.ndarray:
     """Codes (as fp64 values) of t * scale rounded to e4m3 or e5m2, for a tensor
-    whose per-tensor scale is known in advance rather than measured."""
+    whose per-tensor scale is known in advance rather than measured (scale an
+    fp32 value; the product is rounded to fp32 first, as above)."""
     r = e4m3_round if fmt == "e4m3" else e5m2_round
-    return r(np.asarray(t, dtype=np.float64) * scale)
+    return r(_scaled(t, scale))
+
+
+def bound_scale(qmax: float, n: int) -> float:
+    """The fp32 scale qmax / (1/n) of a tensor bounded by 1/n in magnitude:
+    1/n rounded to fp32, then one fp32 division."""
+    inv_n = np.float32(1.0) / np.float32(n)
+    return float(np.float32(qmax) / inv_n)

@@ -21,15 +21,17 @@ gradient operand of the input-gradient and weight-gradient products to e5m2
 the lm_head products in FP8: the logits from e4m3 casts of hf and W_lm, and
 the two gradient products from the logits gradient dz, whose entries
 (softmax - onehot)/n lie in [-1/n, 1/n], quantised with the per-tensor
-scale that bound fixes (448 n, or 57344 n for e5m2), so that splitting the
-rows into chunks does not change the product.  Without ``fp8_lm_head`` the
+scale that bound fixes (448 n, or 57344 n for e5m2, formed in fp32 as
+qmax / fp32(1/n)), so that splitting the rows into chunks does not change
+the product.  Without ``fp8_lm_head`` the
 lm_head stays exact.
 """
 from __future__ import annotations
 
 import numpy as np
 
-from .fp8 import E4M3_MAX, E5M2_MAX, bf16_round, fp8_matmul, fp8_matmul_grad, quantize_e4m3, quantize_fixed
+from .fp8 import (E4M3_MAX, E5M2_MAX, bf16_round, bound_scale, fp8_matmul, fp8_matmul_grad, quantize_e4m3,
+                  quantize_fixed)
 
 
 def _f64(a) -> np.ndarray:
@@ -338,7 +340,7 @@ def lm_head_xent(h, w_lm, targets, fp8=False):
         return loss, (dz @ w).reshape(h.shape), dz.T @ hf
     # |dz| <= 1/n fixes the per-tensor scale of the logits gradient
     fmt = "e5m2" if fp8 == "e5m2" else "e4m3"
-    s_dz = (E5M2_MAX if fmt == "e5m2" else E4M3_MAX) * n
+    s_dz = bound_scale(E5M2_MAX if fmt == "e5m2" else E4M3_MAX, n)
     qdz = quantize_fixed(bf16_round(dz), s_dz, fmt)
     qw, sw = quantize_e4m3(bf16_round(w))
     qh, sh = quantize_e4m3(bf16_round(hf))
