@@ -1,7 +1,7 @@
 // Attention forward on the 5th-generation tensor cores (tcgen05 + TMEM), bf16,
 // hd = 128.  Same math as attention.cuh (causal GQA, sliding window, LSE).
 //
-// CTA = 128 queries of one head; 10 warps:
+// CTA = 128 queries of one head; 2 + 4*SPLIT warps (SPLIT = 2: 10 warps):
 //   warp 0    TMA producer: Q once, then K and V tiles of 128 keys into two
 //             2-stage rings (a K slot is refilled once its S MMA is done, a V
 //             slot once its PV MMA is done; all loads are 64-column boxes of
@@ -32,11 +32,20 @@
 namespace gptb {
 
 constexpr int FA_BM = 128, FA_BN = 128;
-constexpr int FA_THREADS = 320;
-constexpr int FA_SOFTMAX_THREADS = 256;
 constexpr int FA_TILE = 128 * 128 * 2;  // one 128x128 bf16 tile: 32 KB (two 64-column swizzled halves)
-constexpr int FA_SMEM = 1024 /*align*/ + FA_TILE /*Q*/ + 4 * FA_TILE /*K,V x2*/ + 256 /*barriers*/ +
-                        2 * 2 * 128 * 4 /*row max exchange, 2 tiles in flight*/ + 2 * 128 * 4 /*row sums*/;
+// SPLIT softmax warps per TMEM lane quarter, each owning 128/SPLIT keys of a
+// row (and 128/SPLIT columns of O); 2 + 4*SPLIT warps in all
+template <int SPLIT> struct FaShape {
+  static constexpr int SOFTMAX_THREADS = 128 * SPLIT;
+  static constexpr int THREADS = 64 + SOFTMAX_THREADS;
+  static constexpr int KPW = 128 / SPLIT;  // keys (and O columns) per softmax thread
+  static constexpr int SMEM = 1024 /*align*/ + FA_TILE /*Q*/ + 4 * FA_TILE /*K,V x2*/ + 256 /*barriers*/ +
+                              2 * SPLIT * 128 * 4 /*row max exchange, 2 tiles in flight*/ +
+                              SPLIT * 128 * 4 /*row sums*/;
+};
+#ifndef GPTB_FA_SPLIT
+#define GPTB_FA_SPLIT 2
+#endif
 
 
 // K-major SW128 descriptor of a 128-row tile, k-th 16-element K step
@@ -48,9 +57,13 @@ __device__ __forceinline__ uint64_t fa_desc_mn(uint32_t tile, int k) {
   return smem_desc_sw128(tile + (uint32_t)(k * 2048), 16384, 1024);
 }
 
-__global__ void __launch_bounds__(FA_THREADS, 1)
+template <int SPLIT>
+__global__ void __launch_bounds__(FaShape<SPLIT>::THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ o, long long ldo,
                        float* __restrict__ lse, int T, int H, int Hkv, int window, unsigned int* __restrict__ amax_o) {
+  constexpr int FA_SOFTMAX_THREADS = FaShape<SPLIT>::SOFTMAX_THREADS;
+  constexpr int KPW = FaShape<SPLIT>::KPW;
+  constexpr int NSW = 4 * SPLIT;  // softmax warps
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -69,8 +82,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   uint64_t* v_empty = bars + 16;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xmax = reinterpret_cast<float*>(bars + 32);  // [2 tile parities][2 halves][128 rows] (after 256 B of barriers)
-  float* xsum = xmax + 2 * 2 * 128;                   // [2 halves][128 rows]
+  float* xmax = reinterpret_cast<float*>(bars + 32);  // [2 tile parities][SPLIT parts][128 rows] (after 256 B of barriers)
+  float* xsum = xmax + 2 * SPLIT * 128;               // [SPLIT parts][128 rows]
 
   const int nqb = (T + FA_BM - 1) / FA_BM;
   const int qb = nqb - 1 - (int)blockIdx.x;  // heavy (late) query tiles first
@@ -91,8 +104,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 8);
-      mbar_init(&p_full[i], 8);
+      mbar_init(&s_empty[i], NSW);
+      mbar_init(&p_full[i], NSW);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -169,7 +182,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     }
   } else {
     // softmax warps: TMEM lane quarter qw = warp % 4 -> query rows 32*qw ..
-    // 32*qw+31; half hf -> score / output columns 64*hf .. 64*hf+63
+    // 32*qw+31; part hf (0..SPLIT-1) -> score / output columns KPW*hf .. KPW*hf+KPW-1
+    constexpr int NCH = KPW / 32;  // 32-column TMEM chunks per thread
     const int qw = warp & 3;
     const int hf = (warp - 2) >> 2;
     const int r = qw * 32 + lane;  // row within the tile
@@ -187,16 +201,17 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     // warp can be left waiting at a barrier that another warp never reaches.
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
-      const int k0 = (kb_lo + j) * FA_BN + hf * 64;  // first key of this half
+      const int k0 = (kb_lo + j) * FA_BN + hf * KPW;  // first key of this part
       ok = ok && mbar_wait_warp(&s_full[sb], (j >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
       tc_fence_after();
-      const bool need_mask = (k0 + 63 > q0) || (k0 + 64 > T) || (window >= 0 && q0 + FA_BM - 1 - k0 > window);
-      // both 32-column chunks of this half go to registers at once; the score
-      // buffer is released right after, so the next-but-one S MMA can start
-      uint32_t v[64];
+      const bool need_mask = (k0 + KPW - 1 > q0) || (k0 + KPW > T) || (window >= 0 && q0 + FA_BM - 1 - k0 > window);
+      // every chunk of this part goes to registers at once; the score buffer is
+      // released right after, so the next-but-one S MMA can start
+      uint32_t v[KPW];
       if (ok) {
-        tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * KPW + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
         tmem_ld_wait();
       }
       tc_fence_before();
@@ -205,22 +220,25 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       // masked scores become -inf; visible keys of row t: kv_lo..kv_hi
       if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < KPW; ++i) {
           const int jk = k0 + i;
           v[i] = (jk >= kv_lo && jk <= kv_hi) ? v[i] : __float_as_uint(-INFINITY);
         }
       }
       float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mp[i & 3] = fmaxf(mp[i & 3], __uint_as_float(v[i]));
-      float* xm = xmax + sb * 256;
+      for (int i = 0; i < KPW; ++i) mp[i & 3] = fmaxf(mp[i & 3], __uint_as_float(v[i]));
+      float* xm = xmax + sb * SPLIT * 128;
       xm[hf * 128 + r] = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
       named_bar_sync(1, FA_SOFTMAX_THREADS);
-      const float mx = fmaxf(xm[r], xm[128 + r]) * sl2;
+      float mxr = xm[r];
+#pragma unroll
+      for (int p = 1; p < SPLIT; ++p) mxr = fmaxf(mxr, xm[p * 128 + r]);
+      const float mx = mxr * sl2;
       // P buffer j&1 was last read by the PV product of tile j-2
       if (j > 1) ok = ok && mbar_wait_warp(&pv_done[sb], ((j >> 1) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_EPILOGUE);
       if (!ok) continue;
-      // rescale decision is per row (identical in both halves) but the TMEM
+      // rescale decision is per row (identical in every part) but the TMEM
       // accesses are warp-collective: the whole warp enters, rows that keep
       // their max use a factor of 1
       const bool grow = mx > m_used + 8.f;
@@ -232,13 +250,13 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           if (!ok) continue;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(lane_addr + 256 + hf * 64 + c * 32, v);
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t w[32];
+            tmem_ld_32x32b_x32(lane_addr + 256 + hf * KPW + c * 32, w);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * corr);
-            tmem_st_32x32b_x32(lane_addr + 256 + hf * 64 + c * 32, v);
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * corr);
+            tmem_st_32x32b_x32(lane_addr + 256 + hf * KPW + c * 32, w);
           }
           tmem_st_wait();
         }
@@ -249,11 +267,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
       // pass 2: P = exp2(s*scale - m) as bf16 pairs (key 2c in the low half)
-      // into TMEM columns 384 + 64*(j&1) + 32*hf .. +31 of this row's lane
-      uint32_t pk[32];
+      // into TMEM columns 384 + 64*(j&1) + (KPW/2)*hf .. of this row's lane
+      uint32_t pk[KPW / 2];
       float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < KPW / 2; ++c) {
         const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * c]), sl2, -mu));  // exp2(-inf) = 0 for masked keys
         const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * c + 1]), sl2, -mu));
         lp[(2 * c) & 3] += p0;
@@ -261,38 +279,44 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         pk[c] = pack_bf16(p0, p1);
       }
       l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-      tmem_st_32x32b_x32(lane_addr + 384 + sb * 64 + hf * 32, pk);
+      if constexpr (KPW == 64) {
+        tmem_st_32x32b_x32(lane_addr + 384 + sb * 64 + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      } else {
+        tmem_st_32x32b_x16(lane_addr + 384 + sb * 64 + hf * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    // the two halves' sums share the same running max: add them
+    // every part's sum shares the same running max: add them
     xsum[hf * 128 + r] = l;
     named_bar_sync(1, FA_SOFTMAX_THREADS);
-    const float lt = xsum[r] + xsum[128 + r];
+    float lt = 0.f;
+#pragma unroll
+    for (int p = 0; p < SPLIT; ++p) lt += xsum[p * 128 + r];
     if (__all_sync(0xffffffffu, ok) &&
         mbar_wait_warp(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
       tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      bf16* orow = o + ((long long)b * T + t) * ldo + h * 128 + hf * 64;
+      bf16* orow = o + ((long long)b * T + t) * ldo + h * 128 + hf * KPW;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_addr + 256 + hf * 64 + c * 32, v);
+      for (int c = 0; c < NCH; ++c) {
+        uint32_t w[32];
+        tmem_ld_32x32b_x32(lane_addr + 256 + hf * KPW + c * 32, w);
         tmem_ld_wait();
         if (t < T) {
           if (amax_o) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) oam = fmaxf(oam, fabsf(__uint_as_float(v[i]) * inv));
+            for (int i = 0; i < 32; ++i) oam = fmaxf(oam, fabsf(__uint_as_float(w[i]) * inv));
           }
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             uint4 u;
-            u.x = pack_bf16(__uint_as_float(v[g * 8 + 0]) * inv, __uint_as_float(v[g * 8 + 1]) * inv);
-            u.y = pack_bf16(__uint_as_float(v[g * 8 + 2]) * inv, __uint_as_float(v[g * 8 + 3]) * inv);
-            u.z = pack_bf16(__uint_as_float(v[g * 8 + 4]) * inv, __uint_as_float(v[g * 8 + 5]) * inv);
-            u.w = pack_bf16(__uint_as_float(v[g * 8 + 6]) * inv, __uint_as_float(v[g * 8 + 7]) * inv);
+            u.x = pack_bf16(__uint_as_float(w[g * 8 + 0]) * inv, __uint_as_float(w[g * 8 + 1]) * inv);
+            u.y = pack_bf16(__uint_as_float(w[g * 8 + 2]) * inv, __uint_as_float(w[g * 8 + 3]) * inv);
+            u.z = pack_bf16(__uint_as_float(w[g * 8 + 4]) * inv, __uint_as_float(w[g * 8 + 5]) * inv);
+            u.w = pack_bf16(__uint_as_float(w[g * 8 + 6]) * inv, __uint_as_float(w[g * 8 + 7]) * inv);
             *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = u;
           }
         }
@@ -306,7 +330,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       named_bar_sync(1, FA_SOFTMAX_THREADS);
       if (warp == 2 && lane == 0) {
         float mm = 0.f;
-        for (int w = 0; w < FA_SOFTMAX_THREADS / 32; ++w) mm = fmaxf(mm, xsum[w]);
+        for (int w = 0; w < NSW; ++w) mm = fmaxf(mm, xsum[w]);
         atomicMax(amax_o, __float_as_uint(stored_abs_max_bf16(mm)));
       }
     }
