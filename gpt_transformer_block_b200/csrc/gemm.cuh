@@ -588,8 +588,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = fmaf(beta, a[i], v[i]);
               } else if (ep.kind == EPI_DRELU2) {
+                // 2 relu(u) = 2 sqrt(a) as a * rsqrt(a) (one MUFU op; the IEEE
+                // sqrt's zero-input path would be taken for every a = 0)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= 2.f * sqrtf(fmaxf(a[i], 0.f));
+                for (int i = 0; i < 8; ++i) v[i] *= (a[i] > 0.f) ? 2.f * a[i] * rsqrtf(a[i]) : 0.f;
               } else {
                 // the dot takes the values as stored (rounded to bf16)
 #pragma unroll
