@@ -163,7 +163,11 @@ constexpr int TC_BN = 256;   // columns of D per CTA (one TMEM accumulator)
 constexpr int TC_THREADS = 192;
 constexpr int TC_GROUP_M = 8;
 
-constexpr int TC_EPI_BYTES = 4 * 8192;  // per epilogue warp: two 32-row x 128-byte staging tiles
+// per epilogue warp: four 32-row x 128-byte staging tiles (two output tiles
+// written alternately, so a chunk's store overlaps the next chunk, and two
+// input tiles of the residual / saved activation, loaded one chunk ahead)
+constexpr int TC_EPI_TILE = 4096;
+constexpr int TC_EPI_BYTES = 4 * 4 * TC_EPI_TILE;
 
 // Tile shape of the two kernel forms.
 //   single: one CTA computes a 128 x 256 tile (A 128 rows, B 256 rows per stage)
@@ -174,11 +178,12 @@ constexpr int TC_EPI_BYTES = 4 * 8192;  // per epilogue warp: two 32-row x 128-b
 template <bool PAIR> struct TcShape {
   static constexpr int TILE_M = PAIR ? 256 : 128;
   static constexpr int B_ROWS = PAIR ? 128 : 256;
-  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int STAGES = PAIR ? 5 : 3;
   static constexpr int A_BYTES = TC_BM * 128;
   static constexpr int B_BYTES = B_ROWS * 128;
   // stages * (A + B) + epilogue staging + barriers + 1 KB alignment slack
   static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES) + TC_EPI_BYTES + 256 + 1024;
+  static_assert(SMEM <= 232448, "GEMM shared memory above the per-CTA limit");
 };
 
 __device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, int& tm, int& tn, int& split) {
@@ -303,8 +308,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* aux_bar = drain + 1;  // [4] one per epilogue warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + 4);
+  uint64_t* aux_bar = drain + 1;  // [8] two per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux_bar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -328,7 +333,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&tempty[b], PAIR ? 8 : 4);  // the epilogue warps of both CTAs drain an accumulator
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&aux_bar[i], 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&aux_bar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -483,13 +488,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint8_t* stg0 = sEpi + (warp - 2) * 8192;  // this warp's two staging tiles
-    uint8_t* stg1 = stg0 + 4096;
-    uint64_t* abar = &aux_bar[warp - 2];
-    uint32_t aphase = 0;
+    uint8_t* ebuf = sEpi + (warp - 2) * (4 * TC_EPI_TILE);  // this warp's four staging tiles
+    uint64_t* abar = &aux_bar[(warp - 2) * 2];
     const bool has_aux = (ep.kind == EPI_RESID || ep.kind == EPI_DRELU2 || ep.kind == EPI_DOT);
     const bool acc32 = (ep.kind == EPI_ACCUM_F32);
     const int swz = (lane & 7);  // 16-byte chunk swizzle of this lane's 128-byte staging row
+    // Staging tiles: bf16 output chunks alternate between tiles 0 and 1, and
+    // the input chunks (residual, saved activation, O) between tiles 2 and 3;
+    // fp32 chunks and the q/k/v heads take two tiles each, alternating
+    // between tiles 0-1 and 2-3.  Every chunk commits one bulk group, so
+    // waiting until at most one group is still reading frees the tile(s) of
+    // the chunk before last.
+    uint32_t ns = 0;          // bulk groups committed by this warp
+    uint32_t na = 0, nw = 0;  // input-tile loads issued / consumed by this warp
+    auto chunks_of = [&](int tn_) { return min(TC_BN / 64, (N - tn_ * TC_BN + 63) / 64); };
+    // load the input chunk cc_ of unit u_ into the next input tile (lane 0; the count advances on every lane)
+    auto issue_aux = [&](int u_, int cc_) {
+      if (lane == 0) {
+        int tm_, tn_, sp_;
+        tc_unit_coords(u_, tiles_m, tiles_n, tm_, tn_, sp_);
+        uint64_t* bar = &abar[na & 1u];
+        mbar_arrive_expect_tx(bar, TC_EPI_TILE);
+        tma_load_2d(ebuf + (2 + (na & 1u)) * TC_EPI_TILE, &tmX, bar, tn_ * TC_BN + cc_ * 64,
+                    tm_ * SH::TILE_M + (int)rank * TC_BM + q * 32);
+      }
+      ++na;
+    };
+    if (has_aux && unit0 < units) issue_aux(unit0, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     const float alpha = epi_alpha(ep);
@@ -507,54 +532,72 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int hb = 0; hb < TC_BN / 128; ++hb) {
           const int col0 = tn * TC_BN + hb * 128;
           if (col0 >= N) break;  // warp-uniform
-          if (lane == 0) bulk_wait_read0();
+          uint8_t* st0 = ebuf + (ns & 1u) * 2 * TC_EPI_TILE;
+          if (lane == 0) bulk_wait_read1();
           __syncwarp();
           const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + hb * 128);
-          epi_qkv_head(ep, ta, stg0, stg1, lane, alpha, col0 / 128, row0 + lane, row0 + lane < M);
+          epi_qkv_head(ep, ta, st0, st0 + TC_EPI_TILE, lane, alpha, col0 / 128, row0 + lane, row0 + lane < M);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmO, stg0, col0, row0);
-            tma_store_2d(&tmO, stg1, col0 + 64, row0);
+            tma_store_2d(&tmO, st0, col0, row0);
+            tma_store_2d(&tmO, st0 + TC_EPI_TILE, col0 + 64, row0);
             bulk_commit_group();
           }
+          ++ns;
         }
       }
       float dsum = 0.f;  // EPI_DOT: this row's running sum over the current 128-column group
       // EPI_XENT: this row's running max and sum of exp2((z - max) * log2 e) over the tile
       float xm = -INFINITY, xs = 0.f;
       const int xy = (ep.kind == EPI_XENT && row0 + lane < M) ? ep.targets[row0 + lane] : -1;
+      const int nch = (ep.kind == EPI_QKV) ? 0 : chunks_of(tn);
 #pragma unroll 1
-      for (int cc = 0; cc < (ep.kind == EPI_QKV ? 0 : TC_BN / 64); ++cc) {
+      for (int cc = 0; cc < nch; ++cc) {
         const int col0 = tn * TC_BN + cc * 64;
-        if (col0 >= N) break;  // warp-uniform
+        const bool tail = col0 + 64 > N;  // warp-uniform: the last chunk of a ragged N
         uint32_t r0[32], r1[32];
         const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + cc * 64);
         tmem_ld_32x32b_x32(ta, r0);
         tmem_ld_32x32b_x32(ta + 32, r1);
-        // the staging tiles are free once this warp's previous bulk copies have read them
-        if (lane == 0) bulk_wait_read0();
-        __syncwarp();
-        if (has_aux && lane == 0) {
-          mbar_arrive_expect_tx(abar, 4096);
-          tma_load_2d(stg1, &tmX, abar, col0, row0);
-        }
-        tmem_ld_wait();
         if (has_aux) {
-          if (!mbar_wait_warp(abar, aphase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
+          // the next input chunk (of this tile, else of the next unit) goes
+          // into the other input tile, read by the chunk before this one
+          if (cc + 1 < nch) issue_aux(u, cc + 1);
+          else if (u + ustep < units) issue_aux(u + ustep, 0);
+        }
+        // this chunk's output tile(s) are free once the bulk group of the chunk before last has read them
+        if (lane == 0) bulk_wait_read1();
+        __syncwarp();
+        tmem_ld_wait();
+        uint8_t* cur_in = ebuf + (2 + (nw & 1u)) * TC_EPI_TILE;
+        if (has_aux) {
+          if (!mbar_wait_warp(&abar[nw & 1u], (nw >> 1) & 1u, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
             ok = false;
             break;
           }
-          aphase ^= 1u;
+          ++nw;
         }
-        uint8_t* p0 = stg0 + lane * 128;
-        uint8_t* p1 = stg1 + lane * 128;
+        uint8_t* p0 = ebuf + (acc32 ? (ns & 1u) * 2 * TC_EPI_TILE : (ns & 1u) * TC_EPI_TILE) + lane * 128;
+        uint8_t* p1 = acc32 ? p0 + TC_EPI_TILE : cur_in + lane * 128;
         float xml2 = 0.f;  // EPI_XENT: running max * log2 e after this chunk
         if (ep.kind == EPI_XENT) {
-          float cm = xm;
+          // the chunk's max as eight independent chains (columns past N left out)
+          float cm8[8];
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (col0 + i < N) cm = fmaxf(cm, __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
+          for (int j = 0; j < 8; ++j) cm8[j] = xm;
+          if (!tail) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              cm8[i & 7] = fmaxf(cm8[i & 7], __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (col0 + i < N) cm8[i & 7] = fmaxf(cm8[i & 7], __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
+          }
+#pragma unroll
+          for (int j = 1; j < 8; ++j) cm8[0] = fmaxf(cm8[0], cm8[j]);
+          const float cm = cm8[0];
           if (cm > xm) {  // rescale the sum to the new max (0 while the max was -inf)
             xs = (xm == -INFINITY) ? 0.f : xs * fast_exp2((xm - cm) * LOG2E);
             xm = cm;
@@ -573,25 +616,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                             __uint_as_float(r1[4 * g + 2]) * alpha, __uint_as_float(r1[4 * g + 3]) * alpha);
           }
         } else {
-          // bf16: 8 chunks of 8 columns; aux (if any) sits in tile 1 with the same swizzle
+          // bf16: 8 chunks of 8 columns; the input chunk (if any) has the same swizzle
+          float xsum[8];
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
             float v[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(g < 4 ? r0[g * 8 + i] : r1[(g - 4) * 8 + i]) * alpha;
             uint8_t* cp0 = p0 + ((g ^ swz) << 4);
-            uint8_t* cp1 = p1 + ((g ^ swz) << 4);
             if (has_aux) {
               float a[8];
-              load8(reinterpret_cast<const bf16*>(cp1), a);
+              load8(reinterpret_cast<const bf16*>(p1 + ((g ^ swz) << 4)), a);
               if (ep.kind == EPI_RESID) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = fmaf(beta, a[i], v[i]);
               } else if (ep.kind == EPI_DRELU2) {
-                // 2 relu(u) = 2 sqrt(a) as a * rsqrt(a) (one MUFU op; the IEEE
-                // sqrt's zero-input path would be taken for every a = 0)
+                // 2 relu(u) = 2 sqrt(a) as a * rsqrt(a); a below the smallest
+                // normal float (where the flushing rsqrt gives inf) counts as 0
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= (a[i] > 0.f) ? 2.f * a[i] * rsqrtf(a[i]) : 0.f;
+                for (int i = 0; i < 8; ++i) v[i] *= (a[i] >= 1.17549435e-38f) ? 2.f * a[i] * fast_rsqrt(a[i]) : 0.f;
               } else {
                 // the dot takes the values as stored (rounded to bf16)
 #pragma unroll
@@ -599,12 +642,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               }
             }
             if (ep.kind == EPI_XENT) {
-              // columns past N (the last tile's tail) do not take part
               const int c8 = col0 + g * 8;
-              float acc = 0.f;
+              float e[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) acc += (c8 + i < N) ? fast_exp2(fmaf(v[i], LOG2E, -xml2)) : 0.f;
-              xs += acc;
+              for (int i = 0; i < 8; ++i) e[i] = fast_exp2(fmaf(v[i], LOG2E, -xml2));
+              if (tail) {  // columns past N (the last tile's tail) do not take part
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  if (c8 + i >= N) e[i] = 0.f;
+              }
+              xsum[g] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
               if (xy >= c8 && xy < c8 + 8) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
@@ -626,6 +673,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             store8(reinterpret_cast<bf16*>(cp0), v);
           }
+          if (ep.kind == EPI_XENT)
+            xs += ((xsum[0] + xsum[1]) + (xsum[2] + xsum[3])) + ((xsum[4] + xsum[5]) + (xsum[6] + xsum[7]));
         }
         if (ep.kind == EPI_DOT && (cc & 1)) {  // a 128-column group (one head) is complete
           const int row = row0 + lane;
@@ -638,14 +687,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+          uint8_t* t0 = p0 - lane * 128;
           if (acc32) {
-            tma_reduce_add_2d(&tmO, stg0, col0, row0);
-            tma_reduce_add_2d(&tmO, stg1, col0 + 32, row0);
+            tma_reduce_add_2d(&tmO, t0, col0, row0);
+            tma_reduce_add_2d(&tmO, t0 + TC_EPI_TILE, col0 + 32, row0);
           } else {
-            tma_store_2d(&tmO, stg0, col0, row0);
+            tma_store_2d(&tmO, t0, col0, row0);
           }
           bulk_commit_group();
         }
+        ++ns;
       }
       // (a tile cut short by the N tail still covers at least one chunk)
       if (ep.kind == EPI_XENT && ok && row0 + lane < M)
@@ -658,6 +709,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+    }
+    // input-tile loads still in flight (issued ahead of an abort) land before the CTA exits
+    while (nw < na) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(&abar[nw & 1u], (nw >> 1) & 1u)) {
+        if (globaltimer_ns() - t0 > 100000000ull) {
+          record_error(ERRW_TIMEOUT_DRAIN);
+          break;
+        }
+      }
+      ++nw;
     }
     if (lane == 0) bulk_wait0();
     if (ep.amax_out) {

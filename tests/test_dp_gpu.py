@@ -78,11 +78,20 @@ def test_zero2_trainer_world1_matches_direct_updates(cuda_lib):
                 gb.gptb_muon_step(master, pb, g, torch.zeros_like(master), torch.zeros(m, device="cuda"), m, n,
                                   coeffs, hp["lr_muon"], hp["momentum"], hp["beta2_muon"], hp["weight_decay"], ws)
                 torch.cuda.synchronize()
-                # NorMuon's two sums use float atomics: a last-bit difference may
-                # move a bf16 rounding
-                got, base = tr.param(s.name).double().cpu(), p0.double().cpu()
-                err = relerr((got - base).numpy(), (pb.double().cpu() - base).numpy())
-                assert err <= 1e-2, (s.name, err)
+                st = tr.state[s.name]
+                # the reduced bf16 gradient reached the Muon step: with a zero
+                # buffer the momentum update leaves exactly that gradient
+                assert torch.equal(st["buf"], g), s.name
+                # NorMuon's two sums are float atomics, so the fp32 masters may
+                # differ in the last bits; the update they received agrees to
+                # far below the bf16 tolerance
+                err = relerr((st["master"] - p0.float()).double().cpu().numpy(),
+                             (master - p0.float()).double().cpu().numpy())
+                assert err <= 1e-4, (s.name, err)
+                # and the bf16 working weight is the rounding of the trainer's own
+                # master (a last-bit master difference may move that rounding by
+                # one step against the direct call's, so it is not compared)
+                assert torch.equal(tr.param(s.name), st["master"].bfloat16()), s.name
     finally:
         dist.destroy_process_group()
 
