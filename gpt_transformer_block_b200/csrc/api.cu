@@ -714,9 +714,8 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     // over the packed qkv buffer serves the Q, K and V tiles
     CUtensorMap tq;
     if (!make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128)) return GPTB_ERR_CUDA;
-    using FS = FaShape<GPTB_FA_SPLIT>;
-    CK(cudaFuncSetAttribute(attn_fwd_tc_kernel<GPTB_FA_SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, FS::SMEM));
-    attn_fwd_tc_kernel<GPTB_FA_SPLIT><<<dim3((m.T + FA_BM - 1) / FA_BM, m.H, m.B), FS::THREADS, FS::SMEM, st>>>(
+    CK(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM));
+    attn_fwd_tc_kernel<<<(unsigned)(((m.T + FA_QB - 1) / FA_QB) * m.H * m.B), FA_THREADS, FA_SMEM, st>>>(
         tq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W, am ? am + 1 : nullptr);
     CKL();
   }

@@ -1,31 +1,33 @@
 // Attention forward on the 5th-generation tensor cores (tcgen05 + TMEM), bf16,
 // hd = 128.  Same math as attention.cuh (causal GQA, sliding window, LSE).
 //
-// CTA = 128 queries of one head; 2 + 4*SPLIT warps (SPLIT = 2: 10 warps):
-//   warp 0    TMA producer: Q once, then K and V tiles of 128 keys into two
-//             2-stage rings (a K slot is refilled once its S MMA is done, a V
-//             slot once its PV MMA is done; all loads are 64-column boxes of
-//             the packed qkv buffer, 128-byte swizzle)
-//   warp 1    TMEM owner + single-thread MMA issuer:
-//               S_j = Q K_j^T   (M=128, N=128, K=128) into one of two TMEM
-//                               score buffers (columns 0..127 / 128..255)
-//               O  += P_j V_j   (M=128, N=128, K=128; P read from TMEM,
-//                               V as MN-major smem operand) into TMEM
-//                               columns 256..383
-//             S_{j+1} is issued before O += P_j V_j so the scores of the next
-//             tile are ready when the softmax finishes the current one.
-//   warps 2-9 softmax: two warps per TMEM lane quarter; thread = one query
-//             row (its TMEM lane) and one half (64 keys) of the score tile.
-//             Masks (causal / window / sequence end), combines the two halves'
-//             row max through shared memory, keeps a running max in base 2 and
-//             rescales O in TMEM only when the max grows by more than 8 (a
-//             factor 256; P stays below 256 in bf16 and the final
+// CTA = two tiles of 128 queries (256 consecutive queries) of one head; 10 warps:
+//   warp 0    TMA producer: both query tiles once, then K and V tiles of 128
+//             keys into two 2-stage rings (64-column boxes of the packed qkv
+//             buffer, 128-byte swizzle).  A K slot is refilled once every
+//             score product that reads it is done, a V slot once every PV
+//             product is.
+//   warp 1    TMEM owner + single-thread MMA issuer.  For query tile t and key tile j:
+//               S_t  = Q_t K_j^T  (M=128, N=128, K=128) into TMEM columns 128t .. 128t+127
+//               O_t += P_t V_j    (M=128, N=128, K=128; P_t read from TMEM, V an
+//                                 MN-major smem operand) into columns 256+128t ..
+//             P_t (bf16 pairs) overwrites the first 64 columns of S_t: the
+//             products of one thread run in issue order, so the next S_t,
+//             issued after the PV product that reads P_t, cannot overwrite it
+//             early.  Issue order S_0 S_1 | PV_0 S_0' | PV_1 S_1' | ...: the
+//             tensor core works on one tile's products while the other
+//             tile's softmax runs.
+//   warps 2-5 softmax of query tile 0, warps 6-9 of query tile 1: thread =
+//             one query row (its TMEM lane) over all 128 keys of the key tile,
+//             so the row max needs no exchange between threads.  Masks
+//             (causal / window / sequence end), keeps a running max in base 2
+//             and rescales O_t in TMEM only when the max grows by more than 8
+//             (a factor 256; P stays below 256 in bf16 and the final
 //             normalisation uses the same max, so the result is exact), writes
-//             P (bf16 pairs) into one of two TMEM buffers (columns 384..447 /
-//             448..511), the A operand of the PV MMA, so P costs no shared-
-//             memory bandwidth, and at the end normalises its half of O and
-//             writes o and the LSE.
-// Only key tiles that intersect [q0 - W, q0 + 127] are visited.
+//             P_t, and at the end normalises O_t and writes o and the LSE.
+// Only key tiles that intersect a query tile's visible range are visited.
+// The grid is one-dimensional and ordered longest-first (see the CTA index
+// mapping).
 #pragma once
 #include "common.cuh"
 
@@ -33,20 +35,9 @@ namespace gptb {
 
 constexpr int FA_BM = 128, FA_BN = 128;
 constexpr int FA_TILE = 128 * 128 * 2;  // one 128x128 bf16 tile: 32 KB (two 64-column swizzled halves)
-// SPLIT softmax warps per TMEM lane quarter, each owning 128/SPLIT keys of a
-// row (and 128/SPLIT columns of O); 2 + 4*SPLIT warps in all
-template <int SPLIT> struct FaShape {
-  static constexpr int SOFTMAX_THREADS = 128 * SPLIT;
-  static constexpr int THREADS = 64 + SOFTMAX_THREADS;
-  static constexpr int KPW = 128 / SPLIT;  // keys (and O columns) per softmax thread
-  static constexpr int SMEM = 1024 /*align*/ + FA_TILE /*Q*/ + 4 * FA_TILE /*K,V x2*/ + 256 /*barriers*/ +
-                              2 * SPLIT * 128 * 4 /*row max exchange, 2 tiles in flight*/ +
-                              SPLIT * 128 * 4 /*row sums*/;
-};
-#ifndef GPTB_FA_SPLIT
-#define GPTB_FA_SPLIT 2
-#endif
-
+constexpr int FA_QB = 2 * FA_BM;        // queries per CTA
+constexpr int FA_THREADS = 320;
+constexpr int FA_SMEM = 1024 /*align*/ + 2 * FA_TILE /*Q tiles*/ + 4 * FA_TILE /*K,V x2*/ + 256 /*barriers*/;
 
 // K-major SW128 descriptor of a 128-row tile, k-th 16-element K step
 __device__ __forceinline__ uint64_t fa_desc_k(uint32_t tile, int k) {
@@ -57,42 +48,48 @@ __device__ __forceinline__ uint64_t fa_desc_mn(uint32_t tile, int k) {
   return smem_desc_sw128(tile + (uint32_t)(k * 2048), 16384, 1024);
 }
 
-template <int SPLIT>
-__global__ void __launch_bounds__(FaShape<SPLIT>::THREADS, 1)
+__global__ void __launch_bounds__(FA_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ o, long long ldo,
                        float* __restrict__ lse, int T, int H, int Hkv, int window, unsigned int* __restrict__ amax_o) {
-  constexpr int FA_SOFTMAX_THREADS = FaShape<SPLIT>::SOFTMAX_THREADS;
-  constexpr int KPW = FaShape<SPLIT>::KPW;
-  constexpr int NSW = 4 * SPLIT;  // softmax warps
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + FA_TILE;          // 2 stages
-  uint8_t* sV = sK + 2 * FA_TILE;      // 2 stages
+  uint8_t* sQ = smem;                // 2 query tiles
+  uint8_t* sK = sQ + 2 * FA_TILE;    // 2 stages
+  uint8_t* sV = sK + 2 * FA_TILE;    // 2 stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * FA_TILE);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]  K ring: a slot is free once S_j = Q K_j^T is done
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_empty = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;    // [2]  P buffer j&1 written
-  uint64_t* pv_done = bars + 11;  // [2]  O += P_j V_j done (P buffer j&1 free again)
-  uint64_t* drain = bars + 13;
-  uint64_t* v_full = bars + 14;   // [2]  V ring: a slot is free once O += P_j V_j is done
-  uint64_t* v_empty = bars + 16;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* k_full = bars + 1;    // [2 slots]
+  uint64_t* k_empty = bars + 3;   // [2 slots]
+  uint64_t* v_full = bars + 5;    // [2 slots]
+  uint64_t* v_empty = bars + 7;   // [2 slots]
+  uint64_t* s_full = bars + 9;    // [2 query tiles] S_t of the next key tile computed
+  uint64_t* p_full = bars + 11;   // [2 query tiles] P_t written (one arrival per softmax warp)
+  uint64_t* o_done = bars + 13;   // [2 query tiles] O_t += P_t V_j done
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xmax = reinterpret_cast<float*>(bars + 32);  // [2 tile parities][SPLIT parts][128 rows] (after 256 B of barriers)
-  float* xsum = xmax + 2 * SPLIT * 128;               // [SPLIT parts][128 rows]
 
-  const int nqb = (T + FA_BM - 1) / FA_BM;
-  const int qb = nqb - 1 - (int)blockIdx.x;  // heavy (late) query tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // one CTA per (256-query block, head, sequence), heaviest work first: every
+  // (head, sequence)'s last query block (the most key tiles under a causal
+  // mask), then every second-to-last one, ..., so that the CTAs still running
+  // at the end of the grid are the short ones
+  const int nqb = (T + FA_QB - 1) / FA_QB;
+  const int nhb = (int)gridDim.x / nqb;  // heads x sequences
+  const int qb = nqb - 1 - (int)blockIdx.x / nhb;
+  const int h = ((int)blockIdx.x % nhb) % H, b = ((int)blockIdx.x % nhb) / H;
   const int kvh = h / (H / Hkv);
-  const int q0 = qb * FA_BM;
-  const int kb_lo = (window >= 0) ? max(0, q0 - window) / FA_BN : 0;
-  const int kb_hi = min(T - 1, q0 + FA_BM - 1) / FA_BN;
-  const int ntiles = kb_hi - kb_lo + 1;
+  const int q0 = qb * FA_QB;
+  // key tiles that intersect the visible keys of query tile t (empty past T)
+  int lo[2], hi[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = q0 + t * FA_BM;
+    lo[t] = (window >= 0) ? max(0, qt - window) / FA_BN : 0;
+    hi[t] = (qt < T) ? min(qt + FA_BM - 1, T - 1) / FA_BN : lo[t] - 1;
+  }
+  // the ranges are monotone in t and overlap or touch, so their union is one range
+  const int jlo = lo[0];
+  const int jhi = max(hi[0], hi[1]);
   const int row_base = b * T;  // row of token (b, 0) in the packed [B*T, Wq] buffer
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -104,9 +101,8 @@ __global__ void __launch_bounds__(FaShape<SPLIT>::THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], NSW);
-      mbar_init(&p_full[i], NSW);
-      mbar_init(&pv_done[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_done[i], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -121,13 +117,16 @@ __global__ void __launch_bounds__(FaShape<SPLIT>::THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, FA_TILE);
-      tma_load_2d(sQ, &tm_qkv, q_full, h * 128, row_base + q0);
-      tma_load_2d(sQ + 16384, &tm_qkv, q_full, h * 128 + 64, row_base + q0);
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = j & 1;
-        const uint32_t par = ((j >> 1) & 1) ^ 1u;
-        const int kr = row_base + (kb_lo + j) * FA_BN;
+      const int nq = (hi[1] >= lo[1]) ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, nq * FA_TILE);
+      for (int t = 0; t < nq; ++t) {
+        tma_load_2d(sQ + t * FA_TILE, &tm_qkv, q_full, h * 128, row_base + q0 + t * FA_BM);
+        tma_load_2d(sQ + t * FA_TILE + 16384, &tm_qkv, q_full, h * 128 + 64, row_base + q0 + t * FA_BM);
+      }
+      for (int j = jlo; j <= jhi; ++j) {
+        const int i = j - jlo, st = i & 1;
+        const uint32_t par = ((i >> 1) & 1) ^ 1u;
+        const int kr = row_base + j * FA_BN;
         if (!mbar_wait(&k_empty[st], par, abort_flag, ERRW_TIMEOUT_PRODUCER)) break;
         mbar_arrive_expect_tx(&k_full[st], FA_TILE);
         uint8_t* k = sK + st * FA_TILE;
@@ -144,35 +143,47 @@ __global__ void __launch_bounds__(FaShape<SPLIT>::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = make_idesc(128, 128, false, false, false);
       constexpr uint32_t IDESC_O = make_idesc(128, 128, false, true, false);
-      const uint32_t aQ = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, abort_flag, ERRW_TIMEOUT_MMA);
-      auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(&v_full[i & 1], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
+      auto in = [&](int t, int j) { return j >= lo[t] && j <= hi[t]; };
+      // S_t for key tile j; the K slot is released after its last score product
+      auto issue_s = [&](int t, int j) -> bool {
+        const int i = j - jlo, st = i & 1;
+        if (!mbar_wait(&k_full[st], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t aV = smem_u32(sV + (i & 1) * FA_TILE);
-        // A = P_i from TMEM (lane = query row, 8 columns per 16 keys)
+        const uint32_t aQ = smem_u32(sQ + t * FA_TILE), aK = smem_u32(sK + st * FA_TILE);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_bf16_ts(tmem + 256, tmem + 384 + (i & 1) * 64 + k * 8, fa_desc_mn(aV, k), IDESC_O,
-                      (i > 0 || k > 0) ? 1u : 0u);
-        mma_commit(&pv_done[i & 1]);
-        mma_commit(&v_empty[i & 1]);
+          mma_bf16_ss(tmem + t * 128, fa_desc_k(aQ, k), fa_desc_k(aK, k), IDESC_S, k > 0 ? 1u : 0u);
+        mma_commit(&s_full[t]);
+        if (t == 1 || !in(1, j)) mma_commit(&k_empty[st]);
         return true;
       };
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int sb = j & 1;
-        if (!mbar_wait(&k_full[sb], (j >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
-        if (!mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) { ok = false; break; }
+      // O_t += P_t V_j once the softmax has written P_t; the V slot is released after its last PV product
+      auto issue_pv = [&](int t, int j) -> bool {
+        const int i = j - jlo, st = i & 1;
+        const int c = j - lo[t];
+        if (!mbar_wait(&v_full[st], (i >> 1) & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
+        if (!mbar_wait(&p_full[t], c & 1, abort_flag, ERRW_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t aK = smem_u32(sK + sb * FA_TILE);
+        const uint32_t aV = smem_u32(sV + st * FA_TILE);
+        // A = P_t from TMEM (lane = query row, 8 columns per 16 keys)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mma_bf16_ss(tmem + sb * 128, fa_desc_k(aQ, k), fa_desc_k(aK, k), IDESC_S, k > 0 ? 1u : 0u);
-        mma_commit(&s_full[sb]);
-        mma_commit(&k_empty[sb]);
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+        for (int k = 0; k < 8; ++k)
+          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, fa_desc_mn(aV, k), IDESC_O,
+                      (c > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&o_done[t]);
+        if (t == 1 || !in(1, j)) mma_commit(&v_empty[st]);
+        return true;
+      };
+      if (ok && in(0, jlo)) ok = issue_s(0, jlo);
+      if (ok && hi[1] >= lo[1]) ok = issue_s(1, lo[1]);
+      for (int j = jlo; ok && j <= jhi; ++j) {
+        if (in(0, j)) {
+          ok = issue_pv(0, j) && (j + 1 > hi[0] || issue_s(0, j + 1));
+          if (!ok) break;
+        }
+        if (in(1, j)) ok = issue_pv(1, j) && (j + 1 > hi[1] || issue_s(1, j + 1));
       }
-      if (ok) ok = issue_pv(ntiles - 1);
       if (*abort_flag) {
         mma_commit(drain);
         const unsigned long long t0 = globaltimer_ns();
@@ -181,131 +192,110 @@ __global__ void __launch_bounds__(FaShape<SPLIT>::THREADS, 1)
       }
     }
   } else {
-    // softmax warps: TMEM lane quarter qw = warp % 4 -> query rows 32*qw ..
-    // 32*qw+31; part hf (0..SPLIT-1) -> score / output columns KPW*hf .. KPW*hf+KPW-1
-    constexpr int NCH = KPW / 32;  // 32-column TMEM chunks per thread
+    // softmax of query tile tt: TMEM lane quarter qw = warp % 4 -> rows 32*qw .. 32*qw+31
+    const int tt = (warp - 2) >> 2;
     const int qw = warp & 3;
-    const int hf = (warp - 2) >> 2;
-    const int r = qw * 32 + lane;  // row within the tile
-    const int t = q0 + r;          // query position
+    const int r = qw * 32 + lane;        // row within the query tile
+    const int tq = q0 + tt * FA_BM + r;  // query position
     const uint32_t lane_addr = tmem + ((uint32_t)(qw * 32) << 16);
+    const uint32_t s_col = (uint32_t)(tt * 128), o_col = (uint32_t)(256 + tt * 128);
     const float sl2 = LOG2E / sqrtf(128.f);
-    float oam = 0.f;  // max |o| this thread stores (FP8 amax)
-    // keys visible from query t: [t - W, t] (or [0, t]) clipped to the sequence
-    const int kv_lo = (window >= 0) ? t - window : 0;
-    const int kv_hi = min(t, T - 1);
+    const int qt0 = q0 + tt * FA_BM;  // first query of the tile
+    // keys visible from query tq: [tq - W, tq] (or [0, tq]) clipped to the sequence
+    const int kv_lo = (window >= 0) ? tq - window : 0;
+    const int kv_hi = min(tq, T - 1);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    // Every softmax warp runs every iteration and passes every named barrier,
-    // also after a failed (timed-out) wait: then it only skips the work, so no
-    // warp can be left waiting at a barrier that another warp never reaches.
-    for (int j = 0; j < ntiles; ++j) {
-      const int sb = j & 1;
-      const int k0 = (kb_lo + j) * FA_BN + hf * KPW;  // first key of this part
-      ok = ok && mbar_wait_warp(&s_full[sb], (j >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+    const int lo_t = tt ? lo[1] : lo[0];
+    const int n = (tt ? hi[1] : hi[0]) - lo_t + 1;  // key tiles of this query tile (0 past T)
+    for (int c = 0; c < n && ok; ++c) {
+      const int k0 = (lo_t + c) * FA_BN;
+      ok = mbar_wait_warp(&s_full[tt], c & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+      if (!ok) break;
       tc_fence_after();
-      const bool need_mask = (k0 + KPW - 1 > q0) || (k0 + KPW > T) || (window >= 0 && q0 + FA_BM - 1 - k0 > window);
-      // every chunk of this part goes to registers at once; the score buffer is
-      // released right after, so the next-but-one S MMA can start
-      uint32_t v[KPW];
-      if (ok) {
+      uint32_t v[128];
 #pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          tmem_ld_32x32b_x32(lane_addr + sb * 128 + hf * KPW + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
-        tmem_ld_wait();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
-      // masked scores become -inf; visible keys of row t: kv_lo..kv_hi
+      for (int k = 0; k < 4; ++k)
+        tmem_ld_32x32b_x32(lane_addr + s_col + k * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[k * 32]));
+      tmem_ld_wait();
+      const bool need_mask =
+          (k0 + FA_BN - 1 > qt0) || (k0 + FA_BN > T) || (window >= 0 && qt0 + FA_BM - 1 - k0 > window);
+      // masked scores become -inf; visible keys of row tq: kv_lo..kv_hi
       if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < KPW; ++i) {
+        for (int i = 0; i < 128; ++i) {
           const int jk = k0 + i;
           v[i] = (jk >= kv_lo && jk <= kv_hi) ? v[i] : __float_as_uint(-INFINITY);
         }
       }
-      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float mp[8];
 #pragma unroll
-      for (int i = 0; i < KPW; ++i) mp[i & 3] = fmaxf(mp[i & 3], __uint_as_float(v[i]));
-      float* xm = xmax + sb * SPLIT * 128;
-      xm[hf * 128 + r] = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-      named_bar_sync(1, FA_SOFTMAX_THREADS);
-      float mxr = xm[r];
+      for (int i = 0; i < 8; ++i) mp[i] = __uint_as_float(v[i]);
 #pragma unroll
-      for (int p = 1; p < SPLIT; ++p) mxr = fmaxf(mxr, xm[p * 128 + r]);
-      const float mx = mxr * sl2;
-      // P buffer j&1 was last read by the PV product of tile j-2
-      if (j > 1) ok = ok && mbar_wait_warp(&pv_done[sb], ((j >> 1) & 1) ^ 1u, abort_flag, ERRW_TIMEOUT_EPILOGUE);
-      if (!ok) continue;
-      // rescale decision is per row (identical in every part) but the TMEM
-      // accesses are warp-collective: the whole warp enters, rows that keep
-      // their max use a factor of 1
+      for (int i = 8; i < 128; ++i) mp[i & 7] = fmaxf(mp[i & 7], __uint_as_float(v[i]));
+      const float mx =
+          fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * sl2;
+      // the running max moves only when it grows by more than 8 (base 2)
       const bool grow = mx > m_used + 8.f;
-      if (__any_sync(0xffffffffu, grow)) {
-        const float corr = grow ? fast_exp2(m_used - mx) : 1.f;  // 0 when m_used is -inf
-        if (j > 0) {
-          // O may only be rescaled once every issued PV product (up to tile j-1) is done
-          ok = mbar_wait_warp(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
-          if (!ok) continue;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            uint32_t w[32];
-            tmem_ld_32x32b_x32(lane_addr + 256 + hf * KPW + c * 32, w);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * corr);
-            tmem_st_32x32b_x32(lane_addr + 256 + hf * KPW + c * 32, w);
-          }
-          tmem_st_wait();
-        }
-        if (grow) {
-          l *= corr;
-          m_used = mx;
-        }
+      const float corr = grow ? fast_exp2(m_used - mx) : 1.f;  // 0 when m_used is -inf
+      if (grow) {
+        l *= corr;
+        m_used = mx;
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      // pass 2: P = exp2(s*scale - m) as bf16 pairs (key 2c in the low half)
-      // into TMEM columns 384 + 64*(j&1) + (KPW/2)*hf .. of this row's lane
-      uint32_t pk[KPW / 2];
+      // P = exp2(s*scale - m) as bf16 pairs (key 2c in the low half) over the
+      // first 64 columns of S_t
       float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < KPW / 2; ++c) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * c]), sl2, -mu));  // exp2(-inf) = 0 for masked keys
-        const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * c + 1]), sl2, -mu));
-        lp[(2 * c) & 3] += p0;
-        lp[(2 * c + 1) & 3] += p1;
-        pk[c] = pack_bf16(p0, p1);
+      for (int hq = 0; hq < 4; ++hq) {  // 32 keys (16 columns of P) at a time
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i = hq * 32 + 2 * e;
+          const float p0 = fast_exp2(fmaf(__uint_as_float(v[i]), sl2, -mu));  // exp2(-inf) = 0 for masked keys
+          const float p1 = fast_exp2(fmaf(__uint_as_float(v[i + 1]), sl2, -mu));
+          lp[(2 * e) & 3] += p0;
+          lp[(2 * e + 1) & 3] += p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st_32x32b_x16(lane_addr + s_col + hq * 16, pk);
       }
       l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-      if constexpr (KPW == 64) {
-        tmem_st_32x32b_x32(lane_addr + 384 + sb * 64 + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      } else {
-        tmem_st_32x32b_x16(lane_addr + 384 + sb * 64 + hf * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+      // O_t to the new max (the TMEM accesses are warp-collective: the whole
+      // warp enters, rows that keep their max use 1).  O_t holds every PV
+      // product up to key tile c-1 (the commit of S_t above follows them);
+      // the wait states it.
+      if (c > 0 && __any_sync(0xffffffffu, grow)) {
+        ok = mbar_wait_warp(&o_done[tt], (c - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          uint32_t w[32];
+          tmem_ld_32x32b_x32(lane_addr + o_col + k * 32, w);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * corr);
+          tmem_st_32x32b_x32(lane_addr + o_col + k * 32, w);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (lane == 0) mbar_arrive(&p_full[tt]);
     }
-    // every part's sum shares the same running max: add them
-    xsum[hf * 128 + r] = l;
-    named_bar_sync(1, FA_SOFTMAX_THREADS);
-    float lt = 0.f;
-#pragma unroll
-    for (int p = 0; p < SPLIT; ++p) lt += xsum[p * 128 + r];
-    if (__all_sync(0xffffffffu, ok) &&
-        mbar_wait_warp(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
+    float oam = 0.f;  // max |o| this thread stores (FP8 amax)
+    if (n > 0 && __all_sync(0xffffffffu, ok) &&
+        mbar_wait_warp(&o_done[tt], (n - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
       tc_fence_after();
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      bf16* orow = o + ((long long)b * T + t) * ldo + h * 128 + hf * KPW;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      bf16* orow = o + ((long long)b * T + tq) * ldo + h * 128;
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
+      for (int k = 0; k < 4; ++k) {
         uint32_t w[32];
-        tmem_ld_32x32b_x32(lane_addr + 256 + hf * KPW + c * 32, w);
+        tmem_ld_32x32b_x32(lane_addr + o_col + k * 32, w);
         tmem_ld_wait();
-        if (t < T) {
+        if (tq < T) {
           if (amax_o) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) oam = fmaxf(oam, fabsf(__uint_as_float(w[i]) * inv));
@@ -317,22 +307,15 @@ __global__ void __launch_bounds__(FaShape<SPLIT>::THREADS, 1)
             u.y = pack_bf16(__uint_as_float(w[g * 8 + 2]) * inv, __uint_as_float(w[g * 8 + 3]) * inv);
             u.z = pack_bf16(__uint_as_float(w[g * 8 + 4]) * inv, __uint_as_float(w[g * 8 + 5]) * inv);
             u.w = pack_bf16(__uint_as_float(w[g * 8 + 6]) * inv, __uint_as_float(w[g * 8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = u;
+            *reinterpret_cast<uint4*>(orow + k * 32 + g * 8) = u;
           }
         }
       }
-      if (t < T && hf == 0) lse[((long long)b * H + h) * T + t] = (m_used + log2f(lt)) * LN2;
+      if (tq < T) lse[((long long)b * H + h) * T + tq] = (m_used + log2f(l)) * LN2;
     }
-    if (amax_o) {  // the softmax warps' max |o| (FP8 amax): one atomic per CTA
+    if (amax_o) {  // the warp's max |o| (FP8 amax)
       oam = warp_max(oam);
-      named_bar_sync(1, FA_SOFTMAX_THREADS);
-      if (lane == 0) xsum[warp - 2] = oam;  // xsum is free once every row's sum has been read
-      named_bar_sync(1, FA_SOFTMAX_THREADS);
-      if (warp == 2 && lane == 0) {
-        float mm = 0.f;
-        for (int w = 0; w < NSW; ++w) mm = fmaxf(mm, xsum[w]);
-        atomicMax(amax_o, __float_as_uint(stored_abs_max_bf16(mm)));
-      }
+      if (lane == 0 && oam > 0.f) atomicMax(amax_o, __float_as_uint(stored_abs_max_bf16(oam)));
     }
   }
   tc_fence_before();
