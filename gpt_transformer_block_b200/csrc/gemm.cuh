@@ -26,6 +26,8 @@
 //   the fp32 configuration whose 1e-5 tolerance tensor-core fp32 (tf32)
 //   inputs cannot meet.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace gptb {
@@ -279,6 +281,258 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, uint32_t ta, u
   }
 }
 
+// The epilogue warps' role for one epilogue kind (the kind is a template
+// parameter, so each kind's per-chunk loop is compact straight-line code).
+template <int KIND, bool PAIR>
+__device__ __forceinline__ void tc_epilogue(const EpiParams& ep, const CUtensorMap* tmO_, const CUtensorMap* tmX_,
+                                            uint32_t tmem_base, uint8_t* sEpi, uint64_t* aux_bar, uint64_t* tfull,
+                                            uint64_t* tempty, volatile int* abort_flag, int M, int N, int unit0,
+                                            int ustep, int units, int tiles_m, int tiles_n, int warp, int lane,
+                                            uint32_t rank) {
+  using SH = TcShape<PAIR>;
+  const CUtensorMap& tmO = *tmO_;
+  const CUtensorMap& tmX = *tmX_;
+  const int q = warp & 3;  // TMEM lane quarter this warp may access
+  uint8_t* ebuf = sEpi + (warp - 2) * (4 * TC_EPI_TILE);  // this warp's four staging tiles
+  uint64_t* abar = &aux_bar[(warp - 2) * 2];
+  constexpr bool has_aux = (KIND == EPI_RESID || KIND == EPI_DRELU2 || KIND == EPI_DOT);
+  constexpr bool acc32 = (KIND == EPI_ACCUM_F32);
+  const int swz = (lane & 7);  // 16-byte chunk swizzle of this lane's 128-byte staging row
+  // Staging tiles: bf16 output chunks alternate between tiles 0 and 1, and
+  // the input chunks (residual, saved activation, O) between tiles 2 and 3;
+  // fp32 chunks and the q/k/v heads take two tiles each, alternating
+  // between tiles 0-1 and 2-3.  Every chunk commits one bulk group, so
+  // waiting until at most one group is still reading frees the tile(s) of
+  // the chunk before last.
+  uint32_t ns = 0;          // bulk groups committed by this warp
+  uint32_t na = 0, nw = 0;  // input-tile loads issued / consumed by this warp
+  auto chunks_of = [&](int tn_) { return min(TC_BN / 64, (N - tn_ * TC_BN + 63) / 64); };
+  // load the input chunk cc_ of unit u_ into the next input tile (lane 0; the count advances on every lane)
+  auto issue_aux = [&](int u_, int cc_) {
+    if (lane == 0) {
+      int tm_, tn_, sp_;
+      tc_unit_coords(u_, tiles_m, tiles_n, tm_, tn_, sp_);
+      uint64_t* bar = &abar[na & 1u];
+      mbar_arrive_expect_tx(bar, TC_EPI_TILE);
+      tma_load_2d(ebuf + (2 + (na & 1u)) * TC_EPI_TILE, &tmX, bar, tn_ * TC_BN + cc_ * 64,
+                  tm_ * SH::TILE_M + (int)rank * TC_BM + q * 32);
+    }
+    ++na;
+  };
+  if (has_aux && unit0 < units) issue_aux(unit0, 0);
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  const float alpha = epi_alpha(ep);
+  const float beta = epi_beta(ep);
+  float oam = 0.f;  // max |out| stored by this thread (FP8 amax of EPI_RELU2 / EPI_DRELU2 outputs)
+  bool ok = true;
+  for (int u = unit0; u < units && ok; u += ustep) {
+    int tm, tn, split;
+    tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
+    if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
+    tc_fence_after();
+    const int row0 = tm * SH::TILE_M + (int)rank * TC_BM + q * 32;
+    if constexpr (KIND == EPI_QKV) {
+#pragma unroll 1
+      for (int hb = 0; hb < TC_BN / 128; ++hb) {
+        const int col0 = tn * TC_BN + hb * 128;
+        if (col0 >= N) break;  // warp-uniform
+        uint8_t* st0 = ebuf + (ns & 1u) * 2 * TC_EPI_TILE;
+        if (lane == 0) bulk_wait_read1();
+        __syncwarp();
+        const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + hb * 128);
+        epi_qkv_head(ep, ta, st0, st0 + TC_EPI_TILE, lane, alpha, col0 / 128, row0 + lane, row0 + lane < M);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmO, st0, col0, row0);
+          tma_store_2d(&tmO, st0 + TC_EPI_TILE, col0 + 64, row0);
+          bulk_commit_group();
+        }
+        ++ns;
+      }
+    }
+    float dsum = 0.f;  // EPI_DOT: this row's running sum over the current 128-column group
+    // EPI_XENT: this row's running max and sum of exp2((z - max) * log2 e) over the tile
+    float xm = -INFINITY, xs = 0.f;
+    const int xy = (KIND == EPI_XENT && row0 + lane < M) ? ep.targets[row0 + lane] : -1;
+    const int nch = (KIND == EPI_QKV) ? 0 : chunks_of(tn);
+#pragma unroll 1
+    for (int cc = 0; cc < nch; ++cc) {
+      const int col0 = tn * TC_BN + cc * 64;
+      const bool tail = col0 + 64 > N;  // warp-uniform: the last chunk of a ragged N
+      uint32_t r0[32], r1[32];
+      const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + cc * 64);
+      tmem_ld_32x32b_x32(ta, r0);
+      tmem_ld_32x32b_x32(ta + 32, r1);
+      if constexpr (has_aux) {
+        // the next input chunk (of this tile, else of the next unit) goes
+        // into the other input tile, read by the chunk before this one
+        if (cc + 1 < nch) issue_aux(u, cc + 1);
+        else if (u + ustep < units) issue_aux(u + ustep, 0);
+      }
+      // this chunk's output tile(s) are free once the bulk group of the chunk before last has read them
+      if (lane == 0) bulk_wait_read1();
+      __syncwarp();
+      tmem_ld_wait();
+      uint8_t* cur_in = ebuf + (2 + (nw & 1u)) * TC_EPI_TILE;
+      if constexpr (has_aux) {
+        if (!mbar_wait_warp(&abar[nw & 1u], (nw >> 1) & 1u, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
+          ok = false;
+          break;
+        }
+        ++nw;
+      }
+      uint8_t* p0 = ebuf + (acc32 ? (ns & 1u) * 2 * TC_EPI_TILE : (ns & 1u) * TC_EPI_TILE) + lane * 128;
+      uint8_t* p1 = acc32 ? p0 + TC_EPI_TILE : cur_in + lane * 128;
+      float xml2 = 0.f;  // EPI_XENT: running max * log2 e after this chunk
+      if constexpr (KIND == EPI_XENT) {
+        // the chunk's max as eight independent chains (columns past N left out)
+        float cm8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cm8[j] = xm;
+        if (!tail) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            cm8[i & 7] = fmaxf(cm8[i & 7], __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (col0 + i < N) cm8[i & 7] = fmaxf(cm8[i & 7], __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
+        }
+#pragma unroll
+        for (int j = 1; j < 8; ++j) cm8[0] = fmaxf(cm8[0], cm8[j]);
+        const float cm = cm8[0];
+        if (cm > xm) {  // rescale the sum to the new max (0 while the max was -inf)
+          xs = (xm == -INFINITY) ? 0.f : xs * fast_exp2((xm - cm) * LOG2E);
+          xm = cm;
+        }
+        xml2 = xm * LOG2E;
+      }
+      if constexpr (acc32) {
+        // fp32: columns 0..31 -> tile 0, 32..63 -> tile 1 (32 x 128-byte rows each)
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          *reinterpret_cast<float4*>(p0 + ((g ^ swz) << 4)) =
+              make_float4(__uint_as_float(r0[4 * g]) * alpha, __uint_as_float(r0[4 * g + 1]) * alpha,
+                          __uint_as_float(r0[4 * g + 2]) * alpha, __uint_as_float(r0[4 * g + 3]) * alpha);
+          *reinterpret_cast<float4*>(p1 + ((g ^ swz) << 4)) =
+              make_float4(__uint_as_float(r1[4 * g]) * alpha, __uint_as_float(r1[4 * g + 1]) * alpha,
+                          __uint_as_float(r1[4 * g + 2]) * alpha, __uint_as_float(r1[4 * g + 3]) * alpha);
+        }
+      } else {
+        // bf16: 8 chunks of 8 columns; the input chunk (if any) has the same swizzle
+        float xsum[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          float v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(g < 4 ? r0[g * 8 + i] : r1[(g - 4) * 8 + i]) * alpha;
+          uint8_t* cp0 = p0 + ((g ^ swz) << 4);
+          if constexpr (has_aux) {
+            float a[8];
+            load8(reinterpret_cast<const bf16*>(p1 + ((g ^ swz) << 4)), a);
+            if constexpr (KIND == EPI_RESID) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = fmaf(beta, a[i], v[i]);
+            } else if constexpr (KIND == EPI_DRELU2) {
+              // 2 relu(u) = 2 sqrt(a) as a * rsqrt(a); a below the smallest
+              // normal float (where the flushing rsqrt gives inf) counts as 0
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] *= (a[i] >= 1.17549435e-38f) ? 2.f * a[i] * fast_rsqrt(a[i]) : 0.f;
+            } else {
+              // the dot takes the values as stored (rounded to bf16)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dsum = fmaf(__bfloat162float(__float2bfloat16_rn(v[i])), a[i], dsum);
+            }
+          }
+          if constexpr (KIND == EPI_XENT) {
+            const int c8 = col0 + g * 8;
+            float e[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) e[i] = fast_exp2(fmaf(v[i], LOG2E, -xml2));
+            if (tail) {  // columns past N (the last tile's tail) do not take part
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (c8 + i >= N) e[i] = 0.f;
+            }
+            xsum[g] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
+            if (xy >= c8 && xy < c8 + 8) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (xy == c8 + i) ep.xent_zy[row0 + lane] = v[i];
+            }
+          }
+          if constexpr (KIND == EPI_RELU2) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float t = fmaxf(v[i], 0.f);
+              v[i] = t * t;
+            }
+          }
+          if ((KIND == EPI_RELU2 || KIND == EPI_DRELU2) && ep.amax_out && row0 + lane < M) {
+            const int c8 = col0 + g * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (c8 + i < N) oam = fmaxf(oam, fabsf(v[i]));
+          }
+          store8(reinterpret_cast<bf16*>(cp0), v);
+        }
+        if constexpr (KIND == EPI_XENT)
+          xs += ((xsum[0] + xsum[1]) + (xsum[2] + xsum[3])) + ((xsum[4] + xsum[5]) + (xsum[6] + xsum[7]));
+      }
+      if (KIND == EPI_DOT && (cc & 1)) {  // a 128-column group (one head) is complete
+        const int row = row0 + lane;
+        if (row < M) {
+          const int bb = row / ep.T, t = row - bb * ep.T;
+          ep.rowdot[((long long)bb * ep.H + col0 / 128) * ep.T + t] = dsum;
+        }
+        dsum = 0.f;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        uint8_t* t0 = p0 - lane * 128;
+        if constexpr (acc32) {
+          tma_reduce_add_2d(&tmO, t0, col0, row0);
+          tma_reduce_add_2d(&tmO, t0 + TC_EPI_TILE, col0 + 32, row0);
+        } else {
+          tma_store_2d(&tmO, t0, col0, row0);
+        }
+        bulk_commit_group();
+      }
+      ++ns;
+    }
+    // (a tile cut short by the N tail still covers at least one chunk)
+    if (KIND == EPI_XENT && ok && row0 + lane < M)
+      ep.xent_part[(long long)(row0 + lane) * ep.xent_nt + tn] = make_float2(xm, xs);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      if (PAIR) mbar_arrive_cluster(map_shared_rank(&tempty[acc], 0));
+      else mbar_arrive(&tempty[acc]);
+    }
+    acc ^= 1;
+    if (acc == 0) acc_phase ^= 1u;
+  }
+  // input-tile loads still in flight (issued ahead of an abort) land before the CTA exits
+  while (nw < na) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(&abar[nw & 1u], (nw >> 1) & 1u)) {
+      if (globaltimer_ns() - t0 > 100000000ull) {
+        record_error(ERRW_TIMEOUT_DRAIN);
+        break;
+      }
+    }
+    ++nw;
+  }
+  if (lane == 0) bulk_wait0();
+  if ((KIND == EPI_RELU2 || KIND == EPI_DRELU2) && ep.amax_out) {
+    oam = warp_max(oam);
+    if (lane == 0) atomicMax(ep.amax_out, __float_as_uint(stored_abs_max_bf16(oam)));
+  }
+}
+
 template <bool A_MN, bool B_MN, bool FP8, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -487,244 +741,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint8_t* ebuf = sEpi + (warp - 2) * (4 * TC_EPI_TILE);  // this warp's four staging tiles
-    uint64_t* abar = &aux_bar[(warp - 2) * 2];
-    const bool has_aux = (ep.kind == EPI_RESID || ep.kind == EPI_DRELU2 || ep.kind == EPI_DOT);
-    const bool acc32 = (ep.kind == EPI_ACCUM_F32);
-    const int swz = (lane & 7);  // 16-byte chunk swizzle of this lane's 128-byte staging row
-    // Staging tiles: bf16 output chunks alternate between tiles 0 and 1, and
-    // the input chunks (residual, saved activation, O) between tiles 2 and 3;
-    // fp32 chunks and the q/k/v heads take two tiles each, alternating
-    // between tiles 0-1 and 2-3.  Every chunk commits one bulk group, so
-    // waiting until at most one group is still reading frees the tile(s) of
-    // the chunk before last.
-    uint32_t ns = 0;          // bulk groups committed by this warp
-    uint32_t na = 0, nw = 0;  // input-tile loads issued / consumed by this warp
-    auto chunks_of = [&](int tn_) { return min(TC_BN / 64, (N - tn_ * TC_BN + 63) / 64); };
-    // load the input chunk cc_ of unit u_ into the next input tile (lane 0; the count advances on every lane)
-    auto issue_aux = [&](int u_, int cc_) {
-      if (lane == 0) {
-        int tm_, tn_, sp_;
-        tc_unit_coords(u_, tiles_m, tiles_n, tm_, tn_, sp_);
-        uint64_t* bar = &abar[na & 1u];
-        mbar_arrive_expect_tx(bar, TC_EPI_TILE);
-        tma_load_2d(ebuf + (2 + (na & 1u)) * TC_EPI_TILE, &tmX, bar, tn_ * TC_BN + cc_ * 64,
-                    tm_ * SH::TILE_M + (int)rank * TC_BM + q * 32);
-      }
-      ++na;
+    // one code path per epilogue kind
+    auto run = [&](auto kind) {
+      tc_epilogue<decltype(kind)::value, PAIR>(ep, &tmO, &tmX, tmem_base, sEpi, aux_bar, tfull, tempty, abort_flag, M, N,
+                                               unit0, ustep, units, tiles_m, tiles_n, warp, lane, rank);
     };
-    if (has_aux && unit0 < units) issue_aux(unit0, 0);
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    const float alpha = epi_alpha(ep);
-    const float beta = epi_beta(ep);
-    float oam = 0.f;  // max |out| stored by this thread (FP8 amax of EPI_RELU2 / EPI_DRELU2 outputs)
-    bool ok = true;
-    for (int u = unit0; u < units && ok; u += ustep) {
-      int tm, tn, split;
-      tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
-      if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
-      tc_fence_after();
-      const int row0 = tm * SH::TILE_M + (int)rank * TC_BM + q * 32;
-      if (ep.kind == EPI_QKV) {
-#pragma unroll 1
-        for (int hb = 0; hb < TC_BN / 128; ++hb) {
-          const int col0 = tn * TC_BN + hb * 128;
-          if (col0 >= N) break;  // warp-uniform
-          uint8_t* st0 = ebuf + (ns & 1u) * 2 * TC_EPI_TILE;
-          if (lane == 0) bulk_wait_read1();
-          __syncwarp();
-          const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + hb * 128);
-          epi_qkv_head(ep, ta, st0, st0 + TC_EPI_TILE, lane, alpha, col0 / 128, row0 + lane, row0 + lane < M);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmO, st0, col0, row0);
-            tma_store_2d(&tmO, st0 + TC_EPI_TILE, col0 + 64, row0);
-            bulk_commit_group();
-          }
-          ++ns;
-        }
-      }
-      float dsum = 0.f;  // EPI_DOT: this row's running sum over the current 128-column group
-      // EPI_XENT: this row's running max and sum of exp2((z - max) * log2 e) over the tile
-      float xm = -INFINITY, xs = 0.f;
-      const int xy = (ep.kind == EPI_XENT && row0 + lane < M) ? ep.targets[row0 + lane] : -1;
-      const int nch = (ep.kind == EPI_QKV) ? 0 : chunks_of(tn);
-#pragma unroll 1
-      for (int cc = 0; cc < nch; ++cc) {
-        const int col0 = tn * TC_BN + cc * 64;
-        const bool tail = col0 + 64 > N;  // warp-uniform: the last chunk of a ragged N
-        uint32_t r0[32], r1[32];
-        const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TC_BN + cc * 64);
-        tmem_ld_32x32b_x32(ta, r0);
-        tmem_ld_32x32b_x32(ta + 32, r1);
-        if (has_aux) {
-          // the next input chunk (of this tile, else of the next unit) goes
-          // into the other input tile, read by the chunk before this one
-          if (cc + 1 < nch) issue_aux(u, cc + 1);
-          else if (u + ustep < units) issue_aux(u + ustep, 0);
-        }
-        // this chunk's output tile(s) are free once the bulk group of the chunk before last has read them
-        if (lane == 0) bulk_wait_read1();
-        __syncwarp();
-        tmem_ld_wait();
-        uint8_t* cur_in = ebuf + (2 + (nw & 1u)) * TC_EPI_TILE;
-        if (has_aux) {
-          if (!mbar_wait_warp(&abar[nw & 1u], (nw >> 1) & 1u, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
-            ok = false;
-            break;
-          }
-          ++nw;
-        }
-        uint8_t* p0 = ebuf + (acc32 ? (ns & 1u) * 2 * TC_EPI_TILE : (ns & 1u) * TC_EPI_TILE) + lane * 128;
-        uint8_t* p1 = acc32 ? p0 + TC_EPI_TILE : cur_in + lane * 128;
-        float xml2 = 0.f;  // EPI_XENT: running max * log2 e after this chunk
-        if (ep.kind == EPI_XENT) {
-          // the chunk's max as eight independent chains (columns past N left out)
-          float cm8[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) cm8[j] = xm;
-          if (!tail) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-              cm8[i & 7] = fmaxf(cm8[i & 7], __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (col0 + i < N) cm8[i & 7] = fmaxf(cm8[i & 7], __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * alpha);
-          }
-#pragma unroll
-          for (int j = 1; j < 8; ++j) cm8[0] = fmaxf(cm8[0], cm8[j]);
-          const float cm = cm8[0];
-          if (cm > xm) {  // rescale the sum to the new max (0 while the max was -inf)
-            xs = (xm == -INFINITY) ? 0.f : xs * fast_exp2((xm - cm) * LOG2E);
-            xm = cm;
-          }
-          xml2 = xm * LOG2E;
-        }
-        if (acc32) {
-          // fp32: columns 0..31 -> tile 0, 32..63 -> tile 1 (32 x 128-byte rows each)
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            *reinterpret_cast<float4*>(p0 + ((g ^ swz) << 4)) =
-                make_float4(__uint_as_float(r0[4 * g]) * alpha, __uint_as_float(r0[4 * g + 1]) * alpha,
-                            __uint_as_float(r0[4 * g + 2]) * alpha, __uint_as_float(r0[4 * g + 3]) * alpha);
-            *reinterpret_cast<float4*>(p1 + ((g ^ swz) << 4)) =
-                make_float4(__uint_as_float(r1[4 * g]) * alpha, __uint_as_float(r1[4 * g + 1]) * alpha,
-                            __uint_as_float(r1[4 * g + 2]) * alpha, __uint_as_float(r1[4 * g + 3]) * alpha);
-          }
-        } else {
-          // bf16: 8 chunks of 8 columns; the input chunk (if any) has the same swizzle
-          float xsum[8];
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(g < 4 ? r0[g * 8 + i] : r1[(g - 4) * 8 + i]) * alpha;
-            uint8_t* cp0 = p0 + ((g ^ swz) << 4);
-            if (has_aux) {
-              float a[8];
-              load8(reinterpret_cast<const bf16*>(p1 + ((g ^ swz) << 4)), a);
-              if (ep.kind == EPI_RESID) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = fmaf(beta, a[i], v[i]);
-              } else if (ep.kind == EPI_DRELU2) {
-                // 2 relu(u) = 2 sqrt(a) as a * rsqrt(a); a below the smallest
-                // normal float (where the flushing rsqrt gives inf) counts as 0
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= (a[i] >= 1.17549435e-38f) ? 2.f * a[i] * fast_rsqrt(a[i]) : 0.f;
-              } else {
-                // the dot takes the values as stored (rounded to bf16)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) dsum = fmaf(__bfloat162float(__float2bfloat16_rn(v[i])), a[i], dsum);
-              }
-            }
-            if (ep.kind == EPI_XENT) {
-              const int c8 = col0 + g * 8;
-              float e[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) e[i] = fast_exp2(fmaf(v[i], LOG2E, -xml2));
-              if (tail) {  // columns past N (the last tile's tail) do not take part
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  if (c8 + i >= N) e[i] = 0.f;
-              }
-              xsum[g] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-              if (xy >= c8 && xy < c8 + 8) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  if (xy == c8 + i) ep.xent_zy[row0 + lane] = v[i];
-              }
-            }
-            if (ep.kind == EPI_RELU2) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float t = fmaxf(v[i], 0.f);
-                v[i] = t * t;
-              }
-            }
-            if (ep.amax_out && row0 + lane < M) {
-              const int c8 = col0 + g * 8;
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                if (c8 + i < N) oam = fmaxf(oam, fabsf(v[i]));
-            }
-            store8(reinterpret_cast<bf16*>(cp0), v);
-          }
-          if (ep.kind == EPI_XENT)
-            xs += ((xsum[0] + xsum[1]) + (xsum[2] + xsum[3])) + ((xsum[4] + xsum[5]) + (xsum[6] + xsum[7]));
-        }
-        if (ep.kind == EPI_DOT && (cc & 1)) {  // a 128-column group (one head) is complete
-          const int row = row0 + lane;
-          if (row < M) {
-            const int bb = row / ep.T, t = row - bb * ep.T;
-            ep.rowdot[((long long)bb * ep.H + col0 / 128) * ep.T + t] = dsum;
-          }
-          dsum = 0.f;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          uint8_t* t0 = p0 - lane * 128;
-          if (acc32) {
-            tma_reduce_add_2d(&tmO, t0, col0, row0);
-            tma_reduce_add_2d(&tmO, t0 + TC_EPI_TILE, col0 + 32, row0);
-          } else {
-            tma_store_2d(&tmO, t0, col0, row0);
-          }
-          bulk_commit_group();
-        }
-        ++ns;
-      }
-      // (a tile cut short by the N tail still covers at least one chunk)
-      if (ep.kind == EPI_XENT && ok && row0 + lane < M)
-        ep.xent_part[(long long)(row0 + lane) * ep.xent_nt + tn] = make_float2(xm, xs);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (PAIR) mbar_arrive_cluster(map_shared_rank(&tempty[acc], 0));
-        else mbar_arrive(&tempty[acc]);
-      }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
-    }
-    // input-tile loads still in flight (issued ahead of an abort) land before the CTA exits
-    while (nw < na) {
-      const unsigned long long t0 = globaltimer_ns();
-      while (!mbar_try_wait(&abar[nw & 1u], (nw >> 1) & 1u)) {
-        if (globaltimer_ns() - t0 > 100000000ull) {
-          record_error(ERRW_TIMEOUT_DRAIN);
-          break;
-        }
-      }
-      ++nw;
-    }
-    if (lane == 0) bulk_wait0();
-    if (ep.amax_out) {
-      oam = warp_max(oam);
-      if (lane == 0) atomicMax(ep.amax_out, __float_as_uint(stored_abs_max_bf16(oam)));
+    switch (ep.kind) {
+      case EPI_STORE: run(std::integral_constant<int, EPI_STORE>{}); break;
+      case EPI_RESID: run(std::integral_constant<int, EPI_RESID>{}); break;
+      case EPI_RELU2: run(std::integral_constant<int, EPI_RELU2>{}); break;
+      case EPI_DRELU2: run(std::integral_constant<int, EPI_DRELU2>{}); break;
+      case EPI_ACCUM_F32: run(std::integral_constant<int, EPI_ACCUM_F32>{}); break;
+      case EPI_QKV: run(std::integral_constant<int, EPI_QKV>{}); break;
+      case EPI_DOT: run(std::integral_constant<int, EPI_DOT>{}); break;
+      case EPI_XENT: run(std::integral_constant<int, EPI_XENT>{}); break;
+      default: break;
     }
   }
   tc_fence_before();
