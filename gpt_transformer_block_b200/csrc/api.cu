@@ -136,19 +136,21 @@ bool make_tmap_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
   return r == CUDA_SUCCESS;
 }
 
-// fp32 [outer2][outer1][inner] view (row stride ld, plane stride ld*outer1), 128-byte swizzle;
-// a store box that runs past outer1 is clipped there (the sequence end)
-bool make_tmap_f32_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer1, uint64_t outer2, uint64_t ld,
-                      uint32_t box_inner, uint32_t box_outer) {
+// fp32 or bf16 [outer2][outer1][inner] view (row stride ld, plane stride
+// ld*outer1), 128-byte swizzle; a store box that runs past outer1 is clipped
+// there (the sequence end)
+bool make_tmap_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint64_t outer1, uint64_t outer2,
+                  uint64_t ld, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const uint64_t esz = f32 ? 4 : 2;
   cuuint64_t dims[3] = {inner, outer1, outer2};
-  cuuint64_t strides[2] = {ld * 4, ld * 4 * outer1};
+  cuuint64_t strides[2] = {ld * esz, ld * esz * outer1};
   cuuint32_t box[3] = {box_inner, box_outer, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -810,13 +812,13 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   } else {
     // tcgen05 flash backward: K/V tiles (128 rows) and Q/dO tiles (64 rows) by
     // TMA, dQ accumulated with fp32 reductions at L2 into the zeroed buffer,
-    // dK / dV written whole by TMA stores (every key row of every tile)
+    // dK / dV (bf16) written whole by TMA stores (every key row of every tile)
     CUtensorMap tkv, tq, tdo, tdk, tdv;
     bool okm = make_tmap(&tkv, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128);
     okm = okm && make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 64);
     okm = okm && make_tmap(&tdo, X.dO, false, (uint64_t)Ho, (uint64_t)m.N, (uint64_t)Ho, 64, 64);
-    okm = okm && make_tmap_f32_3d(&tdk, X.dk, (uint64_t)Kv, (uint64_t)m.T, (uint64_t)m.B, (uint64_t)Kv, 32, 32);
-    okm = okm && make_tmap_f32_3d(&tdv, X.dv, (uint64_t)Kv, (uint64_t)m.T, (uint64_t)m.B, (uint64_t)Kv, 32, 32);
+    okm = okm && make_tmap_3d(&tdk, X.dk, false, (uint64_t)Kv, (uint64_t)m.T, (uint64_t)m.B, (uint64_t)Kv, 64, 32);
+    okm = okm && make_tmap_3d(&tdv, X.dv, false, (uint64_t)Kv, (uint64_t)m.T, (uint64_t)m.B, (uint64_t)Kv, 64, 32);
     if (!okm) return GPTB_ERR_CUDA;
     CK(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AB2_SMEM));
     const int nkb = (m.T + AB2_BK - 1) / AB2_BK;
@@ -826,8 +828,9 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   }
   if constexpr (std::is_same<T, bf16>::value) {
     qkv_post_bwd_h128_kernel<<<grid_rows(m.N), EW_THREADS, 0, st>>>(
-        (const bf16*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (bf16*)X.dqkv, m.T, m.N, m.H, m.Hkv,
-        ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg, ve ? g.ve_table : nullptr, X.dz, gam[3]);
+        (const bf16*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, (const bf16*)X.dk, (const bf16*)X.dv, Kv,
+        (bf16*)X.dqkv, m.T, m.N, m.H, m.Hkv, ve ? (const bf16*)w.ve_table : nullptr, idx, S.sg,
+        ve ? g.ve_table : nullptr, X.dz, gam[3]);
   } else {
     qkv_post_bwd_kernel<T><<<grid_rows(m.N * (m.H + 2 * m.Hkv)), EW_THREADS, 0, st>>>(
         (const T*)S.qkv, m.Wq, S.rstd_qk, X.rope, X.dq, Ho, X.dk, X.dv, Kv, (T*)X.dqkv, m.T, m.N, m.H, m.Hkv, m.hd,
@@ -1315,7 +1318,8 @@ int gptb_device_error(gptb_stream_t stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return GPTB_ERR_CUDA;
-    return (v & 0xf00) == 0x200 ? GPTB_ERR_BAD_INPUT : GPTB_ERR_TIMEOUT;
+    if ((v & 0xf00) == 0x200) return GPTB_ERR_BAD_INPUT;
+    return (v & 0xf00) == 0x300 ? GPTB_ERR_CUDA : GPTB_ERR_TIMEOUT;
   }
   return GPTB_OK;
 }

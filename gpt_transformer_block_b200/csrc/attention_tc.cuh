@@ -351,7 +351,7 @@ namespace gptb {
 // 10-17 dQ epilogue (thread = hd lane of dQ^T, 32 of the 64 queries; two
 // warps per TMEM lane quarter, as the reductions are bound by how many
 // requests each warp keeps in flight).  At the end the softmax warps
-// write dK, dV (fp32) through swizzled staging tiles in the then idle Q/dO
+// write dK, dV (bf16) through swizzled staging tiles in the then idle Q/dO
 // ring and TMA stores that clip at the sequence end.
 // CTA order: groups of AB2_GROUP (kv head, sequence) pairs, key-tile-major
 // inside a group, so the tiles with the most query tiles (the first ones
@@ -367,8 +367,8 @@ constexpr int AB2_PS_TILE = 128 * 64 * 2;   // 16 KB
 constexpr int AB2_STAGES = 4;              // Q / dO / LSE / D ring
 constexpr int AB2_SMEM = 1024 + 2 * AB2_KV_TILE + 2 * AB2_STAGES * AB2_Q_TILE + AB2_PS_TILE + 256 +
                          AB2_STAGES * 2 * 64 * 4;
-// the dK / dV staging (8 warps x 4 tiles of 32 rows x 128 bytes) fits in the Q / dO ring
-static_assert(8 * 4 * 4096 <= 2 * AB2_STAGES * AB2_Q_TILE, "dK/dV staging does not fit the ring");
+// the dK / dV staging (8 warps x 2 tiles of 32 rows x 128 bytes) fits in the Q / dO ring
+static_assert(8 * 2 * 4096 <= 2 * AB2_STAGES * AB2_Q_TILE, "dK/dV staging does not fit the ring");
 
 __global__ void __launch_bounds__(AB2_THREADS, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
@@ -622,35 +622,36 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // dK, dV rows (fp32) for this CTA's keys, columns cb*64 .. cb*64+63, through
-    // four 32x32 swizzled staging tiles per warp in the (now idle) Q/dO ring
+    // dK, dV rows (bf16) for this CTA's keys, columns cb*64 .. cb*64+63, through
+    // two 32-row x 128-byte swizzled staging tiles per warp in the (now idle) Q/dO ring
     if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(acc_done, 0, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
       tc_fence_after();
-      uint8_t* stg = sQ + (warp - 2) * 4 * 4096;
+      uint8_t* stg = sQ + (warp - 2) * 2 * 4096;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(lane_addr + which * 128 + cb * 64, v0);
+        tmem_ld_32x32b_x32(lane_addr + which * 128 + cb * 64 + 32, v1);
+        tmem_ld_wait();
+        uint8_t* prow = stg + which * 4096 + lane * 128;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(lane_addr + which * 128 + cb * 64 + c * 32, v);
-          tmem_ld_wait();
-          uint8_t* prow = stg + (which * 2 + c) * 4096 + lane * 128;
+        for (int g = 0; g < 8; ++g) {  // 16-byte chunk g: columns 8g .. 8g+7
+          uint32_t w[4];
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<float4*>(prow + ((g ^ (lane & 7)) << 4)) =
-                make_float4(__uint_as_float(v[g * 4]), __uint_as_float(v[g * 4 + 1]), __uint_as_float(v[g * 4 + 2]),
-                            __uint_as_float(v[g * 4 + 3]));
+          for (int j = 0; j < 4; ++j) {
+            const int c0 = g * 8 + 2 * j;
+            const float lo = __uint_as_float(c0 < 32 ? v0[c0] : v1[c0 - 32]);
+            const float hi = __uint_as_float(c0 + 1 < 32 ? v0[c0 + 1] : v1[c0 + 1 - 32]);
+            w[j] = pack_bf16(lo, hi);
+          }
+          *reinterpret_cast<uint4*>(prow + ((g ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0 && k0 + qw * 32 < T) {  // (a box wholly past the sequence end is not issued)
-#pragma unroll
-        for (int which = 0; which < 2; ++which)
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            tma_store_3d(which == 0 ? &tm_dk : &tm_dv, stg + (which * 2 + c) * 4096, kvh * 128 + cb * 64 + c * 32,
-                         k0 + qw * 32, b);
+        tma_store_3d(&tm_dk, stg, kvh * 128 + cb * 64, k0 + qw * 32, b);
+        tma_store_3d(&tm_dv, stg + 4096, kvh * 128 + cb * 64, k0 + qw * 32, b);
         bulk_commit_group();
         bulk_wait0();
       }

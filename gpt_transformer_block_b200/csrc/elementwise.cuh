@@ -601,6 +601,12 @@ __device__ __forceinline__ void ld4(const bf16* p, float (&v)[4]) {
   const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
   v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
 }
+__device__ __forceinline__ void load4(const bf16* p, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
 __device__ __forceinline__ void st4(bf16* p, const float (&v)[4]) {
   uint2 u;
   u.x = pack_bf16(v[0], v[1]);
@@ -616,7 +622,7 @@ constexpr int QKV_BWD_HEADS = 2;
 __global__ void __launch_bounds__(EW_THREADS, 4)
     qkv_post_bwd_h128_kernel(const bf16* __restrict__ qkv, long long ld, const float* __restrict__ rstd_qk,
                              const float2* __restrict__ rope, const float* __restrict__ dq, long long lddq,
-                             const float* __restrict__ dk, const float* __restrict__ dv, long long lddkv,
+                             const bf16* __restrict__ dk, const bf16* __restrict__ dv, long long lddkv,
                              bf16* __restrict__ dqkv, int Tn, long long N, int H, int Hkv,
                              const bf16* __restrict__ ve_table, const int32_t* __restrict__ idx,
                              const float* __restrict__ sg, float* __restrict__ dve_table, float* __restrict__ dz,
@@ -651,8 +657,13 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
       for (int b = 0; b < QB; ++b) {
         const int hh = h0 + b;
         if (hh < nqk) {
-          const float* gp = (hh < H) ? dq + n * lddq + (long long)hh * 128 : dk + n * lddkv + (long long)(hh - H) * 128;
-          g4[b] = *reinterpret_cast<const float4*>(gp + lane * 4);
+          if (hh < H) {  // dq: fp32 (summed over key tiles by reductions); dk: bf16
+            g4[b] = *reinterpret_cast<const float4*>(dq + n * lddq + (long long)hh * 128 + lane * 4);
+          } else {
+            float t4[4];
+            load4(dk + n * lddkv + (long long)(hh - H) * 128 + lane * 4, t4);
+            g4[b] = make_float4(t4[0], t4[1], t4[2], t4[3]);
+          }
           yb[b] = *reinterpret_cast<const uint2*>(yrow + (long long)hh * 128);
           r[b] = rstd_qk[n * nqk + hh];
         }
@@ -698,7 +709,9 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
       for (int b = 0; b < QB; ++b) {
         const int kv = k0 + b;
         if (kv < Hkv) {
-          g4[b] = *reinterpret_cast<const float4*>(dv + n * lddkv + (long long)kv * 128 + lane * 4);
+          float t4[4];
+          load4(dv + n * lddkv + (long long)kv * 128 + lane * 4, t4);
+          g4[b] = make_float4(t4[0], t4[1], t4[2], t4[3]);
           if (ve_table) {
             eb[b] = *reinterpret_cast<const uint2*>(ve_table + ve_row + (long long)kv * 128);
             sv[b] = sg[n * Hkv + kv];

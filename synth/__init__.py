@@ -59,6 +59,8 @@ CONFIGS = {
                       [1024 if i % 2 == 0 else -1 for i in range(20)]),
     "d24": _stack("d24", 24, 1536, 12, 12, [-1] * 24),
     "d26_fp8": _stack("d26_fp8", 26, 1664, 13, 13, [-1] * 26, dtype="fp8"),
+    # the d26 shape in bf16: the reference point for the FP8 configuration's step time
+    "d26_bf16": _stack("d26_bf16", 26, 1664, 13, 13, [-1] * 26),
     # the FP8 variant of the next rows: e5m2 gradient operands and an FP8 lm_head
     "d26_fp8_e5m2": dict(_stack("d26_fp8_e5m2", 26, 1664, 13, 13, [-1] * 26, dtype="fp8"),
                          fp8_grad="e5m2", fp8_lm_head=True),
