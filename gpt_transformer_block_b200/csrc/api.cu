@@ -1318,8 +1318,7 @@ int gptb_device_error(gptb_stream_t stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return GPTB_ERR_CUDA;
-    if ((v & 0xf00) == 0x200) return GPTB_ERR_BAD_INPUT;
-    return (v & 0xf00) == 0x300 ? GPTB_ERR_CUDA : GPTB_ERR_TIMEOUT;
+    return (v & 0xf00) == 0x200 ? GPTB_ERR_BAD_INPUT : GPTB_ERR_TIMEOUT;
   }
   return GPTB_OK;
 }

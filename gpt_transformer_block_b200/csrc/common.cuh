@@ -31,8 +31,6 @@ enum : int {
   ERRW_TIMEOUT_PROBE = 0x105,
   // invalid input data found on the device (codes 0x2xx)
   ERRW_BAD_TARGET = 0x201,  // a cross-entropy target outside [0, vocab)
-  // a kernel could not lay out its shared memory (codes 0x3xx)
-  ERRW_SMEM_LAYOUT = 0x301,
 };
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_error_word, 0, code); }
@@ -317,10 +315,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // named barrier over a subset of the CTA's warps
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-// arrive at a named barrier without waiting (the other threads of the count sync on it)
-__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Shared-memory matrix descriptor (tcgen05), 128-byte swizzle.

@@ -354,9 +354,7 @@ int gptb_cast_bf16_f32(const void* x, float* y, long long n, float scale, gptb_s
  * Returns GPTB_OK, GPTB_ERR_TIMEOUT if a bounded wait inside a kernel expired
  * (the kernel recorded it, drained and returned), GPTB_ERR_BAD_INPUT if a
  * kernel found invalid input data (a cross-entropy target outside
- * [0, vocab)), or GPTB_ERR_CUDA (a CUDA error, or a kernel that returned
- * without work because its dynamic shared memory was not aligned as it
- * needs). */
+ * [0, vocab)), or GPTB_ERR_CUDA. */
 int gptb_device_error(gptb_stream_t stream);
 
 /* Self-test of the bounded waits: sets the wait limit to limit_ns, launches
