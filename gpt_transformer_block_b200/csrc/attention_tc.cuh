@@ -565,40 +565,33 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
       const float4* l2v = reinterpret_cast<const float4*>(sLD + st * 128 + cb * 32);
       const float4* ddv = reinterpret_cast<const float4*>(sLD + st * 128 + 64 + cb * 32);
       // P^T and dS^T for this warp's 32 queries, packed to bf16 pairs (query
-      // 2j in the low half), in two halves of 16 queries
+      // 2j in the low half); S^T and dP^T come in with one TMEM round trip
       uint32_t pu[16], du[16];
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sv[16], dv[16];
-        tmem_ld_32x32b_x16(lane_addr + 256 + cb * 32 + hf * 16, sv);
-        tmem_ld_32x32b_x16(lane_addr + 320 + cb * 32 + hf * 16, dv);
-        float l2[16], dd[16];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float4 a = l2v[hf * 4 + g], d = ddv[hf * 4 + g];
-          l2[g * 4] = a.x; l2[g * 4 + 1] = a.y; l2[g * 4 + 2] = a.z; l2[g * 4 + 3] = a.w;
-          dd[g * 4] = d.x; dd[g * 4 + 1] = d.y; dd[g * 4 + 2] = d.z; dd[g * 4 + 3] = d.w;
-        }
+      {
+        uint32_t sv[32], dv[32];
+        tmem_ld_32x32b_x32(lane_addr + 256 + cb * 32, sv);
+        tmem_ld_32x32b_x32(lane_addr + 320 + cb * 32, dv);
         tmem_ld_wait();
-        if (hf == 1) {
-          // S^T / dP^T are in registers: the next step's products may overwrite them
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_empty);
-        }
+        // S^T / dP^T are in registers: the next step's products may overwrite them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty);
 #pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) {
-          float pe[2], de[2];
+        for (int g = 0; g < 8; ++g) {
+          const float4 a = l2v[g], d = ddv[g];
+          const float l2[4] = {a.x, a.y, a.z, a.w}, dd[4] = {d.x, d.y, d.z, d.w};
+          float pe[4], de[4];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = e2 * 2 + h2;
-            const int t = tq + hf * 16 + e;
+          for (int e = 0; e < 4; ++e) {
+            const int t = tq + g * 4 + e;
             const bool vis = !need_mask || (t >= q_vis_lo && t <= q_vis_hi);
-            pe[h2] = vis ? fast_exp2(fmaf(__uint_as_float(sv[e]), sl2, -l2[e])) : 0.f;
-            de[h2] = pe[h2] * (__uint_as_float(dv[e]) - dd[e]) * scale;
+            pe[e] = vis ? fast_exp2(fmaf(__uint_as_float(sv[g * 4 + e]), sl2, -l2[e])) : 0.f;
+            de[e] = pe[e] * (__uint_as_float(dv[g * 4 + e]) - dd[e]) * scale;
           }
-          pu[hf * 8 + e2] = pack_bf16(pe[0], pe[1]);
-          du[hf * 8 + e2] = pack_bf16(de[0], de[1]);
+          pu[g * 2] = pack_bf16(pe[0], pe[1]);
+          pu[g * 2 + 1] = pack_bf16(pe[2], pe[3]);
+          du[g * 2] = pack_bf16(de[0], de[1]);
+          du[g * 2 + 1] = pack_bf16(de[2], de[3]);
         }
       }
       // the previous step's dV/dK/dQ MMAs must be done reading P^T / dS^T
