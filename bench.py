@@ -236,8 +236,17 @@ def run_optimizer(args, c: dict):
         w = torch.randn(m, n, device="cuda", generator=g).mul_(0.02)
         mats.append(dict(w=w, wb=w.bfloat16(), g=torch.randn(m, n, device="cuda", generator=g),
                          buf=torch.zeros(m, n, device="cuda"), v=torch.zeros(m, device="cuda"), m=m, n=n))
-    ws = torch.empty(max(gb.gptb_muon_workspace_bytes(m, n, len(coeffs)) for m, n in shapes),
-                     dtype=torch.uint8, device="cuda")
+    # matrices of one shape (one per layer) take one batched Muon call: every
+    # Polar Express product is one GEMM launch over the whole group
+    groups = {}
+    for x in mats:
+        groups.setdefault((x["m"], x["n"]), []).append(x)
+    if args.muon_per_matrix:
+        ws = torch.empty(max(gb.gptb_muon_workspace_bytes(m, n, len(coeffs)) for m, n in shapes),
+                         dtype=torch.uint8, device="cuda")
+    else:
+        ws = torch.empty(max(gb.gptb_muon_batched_workspace_bytes(len(grp), m, n, len(coeffs))
+                             for (m, n), grp in groups.items()), dtype=torch.uint8, device="cuda")
     n_adam = c["vocab"] * d * 2 + sum(c["has_ve"]) * c["vocab"] * c["n_kv_head"] * c["head_dim"]
     p = torch.randn(n_adam, device="cuda", generator=g)
     gr = torch.randn(n_adam, device="cuda", generator=g)
@@ -245,9 +254,15 @@ def run_optimizer(args, c: dict):
     pb = torch.empty(n_adam, dtype=torch.bfloat16, device="cuda")
 
     def muon_all():
-        for x in mats:
-            gb.gptb_muon_step(x["w"], x["wb"], x["g"], x["buf"], x["v"], x["m"], x["n"], coeffs, 0.02, 0.95, 0.95,
-                              0.0, ws)
+        if args.muon_per_matrix:
+            for x in mats:
+                gb.gptb_muon_step(x["w"], x["wb"], x["g"], x["buf"], x["v"], x["m"], x["n"], coeffs, 0.02, 0.95,
+                                  0.95, 0.0, ws)
+            return
+        for (m, n), grp in groups.items():
+            gb.gptb_muon_step_batched([x["w"] for x in grp], [x["wb"] for x in grp], [x["g"] for x in grp],
+                                      [x["buf"] for x in grp], [x["v"] for x in grp], m, n, coeffs, 0.02, 0.95, 0.95,
+                                      0.0, ws)
 
     def adam(t):
         gb.gptb_adamw_step(p, gr, m1, m2, pb, n_adam, 1e-3, 0.8, 0.95, 1e-10, 0.0, t)
@@ -287,6 +302,7 @@ def run_optimizer(args, c: dict):
             "value": t_mu + t_ad, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": False, "dtype": "bf16 GEMMs / f32 elementwise", "data": "synthetic",
             "config": {"workload": c["name"] + "_optimizer", "matrices": len(shapes), "ns_steps": len(coeffs),
+                       "muon_calls": len(mats) if args.muon_per_matrix else len(groups),
                        "adamw_params": n_adam},
             "muon": {"ms": t_mu, "polar_express_flops": flops, "achieved": tf, "unit": "TFLOP/s",
                      "peak": peaks["bf16_tflops"], "frac": tf / peaks["bf16_tflops"],
@@ -384,6 +400,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
     ap.add_argument("--optimizer", action="store_true",
                     help="time the optimizer step (Muon + AdamW) instead of the training step")
+    ap.add_argument("--muon-per-matrix", action="store_true",
+                    help="with --optimizer: one Muon call per matrix instead of one batched call per shape")
     ap.add_argument("--decode", action="store_true",
                     help="time one decode step of attention over a full KV cache instead of the training step")
     args = ap.parse_args()

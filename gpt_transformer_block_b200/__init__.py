@@ -25,7 +25,8 @@ EXPORTS = [
     "gptb_reset_counters", "gptb_launch_count", "gptb_set_gemm_timing", "gptb_gemm_timing",
     "gptb_error_string", "lm_head_xent_noalloc", "gptb_probe_bounded_wait",
     "gptb_adamw_step", "gptb_polar_express_workspace_bytes", "gptb_polar_express", "gptb_decode_attention",
-    "gptb_muon_workspace_bytes", "gptb_muon_step", "gpt_stack_step_hooked", "gptb_cast_f32_bf16",
+    "gptb_muon_workspace_bytes", "gptb_muon_step", "gptb_muon_batched_workspace_bytes", "gptb_muon_step_batched",
+    "gptb_gemm_bf16_batched", "gpt_stack_step_hooked", "gptb_cast_f32_bf16",
     "gptb_cast_bf16_f32", "gptb_decode_workspace_bytes", "gptb_gemm_fp8_workspace_bytes", "gptb_gemm_fp8",
 ]
 
@@ -124,10 +125,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptb_muon_step.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _fp, ctypes.c_int,
                                    ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp,
                                    ctypes.c_size_t, _vp]
+    lib.gptb_muon_batched_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.gptb_muon_batched_workspace_bytes.restype = ctypes.c_size_t
+    lib.gptb_muon_step_batched.argtypes = [ctypes.c_int, P(_vp), P(_vp), P(_vp), P(_vp), P(_vp), ctypes.c_int,
+                                           ctypes.c_int, _fp, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                           ctypes.c_float, ctypes.c_float, _vp, ctypes.c_size_t, _vp]
+    lib.gptb_gemm_bf16_batched.argtypes = [_vp, ctypes.c_int, ctypes.c_longlong, ctypes.c_longlong, _vp, ctypes.c_int,
+                                           ctypes.c_longlong, ctypes.c_longlong, _vp, ctypes.c_int,
+                                           ctypes.c_longlong, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, _vp]
     for name in EXPORTS:
         if name not in ("gptb_workspace_bytes", "gptb_error_string", "gptb_reset_counters",
                         "gptb_launch_count", "gptb_polar_express_workspace_bytes", "gptb_muon_workspace_bytes",
-                        "gptb_decode_workspace_bytes", "gptb_gemm_fp8_workspace_bytes"):
+                        "gptb_decode_workspace_bytes", "gptb_gemm_fp8_workspace_bytes",
+                        "gptb_muon_batched_workspace_bytes"):
             getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -286,6 +297,11 @@ def gptb_gemm_bf16(A, a_mn, lda, B, b_mn, ldb, C, c_f32, ldc, M, N, K, stream=No
                                  M, N, K, _stream(stream)), "gptb_gemm_bf16")
 
 
+def gptb_gemm_bf16_batched(A, a_mn, lda, sa, B, b_mn, ldb, sb, C, c_f32, ldc, sc, M, N, K, batch, stream=None):
+    _check(load().gptb_gemm_bf16_batched(ptr(A), int(a_mn), lda, sa, ptr(B), int(b_mn), ldb, sb, ptr(C), int(c_f32),
+                                         ldc, sc, M, N, K, int(batch), _stream(stream)), "gptb_gemm_bf16_batched")
+
+
 def gptb_adamw_step(p, g, m, v, p_bf16, n, lr, beta1, beta2, eps, weight_decay, step, stream=None):
     """One AdamW step over n fp32 parameters in place (p, m, v); p_bf16 (or None)
     receives the bf16 copy of the new parameters."""
@@ -320,6 +336,28 @@ def gptb_muon_step(w, w_bf16, g, buf, v, m, n, coeffs, lr, mu, beta2, weight_dec
     _check(load().gptb_muon_step(ptr(w), ptr(w_bf16), ptr(g), ptr(buf), ptr(v), int(m), int(n), arr, len(coeffs),
                                  float(lr), float(mu), float(beta2), float(weight_decay), ptr(workspace), nbytes,
                                  _stream(stream)), "gptb_muon_step")
+
+
+def gptb_muon_batched_workspace_bytes(count: int, m: int, n: int, steps: int) -> int:
+    return int(load().gptb_muon_batched_workspace_bytes(int(count), int(m), int(n), int(steps)))
+
+
+def gptb_muon_step_batched(ws, wbs, gs, bufs, vs, m, n, coeffs, lr, mu, beta2, weight_decay, workspace, stream=None):
+    """gptb_muon_step on len(ws) same-shape matrices at once (lists of tensors; wbs entries may be None)."""
+    count = len(ws)
+    if not (len(wbs) == len(gs) == len(bufs) == len(vs) == count):
+        raise ValueError("gptb_muon_step_batched: the per-matrix lists differ in length")
+    arr_t = _vp * count
+
+    def arr(ts):
+        return arr_t(*[ptr(t) if t is not None else None for t in ts])
+
+    flat = [float(x) for abc in coeffs for x in abc]
+    cf = (ctypes.c_float * len(flat))(*flat)
+    nbytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
+    _check(load().gptb_muon_step_batched(count, arr(ws), arr(wbs), arr(gs), arr(bufs), arr(vs), int(m), int(n), cf,
+                                         len(coeffs), float(lr), float(mu), float(beta2), float(weight_decay),
+                                         ptr(workspace), nbytes, _stream(stream)), "gptb_muon_step_batched")
 
 
 def gptb_decode_workspace_bytes(B: int, H: int, T_max: int) -> int:

@@ -121,18 +121,23 @@ bool make_tmap(CUtensorMap* m, const void* ptr, bool fp8, uint64_t inner, uint64
   return r == CUDA_SUCCESS;
 }
 
-// 2-D fp32 tensor map (TMA store / bulk reduce-add target), optional 128-byte swizzle
-bool make_tmap_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
-                   uint32_t box_outer, bool sw128) {
+// GEMM operand maps: [batch][outer][inner] (row stride ld, batch stride bs
+// elements; batch 1 is the plain matrix), 128-byte swizzle
+bool make_tmap_gemm(CUtensorMap* m, const void* ptr, int esz, uint64_t inner, uint64_t outer, uint64_t ld,
+                    uint32_t box_inner, uint32_t box_outer, int batch, long long bs) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 4};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (batch > 1 && (bs <= 0 || (bs * esz) % 16)) return false;
+  const uint64_t bstride = (batch > 1 ? (uint64_t)bs : ld * outer) * (uint64_t)esz;
+  cuuint64_t dims[3] = {inner, outer, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {ld * (uint64_t)esz, bstride};
+  cuuint32_t box[3] = {box_inner, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType dt = esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -215,15 +220,16 @@ int max_pair_clusters(K kern, int smem) {
 
 template <bool AM, bool BM, bool F8, bool PAIR>
 int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const CUtensorMap& to2,
-              const CUtensorMap& tx, int M, int N, int K, int splits, const EpiParams& ep, cudaStream_t st) {
+              const CUtensorMap& tx, int M, int N, int K, int splits, int nbatch, const EpiParams& ep,
+              cudaStream_t st) {
   auto kern = gemm_tc_kernel<AM, BM, F8, PAIR>;
   const int smem = TcShape<PAIR>::SMEM;
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const long long units = (long long)((M + TcShape<PAIR>::TILE_M - 1) / TcShape<PAIR>::TILE_M) *
-                          ((N + TC_BN - 1) / TC_BN) * splits;
+                          ((N + TC_BN - 1) / TC_BN) * splits * nbatch;
   if (!PAIR) {
     const int grid = (int)std::min<long long>(units, dev_info().sms);
-    kern<<<grid, TC_THREADS, smem, st>>>(ta, tb, to, to2, tx, M, N, K, splits, ep);
+    kern<<<grid, TC_THREADS, smem, st>>>(ta, tb, to, to2, tx, M, N, K, splits, nbatch, ep);
   } else {
     const int clusters = (int)std::min<long long>(units, max_pair_clusters(kern, smem));
     cudaLaunchConfig_t cfg = {};
@@ -238,7 +244,7 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, to2, tx, M, N, K, splits, ep) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, to2, tx, M, N, K, splits, nbatch, ep) != cudaSuccess) {
       cudaGetLastError();
       LAUNCHED();
       return GPTB_ERR_CUDA;
@@ -254,8 +260,16 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
 #define GPTB_PAIR_MIN_M 256
 #endif
 
-int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t st) {
-  if (M <= 0 || N <= 0) return GPTB_OK;
+// C[b] = A[b] op B[b] for b < batch: operand b starts bs* elements after
+// operand 0 (tensor-core path only; the epilogue kinds with per-row side
+// outputs take batch 1)
+int gemm_batched(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, int batch, long long bsA, long long bsB,
+                 long long bsO, long long bsX, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || batch == 0) return GPTB_OK;
+  if (batch < 0) return GPTB_ERR_INVALID_ARG;
+  if (batch > 1 && (dtype == GPTB_F32 || ep.kind == EPI_XENT || ep.kind == EPI_QKV || ep.kind == EPI_DOT ||
+                    ep.amax_out))
+    return GPTB_ERR_UNSUPPORTED;
   if (K <= 0) return ep.kind == EPI_ACCUM_F32 ? GPTB_OK : GPTB_ERR_INVALID_ARG;
   cudaEvent_t ea = nullptr, eb = nullptr;
   bool timed = false;
@@ -304,14 +318,17 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
     const bool pair = M >= GPTB_PAIR_MIN_M;
     const int b_rows = pair ? TcShape<true>::B_ROWS : TcShape<false>::B_ROWS;  // rows of B one CTA stages
     CUtensorMap ta, tb, to, to2, tx;
-    bool ok = A.mn ? make_tmap(&ta, A.p, f8, M, K, A.ld, bk, bk) : make_tmap(&ta, A.p, f8, K, M, A.ld, bk, TC_BM);
-    ok = ok && (B.mn ? make_tmap(&tb, B.p, f8, N, K, B.ld, bk, bk) : make_tmap(&tb, B.p, f8, K, N, B.ld, bk, b_rows));
+    const int oe = f8 ? 1 : 2;  // operand element size
+    bool ok = A.mn ? make_tmap_gemm(&ta, A.p, oe, M, K, A.ld, bk, bk, batch, bsA)
+                   : make_tmap_gemm(&ta, A.p, oe, K, M, A.ld, bk, TC_BM, batch, bsA);
+    ok = ok && (B.mn ? make_tmap_gemm(&tb, B.p, oe, N, K, B.ld, bk, bk, batch, bsB)
+                     : make_tmap_gemm(&tb, B.p, oe, K, N, B.ld, bk, b_rows, batch, bsB));
     // epilogue maps: 32-row boxes of 64 bf16 / 32 fp32 columns, 128-byte swizzle
-    ok = ok && (acc32 ? make_tmap_f32(&to, ep.out, N, M, ep.ldo, 32, 32, true)
-                      : make_tmap(&to, ep.out, false, N, M, ep.ldo, 64, 32));
+    ok = ok && (acc32 ? make_tmap_gemm(&to, ep.out, 4, N, M, ep.ldo, 32, 32, batch, bsO)
+                      : make_tmap_gemm(&to, ep.out, 2, N, M, ep.ldo, 64, 32, batch, bsO));
     to2 = to;
     tx = to;
-    if (ok && has_aux) ok = make_tmap(&tx, ep.aux, false, N, M, ep.ld_aux, 64, 32);
+    if (ok && has_aux) ok = make_tmap_gemm(&tx, ep.aux, 2, N, M, ep.ld_aux, 64, 32, batch, bsX);
     if (!ok) return GPTB_ERR_CUDA;
     int splits = 1;
     if (ep.kind == EPI_ACCUM_F32) {
@@ -321,29 +338,33 @@ int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t 
     }
     const int sel = (A.mn ? 1 : 0) | (B.mn ? 2 : 0) | (f8 ? 4 : 0) | (pair ? 8 : 0);
     switch (sel) {
-      case 0: rc = launch_tc<false, false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 1: rc = launch_tc<true, false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 2: rc = launch_tc<false, true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 3: rc = launch_tc<true, true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 4: rc = launch_tc<false, false, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 6: rc = launch_tc<false, true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 7: rc = launch_tc<true, true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 8: rc = launch_tc<false, false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 9: rc = launch_tc<true, false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 10: rc = launch_tc<false, true, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 11: rc = launch_tc<true, true, false, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 12: rc = launch_tc<false, false, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 14: rc = launch_tc<false, true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
-      case 15: rc = launch_tc<true, true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, ep, st); break;
+      case 0: rc = launch_tc<false, false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 1: rc = launch_tc<true, false, false, false>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 2: rc = launch_tc<false, true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 3: rc = launch_tc<true, true, false, false>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 4: rc = launch_tc<false, false, true, false>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 6: rc = launch_tc<false, true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 7: rc = launch_tc<true, true, true, false>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 8: rc = launch_tc<false, false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 9: rc = launch_tc<true, false, false, true>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 10: rc = launch_tc<false, true, false, true>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 11: rc = launch_tc<true, true, false, true>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 12: rc = launch_tc<false, false, true, true>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 14: rc = launch_tc<false, true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
+      case 15: rc = launch_tc<true, true, true, true>(ta, tb, to, to2, tx, M, N, K, splits, batch, ep, st); break;
       default: rc = GPTB_ERR_UNSUPPORTED;  // e4m3 with A M-major and B K-major: not used
     }
   }
   if (timed) {
     cudaEventRecord(eb, st);
     std::lock_guard<std::mutex> lk(g_timing_mu);
-    g_timed.push_back({ea, eb, 2.0 * M * (double)N * K, dtype == GPTB_FP8_E4M3});
+    g_timed.push_back({ea, eb, 2.0 * M * (double)N * K * batch, dtype == GPTB_FP8_E4M3});
   }
   return rc;
+}
+
+int gemm(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, cudaStream_t st) {
+  return gemm_batched(dtype, A, B, M, N, K, ep, 1, 0, 0, 0, 0, st);
 }
 
 EpiParams epi(int kind, int dtype, void* out, long long ldo, const void* aux = nullptr, long long ld_aux = 0,
@@ -1092,6 +1113,16 @@ int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_
   return gemm(GPTB_BF16, {A, lda, a_mn != 0}, {B, ldb, b_mn != 0}, M, N, K, e, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int gptb_gemm_bf16_batched(const void* A, int a_mn, long long lda, long long stride_a, const void* B, int b_mn,
+                           long long ldb, long long stride_b, void* C, int c_f32, long long ldc, long long stride_c,
+                           int M, int N, int K, int batch, gptb_stream_t stream) {
+  if (!A || !B || !C || M < 0 || N < 0 || K < 0 || batch < 1) return GPTB_ERR_INVALID_ARG;
+  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  EpiParams e = epi(c_f32 ? EPI_ACCUM_F32 : EPI_STORE, GPTB_BF16, C, ldc);
+  return gemm_batched(GPTB_BF16, {A, lda, a_mn != 0}, {B, ldb, b_mn != 0}, M, N, K, e, batch, stride_a, stride_b,
+                      stride_c, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t gptb_gemm_fp8_workspace_bytes(int M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   return ((size_t)M * K + 255) / 256 * 256 + ((size_t)N * K + 255) / 256 * 256 + 256;
@@ -1146,60 +1177,72 @@ constexpr size_t PE_HEADER = 1024;  // sum of squares (4 B) at 0, coefficients (
 size_t pe_align(size_t b) { return (b + 255) & ~size_t(255); }
 }  // namespace
 
-size_t gptb_polar_express_workspace_bytes(int m, int n, int steps) {
-  if (m <= 0 || n <= 0 || steps < 1 || steps > 64) return 0;
+// Polar Express workspace for `count` matrices of m x n: header (per-matrix
+// sums of squares at 0, coefficients at 256), two count x m x n iterates,
+// and count Gram matrices A and B of the smaller side
+constexpr int PE_MAX_BATCH = 64;
+size_t pe_bytes(int count, int m, int n, int steps) {
+  if (count <= 0 || count > PE_MAX_BATCH || m <= 0 || n <= 0 || steps < 1 || steps > 64) return 0;
   const size_t s = (size_t)std::min(m, n);
-  return PE_HEADER + 2 * pe_align((size_t)m * n * 2) + 2 * pe_align(s * s * 2);
+  return PE_HEADER + 2 * pe_align((size_t)count * m * n * 2) + 2 * pe_align((size_t)count * s * s * 2);
 }
+
+size_t gptb_polar_express_workspace_bytes(int m, int n, int steps) { return pe_bytes(1, m, n, steps); }
 
 }  // extern "C"
 
 namespace {
 // The Polar Express loop on a bf16 [m, n] matrix into out (workspace laid out
 // as gptb_polar_express_workspace_bytes describes; arguments already checked).
-int polar_express_impl(const void* G, void* out, int m, int n, const float* coeffs, int steps, uint8_t* w,
+int polar_express_impl(const void* G, void* out, int m, int n, int count, const float* coeffs, int steps, uint8_t* w,
                        cudaStream_t st) {
   const size_t ne = (size_t)m * n;
-  float* sumsq = reinterpret_cast<float*>(w);
+  float* sumsq = reinterpret_cast<float*>(w);  // [count]
   float* cf = reinterpret_cast<float*>(w + 256);
   bf16* X[2];
   X[0] = reinterpret_cast<bf16*>(w + PE_HEADER);
-  X[1] = reinterpret_cast<bf16*>(w + PE_HEADER + pe_align(ne * 2));
+  X[1] = reinterpret_cast<bf16*>(w + PE_HEADER + pe_align(count * ne * 2));
   const bool wide = m < n;
   const int s = wide ? m : n;  // side of the Gram matrix
-  bf16* A = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(ne * 2));
-  bf16* Bm = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(ne * 2) + pe_align((size_t)s * s * 2));
+  const size_t ss = (size_t)s * s;
+  bf16* A = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(count * ne * 2));
+  bf16* Bm = reinterpret_cast<bf16*>(w + PE_HEADER + 2 * pe_align(count * ne * 2) + pe_align(count * ss * 2));
   // the coefficients travel in the launch parameters (the host array is read here)
   HostFloats192 hc;
   std::memcpy(hc.v, coeffs, sizeof(float) * 3 * steps);
-  store_floats_kernel<<<1, 32, 0, st>>>(hc, 3 * steps, cf, sumsq);
+  store_floats_kernel<<<1, 64, 0, st>>>(hc, 3 * steps, cf, sumsq, count);
   CKL();
-  const int grid = (int)std::max<long long>(1, std::min<long long>(((long long)ne + 255) / 256, dev_info().sms * 8LL));
-  sumsq_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16*>(G), (long long)ne, sumsq);
+  const int grid = (int)std::max<long long>(1, std::min<long long>(((long long)ne + 255) / 256, dev_info().sms * 8LL / count + 1));
+  sumsq_bf16_kernel<<<dim3(grid, count), 256, 0, st>>>(static_cast<const bf16*>(G), (long long)ne, sumsq, (long long)ne);
   CKL();
-  scale_by_norm_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16*>(G), X[0], (long long)ne, sumsq, 1e-7f);
+  scale_by_norm_bf16_kernel<<<dim3(grid, count), 256, 0, st>>>(static_cast<const bf16*>(G), X[0], (long long)ne, sumsq,
+                                                               1e-7f, (long long)ne);
   CKL();
+  // every product runs once over the whole batch (one launch, count slices)
+  const long long bne = (long long)ne, bss = (long long)ss;
   bf16* cur = X[0];
   for (int t = 0; t < steps; ++t) {
     const float* a = cf + 3 * t;
     bf16* nxt = (t == steps - 1) ? static_cast<bf16*>(out) : X[(t + 1) & 1];
     // A = Gram matrix of the smaller side (X^T X for a tall X, X X^T for a wide one)
     if (!wide)
-      TRY(gemm(GPTB_BF16, {cur, n, true}, {cur, n, true}, n, n, m, epi(EPI_STORE, GPTB_BF16, A, n), st));
+      TRY(gemm_batched(GPTB_BF16, {cur, n, true}, {cur, n, true}, n, n, m, epi(EPI_STORE, GPTB_BF16, A, n), count, bne,
+                       bne, bss, 0, st));
     else
-      TRY(gemm(GPTB_BF16, {cur, n, false}, {cur, n, false}, m, m, n, epi(EPI_STORE, GPTB_BF16, A, m), st));
+      TRY(gemm_batched(GPTB_BF16, {cur, n, false}, {cur, n, false}, m, m, n, epi(EPI_STORE, GPTB_BF16, A, m), count,
+                       bne, bne, bss, 0, st));
     // B = b A + c A A   (A symmetric, so A A = A A^T)
     EpiParams eb = epi(EPI_RESID, GPTB_BF16, Bm, s, A, s);
     eb.alpha = a + 2;
     eb.beta = a + 1;
-    TRY(gemm(GPTB_BF16, {A, s, false}, {A, s, false}, s, s, s, eb, st));
+    TRY(gemm_batched(GPTB_BF16, {A, s, false}, {A, s, false}, s, s, s, eb, count, bss, bss, bss, bss, st));
     // X = a X + X B   (B symmetric); for a wide X the same update of X^T reads X = a X + B X
     EpiParams ex = epi(EPI_RESID, GPTB_BF16, nxt, n, cur, n);
     ex.beta = a;
     if (!wide)
-      TRY(gemm(GPTB_BF16, {cur, n, false}, {Bm, s, false}, m, n, n, ex, st));
+      TRY(gemm_batched(GPTB_BF16, {cur, n, false}, {Bm, s, false}, m, n, n, ex, count, bne, bss, bne, bne, st));
     else
-      TRY(gemm(GPTB_BF16, {Bm, s, false}, {cur, n, true}, m, n, m, ex, st));
+      TRY(gemm_batched(GPTB_BF16, {Bm, s, false}, {cur, n, true}, m, n, m, ex, count, bss, bne, bne, bne, st));
     cur = nxt;
   }
   return GPTB_OK;
@@ -1220,48 +1263,78 @@ int gptb_polar_express(const void* G, void* out, int m, int n, const float* coef
   }
   if (workspace_bytes < gptb_polar_express_workspace_bytes(m, n, steps)) return GPTB_ERR_WORKSPACE;
   if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
-  return polar_express_impl(G, out, m, n, coeffs, steps, static_cast<uint8_t*>(workspace),
+  return polar_express_impl(G, out, m, n, 1, coeffs, steps, static_cast<uint8_t*>(workspace),
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
-size_t gptb_muon_workspace_bytes(int m, int n, int steps) {
-  const size_t pe = gptb_polar_express_workspace_bytes(m, n, steps);
+// Muon workspace for `count` matrices: the batched Polar Express workspace,
+// the bf16 inputs u and outputs o, per-row step sizes, two sums per matrix
+size_t muon_bytes(int count, int m, int n, int steps) {
+  const size_t pe = pe_bytes(count, m, n, steps);
   if (pe == 0) return 0;
-  // Polar Express workspace, the bf16 input u and output o, per-row step sizes, two sums
-  return pe + 2 * pe_align((size_t)m * n * 2) + pe_align((size_t)m * 4) + 256;
+  return pe + 2 * pe_align((size_t)count * m * n * 2) + pe_align((size_t)count * m * 4) + pe_align((size_t)count * 8);
+}
+
+size_t gptb_muon_workspace_bytes(int m, int n, int steps) { return muon_bytes(1, m, n, steps); }
+size_t gptb_muon_batched_workspace_bytes(int count, int m, int n, int steps) { return muon_bytes(count, m, n, steps); }
+
+// One Muon step on `count` matrices of m x n (pointer arrays on the host)
+int muon_impl(int count, float* const* w, void* const* w_bf16, const float* const* g, float* const* buf,
+              float* const* v, int m, int n, const float* coeffs, int steps, float lr, float mu, float beta2,
+              float weight_decay, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  if (count <= 0 || count > PE_MAX_BATCH || !w || !g || !buf || !v || !coeffs || !workspace || m <= 0 || n <= 0 ||
+      m % 8 || n % 8 || steps < 1 || steps > 64)
+    return GPTB_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (!w[i] || !g[i] || !buf[i] || !v[i]) return GPTB_ERR_INVALID_ARG;
+    if (!aligned16(w[i]) || !aligned16(g[i]) || !aligned16(buf[i]) ||
+        (w_bf16 && w_bf16[i] && (reinterpret_cast<uintptr_t>(w_bf16[i]) & 7u)))
+      return GPTB_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GPTB_ERR_INVALID_ARG;
+  if (workspace_bytes < muon_bytes(count, m, n, steps)) return GPTB_ERR_WORKSPACE;
+  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
+  const size_t ne = (size_t)m * n;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t pe = pe_bytes(count, m, n, steps);
+  bf16* u = reinterpret_cast<bf16*>(ws + pe);
+  bf16* o = reinterpret_cast<bf16*>(ws + pe + pe_align(count * ne * 2));
+  float* step = reinterpret_cast<float*>(ws + pe + 2 * pe_align(count * ne * 2));
+  float* sums = reinterpret_cast<float*>(ws + pe + 2 * pe_align(count * ne * 2) + pe_align((size_t)count * m * 4));
+  const long long n4 = (long long)ne / 4;  // m, n multiples of 8
+  const int grid = (int)std::max<long long>(1, std::min<long long>((n4 + 255) / 256, dev_info().sms * 8LL));
+  // momentum (Nesterov): buf = mu buf + g, u = g + mu buf (bf16), into the batch's slices
+  for (int i = 0; i < count; ++i) {
+    muon_momentum_kernel<<<grid, 256, 0, st>>>(g[i], buf[i], u + i * ne, n4, mu, sums + 2 * i);
+    CKL();
+  }
+  TRY(polar_express_impl(u, o, m, n, count, coeffs, steps, ws, st));
+  // NorMuon: per-row second moment and step size, then the norm-keeping scale and the update
+  for (int i = 0; i < count; ++i) {
+    normuon_rows_kernel<<<grid_rows(m), EW_THREADS, 0, st>>>(o + i * ne, m, n, v[i], beta2, step + (size_t)i * m,
+                                                             sums + 2 * i);
+    CKL();
+    muon_apply_kernel<<<grid, 256, 0, st>>>(w[i], static_cast<bf16*>(w_bf16 ? w_bf16[i] : nullptr), o + i * ne,
+                                            step + (size_t)i * m, sums + 2 * i, m, n, lr, weight_decay);
+    CKL();
+  }
+  return GPTB_OK;
 }
 
 int gptb_muon_step(float* w, void* w_bf16, const float* g, float* buf, float* v, int m, int n, const float* coeffs,
                    int steps, float lr, float mu, float beta2, float weight_decay, void* workspace,
                    size_t workspace_bytes, gptb_stream_t stream) {
-  if (!w || !g || !buf || !v || !coeffs || !workspace || m <= 0 || n <= 0 || m % 8 || n % 8 || steps < 1 ||
-      steps > 64)
-    return GPTB_ERR_INVALID_ARG;
-  if (!aligned16(w) || !aligned16(g) || !aligned16(buf) || (w_bf16 && (reinterpret_cast<uintptr_t>(w_bf16) & 7u)) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return GPTB_ERR_INVALID_ARG;
-  if (workspace_bytes < gptb_muon_workspace_bytes(m, n, steps)) return GPTB_ERR_WORKSPACE;
-  if (dev_info().cc_major != 10) return GPTB_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t ne = (size_t)m * n;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t pe = gptb_polar_express_workspace_bytes(m, n, steps);
-  bf16* u = reinterpret_cast<bf16*>(ws + pe);
-  bf16* o = reinterpret_cast<bf16*>(ws + pe + pe_align(ne * 2));
-  float* step = reinterpret_cast<float*>(ws + pe + 2 * pe_align(ne * 2));
-  float* sums = reinterpret_cast<float*>(ws + pe + 2 * pe_align(ne * 2) + pe_align((size_t)m * 4));
-  const long long n4 = (long long)ne / 4;  // m, n multiples of 8
-  const int grid = (int)std::max<long long>(1, std::min<long long>((n4 + 255) / 256, dev_info().sms * 8LL));
-  // momentum (Nesterov): buf = mu buf + g, u = g + mu buf (bf16)
-  muon_momentum_kernel<<<grid, 256, 0, st>>>(g, buf, u, n4, mu, sums);
-  CKL();
-  TRY(polar_express_impl(u, o, m, n, coeffs, steps, ws, st));
-  // NorMuon: per-row second moment and step size, then the norm-keeping scale and the update
-  normuon_rows_kernel<<<grid_rows(m), EW_THREADS, 0, st>>>(o, m, n, v, beta2, step, sums);
-  CKL();
-  muon_apply_kernel<<<grid, 256, 0, st>>>(w, static_cast<bf16*>(w_bf16), o, step, sums, m, n, lr, weight_decay);
-  CKL();
-  return GPTB_OK;
+  void* wb[1] = {w_bf16};
+  return muon_impl(1, &w, w_bf16 ? wb : nullptr, &g, &buf, &v, m, n, coeffs, steps, lr, mu, beta2, weight_decay,
+                   workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gptb_muon_step_batched(int count, float* const* w, void* const* w_bf16, const float* const* g, float* const* buf,
+                           float* const* v, int m, int n, const float* coeffs, int steps, float lr, float mu,
+                           float beta2, float weight_decay, void* workspace, size_t workspace_bytes,
+                           gptb_stream_t stream) {
+  return muon_impl(count, w, w_bf16, g, buf, v, m, n, coeffs, steps, lr, mu, beta2, weight_decay, workspace,
+                   workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // --------------------------------------------------------------- decode --

@@ -411,14 +411,20 @@ __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
 struct HostFloats192 {
   float v[192];
 };
-__global__ void store_floats_kernel(HostFloats192 src, int n, float* __restrict__ dst, float* __restrict__ zero) {
+__global__ void store_floats_kernel(HostFloats192 src, int n, float* __restrict__ dst, float* __restrict__ zero,
+                                    int nzero) {
   for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src.v[i];
-  if (threadIdx.x == 0 && zero) *zero = 0.f;
+  if (zero)
+    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0.f;
 }
 
-// sum of squares of a bf16 array into *out (fp32, zeroed by the caller)
-__global__ void __launch_bounds__(256) sumsq_bf16_kernel(const bf16* __restrict__ x, long long n, float* __restrict__ out) {
+// sum of squares of a bf16 array into *out (fp32, zeroed by the caller);
+// blockIdx.y selects one of several arrays `stride` elements apart (and out[y])
+__global__ void __launch_bounds__(256)
+    sumsq_bf16_kernel(const bf16* __restrict__ x, long long n, float* __restrict__ out, long long stride) {
   __shared__ float sred[8];
+  x += blockIdx.y * stride;
+  out += blockIdx.y;
   float s = 0.f;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const float t = __bfloat162float(x[i]);
@@ -434,10 +440,13 @@ __global__ void __launch_bounds__(256) sumsq_bf16_kernel(const bf16* __restrict_
   }
 }
 
-// y = x / (sqrt(*sumsq) + eps), rounded to bf16
+// y = x / (sqrt(*sumsq) + eps), rounded to bf16; blockIdx.y selects one of
+// several arrays `stride` elements apart (and sumsq[y])
 __global__ void scale_by_norm_bf16_kernel(const bf16* __restrict__ x, bf16* __restrict__ y, long long n,
-                                          const float* __restrict__ sumsq, float eps) {
-  const float inv = 1.f / (sqrtf(*sumsq) + eps);
+                                          const float* __restrict__ sumsq, float eps, long long stride) {
+  x += blockIdx.y * stride;
+  y += blockIdx.y * stride;
+  const float inv = 1.f / (sqrtf(sumsq[blockIdx.y]) + eps);
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
     y[i] = __float2bfloat16_rn(__bfloat162float(x[i]) * inv);
 }

@@ -188,10 +188,15 @@ template <bool PAIR> struct TcShape {
   static_assert(SMEM <= 232448, "GEMM shared memory above the per-CTA limit");
 };
 
-__device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, int& tm, int& tn, int& split) {
+// unit u -> (split-K part, batch entry, tile row, tile column); the tiles of
+// one (split, batch entry) are walked in groups of TC_GROUP_M tile rows
+__device__ __forceinline__ void tc_unit_coords(int u, int tiles_m, int tiles_n, int nbatch, int& tm, int& tn,
+                                               int& split, int& bz) {
   const int tiles = tiles_m * tiles_n;
-  split = u / tiles;
-  const int t = u - split * tiles;
+  const int sb = u / tiles;
+  split = sb / nbatch;
+  bz = sb - split * nbatch;
+  const int t = u - sb * tiles;
   const int per_group = TC_GROUP_M * tiles_n;
   const int g = t / per_group;
   const int first_m = g * TC_GROUP_M;
@@ -287,8 +292,8 @@ template <int KIND, bool PAIR>
 __device__ __forceinline__ void tc_epilogue(const EpiParams& ep, const CUtensorMap* tmO_, const CUtensorMap* tmX_,
                                             uint32_t tmem_base, uint8_t* sEpi, uint64_t* aux_bar, uint64_t* tfull,
                                             uint64_t* tempty, volatile int* abort_flag, int M, int N, int unit0,
-                                            int ustep, int units, int tiles_m, int tiles_n, int warp, int lane,
-                                            uint32_t rank) {
+                                            int ustep, int units, int tiles_m, int tiles_n, int nbatch, int warp,
+                                            int lane, uint32_t rank) {
   using SH = TcShape<PAIR>;
   const CUtensorMap& tmO = *tmO_;
   const CUtensorMap& tmX = *tmX_;
@@ -310,12 +315,12 @@ __device__ __forceinline__ void tc_epilogue(const EpiParams& ep, const CUtensorM
   // load the input chunk cc_ of unit u_ into the next input tile (lane 0; the count advances on every lane)
   auto issue_aux = [&](int u_, int cc_) {
     if (lane == 0) {
-      int tm_, tn_, sp_;
-      tc_unit_coords(u_, tiles_m, tiles_n, tm_, tn_, sp_);
+      int tm_, tn_, sp_, bz_;
+      tc_unit_coords(u_, tiles_m, tiles_n, nbatch, tm_, tn_, sp_, bz_);
       uint64_t* bar = &abar[na & 1u];
       mbar_arrive_expect_tx(bar, TC_EPI_TILE);
-      tma_load_2d(ebuf + (2 + (na & 1u)) * TC_EPI_TILE, &tmX, bar, tn_ * TC_BN + cc_ * 64,
-                  tm_ * SH::TILE_M + (int)rank * TC_BM + q * 32);
+      tma_load_3d(ebuf + (2 + (na & 1u)) * TC_EPI_TILE, &tmX, bar, tn_ * TC_BN + cc_ * 64,
+                  tm_ * SH::TILE_M + (int)rank * TC_BM + q * 32, bz_);
     }
     ++na;
   };
@@ -327,8 +332,8 @@ __device__ __forceinline__ void tc_epilogue(const EpiParams& ep, const CUtensorM
   float oam = 0.f;  // max |out| stored by this thread (FP8 amax of EPI_RELU2 / EPI_DRELU2 outputs)
   bool ok = true;
   for (int u = unit0; u < units && ok; u += ustep) {
-    int tm, tn, split;
-    tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
+    int tm, tn, split, bz;
+    tc_unit_coords(u, tiles_m, tiles_n, nbatch, tm, tn, split, bz);
     if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, ERRW_TIMEOUT_EPILOGUE)) break;
     tc_fence_after();
     const int row0 = tm * SH::TILE_M + (int)rank * TC_BM + q * 32;
@@ -345,8 +350,8 @@ __device__ __forceinline__ void tc_epilogue(const EpiParams& ep, const CUtensorM
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmO, st0, col0, row0);
-          tma_store_2d(&tmO, st0 + TC_EPI_TILE, col0 + 64, row0);
+          tma_store_3d(&tmO, st0, col0, row0, bz);
+          tma_store_3d(&tmO, st0 + TC_EPI_TILE, col0 + 64, row0, bz);
           bulk_commit_group();
         }
         ++ns;
@@ -494,10 +499,10 @@ __device__ __forceinline__ void tc_epilogue(const EpiParams& ep, const CUtensorM
       if (lane == 0) {
         uint8_t* t0 = p0 - lane * 128;
         if constexpr (acc32) {
-          tma_reduce_add_2d(&tmO, t0, col0, row0);
-          tma_reduce_add_2d(&tmO, t0 + TC_EPI_TILE, col0 + 32, row0);
+          tma_reduce_add_3d(&tmO, t0, col0, row0, bz);
+          tma_reduce_add_3d(&tmO, t0 + TC_EPI_TILE, col0 + 32, row0, bz);
         } else {
-          tma_store_2d(&tmO, t0, col0, row0);
+          tma_store_3d(&tmO, t0, col0, row0, bz);
         }
         bulk_commit_group();
       }
@@ -537,7 +542,8 @@ template <bool A_MN, bool B_MN, bool FP8, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
-                   const __grid_constant__ CUtensorMap tmX, int M, int N, int K, int splits, EpiParams ep) {
+                   const __grid_constant__ CUtensorMap tmX, int M, int N, int K, int splits, int nbatch,
+                   EpiParams ep) {
   using SH = TcShape<PAIR>;
   constexpr int STAGES = SH::STAGES;
   constexpr int ELEM = FP8 ? 1 : 2;
@@ -573,7 +579,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int unit0 = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
   const int ustep = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
   const int tiles_m = (M + SH::TILE_M - 1) / SH::TILE_M, tiles_n = (N + TC_BN - 1) / TC_BN;
-  const int units = tiles_m * tiles_n * splits;
+  const int units = tiles_m * tiles_n * splits * nbatch;
   const int kb_total = (K + BK - 1) / BK;
   const int kb_per = (kb_total + splits - 1) / splits;
 
@@ -610,8 +616,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t armed = 0, armed_par = 0;  // stages with a load in flight, and the phase they complete
       bool ok = true;
       for (int u = unit0; u < units && ok; u += ustep) {
-        int tm, tn, split;
-        tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
+        int tm, tn, split, bz;
+        tc_unit_coords(u, tiles_m, tiles_n, nbatch, tm, tn, split, bz);
         const int kb0 = split * kb_per, kb1 = min(kb_total, kb0 + kb_per);
         const int arow = tm * SH::TILE_M + (int)rank * TC_BM;      // this CTA's rows of A
         const int brow = tn * TC_BN + (int)rank * SH::B_ROWS;      // this CTA's rows of B
@@ -630,8 +636,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           uint8_t* b = sB + stage * B_BYTES;
           const int k0 = kb * BK;
           auto load = [&](void* dst, const CUtensorMap* m, int c0, int c1) {
-            if (PAIR) tma_load_2d_pair(dst, m, map_shared_rank(&full[stage], 0), c0, c1);
-            else tma_load_2d(dst, m, &full[stage], c0, c1);
+            if (PAIR) tma_load_3d_pair(dst, m, map_shared_rank(&full[stage], 0), c0, c1, bz);
+            else tma_load_3d(dst, m, &full[stage], c0, c1, bz);
           };
           if (!A_MN) {
             load(a, &tmA, k0, arow);
@@ -683,8 +689,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int u = unit0; u < units && ok; u += ustep) {
-        int tm, tn, split;
-        tc_unit_coords(u, tiles_m, tiles_n, tm, tn, split);
+        int tm, tn, split, bz;
+        tc_unit_coords(u, tiles_m, tiles_n, nbatch, tm, tn, split, bz);
         const int kb0 = split * kb_per, kb1 = min(kb_total, kb0 + kb_per);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, ERRW_TIMEOUT_MMA)) break;
         tc_fence_after();
@@ -744,7 +750,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // one code path per epilogue kind
     auto run = [&](auto kind) {
       tc_epilogue<decltype(kind)::value, PAIR>(ep, &tmO, &tmX, tmem_base, sEpi, aux_bar, tfull, tempty, abort_flag, M, N,
-                                               unit0, ustep, units, tiles_m, tiles_n, warp, lane, rank);
+                                               unit0, ustep, units, tiles_m, tiles_n, nbatch, warp, lane, rank);
     };
     switch (ep.kind) {
       case EPI_STORE: run(std::integral_constant<int, EPI_STORE>{}); break;

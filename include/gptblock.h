@@ -241,6 +241,15 @@ int gpt_stack_step_hooked(const gptb_config* cfg, const gptb_model_weights* w, c
 int gptb_gemm_bf16(const void* A, int a_mn, long long lda, const void* B, int b_mn, long long ldb, void* C,
                    int c_f32, long long ldc, int M, int N, int K, gptb_stream_t stream);
 
+/* Batched form of gptb_gemm_bf16: for b = 0..batch-1, the matrices starting
+ * b*stride_a, b*stride_b, b*stride_c elements after A, B, C (strides in
+ * elements; their byte sizes multiples of 16) are multiplied as above, all in
+ * one launch (the form the Polar Express products take over same-shape
+ * matrices).  GPTB_ERR_INVALID_ARG for batch < 1 or a misaligned stride. */
+int gptb_gemm_bf16_batched(const void* A, int a_mn, long long lda, long long stride_a, const void* B, int b_mn,
+                           long long ldb, long long stride_b, void* C, int c_f32, long long ldc, long long stride_c,
+                           int M, int N, int K, int batch, gptb_stream_t stream);
+
 /* FP8 GEMM entry point used by the tests of the e4m3 / e5m2 tensor-core path:
  * C[M,N] += dequant(q(A) q(B)^T), fp32 accumulate, where q casts the bf16
  * operand to FP8 per tensor (A: e4m3 with scale 448/amax, or e5m2 with
@@ -314,6 +323,22 @@ size_t gptb_muon_workspace_bytes(int m, int n, int steps);
 int gptb_muon_step(float* w, void* w_bf16, const float* g, float* buf, float* v, int m, int n, const float* coeffs,
                    int steps, float lr, float mu, float beta2, float weight_decay, void* workspace,
                    size_t workspace_bytes, gptb_stream_t stream);
+
+/* gptb_muon_step on `count` (1..64) matrices of the same shape [m, n] at
+ * once: every Polar Express product runs as one batched GEMM over the count
+ * matrices (one launch instead of count, and count times the tiles to spread
+ * over the SMs).  w, w_bf16, g, buf, v: HOST arrays of count device pointers,
+ * each as in gptb_muon_step (w_bf16 may be NULL, or hold NULL entries); the
+ * result for each matrix is that of gptb_muon_step up to the order of float
+ * additions in the two NorMuon sums and the Frobenius norm.  workspace:
+ * device, gptb_muon_batched_workspace_bytes(count, m, n, steps) bytes,
+ * 256-byte aligned.  Errors as gptb_muon_step, and GPTB_ERR_INVALID_ARG for
+ * count outside 1..64. */
+size_t gptb_muon_batched_workspace_bytes(int count, int m, int n, int steps);
+int gptb_muon_step_batched(int count, float* const* w, void* const* w_bf16, const float* const* g, float* const* buf,
+                           float* const* v, int m, int n, const float* coeffs, int steps, float lr, float mu,
+                           float beta2, float weight_decay, void* workspace, size_t workspace_bytes,
+                           gptb_stream_t stream);
 
 /* ---------------------------------------------------------- decode ----
  * One generation step of the inference engine (apidog.com/fr "Comment

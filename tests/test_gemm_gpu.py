@@ -84,3 +84,30 @@ def test_gemm_fp8_matches_oracle_product(cuda_lib, a_mn, b_mn, M, N, K, e5m2):
     torch.cuda.synchronize()
     assert gb.gptb_device_error() == 0
     assert relerr(C.cpu().double().numpy(), ref) < 1e-5
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 1)])
+@pytest.mark.parametrize("M,N,K,batch", [(128, 256, 64, 3), (304, 264, 200, 2), (768, 768, 768, 5)])
+def test_gemm_batched(cuda_lib, a_mn, b_mn, M, N, K, batch):
+    """One launch over `batch` matrices stored one after another (the batch
+    entry is the third coordinate of the tensor maps): each product against an
+    fp64 matmul, for a bf16 store and an fp32 accumulation (split-K may meet
+    the batch), in the single-CTA (M < 256) and CTA-pair forms."""
+    gb = cuda_lib
+    g = torch.Generator().manual_seed(M + N + K + batch)
+    A = [_mk((M, K), g) for _ in range(batch)]
+    B = [_mk((N, K), g) for _ in range(batch)]
+    As = torch.stack([a.t().contiguous() if a_mn else a for a in A]).cuda()
+    Bs = torch.stack([b.t().contiguous() if b_mn else b for b in B]).cuda()
+    lda = M if a_mn else K
+    ldb = N if b_mn else K
+    C = torch.zeros(batch, M, N, dtype=torch.float32, device="cuda")
+    gb.gptb_gemm_bf16_batched(As, a_mn, lda, M * K, Bs, b_mn, ldb, N * K, C, 1, N, M * N, M, N, K, batch)
+    Cb = torch.empty(batch, M, N, dtype=torch.bfloat16, device="cuda")
+    gb.gptb_gemm_bf16_batched(As, a_mn, lda, M * K, Bs, b_mn, ldb, N * K, Cb, 0, N, M * N, M, N, K, batch)
+    torch.cuda.synchronize()
+    assert gb.gptb_device_error() == 0
+    for i in range(batch):
+        ref = A[i].double().numpy() @ B[i].double().numpy().T
+        assert relerr(C[i].cpu().double().numpy(), ref) < 1e-5, i
+        assert relerr(Cb[i].float().cpu().numpy(), ref) < 8e-3, i

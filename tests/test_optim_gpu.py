@@ -108,3 +108,58 @@ def test_muon_step_rejects_bad_shapes(cuda_lib):
     with pytest.raises(gb.GPTBError) as e:
         gb.gptb_muon_step(t, None, t, t, t, 12, 8, oo.POLAR_EXPRESS_COEFFS, 0.1, 0.9, 0.9, 0.0, t)
     assert e.value.code == gb.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("shape,count", [((256, 128), 3), ((128, 384), 2), ((768, 768), 4)])
+def test_muon_step_batched_matches_oracle(cuda_lib, shape, count):
+    """gptb_muon_step_batched on `count` same-shape matrices (every Polar
+    Express product one batched GEMM) against oracle.optim.muon_step per
+    matrix, with the tolerances of the single-matrix test, and against
+    gptb_muon_step on the same inputs (the same products in the same order per
+    tile; only the float sums of the norms may add in another order)."""
+    gb = cuda_lib
+    m, n = shape
+    rng = np.random.default_rng(7 * m + n + count)
+    hp = dict(lr=0.02, mu=0.95, beta2=0.95, weight_decay=0.1)
+    w0 = [rng.standard_normal((m, n)).astype(np.float32) * 0.02 for _ in range(count)]
+    gs = [[rng.standard_normal((m, n)).astype(np.float32) for _ in range(count)] for _ in range(2)]
+    ws = [torch.tensor(x, device="cuda") for x in w0]
+    bufs = [torch.zeros(m, n, device="cuda") for _ in range(count)]
+    vs = [torch.zeros(m, device="cuda") for _ in range(count)]
+    wbs = [torch.empty(m, n, dtype=torch.bfloat16, device="cuda") for _ in range(count)]
+    work = torch.empty(gb.gptb_muon_batched_workspace_bytes(count, m, n, 5), dtype=torch.uint8, device="cuda")
+    # the same steps one matrix at a time
+    ws1 = [torch.tensor(x, device="cuda") for x in w0]
+    bufs1 = [torch.zeros(m, n, device="cuda") for _ in range(count)]
+    vs1 = [torch.zeros(m, device="cuda") for _ in range(count)]
+    work1 = torch.empty(gb.gptb_muon_workspace_bytes(m, n, 5), dtype=torch.uint8, device="cuda")
+    for step in range(2):
+        gt = [torch.tensor(x, device="cuda") for x in gs[step]]
+        gb.gptb_muon_step_batched(ws, wbs, gt, bufs, vs, m, n, oo.POLAR_EXPRESS_COEFFS, hp["lr"], hp["mu"],
+                                  hp["beta2"], hp["weight_decay"], work)
+        for i in range(count):
+            gb.gptb_muon_step(ws1[i], None, gt[i], bufs1[i], vs1[i], m, n, oo.POLAR_EXPRESS_COEFFS, hp["lr"],
+                              hp["mu"], hp["beta2"], hp["weight_decay"], work1)
+    torch.cuda.synchronize()
+    assert gb.gptb_device_error() == 0
+    for i in range(count):
+        rw, rbuf, rv = w0[i].astype(np.float64), np.zeros((m, n)), np.zeros(m)
+        for step in range(2):
+            rw, rbuf, rv = oo.muon_step(rw, gs[step][i], rbuf, rv, hp["lr"], hp["mu"], hp["beta2"],
+                                        hp["weight_decay"])
+        got = ws[i].double().cpu().numpy()
+        assert relerr(got - w0[i], rw - w0[i]) <= TOL["bf16"], i
+        assert relerr(bufs[i].double().cpu().numpy(), rbuf) <= TOL["f32"], i
+        assert relerr(vs[i].double().cpu().numpy(), rv) <= TOL["bf16"], i
+        assert torch.equal(wbs[i], ws[i].bfloat16())
+        one = ws1[i].double().cpu().numpy()
+        assert relerr(got - w0[i], one - w0[i]) <= 1e-3, i
+
+
+def test_muon_step_batched_rejects_bad_count(cuda_lib):
+    gb = cuda_lib
+    t = torch.zeros(64, 64, device="cuda")
+    with pytest.raises(gb.GPTBError) as e:
+        gb.gptb_muon_step_batched([t] * 65, [None] * 65, [t] * 65, [t] * 65, [t] * 65, 64, 64,
+                                  oo.POLAR_EXPRESS_COEFFS, 0.1, 0.9, 0.9, 0.0, t)
+    assert e.value.code == gb.ERR_INVALID_ARG
