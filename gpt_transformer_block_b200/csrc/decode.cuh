@@ -9,12 +9,14 @@
 // are split into pieces of DEC_SPLIT rows handled by separate CTAs (enough
 // CTAs in flight to keep the memory system busy), each serving the G query
 // heads of its group:
-//   decode_split_kernel   per piece: scores of its keys for the G heads
-//                         (thread per key, 16-byte loads of the key row),
-//                         the piece's max and sum of exp per head, and the
-//                         unnormalised sum of p_j v_j (a warp per key, each
-//                         lane 4 columns, so a V row is one 256-byte access);
-//                         writes (max, sum, o[128]) per (head, piece)
+//   decode_split_kernel   per piece: one TMA load of the piece's V rows
+//                         (DEC_SPLIT x 128, bf16) into shared memory, issued
+//                         first so it overlaps the score pass; scores of its
+//                         keys for the G heads (thread per key, the key row as
+//                         16-byte loads); the piece's max and sum of exp per
+//                         head; the unnormalised sum of p_j v_j read from the
+//                         staged tile (thread = output column and half of the
+//                         keys); writes (max, sum, o[128]) per (head, piece)
 //   decode_combine_kernel per (sequence, head): rescales the pieces to the
 //                         common max, o = sum o_p e^(m_p - m) / sum l_p e^(m_p - m)
 #pragma once
@@ -22,23 +24,32 @@
 
 namespace gptb {
 
-constexpr int DEC_THREADS = 256;
+#ifndef GPTB_DEC_SPLIT
+#define GPTB_DEC_SPLIT 256
+#endif
 constexpr int DEC_HD = 128;
-constexpr int DEC_SPLIT = 256;      // keys per piece (one per thread in the score pass)
+constexpr int DEC_SPLIT = GPTB_DEC_SPLIT;  // keys per piece (one per thread in the score pass)
+constexpr int DEC_THREADS = DEC_SPLIT;
+static_assert(DEC_SPLIT == 128 || DEC_SPLIT == 256, "a piece is one or two key halves of 128 threads");
 constexpr int DEC_MAX_G = 16;       // query heads per kv head
 
 __host__ __device__ inline int decode_pieces(int Tmax) { return (Tmax + DEC_SPLIT - 1) / DEC_SPLIT; }
 // workspace floats per (sequence, head, piece): max, sum, o[128]
 constexpr int DEC_PART = 2 + DEC_HD;
 
-__global__ void __launch_bounds__(DEC_THREADS)
-    decode_split_kernel(const bf16* __restrict__ q, const bf16* __restrict__ kc, const bf16* __restrict__ vc,
-                        const int32_t* __restrict__ lens, float* __restrict__ part, int H, int Hkv, int Tmax,
-                        int window) {
+constexpr int DEC_V_BYTES = DEC_SPLIT * DEC_HD * 2;  // the staged V tile (dynamic shared memory)
+
+__global__ void __launch_bounds__(DEC_THREADS, 512 / DEC_THREADS)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_v, const bf16* __restrict__ q,
+                        const bf16* __restrict__ kc, const int32_t* __restrict__ lens, float* __restrict__ part,
+                        int H, int Hkv, int Tmax, int window) {
+  extern __shared__ __align__(128) uint8_t dec_smem[];   // [DEC_SPLIT][DEC_HD] bf16 V rows
   __shared__ __align__(16) float sq[DEC_MAX_G * DEC_HD];     // queries, pre-scaled
   __shared__ __align__(16) float ss[DEC_MAX_G * DEC_SPLIT];  // scores, then exp(s - max)
-  __shared__ __align__(16) float sred[8 * DEC_HD];           // per-warp partial outputs
+  __shared__ __align__(16) float sred[DEC_HD];               // the second key half's partial outputs
   __shared__ float sml[2 * DEC_MAX_G];                       // per-head max, sum
+  __shared__ __align__(8) uint64_t vbar;
+  const bf16* sv = reinterpret_cast<const bf16*>(dec_smem);
   const int G = H / Hkv;
   const int P = decode_pieces(Tmax);
   const int piece = blockIdx.x % P;
@@ -54,7 +65,6 @@ __global__ void __launch_bounds__(DEC_THREADS)
   const int nk = max(0, min(DEC_SPLIT, nvis - j0));    // keys of this piece
   const long long rs = (long long)Hkv * DEC_HD;        // cache row stride
   const bf16* kb = kc + (long long)b * Tmax * rs + (long long)kvh * DEC_HD;
-  const bf16* vb = vc + (long long)b * Tmax * rs + (long long)kvh * DEC_HD;
   float* out = part + ((long long)b * H + kvh * G) * P * DEC_PART;  // [G][P][DEC_PART]
   if (nk == 0) {  // nothing visible here: an empty piece (max -inf, sum 0)
     for (int g = tid; g < G; g += DEC_THREADS) {
@@ -62,6 +72,14 @@ __global__ void __launch_bounds__(DEC_THREADS)
       out[((long long)g * P + piece) * DEC_PART + 1] = 0.f;
     }
     return;
+  }
+  // the V rows of the piece: one TMA box of DEC_SPLIT rows (rows past the
+  // piece or past the cache are read or zero-filled and never used)
+  if (tid == 0) {
+    mbar_init(&vbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&vbar, DEC_V_BYTES);
+    tma_load_2d(dec_smem, &tm_v, &vbar, kvh * DEC_HD, b * Tmax + lo + j0);
   }
   const float scale = rsqrtf((float)DEC_HD);
   for (int i = tid; i < G * DEC_HD; i += DEC_THREADS)
@@ -108,30 +126,34 @@ __global__ void __launch_bounds__(DEC_THREADS)
       sml[2 * g + 1] = l;
     }
   }
-  __syncthreads();
-  // sum of p_j v_j: warp w takes keys w, w+8, ...; lane = columns 4 lane .. 4 lane + 3
+  // the staged V tile (a bounded wait: on expiry the error is recorded, the
+  // copy gets a further bounded wait before the CTA leaves, and nothing is written)
+  volatile int no_abort = 0;
+  bool ok = mbar_wait(&vbar, 0, &no_abort, ERRW_TIMEOUT_EPILOGUE);
+  ok = __syncthreads_and(ok);
+  if (!ok) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(&vbar, 0))
+      if (globaltimer_ns() - t0 > 100000000ull) break;
+    return;
+  }
+  // sum of p_j v_j: thread = column c and one of the DEC_THREADS / 128 parts of the keys
+  const int c = tid & (DEC_HD - 1), kh = tid >> 7;
+  const int jh = (DEC_THREADS == 256) ? (nk + 1) / 2 : nk;
+  const int ja = kh ? jh : 0, jb = kh ? nk : jh;
   for (int g = 0; g < G; ++g) {
     const float* pg = ss + g * DEC_SPLIT;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    for (int j = warp; j < nk; j += DEC_THREADS / 32) {
-      const uint2 vv = *reinterpret_cast<const uint2*>(vb + (long long)(lo + j0 + j) * rs + lane * 4);
-      const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.x));
-      const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv.y));
-      const float p = pg[j];
-      a0 = fmaf(p, v01.x, a0);
-      a1 = fmaf(p, v01.y, a1);
-      a2 = fmaf(p, v23.x, a2);
-      a3 = fmaf(p, v23.y, a3);
+    float a0 = 0.f, a1 = 0.f;  // two chains
+    int j = ja;
+    for (; j + 1 < jb; j += 2) {
+      a0 = fmaf(pg[j], __bfloat162float(sv[j * DEC_HD + c]), a0);
+      a1 = fmaf(pg[j + 1], __bfloat162float(sv[(j + 1) * DEC_HD + c]), a1);
     }
-    *reinterpret_cast<float4*>(sred + warp * DEC_HD + lane * 4) = make_float4(a0, a1, a2, a3);
+    if (j < jb) a0 = fmaf(pg[j], __bfloat162float(sv[j * DEC_HD + c]), a0);
+    if (kh) sred[c] = a0 + a1;
     __syncthreads();
     float* og = out + ((long long)g * P + piece) * DEC_PART;
-    if (tid < DEC_HD) {
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < DEC_THREADS / 32; ++w) s += sred[w * DEC_HD + tid];
-      og[2 + tid] = s;
-    }
+    if (!kh) og[2 + c] = (DEC_THREADS == 256) ? (a0 + a1) + sred[c] : a0 + a1;
     if (tid == 0) {
       og[0] = sml[2 * g];
       og[1] = sml[2 * g + 1];
