@@ -35,5 +35,5 @@ def test_flops_per_token_d24_by_hand():
 
 
 def test_traffic_line_is_read_from_the_committed_summary():
-    assert bench.profile_traffic("d24") == pytest.approx(6.388e8)
+    assert bench.profile_traffic("d24") == pytest.approx(5.065e8)
     assert bench.profile_traffic("no_such_workload") is None
