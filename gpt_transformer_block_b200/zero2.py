@@ -193,10 +193,11 @@ class GpuZero2Trainer:
       reductions start there (reduce_scatter for AdamW tensors, reduce to the
       owner for Muon matrices), overlapping the rest of the backward
       (phase 1);
-    - each reduction is waited for, the owned part updated by the library's
-      gptb_adamw_step / gptb_muon_step on fp32 masters that write the bf16
-      working weights, and the all_gather / broadcast of the new bf16 values
-      launched (phase 2);
+    - each reduction is waited for, the owned AdamW shards updated by
+      gptb_adamw_step and their all_gather launched; the owned Muon matrices
+      are updated by one gptb_muon_step_batched call per shape (fp32 masters
+      that write the bf16 working weights), then every rank launches the
+      Muon broadcasts in the same order (phase 2);
     - the gathers are waited for and the working weights filled (phase 3).
 
     Masters and optimizer state exist only for what this rank owns (ZeRO-2).
@@ -249,9 +250,17 @@ class GpuZero2Trainer:
                 if self.plan.owner[s.name] == self.rank:
                     m, n = s.shape
                     self.state[s.name] = dict(master=p.float().clone(), buf=torch.zeros(s.shape, device=dev),
-                                              v=torch.zeros(m, device=dev), g=torch.zeros(s.shape, device=dev),
-                                              ws=torch.empty(gb.gptb_muon_workspace_bytes(m, n, len(self.coeffs)),
-                                                             dtype=torch.uint8, device=dev))
+                                              v=torch.zeros(m, device=dev), g=torch.zeros(s.shape, device=dev))
+        # the owned Muon matrices by shape: each group takes one batched Muon call
+        # (every Polar Express product one GEMM launch over the group)
+        self.muon_groups = {}
+        for s in self.specs:
+            if s.kind != "adamw" and self.plan.owner[s.name] == self.rank:
+                self.muon_groups.setdefault(tuple(s.shape), []).append(s)
+        self.muon_ws = {shape: torch.empty(gb.gptb_muon_batched_workspace_bytes(len(grp), shape[0], shape[1],
+                                                                                 len(self.coeffs)),
+                                           dtype=torch.uint8, device=dev)
+                        for shape, grp in self.muon_groups.items()}
 
     def _lookup(self, tree: dict, name: str):
         if name.startswith("L"):
@@ -295,7 +304,7 @@ class GpuZero2Trainer:
                                  self.stack.ws, ready, compute)
         hp = self.hp
         gathers = []
-        for s, w in pending:                     # phase 2
+        for s, w in pending:                     # phase 2: AdamW shards, and the owned Muon gradients in fp32
             w.wait()
             full, shard = self.wire[s.name]
             st = self.state.get(s.name)
@@ -307,16 +316,18 @@ class GpuZero2Trainer:
                 src = st["pb"] if st["gathered"].dtype == torch.bfloat16 else st["master"]
                 gathers.append((s, dist.all_gather_into_tensor(st["gathered"], src, group=self.group,
                                                                async_op=True)))
-            else:
-                owner = self.plan.owner[s.name]
-                p = self.param(s.name)
-                if owner == self.rank:
-                    m, n = s.shape
-                    gb.gptb_cast_bf16_f32(full, st["g"], s.numel, 1.0, compute)
-                    gb.gptb_muon_step(st["master"], p, st["g"], st["buf"], st["v"], m, n, self.coeffs,
-                                      hp["lr_muon"], hp["momentum"], hp["beta2_muon"], hp["weight_decay"], st["ws"],
-                                      compute)
-                gathers.append((s, dist.broadcast(p, src=owner, group=self.group, async_op=True)))
+            elif self.plan.owner[s.name] == self.rank:
+                gb.gptb_cast_bf16_f32(full, st["g"], s.numel, 1.0, compute)
+        for (m, n), grp in self.muon_groups.items():
+            sts = [self.state[x.name] for x in grp]
+            gb.gptb_muon_step_batched([x["master"] for x in sts], [self.param(x.name) for x in grp],
+                                      [x["g"] for x in sts], [x["buf"] for x in sts], [x["v"] for x in sts], m, n,
+                                      self.coeffs, hp["lr_muon"], hp["momentum"], hp["beta2_muon"],
+                                      hp["weight_decay"], self.muon_ws[(m, n)], compute)
+        for s, _ in pending:                     # every rank broadcasts the Muon matrices in the same order
+            if s.kind != "adamw":
+                gathers.append((s, dist.broadcast(self.param(s.name), src=self.plan.owner[s.name],
+                                                  group=self.group, async_op=True)))
         for s, w in gathers:                     # phase 3
             w.wait()
             if s.kind == "adamw":
