@@ -620,6 +620,10 @@ int check_config(const gptb_config* c) {
 
 // one CTA per token row: ceil(d/8) threads rounded up to whole warps
 int br_threads(int d) { return ((d / 8 + 31) / 32) * 32; }
+// grid of the warp-per-row kernels (8 rows per 256-thread block in flight, grid-stride beyond)
+int warp_rows_grid(long long rows) {
+  return (int)std::max<long long>(1, std::min<long long>((rows + 7) / 8, (long long)dev_info().sms * 8));
+}
 int br_grid(long long rows, int threads) {
   const long long cap = (long long)dev_info().sms * (2048 / threads) * 2;
   return (int)std::max<long long>(1, std::min(rows, cap));
@@ -745,7 +749,7 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, S.o8, S.amax + 1, true, false, true},
               {w.w_o, Ho, false, m.d * Ho, S.wo8, S.amax + 5, true}, (int)m.N, m.d, (int)Ho,
               epi(EPI_RESID, c.dtype, X.x1, m.d, X.xm, m.d), st));
-  br_norm_kernel<T><<<brg, brt, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
+  br_norm_warp_kernel<T><<<warp_rows_grid(m.N), 256, 0, st>>>((const T*)X.x1, nullptr, nullptr, (T*)S.h2, S.rstd2, m.N, m.d,
                                             c.norm_eps, am ? am + 2 : nullptr);
   CKL();
   EpiParams erelu = epi(EPI_RELU2, c.dtype, S.act, m.F);
@@ -870,10 +874,10 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
                                                                      c.ve_gate_ch, g.w_ve_gate);
     CKL();
   }
-  br_mix_norm_bwd_kernel<T><<<brg, brt, 0, st>>>((const T*)X.dh, ve ? X.dz : nullptr,
-                                                    ve ? (const T*)w.w_ve_gate : nullptr, m.Hkv, c.ve_gate_ch,
-                                                    (const T*)S.h, S.rstd1, (const T*)X.dx1, x, x0, w.lambdas, dx_extra,
-                                                    dx, dx0_acc, g.lambdas, m.N, m.d);
+  br_mix_norm_bwd_warp_kernel<T><<<warp_rows_grid(m.N), 256, 0, st>>>((const T*)X.dh, ve ? X.dz : nullptr,
+                                                         ve ? (const T*)w.w_ve_gate : nullptr, m.Hkv, c.ve_gate_ch,
+                                                         (const T*)S.h, S.rstd1, (const T*)X.dx1, x, x0, w.lambdas,
+                                                         dx_extra, dx, dx0_acc, g.lambdas, m.N, m.d);
   CKL();
   return GPTB_OK;
 }
@@ -965,7 +969,7 @@ int stack_impl(const gptb_config& c, const gptb_model_weights& w, const int32_t*
     TRY(block_fwd_impl<T>(c, i, w.layers[i], (const T*)S.x_in[i], x0, idx, xo, S.saved[i], S.scr, st));
   }
   const T* x_bo = c.backout_layer >= 0 ? (const T*)S.x_in[c.backout_layer] : nullptr;
-  br_norm_kernel<T><<<brg, brt, 0, st>>>((const T*)S.xL, x_bo, w.backout_lambda, (T*)S.hf, S.rstd_f, m.N, m.d,
+  br_norm_warp_kernel<T><<<warp_rows_grid(m.N), 256, 0, st>>>((const T*)S.xL, x_bo, w.backout_lambda, (T*)S.hf, S.rstd_f, m.N, m.d,
                                             c.norm_eps, nullptr);
   CKL();
   TRY(lm_head_impl<T>(c, (const T*)S.hf, (const T*)w.w_lm, targets, loss_out, (T*)S.dhf, g.w_lm, S.lm, st));

@@ -161,37 +161,45 @@ __global__ void __launch_bounds__(256)
   if (amax_h) block_amax_publish(am, amax_h, sa);
 }
 
-// h = rmsnorm(x - lam_bo * x_bo)   (backout + final norm when x_bo != null)
+// h = rmsnorm(x - lam_bo * x_bo)   (backout + final norm when x_bo != null).
+// One warp per row: the sum of squares in a first pass (a warp reduction, no
+// block barrier), the scaled row from a second read (L1 / L2); an SM keeps
+// several times more rows in flight than with a block per row.
 template <class T>
 __global__ void __launch_bounds__(256)
-    br_norm_kernel(const T* __restrict__ x, const T* __restrict__ x_bo, const float* __restrict__ lam_bo,
-                   T* __restrict__ h_out, float* __restrict__ rstd_out, long long N, int d, float eps,
-                   unsigned int* __restrict__ amax_h) {
-  __shared__ float sh[2 * BR_MAX_WARPS];
+    br_norm_warp_kernel(const T* __restrict__ x, const T* __restrict__ x_bo, const float* __restrict__ lam_bo,
+                        T* __restrict__ h_out, float* __restrict__ rstd_out, long long N, int d, float eps,
+                        unsigned int* __restrict__ amax_h) {
   __shared__ float sa[32];
-  const BRow r(d);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float lb = x_bo ? *lam_bo : 0.f;
   float am = 0.f;
-  for (long long n = blockIdx.x; n < N; n += gridDim.x) {
-    float v[8] = {}, w[8] = {};
-    if (r.act) {
-      load8(x + n * d + r.c0, v);
-      if (x_bo) load8(x_bo + n * d + r.c0, w);
-    }
+  for (long long n = (long long)blockIdx.x * 8 + warp; n < N; n += (long long)gridDim.x * 8) {
+    const long long ro = n * d;
     float ss = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+      float v[8], w[8] = {};
+      load8(x + ro + c, v);
+      if (x_bo) load8(x_bo + ro + c, w);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      v[k] -= lb * w[k];
-      ss = fmaf(v[k], v[k], ss);
+      for (int k = 0; k < 8; ++k) {
+        v[k] -= lb * w[k];
+        ss = fmaf(v[k], v[k], ss);
+      }
     }
-    const float rstd = rsqrtf(br_sum(ss, sh, r) / d + eps);
+    const float rstd = rsqrtf(warp_sum(ss) / d + eps);
+    for (int c = lane * 8; c < d; c += 256) {
+      float v[8], w[8] = {};
+      load8(x + ro + c, v);
+      if (x_bo) load8(x_bo + ro + c, w);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      v[k] *= rstd;
-      am = fmaxf(am, fabsf(v[k]));
+      for (int k = 0; k < 8; ++k) {
+        v[k] = (v[k] - lb * w[k]) * rstd;
+        am = fmaxf(am, fabsf(v[k]));
+      }
+      store8(h_out + ro + c, v);
     }
-    if (r.act) store8(h_out + n * d + r.c0, v);
-    if (r.tid == 0) rstd_out[n] = rstd;
+    if (lane == 0) rstd_out[n] = rstd;
   }
   if (amax_h) block_amax_publish(am, amax_h, sa);
 }
@@ -238,57 +246,83 @@ __global__ void __launch_bounds__(256)
 // first RMSNorm, plus the residual path dx1; then the lambda mix:
 //   dxm = dx1 + rstd*(dh - h*mean(dh*h));  dx = a*dxm (+ dx_extra);
 //   dx0_acc += b*dxm;  dlam += (sum dxm*x, sum dxm*x0)
+// One warp per row: a first pass over the row forms mean(dh*h) (a warp
+// reduction, no block barrier), a second reads the row again (from L1 / L2)
+// with the other inputs and writes the outputs.  With no barrier per row and
+// few registers an SM keeps tens of rows in flight (a block per row kept
+// three).
 template <class T>
 __global__ void __launch_bounds__(256)
-    br_mix_norm_bwd_kernel(const T* __restrict__ dh, const float* __restrict__ dz, const T* __restrict__ w_gate,
-                           int Hkv, int Cg, const T* __restrict__ h, const float* __restrict__ rstd,
-                           const T* __restrict__ dx1, const T* __restrict__ x, const T* __restrict__ x0,
-                           const float* __restrict__ lam, const T* __restrict__ dx_extra, T* __restrict__ dx_out,
-                           float* __restrict__ dx0_acc, float* __restrict__ dlam, long long N, int d) {
-  __shared__ float sh[2 * BR_MAX_WARPS];
-  const BRow r(d);
+    br_mix_norm_bwd_warp_kernel(const T* __restrict__ dh, const float* __restrict__ dz, const T* __restrict__ w_gate,
+                                int Hkv, int Cg, const T* __restrict__ h, const float* __restrict__ rstd,
+                                const T* __restrict__ dx1, const T* __restrict__ x, const T* __restrict__ x0,
+                                const float* __restrict__ lam, const T* __restrict__ dx_extra, T* __restrict__ dx_out,
+                                float* __restrict__ dx0_acc, float* __restrict__ dlam, long long N, int d) {
+  __shared__ float sred[16];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float a = lam[0], b = lam[1];
   float pa = 0.f, pb = 0.f;
-  for (long long n = blockIdx.x; n < N; n += gridDim.x) {
-    float g[8] = {}, y[8] = {}, o[8] = {}, xv[8] = {}, x0v[8] = {}, acc[8] = {}, ex[8] = {};
-    if (r.act) {
-      const long long off = n * d + r.c0;
-      load8(dh + off, g);
-      load8(h + off, y);
-      load8(dx1 + off, o);
-      load8(x + off, xv);
-      load8(x0 + off, x0v);
-      load8(dx0_acc + off, acc);
-      if (dx_extra) load8(dx_extra + off, ex);
-      if (dz != nullptr && r.c0 < Cg) {
+  for (long long n = (long long)blockIdx.x * 8 + warp; n < N; n += (long long)gridDim.x * 8) {
+    const long long ro = n * d;
+    // dh of 8 columns from c, plus the value-embedding gate term on the first Cg columns
+    auto grad8 = [&](int c, float (&g)[8]) {
+      load8(dh + ro + c, g);
+      if (dz != nullptr && c < Cg) {
         for (int k = 0; k < Hkv; ++k) {
           const float z = dz[n * Hkv + k];
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            if (r.c0 + e < Cg) g[e] = fmaf(z, to_f(w_gate[(long long)k * Cg + r.c0 + e]), g[e]);
+            if (c + e < Cg) g[e] = fmaf(z, to_f(w_gate[(long long)k * Cg + c + e]), g[e]);
         }
       }
-    }
-    const float rs = rstd[n];
+    };
     float dot = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+      float g[8], y[8];
+      grad8(c, g);
+      load8(h + ro + c, y);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) dot = fmaf(g[k], y[k], dot);
-    const float m = br_sum(dot, sh, r) / d;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float dxm = o[k] + rs * (g[k] - y[k] * m);
-      pa = fmaf(dxm, xv[k], pa);
-      pb = fmaf(dxm, x0v[k], pb);
-      acc[k] = fmaf(b, dxm, acc[k]);
-      o[k] = fmaf(a, dxm, ex[k]);
+      for (int e = 0; e < 8; ++e) dot = fmaf(g[e], y[e], dot);
     }
-    if (r.act) {
-      store8(dx0_acc + n * d + r.c0, acc);
-      store8(dx_out + n * d + r.c0, o);
+    const float m = warp_sum(dot) / d;
+    const float rs = rstd[n];
+    for (int c = lane * 8; c < d; c += 256) {
+      float g[8], y[8], o[8], xv[8], x0v[8], acc[8], ex[8] = {};
+      grad8(c, g);
+      load8(h + ro + c, y);
+      load8(dx1 + ro + c, o);
+      load8(x + ro + c, xv);
+      load8(x0 + ro + c, x0v);
+      load8(dx0_acc + ro + c, acc);
+      if (dx_extra) load8(dx_extra + ro + c, ex);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float dxm = o[e] + rs * (g[e] - y[e] * m);
+        pa = fmaf(dxm, xv[e], pa);
+        pb = fmaf(dxm, x0v[e], pb);
+        acc[e] = fmaf(b, dxm, acc[e]);
+        o[e] = fmaf(a, dxm, ex[e]);
+      }
+      store8(dx0_acc + ro + c, acc);
+      store8(dx_out + ro + c, o);
     }
   }
-  br_add_global(dlam, pa, sh, r);
-  br_add_global(dlam + 1, pb, sh, r);
+  pa = warp_sum(pa);
+  pb = warp_sum(pb);
+  if (lane == 0) {
+    sred[warp] = pa;
+    sred[8 + warp] = pb;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float sa = 0.f, sb = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+      sa += sred[w];
+      sb += sred[8 + w];
+    }
+    atomicAdd(dlam, sa);
+    atomicAdd(dlam + 1, sb);
+  }
 }
 
 // Final norm + backout backward:
