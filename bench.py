@@ -173,6 +173,9 @@ def cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
+_ORACLE_WEIGHTS = {}
+
+
 def oracle_sample(c: dict, seed: int = 7) -> dict:
     """Time the fp64 oracle on one block slice (B=1, full T) forward+backward
     plus the lm_head on 512 tokens, and extrapolate to one full step."""
@@ -184,10 +187,17 @@ def oracle_sample(c: dict, seed: int = 7) -> dict:
     except Exception:
         cores = os.cpu_count()
     cs = dict(c, B=1)
-    w = synth.make_weights(cs, seed=seed, mode="random")
-    inp = synth.make_block_inputs(cs, seed=seed + 1)
     layer = cs["n_layer"] - 1  # the last layer carries a value embedding
-    lw = {k: (v if isinstance(v, float) else np.asarray(v, dtype=np.float64)) for k, v in w["layers"][layer].items()}
+    # the timed layer's weights and the lm_head: drawn once per process for a
+    # one-layer copy of the config (the same layer kind), not for the whole stack
+    key = (c["name"], layer)
+    if key not in _ORACLE_WEIGHTS:
+        c1 = dict(cs, n_layer=1, window=[cs["window"][layer]], has_ve=[cs["has_ve"][layer]], backout_layer=-1)
+        w1 = synth.make_weights(c1, seed=seed, mode="random")
+        _ORACLE_WEIGHTS[key] = ({k: (v if isinstance(v, float) else np.asarray(v, dtype=np.float64))
+                                 for k, v in w1["layers"][0].items()}, np.asarray(w1["w_lm"], dtype=np.float64))
+    lw, wl = _ORACLE_WEIGHTS[key]
+    inp = synth.make_block_inputs(cs, seed=seed + 1)
     x = inp["x"].double().numpy()
     x0 = inp["x0"].double().numpy()
     dy = inp["dy"].double().numpy()
@@ -198,7 +208,6 @@ def oracle_sample(c: dict, seed: int = 7) -> dict:
     t_block = time.perf_counter() - t0
     n_lm = min(512, cs["T"])
     h = np.random.default_rng(seed).standard_normal((n_lm, cs["d"]))
-    wl = np.asarray(w["w_lm"], dtype=np.float64)
     y = np.random.default_rng(seed + 1).integers(0, cs["vocab"], n_lm)
     t0 = time.perf_counter()
     om.lm_head_xent(h, wl, y)
