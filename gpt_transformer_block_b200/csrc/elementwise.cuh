@@ -600,16 +600,7 @@ __global__ void __launch_bounds__(256)
 namespace gptb {
 
 // ------------------------------------------- vectorised hd = 128 variants --
-// Lane l holds elements 4l..4l+3 of a head: lanes 0-15 the first half
-// (rotation partner j), lanes 16-31 the second half (j + 64); the partner
-// value is one shuffle (lane ^ 16) away.
 
-__device__ __forceinline__ void ld4(const bf16* p, float (&v)[4]) {
-  const uint2 u = *reinterpret_cast<const uint2*>(p);
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-}
 __device__ __forceinline__ void load4(const bf16* p, float (&v)[4]) {
   const uint2 u = *reinterpret_cast<const uint2*>(p);
   const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
@@ -624,10 +615,18 @@ __device__ __forceinline__ void st4(bf16* p, const float (&v)[4]) {
 }
 
 // backward of q,k <- rope(rmsnorm(.)) and of the VE term for hd = 128: one
-// warp per token.  The token's rotation row is loaded once; heads are taken
-// QKV_BWD_HEADS at a time with all of their loads issued before any compute,
-// so each warp keeps several kilobytes in flight.
+// warp per token.  For q and k heads lane l holds the rotation pairs
+// (2l, 2l+64) and (2l+1, 2l+65), so undoing the rotation needs no shuffle;
+// the (cos, sin) of the lane's two frequencies are loaded once per token.  Heads are taken QB at a time
+// with all of their loads issued before any compute, so each warp keeps
+// several kilobytes in flight.
+// Two heads at a time with four blocks per SM (64 registers) measured fastest:
+// more heads per warp (at 2 or 3 blocks per SM) or more blocks (with spills)
+// were slower.
 constexpr int QKV_BWD_HEADS = 2;
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+}
 __global__ void __launch_bounds__(EW_THREADS, 4)
     qkv_post_bwd_h128_kernel(const bf16* __restrict__ qkv, long long ld, const float* __restrict__ rstd_qk,
                              const float2* __restrict__ rope, const float* __restrict__ dq, long long lddq,
@@ -640,40 +639,35 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
   __shared__ float sa[32];
   float am = 0.f;  // max |dqkv| this lane stores (FP8 amax)
   const int lane = threadIdx.x & 31;
-  const bool hi = lane >= 16;
   const int nqk = H + Hkv;
   const long long wpb = blockDim.x >> 5;
   for (long long n = blockIdx.x * wpb + (threadIdx.x >> 5); n < N; n += gridDim.x * wpb) {
     const int t = (int)(n % Tn);
-    float2 cs[4];
-    {
-      const float4 c01 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4);
-      const float4 c23 = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + (lane & 15) * 4 + 2);
-      cs[0] = make_float2(c01.x, c01.y);
-      cs[1] = make_float2(c01.z, c01.w);
-      cs[2] = make_float2(c23.x, c23.y);
-      cs[3] = make_float2(c23.z, c23.w);
-    }
-    const bf16* yrow = qkv + n * ld + lane * 4;
-    bf16* orow = dqkv + n * ld + lane * 4;
+    // (cos, sin) of frequencies 2l and 2l+1
+    const float4 cs = *reinterpret_cast<const float4*>(rope + (long long)t * 64 + lane * 2);
+    const bf16* yrow = qkv + n * ld + lane * 2;
+    bf16* orow = dqkv + n * ld + lane * 2;
     // q and k heads: undo the rotation on the gradient and on the stored
     // (rotated, normalised) output, then the RMSNorm backward
     for (int h0 = 0; h0 < nqk; h0 += QB) {
-      float4 g4[QB];
-      uint2 yb[QB];  // 4 bf16, converted at use
+      float2 g1[QB], g2[QB];      // gradient, first / second half
+      uint32_t y1[QB], y2[QB];    // stored output, 2 bf16 each
       float r[QB];
 #pragma unroll
       for (int b = 0; b < QB; ++b) {
         const int hh = h0 + b;
         if (hh < nqk) {
           if (hh < H) {  // dq: fp32 (summed over key tiles by reductions); dk: bf16
-            g4[b] = *reinterpret_cast<const float4*>(dq + n * lddq + (long long)hh * 128 + lane * 4);
+            const float* gp = dq + n * lddq + (long long)hh * 128 + lane * 2;
+            g1[b] = *reinterpret_cast<const float2*>(gp);
+            g2[b] = *reinterpret_cast<const float2*>(gp + 64);
           } else {
-            float t4[4];
-            load4(dk + n * lddkv + (long long)(hh - H) * 128 + lane * 4, t4);
-            g4[b] = make_float4(t4[0], t4[1], t4[2], t4[3]);
+            const bf16* gp = dk + n * lddkv + (long long)(hh - H) * 128 + lane * 2;
+            g1[b] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(gp));
+            g2[b] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(gp + 64));
           }
-          yb[b] = *reinterpret_cast<const uint2*>(yrow + (long long)hh * 128);
+          y1[b] = *reinterpret_cast<const uint32_t*>(yrow + (long long)hh * 128);
+          y2[b] = *reinterpret_cast<const uint32_t*>(yrow + (long long)hh * 128 + 64);
           r[b] = rstd_qk[n * nqk + hh];
         }
       }
@@ -681,32 +675,28 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
       for (int b = 0; b < QB; ++b) {
         const int hh = h0 + b;
         if (hh < nqk) {  // warp-uniform
-        const float g[4] = {g4[b].x, g4[b].y, g4[b].z, g4[b].w};
-        const float2 y01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yb[b].x));
-        const float2 y23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yb[b].y));
-        const float y[4] = {y01.x, y01.y, y23.x, y23.y};
-        // first half: a1 c + a2 s ; second half: -a1 s + a2 c  (a1 = first-half value)
-        float gu[4], yu[4], dot = 0.f;
+          const float2 ya = bf2_to_f2(y1[b]), yb = bf2_to_f2(y2[b]);
+          // inverse rotation: first half a1 c + a2 s, second half -a1 s + a2 c
+          const float gu[4] = {g1[b].x * cs.x + g2[b].x * cs.y, g1[b].y * cs.z + g2[b].y * cs.w,
+                               g2[b].x * cs.x - g1[b].x * cs.y, g2[b].y * cs.z - g1[b].y * cs.w};
+          const float yu[4] = {ya.x * cs.x + yb.x * cs.y, ya.y * cs.z + yb.y * cs.w, yb.x * cs.x - ya.x * cs.y,
+                               yb.y * cs.z - ya.y * cs.w};
+          float dot = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float go = __shfl_xor_sync(0xffffffffu, g[e], 16);
-          const float yo = __shfl_xor_sync(0xffffffffu, y[e], 16);
-          const float c = cs[e].x, sn = cs[e].y;
-          gu[e] = hi ? (g[e] * c - go * sn) : (g[e] * c + go * sn);
-          yu[e] = hi ? (y[e] * c - yo * sn) : (y[e] * c + yo * sn);
-          dot = fmaf(gu[e], yu[e], dot);
-        }
-        const float m = warp_sum(dot) * (1.f / 128.f);
-        float o[4];
+          for (int e = 0; e < 4; ++e) dot = fmaf(gu[e], yu[e], dot);
+          const float m = warp_sum(dot) * (1.f / 128.f);
+          float o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          o[e] = r[b] * (gu[e] - yu[e] * m);
-          am = fmaxf(am, fabsf(o[e]));
-        }
-        st4(orow + (long long)hh * 128, o);
+          for (int e = 0; e < 4; ++e) {
+            o[e] = r[b] * (gu[e] - yu[e] * m);
+            am = fmaxf(am, fabsf(o[e]));
+          }
+          *reinterpret_cast<uint32_t*>(orow + (long long)hh * 128) = pack_bf16(o[0], o[1]);
+          *reinterpret_cast<uint32_t*>(orow + (long long)hh * 128 + 64) = pack_bf16(o[2], o[3]);
         }
       }
     }
+    bf16* vout = dqkv + n * ld + lane * 4;  // v heads: lane l holds elements 4l..4l+3
     // v heads: the gradient passes through; with value embeddings also the
     // VE-table gradient (3*sigmoid(z) * dv, scattered by token id) and dz
     const long long ve_row = ve_table ? (long long)idx[n] * Hkv * 128 + lane * 4 : 0;
@@ -742,7 +732,7 @@ __global__ void __launch_bounds__(EW_THREADS, 4)
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(g[e]));
-        st4(orow + (long long)(nqk + kv) * 128, g);
+        st4(vout + (long long)(nqk + kv) * 128, g);
         }
       }
     }

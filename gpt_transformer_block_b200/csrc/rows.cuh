@@ -79,6 +79,34 @@ __device__ __forceinline__ void br_add_global(float* gdst, float v, float* sh, c
   if (r.tid == 0) atomicAdd(gdst, s);
 }
 
+// Register cache of a warp-per-row kernel: lane l holds the 8-element chunks at
+// columns 8l + 256j (j < BR_CHUNKS) of its row as loaded (16 bytes of bf16, or
+// 32 of fp32), so the row crosses HBM once.  Worth it only with few cached
+// arrays: two (the forward norm) keep ~128 registers; four plus the backward's
+// other streams cost occupancy and measured slower than reading the row twice.
+constexpr int BR_CHUNKS = BR_MAX_WARPS;  // the same 2048-element row limit
+template <class T> struct Raw8;
+template <> struct Raw8<bf16> { uint4 u; };
+template <> struct Raw8<float> { float4 a, b; };
+__device__ __forceinline__ void raw_load(const bf16* p, Raw8<bf16>& r) { r.u = *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ void raw_load(const float* p, Raw8<float>& r) {
+  r.a = *reinterpret_cast<const float4*>(p);
+  r.b = *reinterpret_cast<const float4*>(p + 4);
+}
+__device__ __forceinline__ void raw_unpack(const Raw8<bf16>& r, float (&v)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void raw_unpack(const Raw8<float>& r, float (&v)[8]) {
+  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+  v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+}
+
 // ---------------------------------------------------------------- forward
 
 // x_s[n] = wte[idx[n]] (+ smear from the previous token of the same row)
@@ -162,9 +190,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // h = rmsnorm(x - lam_bo * x_bo)   (backout + final norm when x_bo != null).
-// One warp per row: the sum of squares in a first pass (a warp reduction, no
-// block barrier), the scaled row from a second read (L1 / L2); an SM keeps
-// several times more rows in flight than with a block per row.
+// One warp per row, the row kept in registers between the sum of squares (a
+// warp reduction, no block barrier) and the scaling.
 template <class T>
 __global__ void __launch_bounds__(256)
     br_norm_warp_kernel(const T* __restrict__ x, const T* __restrict__ x_bo, const float* __restrict__ lam_bo,
@@ -176,28 +203,45 @@ __global__ void __launch_bounds__(256)
   float am = 0.f;
   for (long long n = (long long)blockIdx.x * 8 + warp; n < N; n += (long long)gridDim.x * 8) {
     const long long ro = n * d;
-    float ss = 0.f;
-    for (int c = lane * 8; c < d; c += 256) {
-      float v[8], w[8] = {};
-      load8(x + ro + c, v);
-      if (x_bo) load8(x_bo + ro + c, w);
+    Raw8<T> xr[BR_CHUNKS], br[BR_CHUNKS];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        v[k] -= lb * w[k];
-        ss = fmaf(v[k], v[k], ss);
+    for (int j = 0; j < BR_CHUNKS; ++j) {
+      const int c = lane * 8 + j * 256;
+      if (c < d) {
+        raw_load(x + ro + c, xr[j]);
+        if (x_bo) raw_load(x_bo + ro + c, br[j]);
+      }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < BR_CHUNKS; ++j) {
+      const int c = lane * 8 + j * 256;
+      if (c < d) {
+        float v[8], w[8] = {};
+        raw_unpack(xr[j], v);
+        if (x_bo) raw_unpack(br[j], w);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          v[k] -= lb * w[k];
+          ss = fmaf(v[k], v[k], ss);
+        }
       }
     }
     const float rstd = rsqrtf(warp_sum(ss) / d + eps);
-    for (int c = lane * 8; c < d; c += 256) {
-      float v[8], w[8] = {};
-      load8(x + ro + c, v);
-      if (x_bo) load8(x_bo + ro + c, w);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        v[k] = (v[k] - lb * w[k]) * rstd;
-        am = fmaxf(am, fabsf(v[k]));
+    for (int j = 0; j < BR_CHUNKS; ++j) {
+      const int c = lane * 8 + j * 256;
+      if (c < d) {
+        float v[8], w[8] = {};
+        raw_unpack(xr[j], v);
+        if (x_bo) raw_unpack(br[j], w);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          v[k] = (v[k] - lb * w[k]) * rstd;
+          am = fmaxf(am, fabsf(v[k]));
+        }
+        store8(h_out + ro + c, v);
       }
-      store8(h_out + ro + c, v);
     }
     if (lane == 0) rstd_out[n] = rstd;
   }
