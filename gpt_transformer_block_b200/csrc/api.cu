@@ -739,11 +739,14 @@ int block_fwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   } else {
     // tcgen05 flash attention: one tensor map (64-column boxes of 128 rows)
     // over the packed qkv buffer serves the Q, K and V tiles
-    CUtensorMap tq;
+    CUtensorMap tq, to;
     if (!make_tmap(&tq, S.qkv, false, (uint64_t)m.Wq, (uint64_t)m.N, (uint64_t)m.Wq, 64, 128)) return GPTB_ERR_CUDA;
+    // o as [B][T][H*hd]: 64-column x 32-row store boxes that clip at each sequence end
+    if (!make_tmap_3d(&to, S.o, false, (uint64_t)Ho, (uint64_t)m.T, (uint64_t)m.B, (uint64_t)Ho, 64, 32))
+      return GPTB_ERR_CUDA;
     CK(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM));
     attn_fwd_tc_kernel<<<(unsigned)(((m.T + FA_QB - 1) / FA_QB) * m.H * m.B), FA_THREADS, FA_SMEM, st>>>(
-        tq, (bf16*)S.o, (long long)m.H * m.hd, S.lse, m.T, m.H, m.Hkv, W, am ? am + 1 : nullptr);
+        tq, to, S.lse, m.T, m.H, m.Hkv, W, am ? am + 1 : nullptr);
     CKL();
   }
   TRY(proj<T>(c, {S.o, Ho, false, m.N * Ho, S.o8, S.amax + 1, true, false, true},

@@ -24,7 +24,8 @@
 //             and rescales O_t in TMEM only when the max grows by more than 8
 //             (a factor 256; P stays below 256 in bf16 and the final
 //             normalisation uses the same max, so the result is exact), writes
-//             P_t, and at the end normalises O_t and writes o and the LSE.
+//             P_t, and at the end normalises O_t and writes the LSE, and o
+//             through the then idle Q_t tile with TMA stores.
 // Only key tiles that intersect a query tile's visible range are visited.
 // The grid is one-dimensional and ordered longest-first (see the CTA index
 // mapping).
@@ -49,7 +50,7 @@ __device__ __forceinline__ uint64_t fa_desc_mn(uint32_t tile, int k) {
 }
 
 __global__ void __launch_bounds__(FA_THREADS, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ o, long long ldo,
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_o,
                        float* __restrict__ lse, int T, int H, int Hkv, int window, unsigned int* __restrict__ amax_o) {
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_o);
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -289,28 +291,42 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         mbar_wait_warp(&o_done[tt], (n - 1) & 1, abort_flag, ERRW_TIMEOUT_EPILOGUE)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* orow = o + ((long long)b * T + tq) * ldo + h * 128;
+      // O_t (bf16) leaves through the Q_t tile, free once every S_t product
+      // has completed (they precede the last PV_t that o_done follows): two
+      // 64-column halves of 128 rows x 128 bytes, 128-byte swizzle; each warp
+      // stores its 32 rows with two TMA boxes that clip at the sequence end
+      uint8_t* stg = sQ + tt * FA_TILE;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 4; ++k) {  // columns 32k .. 32k+31
         uint32_t w[32];
         tmem_ld_32x32b_x32(lane_addr + o_col + k * 32, w);
         tmem_ld_wait();
-        if (tq < T) {
-          if (amax_o) {
+        if (amax_o && tq < T) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) oam = fmaxf(oam, fabsf(__uint_as_float(w[i]) * inv));
-          }
+          for (int i = 0; i < 32; ++i) oam = fmaxf(oam, fabsf(__uint_as_float(w[i]) * inv));
+        }
+        uint8_t* row = stg + (k >> 1) * 16384 + r * 128;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint4 u;
-            u.x = pack_bf16(__uint_as_float(w[g * 8 + 0]) * inv, __uint_as_float(w[g * 8 + 1]) * inv);
-            u.y = pack_bf16(__uint_as_float(w[g * 8 + 2]) * inv, __uint_as_float(w[g * 8 + 3]) * inv);
-            u.z = pack_bf16(__uint_as_float(w[g * 8 + 4]) * inv, __uint_as_float(w[g * 8 + 5]) * inv);
-            u.w = pack_bf16(__uint_as_float(w[g * 8 + 6]) * inv, __uint_as_float(w[g * 8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + k * 32 + g * 8) = u;
-          }
+        for (int g = 0; g < 4; ++g) {
+          uint4 u;
+          u.x = pack_bf16(__uint_as_float(w[g * 8 + 0]) * inv, __uint_as_float(w[g * 8 + 1]) * inv);
+          u.y = pack_bf16(__uint_as_float(w[g * 8 + 2]) * inv, __uint_as_float(w[g * 8 + 3]) * inv);
+          u.z = pack_bf16(__uint_as_float(w[g * 8 + 4]) * inv, __uint_as_float(w[g * 8 + 5]) * inv);
+          u.w = pack_bf16(__uint_as_float(w[g * 8 + 6]) * inv, __uint_as_float(w[g * 8 + 7]) * inv);
+          const int cg = (k & 1) * 4 + g;  // 16-byte chunk within the 128-byte half row
+          *reinterpret_cast<uint4*>(row + ((cg ^ (r & 7)) << 4)) = u;
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int row0 = q0 + tt * FA_BM + qw * 32;  // first query of this warp's rows
+      if (lane == 0 && row0 < T) {                 // (a box wholly past the sequence end is not issued)
+        tma_store_3d(&tm_o, stg + qw * 4096, h * 128, row0, b);
+        tma_store_3d(&tm_o, stg + 16384 + qw * 4096, h * 128 + 64, row0, b);
+        bulk_commit_group();
+        bulk_wait_read0();  // the tile's shared memory is read before the CTA ends
+      }
+      __syncwarp();
       if (tq < T) lse[((long long)b * H + h) * T + tq] = (m_used + log2f(l)) * LN2;
     }
     if (amax_o) {  // the warp's max |o| (FP8 amax)
@@ -646,7 +662,7 @@ __global__ void __launch_bounds__(AB2_THREADS, 1)
         tma_store_3d(&tm_dk, stg, kvh * 128 + cb * 64, k0 + qw * 32, b);
         tma_store_3d(&tm_dv, stg + 4096, kvh * 128 + cb * 64, k0 + qw * 32, b);
         bulk_commit_group();
-        bulk_wait0();
+        bulk_wait_read0();  // the staging tiles are read before the CTA ends
       }
       __syncwarp();
     }
