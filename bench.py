@@ -403,10 +403,11 @@ def main():
     ap.add_argument("--workload", default="d24", choices=list(synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    # smaller footprints of the same workload for profiler captures; a line
-    # printed with either override is not the workload's measurement
+    # smaller footprints (or other shapes) of the same workload for profiler
+    # captures; a line printed with any override is not the workload's measurement
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling only)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the sequence length (profiling only)")
     ap.add_argument("--optimizer", action="store_true",
                     help="time the optimizer step (Muon + AdamW) instead of the training step")
     ap.add_argument("--muon-per-matrix", action="store_true",
@@ -422,6 +423,8 @@ def main():
         over["B"] = args.batch
     if args.layers:
         over["n_layer"] = args.layers
+    if args.seq_len:
+        over["T"] = args.seq_len
     c = synth.config(args.workload, **over)
     if over:
         c["name"] = c["name"] + "_profiling_" + "_".join(f"{k}{v}" for k, v in over.items())
