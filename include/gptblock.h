@@ -399,9 +399,13 @@ int gptb_set_wait_limit_ns(unsigned long long ns);
 void gptb_reset_counters(void);
 long long gptb_launch_count(void);
 int gptb_set_gemm_timing(int enable);
-/* Sum of GEMM device milliseconds and FLOPs since the last reset (syncs);
- * ms_fp8 / flops_fp8: the part of those from GEMMs with e4m3 operands.  Any
- * output pointer may be NULL. */
+/* GEMM device milliseconds and FLOPs since the last reset (syncs).  The
+ * milliseconds are the time covered by the GEMM launches: the union of their
+ * event intervals on one time base, i.e. the sum of their durations when no
+ * two overlap and each instant counted once when launches on two streams run
+ * together (the bf16 backward issues its weight-gradient GEMMs on a second
+ * stream).  ms_fp8 / flops_fp8: the same for the GEMMs with e4m3 operands.
+ * Any output pointer may be NULL. */
 int gptb_gemm_timing(double* ms, double* flops, double* ms_fp8, double* flops_fp8, long long* launches);
 
 /* Human-readable text for a return code. */
