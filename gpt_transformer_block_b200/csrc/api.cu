@@ -522,7 +522,7 @@ struct Scratch {
   // backward
   void *du, *dh2, *dx1, *dO, *dqkv, *dh;
   float *D, *dq, *dk, *dv, *dz;
-  uint8_t* g8;   // FP8: e4m3 copy of the gradient feeding a GEMM pair
+  uint8_t* g8[4];  // FP8: e4m3 copies of the gradients feeding a GEMM pair [dx_out, du, dx1, dqkv]
   float* gamax;  // FP8: amax of the gradients [dx_out, du, dx1, dqkv]
 };
 Scratch carve_scratch(Carve& cv, const Dims& m) {
@@ -545,11 +545,13 @@ Scratch carve_scratch(Carve& cv, const Dims& m) {
   s.dk = (float*)cv.take(m.N * (long long)m.Hkv * m.hd * 4);
   s.dv = (float*)cv.take(m.N * (long long)m.Hkv * m.hd * 4);
   s.dz = (float*)cv.take(m.N * m.Hkv * 4);
-  s.g8 = nullptr;
+  for (auto& q : s.g8) q = nullptr;
   s.gamax = nullptr;
-  if (m.fp8) {
-    const long long w = std::max<long long>(std::max<long long>(m.Wq, m.F), std::max<long long>(m.d, (long long)m.H * m.hd));
-    s.g8 = (uint8_t*)cv.take(m.N * w);
+  if (m.fp8) {  // one copy per gradient: the weight-gradient GEMM on the side stream may still read one
+    s.g8[0] = (uint8_t*)cv.take(m.N * m.d);
+    s.g8[1] = (uint8_t*)cv.take(m.N * m.F);
+    s.g8[2] = (uint8_t*)cv.take(m.N * m.d);
+    s.g8[3] = (uint8_t*)cv.take(m.N * m.Wq);
     s.gamax = (float*)cv.take(4 * 4);  // [block input gradient, du, dx1, dqkv]
   }
   cv.off = std::max(cv.off, fwd_end);
@@ -824,17 +826,21 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     CK(cudaMemsetAsync(X.gamax + 1, 0, 3 * sizeof(float), st));
   }
   const bool e5 = m.grad_e5m2;
-  // bf16: the weight-gradient GEMMs go to the side stream, each forked as
-  // soon as its inputs are written and issued after the input-gradient GEMM
-  // beside it (measured: 2 % off the d24 step, 4 % of its clock cycles; forking
-  // them next to the memory-bound kernels instead was slower).  FP8 keeps one
-  // stream: there the weight-gradient GEMM writes the gradient's e4m3 copy
-  // that the input-gradient GEMM reads.
+  // The weight-gradient GEMMs go to the side stream, each forked as soon as
+  // its inputs are written and issued after the input-gradient GEMM beside it
+  // (measured: 2 % off the d24 step, 4 % of its clock cycles; forking them
+  // next to the memory-bound kernels instead was slower).  FP8: the gradient's
+  // e4m3 copy, which both GEMMs of a pair read, is made on the main stream
+  // before the fork (on one stream the weight-gradient GEMM makes it).
   SideStream* ss = nullptr;
-  if (!m.fp8 && dt != GPTB_F32) {
+  if (dt != GPTB_F32) {
     SideStream& s2 = side_stream();
     if (s2.ok) ss = &s2;
   }
+  const bool q_first = ss && m.fp8;
+  auto qgrad = [&](int i, const void* p, long long elems, bool amax_ready) -> int {
+    return q_first ? quant<T>((const T*)p, elems, X.g8[i], ga[i], e5, st, amax_ready) : GPTB_OK;
+  };
   cudaStream_t sw = ss ? ss->s : st;  // stream of the weight-gradient GEMMs
   auto fork = [&](int e) -> int {
     if (ss) {
@@ -844,31 +850,33 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     return GPTB_OK;
   };
   auto wgrad_proj = [&]() {
-    return proj<T>(c, {dx2, m.d, true, Nd, X.g8, ga[0], true, e5}, {S.act, m.F, true, 0, S.act8, S.amax + 3, false},
+    return proj<T>(c, {dx2, m.d, true, Nd, X.g8[0], ga[0], !q_first, e5}, {S.act, m.F, true, 0, S.act8, S.amax + 3, false},
                    m.d, m.F, N, epi(EPI_ACCUM_F32, dt, g.w_proj, m.F), sw);
   };
   auto wgrad_fc = [&]() {
-    return proj<T>(c, {X.du, m.F, true, m.N * m.F, X.g8, ga[1], true, e5, true},
+    return proj<T>(c, {X.du, m.F, true, m.N * m.F, X.g8[1], ga[1], !q_first, e5, true},
                    {S.h2, m.d, true, 0, S.h2_8, S.amax + 2, false}, m.F, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_fc, m.d),
                    sw);
   };
   EpiParams edr = epi(EPI_DRELU2, dt, X.du, m.F, S.act, m.F);
   edr.amax_out = gam[1];
   if (ss) {
-    TRY(fork(0));  // dx2 and the saved activations are ready
-    TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, ga[0], false, e5},
+    TRY(qgrad(0, dx2, Nd, false));
+    TRY(fork(0));  // dx2 (and its e4m3 copy) and the saved activations are ready
+    TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8[0], ga[0], false, e5},
                 {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false}, N, m.F, m.d, edr, st));
     TRY(wgrad_proj());
+    TRY(qgrad(1, X.du, m.N * m.F, true));
     TRY(fork(1));  // du
-    TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, ga[1], false, e5},
+    TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8[1], ga[1], false, e5},
                 {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false}, N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
     TRY(wgrad_fc());
   } else {
     TRY(wgrad_proj());
-    TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8, ga[0], false, e5},
+    TRY(proj<T>(c, {dx2, m.d, false, Nd, X.g8[0], ga[0], false, e5},
                 {w.w_proj, m.F, true, 0, S.wproj8, S.amax + 7, false}, N, m.F, m.d, edr, st));
     TRY(wgrad_fc());
-    TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8, ga[1], false, e5},
+    TRY(proj<T>(c, {X.du, m.F, false, m.N * m.F, X.g8[1], ga[1], false, e5},
                 {w.w_fc, m.d, true, 0, S.wfc8, S.amax + 6, false}, N, m.d, m.F, epi(EPI_STORE, dt, X.dh2, m.d), st));
   }
   br_norm_bwd_kernel<T><<<brg, brt, 0, st>>>(dx2, (const T*)X.dh2, (const T*)S.h2, S.rstd2, (T*)X.dx1, m.N, m.d,
@@ -876,11 +884,15 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   CKL();
   // attention output projection
   auto wgrad_o = [&]() {
-    return proj<T>(c, {X.dx1, m.d, true, Nd, X.g8, ga[2], true, e5, true}, {S.o, Ho, true, 0, S.o8, S.amax + 1, false},
+    return proj<T>(c, {X.dx1, m.d, true, Nd, X.g8[2], ga[2], !q_first, e5, true}, {S.o, Ho, true, 0, S.o8, S.amax + 1, false},
                    m.d, (int)Ho, N, epi(EPI_ACCUM_F32, dt, g.w_o, Ho), sw);
   };
-  if (ss) TRY(fork(2));  // dx1
-  else TRY(wgrad_o());
+  if (ss) {
+    TRY(qgrad(2, X.dx1, Nd, true));
+    TRY(fork(2));  // dx1
+  } else {
+    TRY(wgrad_o());
+  }
   // dO = dx1 Wo, and the attention backward's D = rowsum(dO * o) per head
   if constexpr (std::is_same<T, bf16>::value) {
     // bf16 / FP8 configurations: D comes out of the dO GEMM's epilogue (o read by TMA)
@@ -888,11 +900,11 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     ed.rowdot = X.D;
     ed.T = m.T;
     ed.H = m.H;
-    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, ga[2], false, e5}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8[2], ga[2], false, e5}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
                 (int)Ho, m.d, ed, st));
     if (ss) TRY(wgrad_o());
   } else {
-    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8, ga[2], true, e5}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
+    TRY(proj<T>(c, {X.dx1, m.d, false, Nd, X.g8[2], ga[2], true, e5}, {w.w_o, Ho, true, 0, S.wo8, S.amax + 5, false}, N,
                 (int)Ho, m.d, epi(EPI_STORE, dt, X.dO, Ho), st));
     attn_bwd_pre_kernel<T><<<grid_rows(m.N * m.H), EW_THREADS, 0, st>>>((const T*)S.o, Ho, (const T*)X.dO, Ho, X.D,
                                                                        m.B, m.T, m.H, m.hd);
@@ -937,7 +949,7 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
   CKL();
   // QKV projection
   auto wgrad_qkv = [&]() -> int {
-    TRY(proj<T>(c, {X.dqkv, m.Wq, true, m.N * m.Wq, X.g8, ga[3], true, e5, true},
+    TRY(proj<T>(c, {X.dqkv, m.Wq, true, m.N * m.Wq, X.g8[3], ga[3], !q_first, e5, true},
                 {S.h, m.d, true, 0, S.h8, S.amax + 0, false}, m.Wq, m.d, N, epi(EPI_ACCUM_F32, dt, g.w_qkv, m.d), sw));
     if (ve) {
       const int nthreads = ((m.Hkv * c.ve_gate_ch + 31) / 32) * 32;
@@ -948,9 +960,13 @@ int block_bwd_impl(const gptb_config& c, int layer, const gptb_block_weights& w,
     }
     return GPTB_OK;
   };
-  if (ss) TRY(fork(3));  // dqkv, dz
-  else TRY(wgrad_qkv());
-  TRY(proj<T>(c, {X.dqkv, m.Wq, false, m.N * m.Wq, X.g8, ga[3], false, e5},
+  if (ss) {
+    TRY(qgrad(3, X.dqkv, m.N * m.Wq, true));
+    TRY(fork(3));  // dqkv, dz
+  } else {
+    TRY(wgrad_qkv());
+  }
+  TRY(proj<T>(c, {X.dqkv, m.Wq, false, m.N * m.Wq, X.g8[3], ga[3], false, e5},
               {w.w_qkv, m.d, true, 0, S.wqkv8, S.amax + 4, false}, N, m.d, m.Wq, epi(EPI_STORE, dt, X.dh, m.d), st));
   if (ss) TRY(wgrad_qkv());
   br_mix_norm_bwd_warp_kernel<T><<<warp_rows_grid(m.N), 256, 0, st>>>((const T*)X.dh, ve ? X.dz : nullptr,
