@@ -1459,23 +1459,33 @@ int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cach
   if (workspace_bytes < gptb_decode_workspace_bytes(B, H, T_max)) return GPTB_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* part = static_cast<float*>(workspace);
-  // the V cache as a [B*T_max, Hkv*128] bf16 matrix, read in unswizzled boxes of DEC_SPLIT rows x 128 columns
-  CUtensorMap tv;
+  // the K and V caches as [B*T_max, Hkv*128] bf16 matrices: K in two 64-column
+  // boxes of DEC_SPLIT rows with a 128-byte swizzle, V in one unswizzled box of
+  // DEC_SPLIT rows x 128 columns
+  CUtensorMap tk, tv;
   {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return GPTB_ERR_CUDA;
     cuuint64_t dims[2] = {(cuuint64_t)Hkv * DEC_HD, (cuuint64_t)B * T_max};
     cuuint64_t strides[1] = {(cuuint64_t)Hkv * DEC_HD * 2};
-    cuuint32_t box[2] = {DEC_HD, DEC_SPLIT};
+    cuuint32_t boxk[2] = {64, DEC_SPLIT};
+    cuuint32_t boxv[2] = {DEC_HD, DEC_SPLIT};
     cuuint32_t estr[2] = {1, 1};
-    if (fn(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v_cache), dims, strides, box, estr,
+    if (fn(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache), dims, strides, boxk, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GPTB_ERR_CUDA;
+    if (fn(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v_cache), dims, strides, boxv, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return GPTB_ERR_CUDA;
   }
-  CK(cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_V_BYTES));
-  decode_split_kernel<<<B * Hkv * decode_pieces(T_max), DEC_THREADS, DEC_V_BYTES, st>>>(
-      tv, static_cast<const bf16*>(q), static_cast<const bf16*>(k_cache), lens, part, H, Hkv, T_max, window);
+  const long long items = (long long)B * Hkv * decode_pieces(T_max);
+  if (items > INT_MAX) return GPTB_ERR_UNSUPPORTED;
+  const int grid = (int)std::min<long long>(items, std::max(1, dev_info().sms));  // persistent
+  CK(cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM));
+  decode_split_kernel<<<grid, DEC_THREADS, DEC_SMEM, st>>>(tk, tv, static_cast<const bf16*>(q), lens, part, H, Hkv,
+                                                            T_max, window, (int)items);
   CKL();
   decode_combine_kernel<<<B * H, DEC_HD, 0, st>>>(part, lens, static_cast<bf16*>(o), lse, H, T_max);
   CKL();

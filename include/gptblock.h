@@ -358,11 +358,11 @@ int gptb_muon_step_batched(int count, float* const* w, void* const* w_bf16, cons
  *            the softmax denominator incl. its max) or NULL
  *   workspace: device, gptb_decode_workspace_bytes(B, H, T_max) bytes, 16-byte
  *            aligned (partial softmax sums of the key pieces; the keys of a
- *            sequence are split into pieces of 256 handled in parallel, then
- *            combined)
+ *            sequence are split into pieces of 128, spread over the SMs and
+ *            streamed through shared memory, then combined)
  * Errors: GPTB_ERR_INVALID_ARG (null / misaligned pointers, H % H_kv != 0),
  * GPTB_ERR_WORKSPACE (workspace too small), GPTB_ERR_UNSUPPORTED (more than
- * 16 query heads per kv head). */
+ * 8 query heads per kv head). */
 size_t gptb_decode_workspace_bytes(int B, int H, int T_max);
 int gptb_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, void* o,
                           float* lse, int B, int H, int Hkv, int T_max, int window, void* workspace,
