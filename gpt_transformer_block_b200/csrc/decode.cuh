@@ -252,7 +252,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   }
 }
 
-// one CTA of DEC_HD threads per (sequence, query head): combine the pieces
+// one CTA of DEC_HD threads per (sequence, query head): combine the pieces in
+// one pass (running max; the sums so far are rescaled when it grows), four
+// pieces' loads in flight at a time
 __global__ void __launch_bounds__(DEC_HD)
     decode_combine_kernel(const float* __restrict__ part, const int32_t* __restrict__ lens, bf16* __restrict__ o,
                           float* __restrict__ lse, int H, int Tmax) {
@@ -262,16 +264,31 @@ __global__ void __launch_bounds__(DEC_HD)
   const float* pp = part + (long long)bh * P * DEC_PART;
   const int len = lens[b];
   const bool valid = len >= 1 && len <= Tmax;
-  float m = -INFINITY;
-  for (int p = 0; p < P; ++p) m = fmaxf(m, pp[(long long)p * DEC_PART]);
-  float l = 0.f, acc = 0.f;
-  if (valid && m > -INFINITY) {
-    for (int p = 0; p < P; ++p) {
-      const float mp = pp[(long long)p * DEC_PART];
-      if (mp == -INFINITY) continue;
-      const float w = expf(mp - m);
-      l = fmaf(pp[(long long)p * DEC_PART + 1], w, l);
-      acc = fmaf(pp[(long long)p * DEC_PART + 2 + d], w, acc);
+  float m = -INFINITY, l = 0.f, acc = 0.f;
+  if (valid) {
+    for (int p0 = 0; p0 < P; p0 += 4) {
+      float mp[4], lp[4], op[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool in = p0 + u < P;
+        const float* q = pp + (long long)(in ? p0 + u : 0) * DEC_PART;
+        mp[u] = in ? q[0] : -INFINITY;
+        lp[u] = in ? q[1] : 0.f;
+        op[u] = in ? q[2 + d] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (mp[u] == -INFINITY) continue;  // an empty piece
+        if (mp[u] > m) {
+          const float r = expf(m - mp[u]);  // 0 while m is -inf
+          l *= r;
+          acc *= r;
+          m = mp[u];
+        }
+        const float w = expf(mp[u] - m);
+        l = fmaf(lp[u], w, l);
+        acc = fmaf(op[u], w, acc);
+      }
     }
   }
   o[(long long)bh * DEC_HD + d] = __float2bfloat16_rn(l > 0.f ? acc / l : 0.f);
