@@ -360,6 +360,23 @@ def run_decode(args, c: dict):
 METRIC = "training tokens/sec (fwd+bwd) on 1 B200 and MFU vs bf16/FP8 tensor peak"
 
 
+def workload_config(name: str, batch: int = 0, layers: int = 0, seq_len: int = 0) -> dict:
+    """The named workload, with the profiling overrides (0 = keep) applied; an
+    overridden workload is renamed so that its line cannot pass for the
+    workload's own measurement."""
+    over = {}
+    if batch:
+        over["B"] = batch
+    if layers:
+        over["n_layer"] = layers
+    if seq_len:
+        over["T"] = seq_len
+    c = synth.config(name, **over)
+    if over:
+        c["name"] = c["name"] + "_profiling_" + "_".join(f"{k}{v}" for k, v in over.items())
+    return c
+
+
 def step_config(c: dict, world: int) -> dict:
     """The `config` object of the training-step line (both arms)."""
     return {"workload": c["name"], "global_batch": c["B"] * world, "seq_len": c["T"],
@@ -418,16 +435,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    over = {}
-    if args.batch:
-        over["B"] = args.batch
-    if args.layers:
-        over["n_layer"] = args.layers
-    if args.seq_len:
-        over["T"] = args.seq_len
-    c = synth.config(args.workload, **over)
-    if over:
-        c["name"] = c["name"] + "_profiling_" + "_".join(f"{k}{v}" for k, v in over.items())
+    c = workload_config(args.workload, args.batch, args.layers, args.seq_len)
     fl = flops_per_token(c)
     if args.impl == "reference":
         run_reference(args, c, fl)

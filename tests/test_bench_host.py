@@ -1,6 +1,7 @@
 """Host-side arithmetic of bench.py (CPU only): the attention pair count that
 the FLOP and roofline figures rest on, the per-token FLOPs of the headline
-workload, and the committed traffic line that feeds roofline.traffic."""
+workload, the committed traffic line that feeds roofline.traffic, and the
+profiling overrides of the workload's shape."""
 import numpy as np
 import pytest
 
@@ -37,3 +38,15 @@ def test_flops_per_token_d24_by_hand():
 def test_traffic_line_is_read_from_the_committed_summary():
     assert bench.profile_traffic("d24") == pytest.approx(5.065e8)
     assert bench.profile_traffic("no_such_workload") is None
+
+
+def test_profiling_overrides_reshape_and_rename_the_workload():
+    c = bench.workload_config("d24")
+    assert (c["name"], c["B"], c["T"], c["n_layer"]) == ("d24", 16, 2048, 24)
+    o = bench.workload_config("d24", batch=8, layers=2, seq_len=4096)
+    assert (o["B"], o["T"], o["n_layer"]) == (8, 4096, 2)
+    assert o["name"].startswith("d24_profiling_") and o["name"] != "d24"
+    # the per-layer lists follow the layer count, the model width does not change
+    assert len(o["window"]) == 2 and len(o["has_ve"]) == 2 and o["d"] == c["d"]
+    # the FLOP count per token grows with T (attention) and shrinks with the layer count
+    assert bench.flops_per_token(o)["algorithmic"] != bench.flops_per_token(c)["algorithmic"]
