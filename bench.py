@@ -352,7 +352,9 @@ def run_decode(args, c: dict):
                       "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
                       "dtype": "bf16", "data": "synthetic",
                       "config": {"workload": c["name"] + "_decode", "batch": B, "cached_tokens": T, "heads": H,
-                                 "kv_heads": Hk},
+                                 "kv_heads": Hk,
+                                 "l2": f"K/V caches ({2 * B * T * Hk * 128 * 2 / 1e6:.0f} MB) read every step; "
+                                       "no flush between steps"},
                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                                    "frac": gbs / peak, "bytes": nbytes}}))
 
