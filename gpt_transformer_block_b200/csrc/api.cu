@@ -284,9 +284,7 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
 
 // GEMMs with at least this many rows run in the pair form (two CTAs, M = 256
 // per tile); smaller ones in the single-CTA form.
-#ifndef GPTB_PAIR_MIN_M
-#define GPTB_PAIR_MIN_M 256
-#endif
+constexpr int GEMM_PAIR_MIN_M = 256;
 
 // C[b] = A[b] op B[b] for b < batch: operand b starts bs* elements after
 // operand 0 (tensor-core path only; the epilogue kinds with per-row side
@@ -343,7 +341,7 @@ int gemm_batched(int dtype, Op A, Op B, int M, int N, int K, EpiParams ep, int b
         (ep.ldo % (acc32 ? 4 : 8)) || (N % 8))
       return GPTB_ERR_INVALID_ARG;
     if (has_aux && (!aligned16(ep.aux) || ep.ld_aux % 8)) return GPTB_ERR_INVALID_ARG;
-    const bool pair = M >= GPTB_PAIR_MIN_M;
+    const bool pair = M >= GEMM_PAIR_MIN_M;
     const int b_rows = pair ? TcShape<true>::B_ROWS : TcShape<false>::B_ROWS;  // rows of B one CTA stages
     CUtensorMap ta, tb, to, to2, tx;
     const int oe = f8 ? 1 : 2;  // operand element size
